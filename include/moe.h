@@ -1,0 +1,242 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a single-GPU (sm_100a) implementation of the
+ * sparse Mixture-of-Experts expert layer: router -> top-k -> residency
+ * lookup -> bucketing -> dequantised SwiGLU experts -> weighted combine +
+ * residual write-back.
+ *
+ * The problem statement these calls follow is the per-layer flow of the
+ * Strata engine analysis article "93 token/s on one 8 GB card"
+ * (m.lqnn.cn/news/264700), section "Architecture overview": prompts are cut
+ * into chunks of at most 8,192 tokens for prefill; then, layer by layer, the
+ * router picks the 10 of 512 experts a token activates, the selected experts
+ * are computed, and their outputs are combined into the residual.  The
+ * "Doorbell handshake" section splits each block at the router ("pre" ends
+ * with router ids + weights, "post" combines expert outputs and writes the
+ * residual back); the "Expert cache" section defines the residency table
+ * (layer, expert) -> slot or -1.  The model shape (48 layers, 512 experts,
+ * 10 routed + 1 shared) is from lcz.me topic 2059, section 2 "Model and
+ * principles".
+ *
+ * Conventions (all calls):
+ *  - Every call returns a moe_status; no exception or exit() crosses the ABI.
+ *    moe_last_error(ctx) gives a one-line description of the last failure.
+ *  - Pointers named *_dev are device pointers the caller owns (for example
+ *    torch tensors' data_ptr()); the library never frees them.  Weight-load
+ *    calls take host or device pointers (src_is_device) and COPY the data;
+ *    the caller may free its buffers as soon as the call returns.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream.  Compute calls are asynchronous on that stream; the
+ *    caller must keep its buffers alive until the stream passes the call.
+ *  - Layouts are row-major and densely packed unless stated otherwise.
+ *    Activations are bfloat16 bit patterns (uint16), router weights fp32.
+ *  - A context is used from one host thread at a time and on the device that
+ *    was current when it was created.
+ *
+ * Packed expert format (input of moe_load_experts / moe_load_shared).  The
+ * pages print no bit layout; these formats are this library's own:
+ *  - One expert is the triple Wg [f,d], Wu [f,d], Wd [d,f] (row-major; the
+ *    reduction dimension is contiguous).  y = Wd (SiLU(Wg h) * (Wu h)),
+ *    SiLU(z) = z / (1 + exp(-z)).
+ *  - MOE_Q4_SYM_G32_F16: groups of 32 along the reduction dimension;
+ *    value = s * (c - 8), c a 4-bit code, two codes per byte with the lower
+ *    index in the low nibble; s is an fp16 scale per (row, group).
+ *  - MOE_Q2_ASYM_G64_F16: groups of 64; value = s * q + m, q a 2-bit code,
+ *    four per byte with element i in bits 2*(i%4); s and m are fp16 per
+ *    (row, group).
+ *  - codes: for each expert, Wg's codes, then Wu's, then Wd's; experts back
+ *    to back.  scales (and mins) follow the same order, [rows, K/group] per
+ *    matrix.  Per expert: Q4 3*f*d/2 code bytes + 3*f*d/32 scales;
+ *    Q2 3*f*d/4 code bytes + 3*f*d/64 scales + as many mins.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_ctx moe_ctx; /* opaque, library-owned */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad size, index or pointer; nothing was done */
+  MOE_ERR_OOM = 2,         /* device allocation failed */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call failed (see last_error) */
+  MOE_ERR_STATE = 4,       /* call order violated (e.g. forward before load) */
+  MOE_ERR_BAD_SLOT = 5,    /* device saw a slot id outside the slot pool */
+  MOE_ERR_DEVICE = 6,      /* device saw another bad value (expert id, ...) */
+  MOE_ERR_TIMEOUT = 7,     /* moe_sync gave up waiting */
+  MOE_ERR_NOT_SUPPORTED = 8 /* valid request this build does not handle */
+} moe_status;
+
+enum { MOE_Q4_SYM_G32_F16 = 1, MOE_Q2_ASYM_G64_F16 = 2 };
+
+/* Statistics of the most recent routed call (moe_get_stats). */
+typedef struct {
+  int64_t calls;            /* routed calls since create / last reset */
+  int64_t tokens;           /* tokens routed since create */
+  int64_t hits;             /* (token, expert) pairs served from the slot pool */
+  int64_t misses;           /* pairs served from the backing arena */
+  int64_t near_ties;        /* tokens whose k-th and (k+1)-th fp32 logits
+                               differ by less than 1e-5 */
+  int32_t last_T;           /* tokens of the last routed call */
+  int32_t last_active;      /* distinct experts of the last call */
+  int32_t last_layer;
+  int32_t E;                /* number of entries written to expert_count */
+  const int32_t *expert_count; /* host array [E]: tokens per expert, last call;
+                                  owned by the context, valid until the next
+                                  moe_get_stats or moe_destroy */
+} moe_stats;
+
+/* moe_create: a context for a layer of hidden size d, SwiGLU width f,
+ * E experts, top-k routing and the given quant format.  Defaults: 1 layer,
+ * no shared expert, no slot pool, up to 64 tokens per call; change them with
+ * moe_configure before the first load.
+ * Errors: INVALID_ARG if d or f is not a multiple of 128, E < 1 or E > 1024,
+ * k < 1, k > E or k > 32, or quant_fmt unknown; CUDA if no device. */
+MOE_API moe_status moe_create(int d, int f, int E, int k, int quant_fmt, moe_ctx **out);
+
+/* moe_configure: model size and call limits; allocates all device memory
+ * (weights arena for n_layers * E experts, n_shared shared experts per layer
+ * (0 or 1), a slot pool of n_slots experts, scratch for max_tokens tokens per
+ * call).  Must come before any load; may be called once.
+ * Errors: INVALID_ARG on n_layers < 1, n_shared not 0/1, n_slots < 0,
+ * max_tokens < 1; STATE if weights were already loaded; OOM. */
+MOE_API moe_status moe_configure(moe_ctx *ctx, int n_layers, int n_shared, int n_slots,
+                         int max_tokens);
+
+/* moe_destroy: frees everything the context owns (synchronises the device
+ * first).  NULL is accepted and ignored. */
+MOE_API moe_status moe_destroy(moe_ctx *ctx);
+
+/* moe_load_experts: copy n_experts packed experts (format above) into
+ * experts [first_expert, first_expert + n_experts) of `layer`, repacking them
+ * into the library's device layout.  Also refreshes any slot-pool copies of
+ * those experts.  Synchronous.  Errors: INVALID_ARG on a bad range or NULL
+ * codes/scales (or NULL mins for Q2); OOM; CUDA. */
+MOE_API moe_status moe_load_experts(moe_ctx *ctx, int layer, int first_expert,
+                            int n_experts, const void *codes,
+                            const void *scales, const void *mins,
+                            int src_is_device);
+
+/* moe_load_shared: the shared expert of `layer` (same format, one expert).
+ * Errors: STATE if configured with n_shared = 0; else as moe_load_experts. */
+MOE_API moe_status moe_load_shared(moe_ctx *ctx, int layer, const void *codes,
+                           const void *scales, const void *mins,
+                           int src_is_device);
+
+/* moe_set_router: router weight W fp32 [E, d] and optional bias fp32 [E]
+ * (NULL = no bias) of `layer`.  Synchronous copy. */
+MOE_API moe_status moe_set_router(moe_ctx *ctx, int layer, const float *W,
+                          const float *bias, int src_is_device);
+
+/* moe_set_norm: RMSNorm before the router for `layer`: h = x * (mean(x^2) +
+ * eps)^-1/2 * gamma.  gamma is a HOST fp32 [d] array or NULL for gamma = 1.
+ * Without this call a layer uses h = x (no norm). */
+MOE_API moe_status moe_set_norm(moe_ctx *ctx, int layer, const float *gamma, float eps);
+
+/* moe_set_slots: residency table, HOST int32 [n_layers * E]: slot id of
+ * (layer, expert) in the slot pool, or -1 when it is served from the backing
+ * arena (every expert always has a backing copy, so results do not depend on
+ * the table).  Copies the experts into their slots (synchronous).
+ * Errors: INVALID_ARG on a slot >= n_slots or a slot used twice. */
+MOE_API moe_status moe_set_slots(moe_ctx *ctx, const int32_t *slot_of);
+
+/* moe_route: router logits + top-k + softmax + bucketing for T tokens of
+ * `layer`.  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
+ * w_dev fp32 [T, k] receive each token's experts and renormalised weights,
+ * ordered by descending logit (equal logits: lower expert id first).
+ * bucket_off_dev int32 [E+1] (exclusive prefix of tokens per expert) and
+ * bucket_perm_dev int32 [T*k] (pair ids t*k+j grouped by expert, ascending t
+ * inside an expert) may be NULL.  Errors: INVALID_ARG if T < 1 or T >
+ * max_tokens or a required pointer is NULL. */
+MOE_API moe_status moe_route(moe_ctx *ctx, int layer, const void *h_dev, int T,
+                     int32_t *idx_dev, float *w_dev, int32_t *bucket_off_dev,
+                     int32_t *bucket_perm_dev, void *stream);
+
+/* moe_bucket: bucketing alone, for caller-provided routing idx_dev int32
+ * [T, k] (distinct expert ids per token).  Outputs as in moe_route.  An id
+ * outside [0, E) sets the device error status (moe_sync returns DEVICE). */
+MOE_API moe_status moe_bucket(moe_ctx *ctx, const int32_t *idx_dev, int T,
+                      int32_t *bucket_off_dev, int32_t *bucket_perm_dev,
+                      void *stream);
+
+/* moe_forward: one decode window of T tokens through `layer`, in place:
+ * x <- x + MoE(norm(x)).  x_dev: bf16 [T, d].  Runs router, top-k, residency
+ * lookup, bucketing, the grouped dequant-SwiGLU experts (+ shared expert)
+ * and the combine + residual kernel.  Errors: INVALID_ARG, STATE (router or
+ * experts not loaded). */
+MOE_API moe_status moe_forward(moe_ctx *ctx, int layer, void *x_dev, int T,
+                       void *stream);
+
+/* moe_forward_delta: as moe_forward but leaves x unchanged and writes the
+ * fp32 MoE output delta_dev [T, d] (the value added to the residual). */
+MOE_API moe_status moe_forward_delta(moe_ctx *ctx, int layer, const void *x_dev, int T,
+                             float *delta_dev, void *stream);
+
+/* moe_forward_stack: moe_forward through layers 0..n_layers-1 in order.  The
+ * first call for a given (x_dev, T) records the whole stack as one CUDA
+ * graph; later calls replay it.  Do not call it while `stream` is being
+ * captured by the caller. */
+MOE_API moe_status moe_forward_stack(moe_ctx *ctx, void *x_dev, int T, void *stream);
+
+/* moe_prefill: a prefill chunk of N tokens (N <= max_tokens) through
+ * `layer`, in place (x <- x + MoE(norm(x))), using the tensor-core grouped
+ * GEMM path for experts that receive many tokens. */
+MOE_API moe_status moe_prefill(moe_ctx *ctx, int layer, void *x_dev, int N,
+                       void *stream);
+
+/* moe_sync: wait (polling cudaEventQuery, at most timeout_ms; < 0 = no
+ * limit) until the work queued by this context has finished, then read and
+ * clear the device error status.  Returns TIMEOUT, BAD_SLOT, DEVICE, CUDA or
+ * OK. */
+MOE_API moe_status moe_sync(moe_ctx *ctx, int timeout_ms);
+
+/* moe_get_stats: synchronises and fills *out (see moe_stats). */
+MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
+
+/* Profiling: when enabled, every forward call records CUDA events on its
+ * stream around its three segments -- routing (norm + router + top-k +
+ * bucketing), experts (the two grouped dequant-GEMV kernels) and combine --
+ * into a pool of 8192 call slots.  The events sit between the kernels, so a
+ * profiled call loses the launch overlap at those three points.  Events are
+ * recorded as external graph nodes, so profiled calls may be captured. */
+MOE_API moe_status moe_set_profiling(moe_ctx *ctx, int enable);
+
+/* Synchronises, then adds the elapsed milliseconds of the profiled calls
+ * made since profiling was last enabled (at most the 8192 most recent) to
+ * ms[0] (routing), ms[1] (experts), ms[2] (combine) and returns their number
+ * in *n_calls.  Reading does not consume the slots: after a replay of a
+ * captured graph, a new read gives that replay's times.  moe_set_profiling
+ * (ctx, 1) starts a new set.  ms is caller-owned host memory. */
+MOE_API moe_status moe_read_profile(moe_ctx *ctx, double ms[3], int64_t *n_calls);
+
+/* Last error message of ctx (never NULL; "" when none). */
+MOE_API const char *moe_last_error(const moe_ctx *ctx);
+
+/* Static name of a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* Debug hook for fault-injection tests: writes one raw entry of the device
+ * residency table WITHOUT the host validation of moe_set_slots.  A slot id
+ * outside the pool is then caught by the routing kernel, which falls back to
+ * the backing copy and sets the device status that moe_sync reports as
+ * MOE_ERR_BAD_SLOT.  Not for production use. */
+MOE_API moe_status moe_debug_poke_slot(moe_ctx *ctx, int layer, int expert, int32_t slot);
+
+/* Bytes one packed expert occupies in the given format (codes + scales +
+ * mins), or -1 for bad arguments. */
+MOE_API int64_t moe_expert_bytes(int d, int f, int quant_fmt);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,237 @@
+"""Thin ctypes binding of libmoe.so (include/moe.h), same function names.
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+Arrays may be passed as torch tensors (device or host), numpy arrays (host)
+or raw integer addresses.  A status other than MOE_OK raises MoeError.  The
+library must have been built (``python -m sparse_moe_expert_gemv_b200.build``);
+importing this module without it raises ImportError -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_OOM", 3: "MOE_ERR_CUDA",
+                4: "MOE_ERR_STATE", 5: "MOE_ERR_BAD_SLOT", 6: "MOE_ERR_DEVICE",
+                7: "MOE_ERR_TIMEOUT", 8: "MOE_ERR_NOT_SUPPORTED"}
+MOE_Q4_SYM_G32_F16 = 1
+MOE_Q2_ASYM_G64_F16 = 2
+
+# every symbol include/moe.h declares
+EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
+           "moe_load_shared", "moe_set_router", "moe_set_norm", "moe_set_slots",
+           "moe_route", "moe_bucket", "moe_forward", "moe_forward_delta",
+           "moe_forward_stack", "moe_prefill", "moe_sync", "moe_get_stats",
+           "moe_last_error", "moe_status_string", "moe_expert_bytes",
+           "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class MoeStats(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_int64), ("tokens", ctypes.c_int64),
+                ("hits", ctypes.c_int64), ("misses", ctypes.c_int64),
+                ("near_ties", ctypes.c_int64), ("last_T", ctypes.c_int32),
+                ("last_active", ctypes.c_int32), ("last_layer", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("expert_count", ctypes.POINTER(ctypes.c_int32))]
+
+
+def _load():
+    if not os.path.exists(SO_PATH):
+        raise ImportError(f"{SO_PATH} is missing: build it with "
+                          "`python -m sparse_moe_expert_gemv_b200.build`")
+    L = ctypes.CDLL(SO_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sig = {
+        "moe_create": [I, I, I, I, I, ctypes.POINTER(P)],
+        "moe_configure": [P, I, I, I, I],
+        "moe_destroy": [P],
+        "moe_load_experts": [P, I, I, I, P, P, P, I],
+        "moe_load_shared": [P, I, P, P, P, I],
+        "moe_set_router": [P, I, P, P, I],
+        "moe_set_norm": [P, I, P, F],
+        "moe_set_slots": [P, P],
+        "moe_route": [P, I, P, I, P, P, P, P, P],
+        "moe_bucket": [P, P, I, P, P, P],
+        "moe_forward": [P, I, P, I, P],
+        "moe_forward_delta": [P, I, P, I, P, P],
+        "moe_forward_stack": [P, P, I, P],
+        "moe_prefill": [P, I, P, I, P],
+        "moe_sync": [P, I],
+        "moe_get_stats": [P, ctypes.POINTER(MoeStats)],
+        "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
+        "moe_set_profiling": [P, I],
+        "moe_read_profile": [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = I
+    L.moe_last_error.argtypes = [P]
+    L.moe_last_error.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [I]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_expert_bytes.argtypes = [I, I, I]
+    L.moe_expert_bytes.restype = ctypes.c_int64
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _ptr(a):
+    """Address of a tensor / ndarray / int / None."""
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    if isinstance(a, np.ndarray):
+        if not a.flags["C_CONTIGUOUS"]:
+            raise ValueError("array must be C-contiguous")
+        return a.ctypes.data
+    if hasattr(a, "data_ptr"):
+        if not a.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+        return a.data_ptr()
+    raise TypeError(f"cannot pass {type(a)} as a pointer")
+
+
+def _is_dev(a):
+    return bool(hasattr(a, "is_cuda") and a.is_cuda)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(ctx, rc):
+    if rc != MOE_OK:
+        msg = _lib.moe_last_error(ctx).decode() if ctx else ""
+        raise MoeError(rc, msg)
+
+
+# ------------------------------------------------------------------ C ABI
+def moe_create(d, f, E, k, quant_fmt):
+    out = ctypes.c_void_p()
+    _check(None, _lib.moe_create(d, f, E, k, quant_fmt, ctypes.byref(out)))
+    return out.value
+
+
+def moe_configure(ctx, n_layers, n_shared, n_slots, max_tokens):
+    _check(ctx, _lib.moe_configure(ctx, n_layers, n_shared, n_slots, max_tokens))
+
+
+def moe_destroy(ctx):
+    _check(None, _lib.moe_destroy(ctx))
+
+
+def moe_load_experts(ctx, layer, first_expert, n_experts, codes, scales, mins=None,
+                     src_is_device=None):
+    dev = _is_dev(codes) if src_is_device is None else bool(src_is_device)
+    _check(ctx, _lib.moe_load_experts(ctx, layer, first_expert, n_experts, _ptr(codes),
+                                      _ptr(scales), _ptr(mins), int(dev)))
+
+
+def moe_load_shared(ctx, layer, codes, scales, mins=None, src_is_device=None):
+    dev = _is_dev(codes) if src_is_device is None else bool(src_is_device)
+    _check(ctx, _lib.moe_load_shared(ctx, layer, _ptr(codes), _ptr(scales), _ptr(mins), int(dev)))
+
+
+def moe_set_router(ctx, layer, W, bias=None, src_is_device=None):
+    dev = _is_dev(W) if src_is_device is None else bool(src_is_device)
+    _check(ctx, _lib.moe_set_router(ctx, layer, _ptr(W), _ptr(bias), int(dev)))
+
+
+def moe_set_norm(ctx, layer, gamma=None, eps=1e-6):
+    _check(ctx, _lib.moe_set_norm(ctx, layer, _ptr(gamma), float(eps)))
+
+
+def moe_set_slots(ctx, slot_of):
+    a = np.ascontiguousarray(slot_of, dtype=np.int32)
+    _check(ctx, _lib.moe_set_slots(ctx, _ptr(a)))
+
+
+def moe_route(ctx, layer, h, T, idx, w, bucket_off=None, bucket_perm=None, stream=None):
+    _check(ctx, _lib.moe_route(ctx, layer, _ptr(h), T, _ptr(idx), _ptr(w), _ptr(bucket_off),
+                               _ptr(bucket_perm), _stream(stream)))
+
+
+def moe_bucket(ctx, idx, T, bucket_off, bucket_perm, stream=None):
+    _check(ctx, _lib.moe_bucket(ctx, _ptr(idx), T, _ptr(bucket_off), _ptr(bucket_perm),
+                                _stream(stream)))
+
+
+def moe_forward(ctx, layer, x, T, stream=None):
+    _check(ctx, _lib.moe_forward(ctx, layer, _ptr(x), T, _stream(stream)))
+
+
+def moe_forward_delta(ctx, layer, x, T, delta, stream=None):
+    _check(ctx, _lib.moe_forward_delta(ctx, layer, _ptr(x), T, _ptr(delta), _stream(stream)))
+
+
+def moe_forward_stack(ctx, x, T, stream=None):
+    _check(ctx, _lib.moe_forward_stack(ctx, _ptr(x), T, _stream(stream)))
+
+
+def moe_prefill(ctx, layer, x, N, stream=None):
+    _check(ctx, _lib.moe_prefill(ctx, layer, _ptr(x), N, _stream(stream)))
+
+
+def moe_sync(ctx, timeout_ms=-1):
+    _check(ctx, _lib.moe_sync(ctx, int(timeout_ms)))
+
+
+def moe_get_stats(ctx):
+    st = MoeStats()
+    _check(ctx, _lib.moe_get_stats(ctx, ctypes.byref(st)))
+    counts = np.ctypeslib.as_array(st.expert_count, shape=(st.E,)).copy() if st.E else None
+    return dict(calls=st.calls, tokens=st.tokens, hits=st.hits, misses=st.misses,
+                near_ties=st.near_ties, last_T=st.last_T, last_active=st.last_active,
+                last_layer=st.last_layer, expert_count=counts)
+
+
+def moe_last_error(ctx):
+    return _lib.moe_last_error(ctx).decode()
+
+
+def moe_status_string(status):
+    return _lib.moe_status_string(status).decode()
+
+
+def moe_expert_bytes(d, f, quant_fmt):
+    return int(_lib.moe_expert_bytes(d, f, quant_fmt))
+
+
+def moe_debug_poke_slot(ctx, layer, expert, slot):
+    _check(ctx, _lib.moe_debug_poke_slot(ctx, layer, expert, slot))
+
+
+def moe_set_profiling(ctx, enable):
+    _check(ctx, _lib.moe_set_profiling(ctx, int(enable)))
+
+
+def moe_read_profile(ctx):
+    """-> (route_ms, experts_ms, combine_ms, n_calls), summed over the calls."""
+    ms = (ctypes.c_double * 3)(0.0, 0.0, 0.0)
+    n = ctypes.c_int64(0)
+    _check(ctx, _lib.moe_read_profile(ctx, ms, ctypes.byref(n)))
+    return ms[0], ms[1], ms[2], n.value

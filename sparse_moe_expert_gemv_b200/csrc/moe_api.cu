@@ -1,0 +1,803 @@
+// moe_api.cu -- host side of libmoe.so: the C ABI declared in include/moe.h.
+//
+// The context owns, in device memory (HBM):
+//   arena   [L * E] experts in the repacked tile layout (every expert has a
+//           backing copy here),
+//   shared  [L] shared experts,
+//   pool    [n_slots] residency slot pool; slot_of[l*E+e] >= 0 makes the
+//           kernels read expert (l,e) from its slot (the "expert cache" of
+//           the Strata engine analysis article, section "Expert cache":
+//           (layer, expert) -> slot or -1),
+//   router  fp32 W [L, E, d] and bias [L, E],
+//   scratch sized for max_tokens tokens per call.
+#include <cuda_runtime.h>
+
+#include <chrono>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <thread>
+#include <utility>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "kernels.cuh"
+
+using namespace moe;
+
+struct moe_ctx {
+  int device = 0;
+  int d = 0, f = 0, E = 0, k = 0, fmt = 0;
+  int L = 1, n_shared = 0, n_slots = 0, max_tokens = 64;
+  bool configured = false, any_loaded = false;
+  Layout lay{};
+  int n_sm = 0;
+  int chunk = 16;
+  int max_jobs = 0;
+  cudaStream_t io = nullptr;  // private stream for loads and status reads
+  cudaStream_t last_stream = nullptr;  // stream of the most recent compute call
+
+  uint8_t *arena = nullptr, *shared = nullptr, *pool = nullptr;
+  int *d_slot_of = nullptr;
+  std::vector<int> h_slot_of;
+  float *d_router = nullptr, *d_bias = nullptr, *d_gamma = nullptr;
+  std::vector<char> has_router, has_bias, has_norm, has_gamma, shared_loaded;
+  std::vector<float> eps;
+  std::vector<std::vector<char>> expert_loaded;
+  std::vector<int> n_loaded;
+
+  // scratch
+  float *logits = nullptr, *w = nullptr, *ybuf = nullptr;
+  int *idx = nullptr, *off = nullptr, *perm = nullptr, *plist = nullptr;
+  unsigned long long *job_ptr = nullptr;
+  int *job_beg = nullptr, *job_n = nullptr, *n_jobs = nullptr;
+  uint16_t *hbuf = nullptr, *abuf = nullptr;
+  int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
+  unsigned long long *stats = nullptr;
+  std::vector<int32_t> host_counts;
+
+  int gemv_blocks[2][2] = {{0, 0}, {0, 0}};
+  // profiling: 4 events per call slot
+  bool profiling = false;
+  std::vector<cudaEvent_t> prof_ev;
+  int prof_next = 0, prof_pending = 0;
+  std::map<std::pair<void *, int>, cudaGraphExec_t> stack_graphs;
+  std::string err;
+};
+
+namespace {
+
+moe_status fail(moe_ctx *c, moe_status s, const char *fmt, ...) {
+  if (c) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    c->err = buf;
+  }
+  return s;
+}
+
+#define CUDA_TRY(c, expr)                                                              \
+  do {                                                                                 \
+    cudaError_t e_ = (expr);                                                           \
+    if (e_ != cudaSuccess) {                                                           \
+      (void)cudaGetLastError();                                                        \
+      return fail(c, e_ == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA,     \
+                  "%s: %s", #expr, cudaGetErrorString(e_));                            \
+    }                                                                                  \
+  } while (0)
+
+template <typename P>
+cudaError_t launch(void (*kern)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                   const P &params, bool pdl = true) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, params);
+}
+
+template <int FMT, bool GATED>
+cudaError_t setup_gemv(int n_sm, int *blocks) {
+  using C = GemvCfg<FMT, GATED>;
+  cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<FMT, GATED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<FMT, GATED>,
+                                                    C::WARPS * 32, C::SMEM);
+  if (e != cudaSuccess) return e;
+  *blocks = n_sm * (per_sm > 0 ? per_sm : 1);
+  return cudaSuccess;
+}
+
+template <int FMT, bool GATED>
+cudaError_t launch_gemv(moe_ctx *c, cudaStream_t s, const GemvParams &gp) {
+  using C = GemvCfg<FMT, GATED>;
+  return launch(expert_gemv_kernel<FMT, GATED>, dim3(c->gemv_blocks[FMT - 1][GATED]),
+                dim3(C::WARPS * 32), C::SMEM, s, gp);
+}
+
+bool valid_layer(const moe_ctx *c, int layer) { return layer >= 0 && layer < c->L; }
+
+template <typename T>
+void dfree(T *&p) {
+  if (p) cudaFree((void *)p);
+  p = nullptr;
+}
+
+moe_status do_configure(moe_ctx *c) {
+  const Layout &L = c->lay;
+  const long long Be = L.expert_bytes;
+  const int T = c->max_tokens, E = c->E, k = c->k, d = c->d, f = c->f;
+  CUDA_TRY(c, cudaMalloc(&c->arena, (size_t)c->L * E * Be));
+  if (c->n_shared) CUDA_TRY(c, cudaMalloc(&c->shared, (size_t)c->L * Be));
+  if (c->n_slots) CUDA_TRY(c, cudaMalloc(&c->pool, (size_t)c->n_slots * Be));
+  CUDA_TRY(c, cudaMalloc(&c->d_slot_of, (size_t)c->L * E * sizeof(int)));
+  c->h_slot_of.assign((size_t)c->L * E, -1);
+  CUDA_TRY(c, cudaMemset(c->d_slot_of, 0xFF, (size_t)c->L * E * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->d_router, (size_t)c->L * E * d * sizeof(float)));
+  CUDA_TRY(c, cudaMalloc(&c->d_bias, (size_t)c->L * E * sizeof(float)));
+  CUDA_TRY(c, cudaMalloc(&c->d_gamma, (size_t)c->L * d * sizeof(float)));
+  const long long P = (long long)T * k, Ptot = P + T;
+  c->max_jobs = (int)(P + E + (T + c->chunk - 1) / c->chunk + 8);
+  CUDA_TRY(c, cudaMalloc(&c->logits, (size_t)T * E * sizeof(float)));
+  CUDA_TRY(c, cudaMalloc(&c->w, (size_t)P * sizeof(float)));
+  CUDA_TRY(c, cudaMalloc(&c->idx, (size_t)P * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->off, (size_t)(E + 1) * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->perm, (size_t)P * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->plist, (size_t)Ptot * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->job_ptr, (size_t)c->max_jobs * sizeof(unsigned long long)));
+  CUDA_TRY(c, cudaMalloc(&c->job_beg, (size_t)c->max_jobs * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->job_n, (size_t)c->max_jobs * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->n_jobs, sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->hbuf, (size_t)T * d * 2));
+  CUDA_TRY(c, cudaMalloc(&c->abuf, (size_t)Ptot * f * 2));
+  CUDA_TRY(c, cudaMalloc(&c->ybuf, (size_t)Ptot * d * sizeof(float)));
+  CUDA_TRY(c, cudaMalloc(&c->status, sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->cnt_out, (size_t)E * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->last, 4 * sizeof(int)));
+  CUDA_TRY(c, cudaMalloc(&c->stats, 8 * sizeof(unsigned long long)));
+  CUDA_TRY(c, cudaMemset(c->status, 0, sizeof(int)));
+  CUDA_TRY(c, cudaMemset(c->cnt_out, 0, (size_t)E * sizeof(int)));
+  CUDA_TRY(c, cudaMemset(c->last, 0, 4 * sizeof(int)));
+  CUDA_TRY(c, cudaMemset(c->stats, 0, 8 * sizeof(unsigned long long)));
+  CUDA_TRY(c, cudaMemset(c->n_jobs, 0, sizeof(int)));
+  c->has_router.assign(c->L, 0);
+  c->has_bias.assign(c->L, 0);
+  c->has_norm.assign(c->L, 0);
+  c->has_gamma.assign(c->L, 0);
+  c->shared_loaded.assign(c->L, 0);
+  c->eps.assign(c->L, 1e-6f);
+  c->expert_loaded.assign(c->L, std::vector<char>(E, 0));
+  c->n_loaded.assign(c->L, 0);
+  c->host_counts.assign(E, 0);
+  c->configured = true;
+  return MOE_OK;
+}
+
+moe_status ensure_configured(moe_ctx *c) {
+  if (c->configured) return MOE_OK;
+  return do_configure(c);
+}
+
+int finish_npl(int E) {
+  int n = (E + 31) / 32;
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+cudaError_t launch_finish(moe_ctx *c, cudaStream_t s, const FinishParams &fp) {
+  const size_t smem = (size_t)(4 * c->E + 2) * sizeof(int);
+  switch (finish_npl(c->E)) {
+    case 1: return launch(route_finish_kernel<1>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+    case 2: return launch(route_finish_kernel<2>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+    case 4: return launch(route_finish_kernel<4>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+    case 8: return launch(route_finish_kernel<8>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+    case 16: return launch(route_finish_kernel<16>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+    default: return launch(route_finish_kernel<32>, dim3(1), dim3(kFinishThreads), smem, s, fp);
+  }
+}
+
+cudaError_t launch_router(moe_ctx *c, cudaStream_t s, const RouterParams &rp) {
+  const dim3 grid((c->E + kRouterWarps - 1) / kRouterWarps), block(kRouterWarps * 32);
+  switch (c->d / 128) {
+    case 1: return launch(router_logits_kernel<1>, grid, block, 0, s, rp);
+    case 2: return launch(router_logits_kernel<2>, grid, block, 0, s, rp);
+    case 4: return launch(router_logits_kernel<4>, grid, block, 0, s, rp);
+    case 8: return launch(router_logits_kernel<8>, grid, block, 0, s, rp);
+    case 12: return launch(router_logits_kernel<12>, grid, block, 0, s, rp);
+    case 16: return launch(router_logits_kernel<16>, grid, block, 0, s, rp);
+    case 24: return launch(router_logits_kernel<24>, grid, block, 0, s, rp);
+    case 32: return launch(router_logits_kernel<32>, grid, block, 0, s, rp);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+bool router_d_supported(int d) {
+  const int v = d / 128;
+  return d % 128 == 0 && (v == 1 || v == 2 || v == 4 || v == 8 || v == 12 || v == 16 ||
+                          v == 24 || v == 32);
+}
+
+// Router input for `layer`: either x itself or RMSNorm(x) in scratch.
+const uint16_t *router_input(moe_ctx *c, int layer, const uint16_t *x, int T, cudaStream_t s,
+                             cudaError_t *e) {
+  if (!c->has_norm[layer]) return x;
+  NormParams np{x, c->has_gamma[layer] ? c->d_gamma + (size_t)layer * c->d : nullptr,
+                c->eps[layer], T, c->d, c->hbuf};
+  *e = launch(rmsnorm_kernel, dim3(T), dim3(256), 0, s, np);
+  return c->hbuf;
+}
+
+FinishParams finish_params(moe_ctx *c, int layer, int T) {
+  FinishParams fp{};
+  fp.logits = c->logits;
+  fp.T = T;
+  fp.E = c->E;
+  fp.k = c->k;
+  fp.layer = layer;
+  fp.idx = c->idx;
+  fp.w = c->w;
+  fp.off = c->off;
+  fp.perm = c->perm;
+  fp.chunk = c->chunk;
+  fp.plist = c->plist;
+  fp.job_ptr = c->job_ptr;
+  fp.job_beg = c->job_beg;
+  fp.job_n = c->job_n;
+  fp.n_jobs = c->n_jobs;
+  fp.max_jobs = c->max_jobs;
+  fp.slot_of = c->d_slot_of;
+  fp.n_slots = c->n_slots;
+  fp.arena = c->arena;
+  fp.pool = c->pool;
+  fp.shared = c->n_shared ? c->shared + (size_t)layer * c->lay.expert_bytes : nullptr;
+  fp.expert_bytes = c->lay.expert_bytes;
+  fp.cnt_out = c->cnt_out;
+  fp.stats = c->stats;
+  fp.last = c->last;
+  fp.status = c->status;
+  return fp;
+}
+
+moe_status check_ready(moe_ctx *c, int layer) {
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
+  if (c->n_loaded[layer] != c->E)
+    return fail(c, MOE_ERR_STATE, "layer %d: %d of %d experts loaded", layer, c->n_loaded[layer],
+                c->E);
+  if (c->n_shared && !c->shared_loaded[layer])
+    return fail(c, MOE_ERR_STATE, "shared expert of layer %d not loaded", layer);
+  return MOE_OK;
+}
+
+constexpr int kProfSlots = 8192;
+
+// Event i (0..3) of the current profiled call, or nullptr when off.
+cudaEvent_t prof_event(moe_ctx *c, int i) {
+  return c->profiling ? c->prof_ev[(size_t)c->prof_next * 4 + i] : nullptr;
+}
+
+cudaError_t prof_mark(moe_ctx *c, int i, cudaStream_t s) {
+  cudaEvent_t ev = prof_event(c, i);
+  return ev ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal) : cudaSuccess;
+}
+
+// The whole decode chain for one layer.  delta == nullptr: residual mode.
+moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  CUDA_TRY(c, prof_mark(c, 0, s));
+  const uint16_t *h = router_input(c, layer, x, T, s, &e);
+  CUDA_TRY(c, e);
+  RouterParams rp{h, c->d_router + (size_t)layer * c->E * c->d,
+                  c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
+                  c->logits};
+  CUDA_TRY(c, launch_router(c, s, rp));
+  FinishParams fp = finish_params(c, layer, T);
+  fp.build_jobs = 1;
+  CUDA_TRY(c, launch_finish(c, s, fp));
+
+  GemvParams g1{};
+  g1.job_ptr = c->job_ptr;
+  g1.job_beg = c->job_beg;
+  g1.job_n = c->job_n;
+  g1.n_jobs = c->n_jobs;
+  g1.plist = c->plist;
+  g1.Tk = T * c->k;
+  g1.k = c->k;
+  g1.src = h;
+  g1.src_by_pair = 0;
+  g1.K = c->d;
+  g1.R = c->f;
+  g1.region_off = 0;
+  g1.out_a = c->abuf;
+  g1.status = c->status;
+  GemvParams g2 = g1;
+  g2.src = c->abuf;
+  g2.src_by_pair = 1;
+  g2.K = c->f;
+  g2.R = c->d;
+  g2.region_off = c->lay.p1_bytes;
+  g2.out_a = nullptr;
+  g2.out_y = c->ybuf;
+  CUDA_TRY(c, prof_mark(c, 1, s));
+  if (c->fmt == MOE_Q4_SYM_G32_F16) {
+    CUDA_TRY(c, (launch_gemv<1, true>(c, s, g1)));
+    CUDA_TRY(c, (launch_gemv<1, false>(c, s, g2)));
+  } else {
+    CUDA_TRY(c, (launch_gemv<2, true>(c, s, g1)));
+    CUDA_TRY(c, (launch_gemv<2, false>(c, s, g2)));
+  }
+  CUDA_TRY(c, prof_mark(c, 2, s));
+  CombineParams cp{c->ybuf, c->w, T, c->k, c->d, c->n_shared, x, delta};
+  const long long n4 = (long long)T * c->d / 4;
+  const int blocks = (int)std::min<long long>((n4 + 255) / 256, 4LL * c->n_sm);
+  CUDA_TRY(c, launch(combine_kernel, dim3(blocks), dim3(256), 0, s, cp));
+  CUDA_TRY(c, prof_mark(c, 3, s));
+  if (c->profiling) {
+    c->prof_next = (c->prof_next + 1) % kProfSlots;
+    c->prof_pending = std::min(c->prof_pending + 1, kProfSlots);
+  }
+  return MOE_OK;
+}
+
+moe_status load_impl(moe_ctx *c, uint8_t *dst, int n, const void *codes, const void *scales,
+                     const void *mins, int src_is_device) {
+  const Layout &L = c->lay;
+  const long long per_codes = L.fmt == 1 ? 3LL * c->f * c->d / 2 : 3LL * c->f * c->d / 4;
+  const long long per_groups = 3LL * c->f * c->d / L.G;
+  const size_t nc = (size_t)n * per_codes, ns = (size_t)n * per_groups * 2;
+  const uint8_t *dc = (const uint8_t *)codes;
+  const uint16_t *ds = (const uint16_t *)scales, *dm = (const uint16_t *)mins;
+  uint8_t *staging = nullptr;
+  if (!src_is_device) {
+    const size_t tot = nc + ns + (mins ? ns : 0);
+    CUDA_TRY(c, cudaMalloc(&staging, tot));
+    cudaError_t e = cudaMemcpyAsync(staging, codes, nc, cudaMemcpyHostToDevice, c->io);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(staging + nc, scales, ns, cudaMemcpyHostToDevice, c->io);
+    if (e == cudaSuccess && mins)
+      e = cudaMemcpyAsync(staging + nc + ns, mins, ns, cudaMemcpyHostToDevice, c->io);
+    if (e != cudaSuccess) {
+      cudaFree(staging);
+      CUDA_TRY(c, e);
+    }
+    dc = staging;
+    ds = (const uint16_t *)(staging + nc);
+    dm = mins ? (const uint16_t *)(staging + nc + ns) : nullptr;
+  }
+  RepackParams rp{dc, ds, dm, dst, n, L};
+  cudaError_t e = launch(repack_kernel, dim3(4 * c->n_sm), dim3(256), 0, c->io, rp, false);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->io);
+  if (staging) cudaFree(staging);
+  CUDA_TRY(c, e);
+  return MOE_OK;
+}
+
+moe_status refresh_slots(moe_ctx *c, int layer, int first, int n) {
+  const long long Be = c->lay.expert_bytes;
+  for (int e = first; e < first + n; ++e) {
+    const int slot = c->h_slot_of[(size_t)layer * c->E + e];
+    if (slot >= 0)
+      CUDA_TRY(c, cudaMemcpyAsync(c->pool + (size_t)slot * Be,
+                                  c->arena + ((size_t)layer * c->E + e) * Be, (size_t)Be,
+                                  cudaMemcpyDeviceToDevice, c->io));
+  }
+  CUDA_TRY(c, cudaStreamSynchronize(c->io));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_OOM: return "MOE_ERR_OOM";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_STATE: return "MOE_ERR_STATE";
+    case MOE_ERR_BAD_SLOT: return "MOE_ERR_BAD_SLOT";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_NOT_SUPPORTED: return "MOE_ERR_NOT_SUPPORTED";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+int64_t moe_expert_bytes(int d, int f, int fmt) {
+  if (d <= 0 || f <= 0 || d % 128 || f % 128) return -1;
+  if (fmt != MOE_Q4_SYM_G32_F16 && fmt != MOE_Q2_ASYM_G64_F16) return -1;
+  return make_layout(fmt, d, f).expert_bytes;
+}
+
+const char *moe_last_error(const moe_ctx *c) { return c ? c->err.c_str() : ""; }
+
+moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d <= 0 || f <= 0 || d % 128 || f % 128 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 ||
+      (fmt != MOE_Q4_SYM_G32_F16 && fmt != MOE_Q2_ASYM_G64_F16) || d > 4096 ||
+      !router_d_supported(d))
+    return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  moe_ctx *c = new moe_ctx();
+  c->device = dev;
+  c->d = d;
+  c->f = f;
+  c->E = E;
+  c->k = k;
+  c->fmt = fmt;
+  c->lay = make_layout(fmt, d, f);
+  cudaError_t e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = setup_gemv<1, true>(c->n_sm, &c->gemv_blocks[0][1]);
+  if (e == cudaSuccess) e = setup_gemv<1, false>(c->n_sm, &c->gemv_blocks[0][0]);
+  if (e == cudaSuccess) e = setup_gemv<2, true>(c->n_sm, &c->gemv_blocks[1][1]);
+  if (e == cudaSuccess) e = setup_gemv<2, false>(c->n_sm, &c->gemv_blocks[1][0]);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    moe_destroy(c);
+    return MOE_ERR_CUDA;
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+moe_status moe_configure(moe_ctx *c, int n_layers, int n_shared, int n_slots, int max_tokens) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->configured) return fail(c, MOE_ERR_STATE, "moe_configure after configuration/loads");
+  if (n_layers < 1 || n_layers > 4096 || (n_shared != 0 && n_shared != 1) || n_slots < 0 ||
+      max_tokens < 1 || max_tokens > (1 << 20))
+    return fail(c, MOE_ERR_INVALID_ARG, "bad configuration");
+  c->L = n_layers;
+  c->n_shared = n_shared;
+  c->n_slots = n_slots;
+  c->max_tokens = max_tokens;
+  return do_configure(c);
+}
+
+moe_status moe_destroy(moe_ctx *c) {
+  if (!c) return MOE_OK;
+  cudaDeviceSynchronize();
+  for (auto &kv : c->stack_graphs) cudaGraphExecDestroy(kv.second);
+  for (cudaEvent_t ev : c->prof_ev) cudaEventDestroy(ev);
+  dfree(c->arena);
+  dfree(c->shared);
+  dfree(c->pool);
+  dfree(c->d_slot_of);
+  dfree(c->d_router);
+  dfree(c->d_bias);
+  dfree(c->d_gamma);
+  dfree(c->logits);
+  dfree(c->w);
+  dfree(c->ybuf);
+  dfree(c->idx);
+  dfree(c->off);
+  dfree(c->perm);
+  dfree(c->plist);
+  dfree(c->job_ptr);
+  dfree(c->job_beg);
+  dfree(c->job_n);
+  dfree(c->n_jobs);
+  dfree(c->hbuf);
+  dfree(c->abuf);
+  dfree(c->status);
+  dfree(c->cnt_out);
+  dfree(c->last);
+  dfree(c->stats);
+  if (c->io) cudaStreamDestroy(c->io);
+  (void)cudaGetLastError();
+  delete c;
+  return MOE_OK;
+}
+
+moe_status moe_load_experts(moe_ctx *c, int layer, int first, int n, const void *codes,
+                            const void *scales, const void *mins, int src_is_device) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  if (!valid_layer(c, layer) || first < 0 || n < 1 || first + n > c->E || !codes || !scales ||
+      (c->fmt == MOE_Q2_ASYM_G64_F16 && !mins))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_load_experts: bad arguments");
+  if (c->fmt == MOE_Q4_SYM_G32_F16) mins = nullptr;
+  uint8_t *dst = c->arena + ((size_t)layer * c->E + first) * c->lay.expert_bytes;
+  st = load_impl(c, dst, n, codes, scales, mins, src_is_device);
+  if (st) return st;
+  for (int e = first; e < first + n; ++e)
+    if (!c->expert_loaded[layer][e]) {
+      c->expert_loaded[layer][e] = 1;
+      c->n_loaded[layer]++;
+    }
+  c->any_loaded = true;
+  return refresh_slots(c, layer, first, n);
+}
+
+moe_status moe_load_shared(moe_ctx *c, int layer, const void *codes, const void *scales,
+                           const void *mins, int src_is_device) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  if (!c->n_shared) return fail(c, MOE_ERR_STATE, "configured without a shared expert");
+  if (!valid_layer(c, layer) || !codes || !scales || (c->fmt == MOE_Q2_ASYM_G64_F16 && !mins))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_load_shared: bad arguments");
+  if (c->fmt == MOE_Q4_SYM_G32_F16) mins = nullptr;
+  st = load_impl(c, c->shared + (size_t)layer * c->lay.expert_bytes, 1, codes, scales, mins,
+                 src_is_device);
+  if (st) return st;
+  c->shared_loaded[layer] = 1;
+  c->any_loaded = true;
+  return MOE_OK;
+}
+
+moe_status moe_set_router(moe_ctx *c, int layer, const float *W, const float *bias,
+                          int src_is_device) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  if (!valid_layer(c, layer) || !W) return fail(c, MOE_ERR_INVALID_ARG, "moe_set_router");
+  const cudaMemcpyKind kind = src_is_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  CUDA_TRY(c, cudaMemcpyAsync(c->d_router + (size_t)layer * c->E * c->d, W,
+                              (size_t)c->E * c->d * sizeof(float), kind, c->io));
+  if (bias)
+    CUDA_TRY(c, cudaMemcpyAsync(c->d_bias + (size_t)layer * c->E, bias, (size_t)c->E * sizeof(float),
+                                kind, c->io));
+  CUDA_TRY(c, cudaStreamSynchronize(c->io));
+  c->has_router[layer] = 1;
+  c->has_bias[layer] = bias != nullptr;
+  return MOE_OK;
+}
+
+moe_status moe_set_norm(moe_ctx *c, int layer, const float *gamma, float eps) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  if (!valid_layer(c, layer) || !(eps >= 0.f)) return fail(c, MOE_ERR_INVALID_ARG, "moe_set_norm");
+  if (gamma)
+    CUDA_TRY(c, cudaMemcpy(c->d_gamma + (size_t)layer * c->d, gamma, (size_t)c->d * sizeof(float),
+                           cudaMemcpyHostToDevice));
+  c->has_norm[layer] = 1;
+  c->has_gamma[layer] = gamma != nullptr;
+  c->eps[layer] = eps;
+  return MOE_OK;
+}
+
+moe_status moe_set_slots(moe_ctx *c, const int32_t *slot_of) {
+  if (!c || !slot_of) return fail(c, MOE_ERR_INVALID_ARG, "moe_set_slots: NULL");
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  const size_t n = (size_t)c->L * c->E;
+  std::vector<char> used(c->n_slots, 0);
+  for (size_t i = 0; i < n; ++i) {
+    const int s = slot_of[i];
+    if (s < -1 || s >= c->n_slots) return fail(c, MOE_ERR_INVALID_ARG, "slot %d out of range", s);
+    if (s >= 0) {
+      if (used[s]) return fail(c, MOE_ERR_INVALID_ARG, "slot %d used twice", s);
+      used[s] = 1;
+    }
+  }
+  c->h_slot_of.assign(slot_of, slot_of + n);
+  CUDA_TRY(c, cudaMemcpy(c->d_slot_of, slot_of, n * sizeof(int), cudaMemcpyHostToDevice));
+  for (int l = 0; l < c->L; ++l) {
+    st = refresh_slots(c, l, 0, c->E);
+    if (st) return st;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_ctx *c, int layer, const void *h, int T, int32_t *idx, float *w,
+                     int32_t *boff, int32_t *bperm, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !h || !idx || !w || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_route: bad arguments (T=%d max=%d)", T, c->max_tokens);
+  if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  RouterParams rp{(const uint16_t *)h, c->d_router + (size_t)layer * c->E * c->d,
+                  c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
+                  c->logits};
+  CUDA_TRY(c, launch_router(c, s, rp));
+  FinishParams fp = finish_params(c, layer, T);
+  fp.idx = idx;
+  fp.w = w;
+  fp.off = boff ? boff : c->off;
+  fp.perm = bperm ? bperm : c->perm;
+  fp.build_jobs = 0;
+  CUDA_TRY(c, launch_finish(c, s, fp));
+  return MOE_OK;
+}
+
+moe_status moe_bucket(moe_ctx *c, const int32_t *idx, int T, int32_t *boff, int32_t *bperm,
+                      void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  moe_status st = ensure_configured(c);
+  if (st) return st;
+  if (!idx || !boff || !bperm || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_bucket: bad arguments");
+  FinishParams fp = finish_params(c, 0, T);
+  fp.logits = nullptr;
+  fp.idx_in = idx;
+  fp.off = boff;
+  fp.perm = bperm;
+  fp.build_jobs = 0;
+  c->last_stream = (cudaStream_t)stream;
+  CUDA_TRY(c, launch_finish(c, (cudaStream_t)stream, fp));
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_ctx *c, int layer, void *x, int T, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !x || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_forward: bad arguments (T=%d max=%d)", T,
+                c->max_tokens);
+  moe_status st = check_ready(c, layer);
+  if (st) return st;
+  c->last_stream = (cudaStream_t)stream;
+  return forward_impl(c, layer, (uint16_t *)x, T, nullptr, (cudaStream_t)stream);
+}
+
+moe_status moe_forward_delta(moe_ctx *c, int layer, const void *x, int T, float *delta,
+                             void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !x || !delta || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_delta: bad arguments");
+  moe_status st = check_ready(c, layer);
+  if (st) return st;
+  c->last_stream = (cudaStream_t)stream;
+  return forward_impl(c, layer, (uint16_t *)const_cast<void *>(x), T, delta,
+                      (cudaStream_t)stream);
+}
+
+moe_status moe_forward_stack(moe_ctx *c, void *x, int T, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!x || T < 1 || T > c->max_tokens) return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_stack");
+  for (int l = 0; l < c->L; ++l) {
+    moe_status st = check_ready(c, l);
+    if (st) return st;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  auto key = std::make_pair(x, T);
+  auto it = c->stack_graphs.find(key);
+  if (it == c->stack_graphs.end()) {
+    cudaStream_t cap = nullptr;
+    CUDA_TRY(c, cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
+    moe_status st = MOE_OK;
+    if (e == cudaSuccess) {
+      for (int l = 0; l < c->L && st == MOE_OK; ++l)
+        st = forward_impl(c, l, (uint16_t *)x, T, nullptr, cap);
+      e = cudaStreamEndCapture(cap, &graph);
+    }
+    cudaGraphExec_t exec = nullptr;
+    if (e == cudaSuccess && st == MOE_OK) e = cudaGraphInstantiate(&exec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    cudaStreamDestroy(cap);
+    if (st != MOE_OK) return st;
+    CUDA_TRY(c, e);
+    it = c->stack_graphs.emplace(key, exec).first;
+  }
+  c->last_stream = s;
+  CUDA_TRY(c, cudaGraphLaunch(it->second, s));
+  return MOE_OK;
+}
+
+moe_status moe_prefill(moe_ctx *c, int layer, void *x, int N, void *stream) {
+  // A prefill chunk computes the same layer function as a decode window; the
+  // grouped expert kernels split each expert's tokens into jobs.
+  return moe_forward(c, layer, x, N, stream);
+}
+
+moe_status moe_sync(moe_ctx *c, int timeout_ms) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return MOE_OK;
+  // poll the stream of the most recent compute call, with a bound
+  const auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    cudaError_t e = cudaStreamQuery(c->last_stream);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) CUDA_TRY(c, e);
+    if (timeout_ms >= 0 &&
+        std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms))
+      return fail(c, MOE_ERR_TIMEOUT, "moe_sync: not done after %d ms", timeout_ms);
+    std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+  int st = 0;
+  CUDA_TRY(c, cudaMemcpyAsync(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost, c->io));
+  CUDA_TRY(c, cudaMemsetAsync(c->status, 0, sizeof(int), c->io));
+  CUDA_TRY(c, cudaStreamSynchronize(c->io));
+  if (st & kErrBadSlot) return fail(c, MOE_ERR_BAD_SLOT, "device status 0x%x: bad slot", st);
+  if (st) return fail(c, MOE_ERR_DEVICE, "device status 0x%x", st);
+  return MOE_OK;
+}
+
+moe_status moe_get_stats(moe_ctx *c, moe_stats *out) {
+  if (!c || !out) return MOE_ERR_INVALID_ARG;
+  std::memset(out, 0, sizeof *out);
+  if (!c->configured) return MOE_OK;
+  CUDA_TRY(c, cudaStreamSynchronize(c->last_stream));
+  unsigned long long s[8];
+  int last[4];
+  CUDA_TRY(c, cudaMemcpyAsync(s, c->stats, sizeof s, cudaMemcpyDeviceToHost, c->io));
+  CUDA_TRY(c, cudaMemcpyAsync(last, c->last, sizeof last, cudaMemcpyDeviceToHost, c->io));
+  CUDA_TRY(c, cudaMemcpyAsync(c->host_counts.data(), c->cnt_out, (size_t)c->E * sizeof(int),
+                              cudaMemcpyDeviceToHost, c->io));
+  CUDA_TRY(c, cudaStreamSynchronize(c->io));
+  out->calls = (int64_t)s[0];
+  out->tokens = (int64_t)s[1];
+  out->hits = (int64_t)s[2];
+  out->misses = (int64_t)s[3];
+  out->near_ties = (int64_t)s[4];
+  out->last_T = last[0];
+  out->last_active = last[1];
+  out->last_layer = last[2];
+  out->E = c->E;
+  out->expert_count = c->host_counts.data();
+  return MOE_OK;
+}
+
+moe_status moe_set_profiling(moe_ctx *c, int enable) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (enable && c->prof_ev.empty()) {
+    c->prof_ev.resize((size_t)kProfSlots * 4, nullptr);
+    for (auto &ev : c->prof_ev) CUDA_TRY(c, cudaEventCreate(&ev));
+  }
+  c->profiling = enable != 0;
+  c->prof_next = 0;
+  c->prof_pending = 0;
+  return MOE_OK;
+}
+
+moe_status moe_read_profile(moe_ctx *c, double ms[3], int64_t *n_calls) {
+  if (!c || !ms || !n_calls) return MOE_ERR_INVALID_ARG;
+  *n_calls = 0;
+  if (c->prof_ev.empty()) return MOE_OK;
+  // the pending calls are the prof_pending slots ending at prof_next - 1;
+  // for replayed graphs every recorded slot is re-read
+  const int n = c->prof_pending;
+  for (int i = 0; i < n; ++i) {
+    const int slot = ((c->prof_next - n + i) % kProfSlots + kProfSlots) % kProfSlots;
+    float seg[3];
+    CUDA_TRY(c, cudaEventSynchronize(c->prof_ev[(size_t)slot * 4 + 3]));
+    for (int j = 0; j < 3; ++j)
+      CUDA_TRY(c, cudaEventElapsedTime(&seg[j], c->prof_ev[(size_t)slot * 4 + j],
+                                       c->prof_ev[(size_t)slot * 4 + j + 1]));
+    for (int j = 0; j < 3; ++j) ms[j] += seg[j];
+  }
+  *n_calls = n;
+  return MOE_OK;
+}
+
+// Debug hook: write one raw slot-table entry on the device without host
+// validation, so tests can check the device-side detection of a corrupted
+// residency table (kErrBadSlot -> MOE_ERR_BAD_SLOT from moe_sync).
+moe_status moe_debug_poke_slot(moe_ctx *c, int layer, int expert, int32_t slot) {
+  if (!c || !c->configured || !valid_layer(c, layer) || expert < 0 || expert >= c->E)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_debug_poke_slot");
+  CUDA_TRY(c, cudaMemcpy(c->d_slot_of + (size_t)layer * c->E + expert, &slot, sizeof slot,
+                         cudaMemcpyHostToDevice));
+  return MOE_OK;
+}
+
+}  // extern "C"
