@@ -322,7 +322,7 @@ def run_native(args, world, rank, local):
         },
         "e2e": {"value": world * tok / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": K * 5,
+        "gpu_launches": K * (4 if T <= 32 else 5),
         "clocks": clocks,
     }
     B.moe_destroy(ctx)

@@ -219,6 +219,19 @@ MOE_API moe_status moe_set_profiling(moe_ctx *ctx, int enable);
  * (ctx, 1) starts a new set.  ms is caller-owned host memory. */
 MOE_API moe_status moe_read_profile(moe_ctx *ctx, double ms[3], int64_t *n_calls);
 
+/* Device timeline tracing (diagnostics).  When enabled, kernels record the
+ * earliest and latest %globaltimer (ns) at which any CTA reached each of a
+ * fixed list of trace points (kernel start, dependency wait passed, phase
+ * ends, kernel end of the routing, expert and combine kernels).  The trace
+ * buffer is shared by every context of the process on this device; enabling
+ * it synchronises the device.  Costs a few atomics per CTA while on. */
+MOE_API moe_status moe_set_trace(moe_ctx *ctx, int enable);
+
+/* Synchronises, copies the 2 * n_points trace values (first all minima, then
+ * all maxima; unset minima read as -1, unset maxima as 0) into out[0 .. n)
+ * and resets them.  n must be at least 2 * 18. */
+MOE_API moe_status moe_read_trace(moe_ctx *ctx, int64_t *out, int n);
+
 /* Last error message of ctx (never NULL; "" when none). */
 MOE_API const char *moe_last_error(const moe_ctx *ctx);
 

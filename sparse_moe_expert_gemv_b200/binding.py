@@ -29,7 +29,8 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_route", "moe_bucket", "moe_forward", "moe_forward_delta",
            "moe_forward_stack", "moe_prefill", "moe_sync", "moe_get_stats",
            "moe_last_error", "moe_status_string", "moe_expert_bytes",
-           "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile")
+           "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
+           "moe_set_trace", "moe_read_trace")
 
 
 class MoeError(RuntimeError):
@@ -71,6 +72,8 @@ def _load():
         "moe_get_stats": [P, ctypes.POINTER(MoeStats)],
         "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
         "moe_set_profiling": [P, I],
+        "moe_set_trace": [P, I],
+        "moe_read_trace": [P, ctypes.POINTER(ctypes.c_int64), I],
         "moe_read_profile": [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
     for name, args in sig.items():
@@ -235,3 +238,22 @@ def moe_read_profile(ctx):
     n = ctypes.c_int64(0)
     _check(ctx, _lib.moe_read_profile(ctx, ms, ctypes.byref(n)))
     return ms[0], ms[1], ms[2], n.value
+
+
+TRACE_POINTS = ("route_start", "route_waited", "route_logits", "route_last_start", "route_topk",
+                "route_bucket", "route_end", "gate_start", "gate_waited", "gate_first_item",
+                "gate_end", "down_start", "down_waited", "down_end", "comb_start", "comb_end",
+                "route_loaded", "route_selected")
+
+
+def moe_set_trace(ctx, enable):
+    _check(ctx, _lib.moe_set_trace(ctx, int(enable)))
+
+
+def moe_read_trace(ctx):
+    """-> {point: (earliest_ns, latest_ns)}; points no CTA reached are omitted."""
+    n = 2 * len(TRACE_POINTS)
+    buf = (ctypes.c_int64 * n)()
+    _check(ctx, _lib.moe_read_trace(ctx, buf, n))
+    k = len(TRACE_POINTS)
+    return {name: (buf[i], buf[k + i]) for i, name in enumerate(TRACE_POINTS) if buf[i] != -1}

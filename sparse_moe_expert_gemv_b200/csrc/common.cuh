@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #define MOE_DEV __device__ __forceinline__
+#define MOE_HOST_DEV_INLINE __host__ __device__ __forceinline__
 
 namespace moe {
 
@@ -52,6 +53,40 @@ inline Layout make_layout(int fmt, int d, int f) {
   L.expert_bytes = L.p1_bytes + L.p2_bytes;
   return L;
 }
+
+// ----------------------------------------------------------------- tracing
+// Device timeline of one forward call (moe_set_trace): each trace point
+// keeps the earliest and latest %globaltimer (ns) any CTA recorded there.
+// Null when tracing is off; then a trace point costs one load and a branch.
+enum TracePoint : int {
+  kTrRouteStart = 0, kTrRouteWaited, kTrRouteLogits, kTrRouteLastStart, kTrRouteTopk,
+  kTrRouteBucket, kTrRouteEnd,
+  kTrGateStart, kTrGateWaited, kTrGateFirstTile, kTrGateEnd,
+  kTrDownStart, kTrDownWaited, kTrDownEnd,
+  kTrCombStart, kTrCombEnd,
+  kTrRouteLoaded, kTrRouteSelected,
+  kTrCount
+};
+// [2 * kTrCount]: minima then maxima; the library is one translation unit
+__device__ unsigned long long *g_trace = nullptr;
+
+MOE_DEV unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+MOE_DEV void trace_point(int i) {
+  unsigned long long *tr = g_trace;
+  if (tr) {
+    const unsigned long long t = global_ns();
+    atomicMin(tr + i, t);
+    atomicMax(tr + kTrCount + i, t);
+  }
+}
+#define MOE_TRACE(i)                       \
+  do {                                     \
+    if (threadIdx.x == 0) trace_point(i);  \
+  } while (0)
 
 // ------------------------------------------------------- PDL (griddepcontrol)
 MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -153,6 +188,20 @@ MOE_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, 
         "f"(c[2]), "f"(c[3]));
 }
 
+// D = A * B (zero accumulator) when `first`, else D += A * B.
+MOE_DEV void mma_bf16_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                          bool first) {
+  if (first) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+  } else {
+    mma_bf16_16816(d, a, b0, b1, d);
+  }
+}
+
 // ------------------------------------------------------------- code unpack
 MOE_DEV uint32_t lop3_and_or(uint32_t x, uint32_t m, uint32_t c) {
   uint32_t r;  // (x & m) | c
@@ -204,6 +253,18 @@ MOE_DEV float half_lo(uint32_t v) { return __half2float(__ushort_as_half((unsign
 MOE_DEV float half_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 
 MOE_DEV float bf16_bits_to_float(unsigned short b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Order-preserving map of a float to an unsigned key (-0 and +0 equal):
+// a > b  <=>  order_key(a) > order_key(b) for non-NaN a, b.  0 is below every
+// real value's key, so it marks a used or absent entry.
+MOE_DEV uint32_t order_key(float f) {
+  if (f == 0.f) f = 0.f;
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+MOE_DEV float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 MOE_DEV float warp_sum(float v) {
 #pragma unroll

@@ -34,7 +34,7 @@ struct moe_ctx {
   bool configured = false, any_loaded = false;
   Layout lay{};
   int n_sm = 0;
-  int chunk = 16;
+  int chunk_min = 8;  // smallest job size (sizes the job list)
   int max_jobs = 0;
   cudaStream_t io = nullptr;  // private stream for loads and status reads
   cudaStream_t last_stream = nullptr;  // stream of the most recent compute call
@@ -48,17 +48,20 @@ struct moe_ctx {
   std::vector<std::vector<char>> expert_loaded;
   std::vector<int> n_loaded;
 
-  // scratch
+  // scratch: views into one allocation (do_configure)
+  uint8_t *scratch = nullptr;
   float *logits = nullptr, *w = nullptr, *ybuf = nullptr;
   int *idx = nullptr, *off = nullptr, *perm = nullptr, *plist = nullptr;
   unsigned long long *job_ptr = nullptr;
   int *job_beg = nullptr, *job_n = nullptr, *n_jobs = nullptr;
   uint16_t *hbuf = nullptr, *abuf = nullptr;
   int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
+  unsigned int *ticket = nullptr;    // fused-routing CTA counter
+  unsigned long long *trace = nullptr;  // moe_set_trace buffer
   unsigned long long *stats = nullptr;
   std::vector<int32_t> host_counts;
 
-  int gemv_blocks[2][2] = {{0, 0}, {0, 0}};
+  int gemv_blocks[2][2][2] = {};  // [fmt][gated][NTM-1]
   // profiling: 4 events per call slot
   bool profiling = false;
   std::vector<cudaEvent_t> prof_ev;
@@ -107,28 +110,49 @@ cudaError_t launch(void (*kern)(P), dim3 grid, dim3 block, size_t smem, cudaStre
   return cudaLaunchKernelEx(&cfg, kern, params);
 }
 
-template <int FMT, bool GATED>
+template <int FMT, bool GATED, int NTM>
 cudaError_t setup_gemv(int n_sm, int *blocks) {
-  using C = GemvCfg<FMT, GATED>;
-  cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<FMT, GATED>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  using C = GemvCfg<FMT, GATED, NTM>;
+  cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<FMT, GATED, NTM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<FMT, GATED>,
-                                                    C::WARPS * 32, C::SMEM);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<FMT, GATED, NTM>,
+                                                    C::WARPS * 32, kGemvSmem);
   if (e != cudaSuccess) return e;
   *blocks = n_sm * (per_sm > 0 ? per_sm : 1);
   return cudaSuccess;
 }
 
-template <int FMT, bool GATED>
+template <int FMT, bool GATED, int NTM>
 cudaError_t launch_gemv(moe_ctx *c, cudaStream_t s, const GemvParams &gp) {
-  using C = GemvCfg<FMT, GATED>;
-  return launch(expert_gemv_kernel<FMT, GATED>, dim3(c->gemv_blocks[FMT - 1][GATED]),
-                dim3(C::WARPS * 32), C::SMEM, s, gp);
+  using C = GemvCfg<FMT, GATED, NTM>;
+  return launch(expert_gemv_kernel<FMT, GATED, NTM>,
+                dim3(c->gemv_blocks[FMT - 1][GATED][NTM - 1]), dim3(C::WARPS * 32), kGemvSmem, s,
+                gp);
+}
+
+// tokens per expert job: 8 for windows of <= 8 tokens (NTM = 1), else 16
+int job_chunk(int T) { return T <= 8 ? 8 : 16; }
+
+template <int FMT>
+cudaError_t launch_experts(moe_ctx *c, cudaStream_t s, int T, const GemvParams &g1,
+                           const GemvParams &g2) {
+  cudaError_t e;
+  if (job_chunk(T) == 8) {
+    e = launch_gemv<FMT, true, 1>(c, s, g1);
+    if (e == cudaSuccess) e = launch_gemv<FMT, false, 1>(c, s, g2);
+  } else {
+    e = launch_gemv<FMT, true, 2>(c, s, g1);
+    if (e == cudaSuccess) e = launch_gemv<FMT, false, 2>(c, s, g2);
+  }
+  return e;
 }
 
 bool valid_layer(const moe_ctx *c, int layer) { return layer >= 0 && layer < c->L; }
+
+// activations are read with 16-byte vector loads and bulk copies
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 template <typename T>
 void dfree(T *&p) {
@@ -150,29 +174,49 @@ moe_status do_configure(moe_ctx *c) {
   CUDA_TRY(c, cudaMalloc(&c->d_bias, (size_t)c->L * E * sizeof(float)));
   CUDA_TRY(c, cudaMalloc(&c->d_gamma, (size_t)c->L * d * sizeof(float)));
   const long long P = (long long)T * k, Ptot = P + T;
-  c->max_jobs = (int)(P + E + (T + c->chunk - 1) / c->chunk + 8);
-  CUDA_TRY(c, cudaMalloc(&c->logits, (size_t)T * E * sizeof(float)));
-  CUDA_TRY(c, cudaMalloc(&c->w, (size_t)P * sizeof(float)));
-  CUDA_TRY(c, cudaMalloc(&c->idx, (size_t)P * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->off, (size_t)(E + 1) * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->perm, (size_t)P * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->plist, (size_t)Ptot * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->job_ptr, (size_t)c->max_jobs * sizeof(unsigned long long)));
-  CUDA_TRY(c, cudaMalloc(&c->job_beg, (size_t)c->max_jobs * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->job_n, (size_t)c->max_jobs * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->n_jobs, sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->hbuf, (size_t)T * d * 2));
-  CUDA_TRY(c, cudaMalloc(&c->abuf, (size_t)Ptot * f * 2));
-  CUDA_TRY(c, cudaMalloc(&c->ybuf, (size_t)Ptot * d * sizeof(float)));
-  CUDA_TRY(c, cudaMalloc(&c->status, sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->cnt_out, (size_t)E * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->last, 4 * sizeof(int)));
-  CUDA_TRY(c, cudaMalloc(&c->stats, 8 * sizeof(unsigned long long)));
-  CUDA_TRY(c, cudaMemset(c->status, 0, sizeof(int)));
-  CUDA_TRY(c, cudaMemset(c->cnt_out, 0, (size_t)E * sizeof(int)));
-  CUDA_TRY(c, cudaMemset(c->last, 0, 4 * sizeof(int)));
-  CUDA_TRY(c, cudaMemset(c->stats, 0, 8 * sizeof(unsigned long long)));
-  CUDA_TRY(c, cudaMemset(c->n_jobs, 0, sizeof(int)));
+  c->max_jobs = (int)(P + E + (T + c->chunk_min - 1) / c->chunk_min + 8);
+  // All per-call scratch lives in one allocation, small and hot buffers
+  // first, so a call touches few pages (the expert stream evicts the
+  // translations of scattered small buffers between calls).
+  size_t off = 0;
+  auto carve = [&](size_t bytes) {
+    const size_t at = off;
+    off += (bytes + 255) / 256 * 256;
+    return at;
+  };
+  const size_t o_status = carve(sizeof(int)), o_ticket = carve(sizeof(unsigned int));
+  const size_t o_njobs = carve(sizeof(int)), o_last = carve(4 * sizeof(int));
+  const size_t o_stats = carve(8 * sizeof(unsigned long long));
+  const size_t o_jptr = carve((size_t)c->max_jobs * sizeof(unsigned long long));
+  const size_t o_jbeg = carve((size_t)c->max_jobs * sizeof(int));
+  const size_t o_jn = carve((size_t)c->max_jobs * sizeof(int));
+  const size_t o_idx = carve((size_t)P * sizeof(int)), o_w = carve((size_t)P * sizeof(float));
+  const size_t o_off = carve((size_t)(E + 1) * sizeof(int)), o_perm = carve((size_t)P * sizeof(int));
+  const size_t o_plist = carve((size_t)Ptot * sizeof(int)), o_cnt = carve((size_t)E * sizeof(int));
+  const size_t o_logits = carve((size_t)T * E * sizeof(float));
+  const size_t o_h = carve((size_t)T * d * 2), o_a = carve((size_t)Ptot * f * 2);
+  const size_t o_y = carve((size_t)Ptot * d * sizeof(float));
+  CUDA_TRY(c, cudaMalloc(&c->scratch, off));
+  CUDA_TRY(c, cudaMemset(c->scratch, 0, off));
+  uint8_t *b = c->scratch;
+  c->status = (int *)(b + o_status);
+  c->ticket = (unsigned int *)(b + o_ticket);
+  c->n_jobs = (int *)(b + o_njobs);
+  c->last = (int *)(b + o_last);
+  c->stats = (unsigned long long *)(b + o_stats);
+  c->job_ptr = (unsigned long long *)(b + o_jptr);
+  c->job_beg = (int *)(b + o_jbeg);
+  c->job_n = (int *)(b + o_jn);
+  c->idx = (int *)(b + o_idx);
+  c->w = (float *)(b + o_w);
+  c->off = (int *)(b + o_off);
+  c->perm = (int *)(b + o_perm);
+  c->plist = (int *)(b + o_plist);
+  c->cnt_out = (int *)(b + o_cnt);
+  c->logits = (float *)(b + o_logits);
+  c->hbuf = (uint16_t *)(b + o_h);
+  c->abuf = (uint16_t *)(b + o_a);
+  c->ybuf = (float *)(b + o_y);
   c->has_router.assign(c->L, 0);
   c->has_bias.assign(c->L, 0);
   c->has_norm.assign(c->L, 0);
@@ -199,7 +243,7 @@ int finish_npl(int E) {
 }
 
 cudaError_t launch_finish(moe_ctx *c, cudaStream_t s, const FinishParams &fp) {
-  const size_t smem = (size_t)(4 * c->E + 2) * sizeof(int);
+  const size_t smem = (size_t)finish_smem_ints(c->E, fp.T * c->k) * sizeof(int);
   switch (finish_npl(c->E)) {
     case 1: return launch(route_finish_kernel<1>, dim3(1), dim3(kFinishThreads), smem, s, fp);
     case 2: return launch(route_finish_kernel<2>, dim3(1), dim3(kFinishThreads), smem, s, fp);
@@ -210,17 +254,63 @@ cudaError_t launch_finish(moe_ctx *c, cudaStream_t s, const FinishParams &fp) {
   }
 }
 
+// The one-launch routing step (route_fused_kernel) serves windows whose
+// tokens fit its shared-memory staging.
+bool use_fused_route(const moe_ctx *c, int T) {
+  const size_t need = std::max((size_t)T * c->d * 2,
+                               (size_t)finish_smem_ints(c->E, T * c->k) * sizeof(int));
+  return T <= kFusedMaxT && need <= (size_t)kFusedSmem;
+}
+
+cudaError_t launch_route_fused(moe_ctx *c, cudaStream_t s, const RouteFusedParams &rp) {
+  const int warps = rp.f.T <= 8 ? 4 : kFusedWarps;
+  const dim3 grid((c->E + warps - 1) / warps), block(warps * 32);
+  const size_t sm = std::max((size_t)rp.f.T * c->d * 2,
+                             (size_t)finish_smem_ints(c->E, rp.f.T * c->k) * sizeof(int));
+  switch (finish_npl(c->E)) {
+    case 1: return launch(route_fused_kernel<1>, grid, block, sm, s, rp);
+    case 2: return launch(route_fused_kernel<2>, grid, block, sm, s, rp);
+    case 4: return launch(route_fused_kernel<4>, grid, block, sm, s, rp);
+    case 8: return launch(route_fused_kernel<8>, grid, block, sm, s, rp);
+    case 16: return launch(route_fused_kernel<16>, grid, block, sm, s, rp);
+    default: return launch(route_fused_kernel<32>, grid, block, sm, s, rp);
+  }
+}
+
+cudaError_t setup_route_fused() {
+  cudaError_t e = cudaSuccess;
+  void (*ks[])(RouteFusedParams) = {route_fused_kernel<1>, route_fused_kernel<2>,
+                                    route_fused_kernel<4>, route_fused_kernel<8>,
+                                    route_fused_kernel<16>, route_fused_kernel<32>};
+  for (auto k : ks)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+  return e;
+}
+
+cudaError_t setup_finish() {
+  cudaError_t e = cudaSuccess;
+  void (*ks[])(FinishParams) = {route_finish_kernel<1>, route_finish_kernel<2>,
+                                route_finish_kernel<4>, route_finish_kernel<8>,
+                                route_finish_kernel<16>, route_finish_kernel<32>};
+  for (auto k : ks)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  return e;
+}
+
 cudaError_t launch_router(moe_ctx *c, cudaStream_t s, const RouterParams &rp) {
   const dim3 grid((c->E + kRouterWarps - 1) / kRouterWarps), block(kRouterWarps * 32);
+  const size_t sm = (size_t)std::min(rp.T, kRouterSmem / (2 * c->d)) * c->d * 2;
   switch (c->d / 128) {
-    case 1: return launch(router_logits_kernel<1>, grid, block, 0, s, rp);
-    case 2: return launch(router_logits_kernel<2>, grid, block, 0, s, rp);
-    case 4: return launch(router_logits_kernel<4>, grid, block, 0, s, rp);
-    case 8: return launch(router_logits_kernel<8>, grid, block, 0, s, rp);
-    case 12: return launch(router_logits_kernel<12>, grid, block, 0, s, rp);
-    case 16: return launch(router_logits_kernel<16>, grid, block, 0, s, rp);
-    case 24: return launch(router_logits_kernel<24>, grid, block, 0, s, rp);
-    case 32: return launch(router_logits_kernel<32>, grid, block, 0, s, rp);
+    case 1: return launch(router_logits_kernel<1>, grid, block, sm, s, rp);
+    case 2: return launch(router_logits_kernel<2>, grid, block, sm, s, rp);
+    case 4: return launch(router_logits_kernel<4>, grid, block, sm, s, rp);
+    case 8: return launch(router_logits_kernel<8>, grid, block, sm, s, rp);
+    case 12: return launch(router_logits_kernel<12>, grid, block, sm, s, rp);
+    case 16: return launch(router_logits_kernel<16>, grid, block, sm, s, rp);
+    case 24: return launch(router_logits_kernel<24>, grid, block, sm, s, rp);
+    case 32: return launch(router_logits_kernel<32>, grid, block, sm, s, rp);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -252,7 +342,7 @@ FinishParams finish_params(moe_ctx *c, int layer, int T) {
   fp.w = c->w;
   fp.off = c->off;
   fp.perm = c->perm;
-  fp.chunk = c->chunk;
+  fp.chunk = job_chunk(T);
   fp.plist = c->plist;
   fp.job_ptr = c->job_ptr;
   fp.job_beg = c->job_beg;
@@ -296,18 +386,49 @@ cudaError_t prof_mark(moe_ctx *c, int i, cudaStream_t s) {
 }
 
 // The whole decode chain for one layer.  delta == nullptr: residual mode.
-moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta, cudaStream_t s) {
+// Routing for `layer` (norm + logits + top-k + buckets + jobs when
+// build_jobs); returns the router input h (x, or the normalised copy).
+moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const FinishParams &fp,
+                      cudaStream_t s, const uint16_t **h_out) {
+  if (use_fused_route(c, T)) {
+    RouteFusedParams rp{};
+    rp.x = x;
+    rp.gamma = c->has_gamma[layer] ? c->d_gamma + (size_t)layer * c->d : nullptr;
+    rp.eps = c->eps[layer];
+    rp.use_norm = c->has_norm[layer];
+    rp.h_out = c->hbuf;
+    rp.W = c->d_router + (size_t)layer * c->E * c->d;
+    rp.bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr;
+    rp.d = c->d;
+    rp.logits = c->logits;
+    rp.ticket = c->ticket;
+    rp.f = fp;
+    CUDA_TRY(c, launch_route_fused(c, s, rp));
+    if (h_out) *h_out = rp.use_norm ? c->hbuf : x;
+    return MOE_OK;
+  }
   cudaError_t e = cudaSuccess;
-  CUDA_TRY(c, prof_mark(c, 0, s));
   const uint16_t *h = router_input(c, layer, x, T, s, &e);
   CUDA_TRY(c, e);
   RouterParams rp{h, c->d_router + (size_t)layer * c->E * c->d,
                   c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
                   c->logits};
   CUDA_TRY(c, launch_router(c, s, rp));
+  CUDA_TRY(c, launch_finish(c, s, fp));
+  if (h_out) *h_out = h;
+  return MOE_OK;
+}
+
+// The whole decode chain for one layer.  delta == nullptr: residual mode.
+// Windows of <= kFusedMaxT tokens take four launches: fused routing, the
+// gated expert GEMV, the down GEMV and the combine + residual.
+moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta, cudaStream_t s) {
+  CUDA_TRY(c, prof_mark(c, 0, s));
   FinishParams fp = finish_params(c, layer, T);
   fp.build_jobs = 1;
-  CUDA_TRY(c, launch_finish(c, s, fp));
+  const uint16_t *h = nullptr;
+  moe_status st = route_impl(c, layer, x, T, fp, s, &h);
+  if (st) return st;
 
   GemvParams g1{};
   g1.job_ptr = c->job_ptr;
@@ -333,18 +454,17 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
   g2.out_a = nullptr;
   g2.out_y = c->ybuf;
   CUDA_TRY(c, prof_mark(c, 1, s));
-  if (c->fmt == MOE_Q4_SYM_G32_F16) {
-    CUDA_TRY(c, (launch_gemv<1, true>(c, s, g1)));
-    CUDA_TRY(c, (launch_gemv<1, false>(c, s, g2)));
-  } else {
-    CUDA_TRY(c, (launch_gemv<2, true>(c, s, g1)));
-    CUDA_TRY(c, (launch_gemv<2, false>(c, s, g2)));
-  }
+  if (c->fmt == MOE_Q4_SYM_G32_F16)
+    CUDA_TRY(c, launch_experts<1>(c, s, T, g1, g2));
+  else
+    CUDA_TRY(c, launch_experts<2>(c, s, T, g1, g2));
   CUDA_TRY(c, prof_mark(c, 2, s));
-  CombineParams cp{c->ybuf, c->w, T, c->k, c->d, c->n_shared, x, delta};
-  const long long n4 = (long long)T * c->d / 4;
-  const int blocks = (int)std::min<long long>((n4 + 255) / 256, 4LL * c->n_sm);
-  CUDA_TRY(c, launch(combine_kernel, dim3(blocks), dim3(256), 0, s, cp));
+  {
+    CombineParams cp{c->ybuf, c->w, T, c->k, c->d, c->n_shared, x, delta};
+    const long long n4 = (long long)T * c->d / 4;
+    const int blocks = (int)std::min<long long>((n4 + 127) / 128, 8LL * c->n_sm);
+    CUDA_TRY(c, launch(combine_kernel, dim3(blocks), dim3(128), 0, s, cp));
+  }
   CUDA_TRY(c, prof_mark(c, 3, s));
   if (c->profiling) {
     c->prof_next = (c->prof_next + 1) % kProfSlots;
@@ -448,10 +568,16 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   c->lay = make_layout(fmt, d, f);
   cudaError_t e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = setup_gemv<1, true>(c->n_sm, &c->gemv_blocks[0][1]);
-  if (e == cudaSuccess) e = setup_gemv<1, false>(c->n_sm, &c->gemv_blocks[0][0]);
-  if (e == cudaSuccess) e = setup_gemv<2, true>(c->n_sm, &c->gemv_blocks[1][1]);
-  if (e == cudaSuccess) e = setup_gemv<2, false>(c->n_sm, &c->gemv_blocks[1][0]);
+  if (e == cudaSuccess) e = setup_route_fused();
+  if (e == cudaSuccess) e = setup_finish();
+  if (e == cudaSuccess) e = setup_gemv<1, true, 1>(c->n_sm, &c->gemv_blocks[0][1][0]);
+  if (e == cudaSuccess) e = setup_gemv<1, false, 1>(c->n_sm, &c->gemv_blocks[0][0][0]);
+  if (e == cudaSuccess) e = setup_gemv<2, true, 1>(c->n_sm, &c->gemv_blocks[1][1][0]);
+  if (e == cudaSuccess) e = setup_gemv<2, false, 1>(c->n_sm, &c->gemv_blocks[1][0][0]);
+  if (e == cudaSuccess) e = setup_gemv<1, true, 2>(c->n_sm, &c->gemv_blocks[0][1][1]);
+  if (e == cudaSuccess) e = setup_gemv<1, false, 2>(c->n_sm, &c->gemv_blocks[0][0][1]);
+  if (e == cudaSuccess) e = setup_gemv<2, true, 2>(c->n_sm, &c->gemv_blocks[1][1][1]);
+  if (e == cudaSuccess) e = setup_gemv<2, false, 2>(c->n_sm, &c->gemv_blocks[1][0][1]);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     moe_destroy(c);
@@ -486,23 +612,12 @@ moe_status moe_destroy(moe_ctx *c) {
   dfree(c->d_router);
   dfree(c->d_bias);
   dfree(c->d_gamma);
-  dfree(c->logits);
-  dfree(c->w);
-  dfree(c->ybuf);
-  dfree(c->idx);
-  dfree(c->off);
-  dfree(c->perm);
-  dfree(c->plist);
-  dfree(c->job_ptr);
-  dfree(c->job_beg);
-  dfree(c->job_n);
-  dfree(c->n_jobs);
-  dfree(c->hbuf);
-  dfree(c->abuf);
-  dfree(c->status);
-  dfree(c->cnt_out);
-  dfree(c->last);
-  dfree(c->stats);
+  dfree(c->scratch);
+  if (c->trace) {
+    unsigned long long *null_ptr = nullptr;
+    cudaMemcpyToSymbol(g_trace, &null_ptr, sizeof null_ptr);
+    dfree(c->trace);
+  }
   if (c->io) cudaStreamDestroy(c->io);
   (void)cudaGetLastError();
   delete c;
@@ -606,23 +721,23 @@ moe_status moe_route(moe_ctx *c, int layer, const void *h, int T, int32_t *idx, 
                      int32_t *boff, int32_t *bperm, void *stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
-  if (!valid_layer(c, layer) || !h || !idx || !w || T < 1 || T > c->max_tokens)
+  if (!valid_layer(c, layer) || !h || !idx || !w || T < 1 || T > c->max_tokens || !aligned16(h))
     return fail(c, MOE_ERR_INVALID_ARG, "moe_route: bad arguments (T=%d max=%d)", T, c->max_tokens);
   if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
-  RouterParams rp{(const uint16_t *)h, c->d_router + (size_t)layer * c->E * c->d,
-                  c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
-                  c->logits};
-  CUDA_TRY(c, launch_router(c, s, rp));
   FinishParams fp = finish_params(c, layer, T);
   fp.idx = idx;
   fp.w = w;
   fp.off = boff ? boff : c->off;
   fp.perm = bperm ? bperm : c->perm;
   fp.build_jobs = 0;
-  CUDA_TRY(c, launch_finish(c, s, fp));
-  return MOE_OK;
+  // moe_route takes the router input directly: no RMSNorm here
+  const char saved = c->has_norm[layer];
+  c->has_norm[layer] = 0;
+  moe_status st = route_impl(c, layer, (const uint16_t *)h, T, fp, s, nullptr);
+  c->has_norm[layer] = saved;
+  return st;
 }
 
 moe_status moe_bucket(moe_ctx *c, const int32_t *idx, int T, int32_t *boff, int32_t *bperm,
@@ -646,7 +761,7 @@ moe_status moe_bucket(moe_ctx *c, const int32_t *idx, int T, int32_t *boff, int3
 moe_status moe_forward(moe_ctx *c, int layer, void *x, int T, void *stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
-  if (!valid_layer(c, layer) || !x || T < 1 || T > c->max_tokens)
+  if (!valid_layer(c, layer) || !x || T < 1 || T > c->max_tokens || !aligned16(x))
     return fail(c, MOE_ERR_INVALID_ARG, "moe_forward: bad arguments (T=%d max=%d)", T,
                 c->max_tokens);
   moe_status st = check_ready(c, layer);
@@ -659,7 +774,8 @@ moe_status moe_forward_delta(moe_ctx *c, int layer, const void *x, int T, float 
                              void *stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
-  if (!valid_layer(c, layer) || !x || !delta || T < 1 || T > c->max_tokens)
+  if (!valid_layer(c, layer) || !x || !delta || T < 1 || T > c->max_tokens || !aligned16(x) ||
+      !aligned16(delta))
     return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_delta: bad arguments");
   moe_status st = check_ready(c, layer);
   if (st) return st;
@@ -671,7 +787,8 @@ moe_status moe_forward_delta(moe_ctx *c, int layer, const void *x, int T, float 
 moe_status moe_forward_stack(moe_ctx *c, void *x, int T, void *stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
-  if (!x || T < 1 || T > c->max_tokens) return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_stack");
+  if (!x || T < 1 || T > c->max_tokens || !aligned16(x))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_stack");
   for (int l = 0; l < c->L; ++l) {
     moe_status st = check_ready(c, l);
     if (st) return st;
@@ -786,6 +903,30 @@ moe_status moe_read_profile(moe_ctx *c, double ms[3], int64_t *n_calls) {
     for (int j = 0; j < 3; ++j) ms[j] += seg[j];
   }
   *n_calls = n;
+  return MOE_OK;
+}
+
+moe_status moe_set_trace(moe_ctx *c, int enable) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  unsigned long long *buf = nullptr;
+  if (enable) {
+    if (!c->trace) CUDA_TRY(c, cudaMalloc(&c->trace, 2 * kTrCount * sizeof(unsigned long long)));
+    CUDA_TRY(c, cudaMemset(c->trace, 0xFF, kTrCount * sizeof(unsigned long long)));
+    CUDA_TRY(c, cudaMemset(c->trace + kTrCount, 0, kTrCount * sizeof(unsigned long long)));
+    buf = c->trace;
+  }
+  CUDA_TRY(c, cudaDeviceSynchronize());
+  CUDA_TRY(c, cudaMemcpyToSymbol(g_trace, &buf, sizeof buf));
+  return MOE_OK;
+}
+
+moe_status moe_read_trace(moe_ctx *c, int64_t *out, int n) {
+  if (!c || !out || n < 2 * kTrCount) return fail(c, MOE_ERR_INVALID_ARG, "moe_read_trace");
+  if (!c->trace) return fail(c, MOE_ERR_STATE, "tracing was never enabled");
+  CUDA_TRY(c, cudaDeviceSynchronize());
+  CUDA_TRY(c, cudaMemcpy(out, c->trace, 2 * kTrCount * sizeof(int64_t), cudaMemcpyDeviceToHost));
+  CUDA_TRY(c, cudaMemset(c->trace, 0xFF, kTrCount * sizeof(unsigned long long)));
+  CUDA_TRY(c, cudaMemset(c->trace + kTrCount, 0, kTrCount * sizeof(unsigned long long)));
   return MOE_OK;
 }
 

@@ -56,8 +56,9 @@ def _mix_int(x: int) -> int:
 
 
 def stream_id(kind: int, layer: int = 0, index: int = 0) -> int:
-    assert 0 <= kind < 256 and 0 <= layer < 4096 and 0 <= index < 4096
-    return (kind << 24) ^ (layer << 12) ^ index
+    """32-bit stream id of (kind, layer, index), each a non-negative int < 2^32."""
+    assert 0 <= kind < 256 and 0 <= layer <= M32 and 0 <= index <= M32
+    return _mix_int(_mix_int(_mix_int(kind) ^ layer) + 0x632BE5AB ^ index)
 
 
 def stream_keys(seed: int, stream: int):
