@@ -259,7 +259,7 @@ cudaError_t launch_finish(moe_ctx *c, cudaStream_t s, const FinishParams &fp) {
 bool use_fused_route(const moe_ctx *c, int T) {
   const size_t need = std::max((size_t)T * c->d * 2,
                                (size_t)finish_smem_ints(c->E, T * c->k) * sizeof(int));
-  return T <= kFusedMaxT && need <= (size_t)kFusedSmem;
+  return T <= kFusedMaxT && c->d <= kFusedMaxV * 128 && need <= (size_t)kFusedSmem;
 }
 
 cudaError_t launch_route_fused(moe_ctx *c, cudaStream_t s, const RouteFusedParams &rp) {
