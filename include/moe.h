@@ -203,6 +203,34 @@ MOE_API moe_status moe_sync(moe_ctx *ctx, int timeout_ms);
 /* moe_get_stats: synchronises and fills *out (see moe_stats). */
 MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
 
+/* moe_route_static: the routing step of moe_route (router logits, top-k
+ * with renormalised softmax, bucketing) with NO allocation and no context,
+ * for callers that cannot call cudaMalloc (for example code that runs under
+ * a fixed device-memory budget handed to its own pool, or a plugin that is
+ * only given raw device pointers).  The pages this library follows have no
+ * counterpart of this call; it is a deployment convenience.
+ *  h_dev     bf16 [T, d] router input (16-byte aligned)
+ *  W_dev     fp32 [E, d] router weights (16-byte aligned); bias_dev fp32 [E]
+ *            or NULL
+ *  idx_dev, w_dev, bucket_off_dev, bucket_perm_dev: outputs exactly as in
+ *            moe_route (none may be NULL).
+ * Limits: 1 <= T <= 32, d a multiple of 128 and <= 2048, 1 <= E <= 1024,
+ * 1 <= k <= min(E, 32); anything else returns MOE_ERR_INVALID_ARG before any
+ * GPU work.  Scratch (logits, a completion ticket, a status word) lives in a
+ * static device array of about 129 KB that every GPU loading this library
+ * holds until the process exits.  The first call on a device, with that
+ * device current, looks up the array's device address and sets the routing
+ * kernels' shared-memory limit; make that first call before any stream
+ * capture.  Each call clears the array's counters on `stream` before use;
+ * calls whose execution overlaps on the GPU (other streams, other threads)
+ * race on the array.  Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA;
+ * an out-of-range routing id cannot occur (ids come from the top-k). */
+MOE_API moe_status moe_route_static(const void *h_dev, int T, int d, int E, int k,
+                                    const float *W_dev, const float *bias_dev,
+                                    int32_t *idx_dev, float *w_dev,
+                                    int32_t *bucket_off_dev, int32_t *bucket_perm_dev,
+                                    void *stream);
+
 /* Profiling: when enabled, every forward call records CUDA events on its
  * stream around its three segments -- routing (norm + router + top-k +
  * bucketing), experts (the two grouped dequant-GEMV kernels) and combine --

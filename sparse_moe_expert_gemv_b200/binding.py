@@ -30,7 +30,7 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_forward_stack", "moe_prefill", "moe_sync", "moe_get_stats",
            "moe_last_error", "moe_status_string", "moe_expert_bytes",
            "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
-           "moe_set_trace", "moe_read_trace")
+           "moe_set_trace", "moe_read_trace", "moe_route_static")
 
 
 class MoeError(RuntimeError):
@@ -73,6 +73,7 @@ def _load():
         "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
         "moe_set_profiling": [P, I],
         "moe_set_trace": [P, I],
+        "moe_route_static": [P, I, I, I, I, P, P, P, P, P, P, P],
         "moe_read_trace": [P, ctypes.POINTER(ctypes.c_int64), I],
         "moe_read_profile": [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -257,3 +258,10 @@ def moe_read_trace(ctx):
     _check(ctx, _lib.moe_read_trace(ctx, buf, n))
     k = len(TRACE_POINTS)
     return {name: (buf[i], buf[k + i]) for i, name in enumerate(TRACE_POINTS) if buf[i] != -1}
+
+
+def moe_route_static(h, T, d, E, k, W, bias, idx, w, bucket_off, bucket_perm, stream=None):
+    """Routing that allocates nothing (see include/moe.h)."""
+    _check(None, _lib.moe_route_static(_ptr(h), T, d, E, k, _ptr(W), _ptr(bias), _ptr(idx),
+                                       _ptr(w), _ptr(bucket_off), _ptr(bucket_perm),
+                                       _stream(stream)))

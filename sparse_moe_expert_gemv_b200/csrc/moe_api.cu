@@ -17,6 +17,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <thread>
 #include <utility>
@@ -938,6 +939,122 @@ moe_status moe_debug_poke_slot(moe_ctx *c, int layer, int expert, int32_t slot) 
     return fail(c, MOE_ERR_INVALID_ARG, "moe_debug_poke_slot");
   CUDA_TRY(c, cudaMemcpy(c->d_slot_of + (size_t)layer * c->E + expert, &slot, sizeof slot,
                          cudaMemcpyHostToDevice));
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+// ======================================================================
+// Routing with no allocation at all.
+//
+// Some callers cannot call cudaMalloc: code running inside a CUDA graph
+// that is being captured or re-instantiated under a fixed memory budget,
+// engines that hand every byte of device memory to their own pool up front
+// and forbid the driver allocator afterwards, or plugins that are given only
+// raw device pointers by a host framework.  moe_route_static serves them:
+// it needs no context, takes the router weights as a device pointer, and
+// keeps its only scratch -- the fp32 logits, the CTA completion ticket and a
+// status word -- in the file-scope device array below.  Every GPU that loads
+// this library holds that array (kStaticScratchBytes) until the process
+// exits.  The array is shared by every call on a device and keeps the last
+// call's contents; each call clears the words that must start at zero.  Two
+// calls whose execution overlaps on the GPU race on it.
+namespace {
+
+constexpr int kStaticMaxT = kFusedMaxT;  // tokens per call
+constexpr int kStaticMaxE = 1024;        // experts
+constexpr int kStaticMaxD = kFusedMaxV * 128;
+constexpr size_t kStaticHeader = 256;    // ticket, status, statistics words
+constexpr size_t kStaticScratchBytes =
+    kStaticHeader + (size_t)kStaticMaxT * kStaticMaxE * sizeof(float);
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+unsigned char *g_static_addr[kMaxDevices] = {};  // device address, per device
+
+// Once per device, with that device current: the device address of the
+// scratch array (a host-side name of a __device__ array is not a device
+// address) and the shared-memory limit of the routing kernels.
+cudaError_t static_scratch(int dev, unsigned char **out) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    e = setup_route_fused();
+    if (e != cudaSuccess) return e;
+    g_static_addr[dev] = static_cast<unsigned char *>(p);
+  }
+  *out = g_static_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route_static(const void *h, int T, int d, int E, int k, const float *W,
+                            const float *bias, int32_t *idx, float *w, int32_t *boff,
+                            int32_t *bperm, void *stream) {
+  if (!h || !W || !idx || !w || !boff || !bperm || T < 1 || T > kStaticMaxT || d < 128 ||
+      d % 128 || d > kStaticMaxD || E < 1 || E > kStaticMaxE || k < 1 || k > E || k > 32 ||
+      !aligned16(h) || !aligned16(W))
+    return MOE_ERR_INVALID_ARG;
+  const size_t smem = std::max((size_t)T * d * 2, (size_t)finish_smem_ints(E, T * k) * sizeof(int));
+  if (smem > (size_t)kFusedSmem) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  unsigned char *base = nullptr;
+  if (static_scratch(dev, &base) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // ticket, status and the statistics words must start at zero
+  if (cudaMemsetAsync(base, 0, kStaticHeader, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  RouteFusedParams rp{};
+  rp.x = (const uint16_t *)h;
+  rp.use_norm = 0;
+  rp.W = W;
+  rp.bias = bias;
+  rp.d = d;
+  rp.logits = reinterpret_cast<float *>(base + kStaticHeader);
+  rp.ticket = reinterpret_cast<unsigned int *>(base);
+  FinishParams &fp = rp.f;
+  fp.T = T;
+  fp.E = E;
+  fp.k = k;
+  fp.logits = rp.logits;
+  fp.idx = idx;
+  fp.w = w;
+  fp.off = boff;
+  fp.perm = bperm;
+  fp.build_jobs = 0;
+  fp.status = reinterpret_cast<int *>(base + 16);
+  fp.stats = reinterpret_cast<unsigned long long *>(base + 64);
+  const int warps = T <= 8 ? 4 : kFusedWarps;
+  const dim3 grid((E + warps - 1) / warps), block(warps * 32);
+  cudaError_t e;
+  switch (finish_npl(E)) {
+    case 1: e = launch(route_fused_kernel<1>, grid, block, smem, s, rp); break;
+    case 2: e = launch(route_fused_kernel<2>, grid, block, smem, s, rp); break;
+    case 4: e = launch(route_fused_kernel<4>, grid, block, smem, s, rp); break;
+    case 8: e = launch(route_fused_kernel<8>, grid, block, smem, s, rp); break;
+    case 16: e = launch(route_fused_kernel<16>, grid, block, smem, s, rp); break;
+    default: e = launch(route_fused_kernel<32>, grid, block, smem, s, rp); break;
+  }
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }
 
