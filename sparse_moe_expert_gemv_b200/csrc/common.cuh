@@ -157,6 +157,27 @@ MOE_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t ba
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// The same copy with an L2 cache policy (see l2_evict_first).
+MOE_DEV void bulk_g2s_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                           uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+// Policy for data read once: its L2 lines are the first to be evicted, so a
+// stream of them does not push other data (or code) out of L2.
+MOE_DEV uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// Start moving [src, src + bytes) from HBM into L2 (16-byte aligned, bytes a
+// multiple of 16); no completion to wait for.
+MOE_DEV void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 MOE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -1,0 +1,736 @@
+// decode.cuh -- the whole MoE layer of one decode window in one launch
+// (sm_100a).
+//
+// Per window of T <= 32 tokens (Strata engine analysis article "93 token/s on
+// one 8 GB card", section "Architecture overview": router -> the selected
+// experts, from wherever they reside -> combine into the residual), one
+// persistent CTA per SM runs five phases separated by grid-wide barriers:
+//
+//   1  stage the window in shared memory (RMSNorm applied when configured)
+//      and compute this CTA's slice of the router logits;       barrier
+//   2  every CTA reads all logits and, redundantly, selects the top-k of
+//      each token, buckets the pairs by expert, looks every selected expert
+//      up in the residency table and builds the job list in shared memory
+//      (no second barrier is needed: every CTA derives the same list);
+//   3  gate/up GEMV: the job list's weight units are split evenly over all
+//      warps of the grid (stream-K); an item cut between warps is finished
+//      by the warp holding its first unit, which adds the later warps'
+//      partial sums in warp order (deterministic), then a = SiLU(g) * u;
+//   4  the down projection's weight stream starts before the barrier that
+//      makes a visible;                                         barrier
+//      down GEMV, split the same way;                           barrier
+//   5  combine: x += sum_j w_j y_j + y_shared (j in order).
+//
+// Compared with one launch per step, this removes three kernel boundaries
+// and the single-CTA routing tail from the critical path, and no warp idles
+// while another still streams: every warp gets the same number of weight
+// bytes.  The grid is one CTA per SM (all co-resident); every wait is
+// bounded and reports kErrTimeout.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+#include "route.cuh"
+
+namespace moe {
+
+constexpr int kDecMaxT = 32;        // tokens per window (token sets are 32-bit masks)
+constexpr int kDecMaxPairs = 512;   // T * k
+constexpr int kDecMaxE = 1024;      // experts (top-k holds <= 32 logits per lane)
+constexpr int kDecMaxK = 32;        // lane j of the top-k warp returns selection j
+constexpr int kDecSmem = 224 * 1024;
+constexpr int kDecWv = 8;           // router-row float4s per lane held in registers
+
+// ------------------------------------------------ memory-model helpers
+MOE_DEV unsigned long long ld_acquire_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+MOE_DEV void st_release_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+MOE_DEV void red_release_add_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Orders this thread's earlier generic-proxy global accesses (and those it
+// has observed) before its later bulk-copy (async-proxy) reads of global memory.
+MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Grid-wide barrier of a launch whose CTAs are all resident.  *count only
+// grows (one arrival per CTA per barrier); a launch reads it once after its
+// dependency wait (a multiple of gridDim.x, every earlier barrier being
+// complete), so its n-th barrier completes when the counter reaches
+// base + n * gridDim.x: the arrival needs no reply.  Returns false if the
+// wait gave up.
+MOE_DEV bool grid_sync(unsigned long long *count, unsigned long long target) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_add_u64(count, 1ull);
+    bool ok = false;
+    for (uint32_t i = 0; !ok && i < (1u << 22); ++i) ok = ld_acquire_u64(count) >= target;
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Bounded wait for a partial-sum flag to carry this barrier epoch.
+MOE_DEV bool wait_flag(const unsigned long long *f, unsigned long long epoch) {
+  for (uint32_t i = 0; i < (1u << 20); ++i) {
+    if (ld_acquire_u64(f) == epoch) return true;
+    if (i >= 64) __nanosleep(64);
+  }
+  return false;
+}
+
+// ------------------------------------------------ shared-memory carve
+// Byte offsets from the dynamic shared-memory base.  The weight ring of
+// every warp comes first (offset 0).
+struct DecSmem {
+  int bars;          // ring mbarriers of every warp, then the window and staging barriers
+  int slot;          // int [E]      residency slots of this layer
+  int mask;          // u32 [E]      token set of every expert
+  int cnt;           // int [E+1]    per expert (jobs << 16 | tokens), then its exclusive scan
+  int idx, w;        // int / float [T*k] selections and weights
+  int plist;         // int [T*k + T] pair ids in job order
+  int jptr, jbeg, jn;  // job list: u64 expert address, first pair, tokens
+  int part;          // float [rpc * qp * T] router partial dots
+  int stage;         // window rows (phase 1-3), then down-projection B rows
+  int stage_bytes;
+  int rsh, rsa;      // padded row strides (bytes) of staged h and a rows
+  int rpc, qp;       // router rows per CTA, parts per row
+  int max_jobs;
+  int npl;           // logits per lane of the top-k warp
+};
+
+MOE_HOST_DEV_INLINE int dec_align(int x, int a) { return (x + a - 1) / a * a; }
+
+// The carve for one launch shape; ring = bytes of the warps' rings.  The
+// caller checks T * rsh <= stage_bytes.
+inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, int E, int k,
+                          int grid) {
+  DecSmem L{};
+  int off = ring;
+  auto carve = [&](int bytes, int align) {
+    off = dec_align(off, align);
+    const int at = off;
+    off += bytes;
+    return at;
+  };
+  const int P = T * k;
+  L.max_jobs = P + (T + chunk - 1) / chunk;
+  L.bars = carve((warps * kRingD + 2) * 8, 8);
+  L.slot = carve(E * 4, 16);
+  L.mask = carve(E * 4, 16);
+  L.cnt = carve((E + 1) * 4, 16);
+  L.idx = carve(P * 4, 16);
+  L.w = carve(P * 4, 16);
+  L.plist = carve((P + T) * 4, 16);
+  L.jptr = carve(L.max_jobs * 8, 16);
+  L.jbeg = carve(L.max_jobs * 4, 16);
+  L.jn = carve(L.max_jobs * 4, 16);
+  L.rpc = (E + grid - 1) / grid;
+  const int nch = d / 128;
+  L.qp = 1;
+  while (L.rpc * L.qp * 2 <= warps && nch % (L.qp * 2) == 0) L.qp *= 2;
+  L.part = carve(L.rpc * L.qp * T * 4, 16);
+  L.stage = carve(0, 128);
+  L.stage_bytes = kDecSmem - L.stage;
+  L.rsh = 2 * d + 64;
+  L.rsa = 2 * f + 64;
+  L.npl = E <= 128 ? 4 : E <= 512 ? 16 : 32;
+  return L;
+}
+
+struct DecodeParams {
+  uint16_t *x;          // bf16 [T, d] layer input; residual mode: x += moe(x)
+  float *delta;         // fp32 [T, d] or null; when set, moe(x) goes here and x is untouched
+  const float *gamma;   // RMSNorm weight [d] or null (gamma = 1)
+  float eps;
+  int use_norm;
+  const float *W;       // router fp32 [E, d]
+  const float *bias;    // fp32 [E] or null
+  int T, d, f, E, k, layer, chunk;
+  const int *slot_of;   // [L*E] residency table
+  int n_slots;
+  const uint8_t *arena, *pool, *shared;
+  long long expert_bytes, p1_bytes;
+  float *logits;        // [T, E]
+  uint16_t *abuf;       // bf16 [T*k + T, f]
+  float *ybuf;          // fp32 [T*k + T, d]
+  float *ws;            // stream-K partial sums [warps of the grid][32][16]
+  unsigned long long *flags;  // [2][warps of the grid]
+  unsigned long long *bar;    // grid barrier counter
+  int *cnt_out;
+  unsigned long long *stats;  // [0]=calls [1]=tokens [2]=hits [3]=misses [4]=near_ties
+  int *last;
+  int *status;
+  DecSmem sm;
+};
+
+// ------------------------------------------------ phase 2: routing
+// Top-k of every token, one warp per token; selections and weights into
+// shared memory and the token into its experts' token sets.
+template <int NPL>
+__device__ __noinline__ void decode_topk(const float *logits, int T, int E, int k, int nw,
+                                         int *s_idx, float *s_w, unsigned *s_mask,
+                                         unsigned long long *near_ties) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int t = wid; t < T; t += nw) {
+    int e;
+    float w;
+    warp_topk<NPL>(logits + (long long)t * E, E, k, lane, t == 0 && near_ties != nullptr, e, w,
+                   near_ties);
+    if (lane < k) {
+      s_idx[t * k + lane] = e;
+      s_w[t * k + lane] = w;
+      atomicOr(&s_mask[e], 1u << t);
+    }
+  }
+}
+
+// All threads of the CTA: the bucketing of the pairs by expert and the job
+// list.  Experts come in ascending id, each split into jobs of <= chunk
+// tokens in ascending t; one exclusive scan over the experts' packed
+// (jobs, tokens) counts gives every expert its first job and first pair.
+// Each selected expert is looked up in the residency table (slot pool, else
+// the backing arena; Strata engine analysis article "93 token/s on one 8 GB
+// card", section "Expert cache").  The shared expert's jobs come last.  CTA
+// 0 also writes the statistics.
+MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned *s_mask,
+                        const int *s_idx, int *s_cnt, int *s_plist, unsigned long long *s_jptr,
+                        int *s_jbeg, int *s_jn) {
+  __shared__ int s_red[32];
+  __shared__ unsigned long long s_hm[3];  // hits, misses, active experts (CTA 0)
+  const int tid = threadIdx.x;
+  const int E = p.E, k = p.k, T = p.T, P = T * k, CH = p.chunk;
+  const bool cta0 = blockIdx.x == 0;
+  if (tid < 3) s_hm[tid] = 0;
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int n = __popc(s_mask[e]);
+    s_cnt[e] = (((n + CH - 1) / CH) << 16) | n;
+  }
+  block_exclusive_scan(s_cnt, s_cnt, E, s_red);
+  const int routed_jobs = s_cnt[E] >> 16;
+  for (int e = tid; e < E; e += blockDim.x) {
+    unsigned m = s_mask[e];
+    const int n = __popc(m);
+    if (cta0) p.cnt_out[e] = n;
+    if (!n) continue;
+    int jx = s_cnt[e] >> 16;
+    const int px = s_cnt[e] & 0xFFFF;
+    const int slot = s_slot[e];
+    const uint8_t *ptr;
+    const bool hit = slot >= 0 && slot < p.n_slots;
+    if (hit) {
+      ptr = p.pool + (long long)slot * p.expert_bytes;
+    } else {
+      if (slot >= p.n_slots && cta0) atomicOr(p.status, kErrBadSlot);
+      ptr = p.arena + ((long long)p.layer * E + e) * p.expert_bytes;
+    }
+    if (cta0) {
+      atomicAdd(&s_hm[hit ? 0 : 1], (unsigned long long)n);
+      atomicAdd(&s_hm[2], 1ull);
+    }
+    for (int b = 0; m; ++b) {
+      const int t = __ffs(m) - 1;
+      m &= m - 1;
+      int j = 0;
+      while (j < k - 1 && s_idx[t * k + j] != e) ++j;
+      s_plist[px + b] = t * k + j;
+    }
+    for (int c0 = 0; c0 < n; c0 += CH, ++jx) {
+      s_jptr[jx] = (unsigned long long)ptr;
+      s_jbeg[jx] = px + c0;
+      s_jn[jx] = min(CH, n - c0);
+    }
+  }
+  int shared_jobs = 0;
+  if (p.shared) {
+    shared_jobs = (T + CH - 1) / CH;
+    for (int t = tid; t < T; t += blockDim.x) s_plist[P + t] = P + t;
+    for (int q = tid; q < shared_jobs; q += blockDim.x) {
+      s_jptr[routed_jobs + q] = (unsigned long long)p.shared;
+      s_jbeg[routed_jobs + q] = P + q * CH;
+      s_jn[routed_jobs + q] = min(CH, T - q * CH);
+    }
+  }
+  __syncthreads();
+  if (cta0 && tid == 0) {
+    atomicAdd(&p.stats[0], 1ULL);
+    atomicAdd(&p.stats[1], (unsigned long long)T);
+    atomicAdd(&p.stats[2], s_hm[0]);
+    atomicAdd(&p.stats[3], s_hm[1]);
+    p.last[0] = T;
+    p.last[1] = (int)s_hm[2];
+    p.last[2] = p.layer;
+  }
+  return routed_jobs + shared_jobs;
+}
+
+// ------------------------------------------------ phases 3 and 4: stream-K GEMV
+// The phase's U weight units (job-major, then row block, then unit) are
+// split over the W warps of the grid: warp w owns [U w / W, U (w+1) / W).
+struct SKCtx {
+  long long U;
+  int W, gw;
+  unsigned long long epoch;   // this phase's barrier number
+  float *ws;                  // [W][32 lanes][16] partial sums
+  unsigned long long *flags;  // [W] this phase's hand-over flags
+};
+
+MOE_DEV long long sk_start(const SKCtx &sk, int w) { return sk.U * w / sk.W; }
+
+// One item of the warp's range: units [ua, ub) of item `it`.
+//  ua > 0   the item began in an earlier warp's range: publish the partial
+//           sum (ws[gw], then flags[gw] = epoch) for that warp to add;
+//  ub < UPI the item continues in later warps' ranges: add their partial
+//           sums in warp order, then store;
+//  else     the whole item is here: store.
+template <int FMT, bool GATED, int NTA>
+MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, long long it, int ua, int ub,
+                     int lane, int rb, const BRows &br, const int (&epair)[2][2], int R,
+                     uint16_t *out_a, float *out_y) {
+  using Run = ItemRun<FMT, GATED, NTA>;
+  constexpr int NM = Run::C::NM;
+  float acc[NM][NTA][4];
+  if (!Run::run(r, ph, lane, ua, ub, br, acc)) return false;
+  if (ua > 0) {
+    float4 *mine = reinterpret_cast<float4 *>(sk.ws + ((long long)sk.gw * 32 + lane) * 16);
+#pragma unroll
+    for (int m = 0; m < NM; ++m)
+#pragma unroll
+      for (int nt = 0; nt < NTA; ++nt)
+        mine[m * NTA + nt] = make_float4(acc[m][nt][0], acc[m][nt][1], acc[m][nt][2], acc[m][nt][3]);
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      st_release_u64(sk.flags + sk.gw, sk.epoch);
+    }
+    return true;
+  }
+  if (ub < ph.UPI) {
+    const long long iend = (it + 1) * ph.UPI;
+    for (int w2 = sk.gw + 1; w2 < sk.W; ++w2) {
+      const long long s2 = sk_start(sk, w2);
+      if (s2 >= iend) break;
+      if (sk_start(sk, w2 + 1) == s2) continue;  // empty range: nothing to add
+      if (__any_sync(0xffffffffu, !wait_flag(sk.flags + w2, sk.epoch))) return false;
+      const float *src = sk.ws + ((long long)w2 * 32 + lane) * 16;
+#pragma unroll
+      for (int m = 0; m < NM; ++m)
+#pragma unroll
+        for (int nt = 0; nt < NTA; ++nt) {
+          const float4 v = ldcg_f4(src + 4 * (m * NTA + nt));
+          acc[m][nt][0] += v.x;
+          acc[m][nt][1] += v.y;
+          acc[m][nt][2] += v.z;
+          acc[m][nt][3] += v.w;
+        }
+    }
+  }
+  Run::store(acc, epair, rb, lane, R, out_a, out_y);
+  return true;
+}
+
+// Gate/up pass over this warp's units.  B rows are the window's token rows,
+// all staged in shared memory (row stride rsh) at stage_g.
+template <int FMT, int NTM>
+MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, long long u0, long long u1,
+                          const DecodeParams &p, const int *s_plist, const int *s_jbeg,
+                          const int *s_jn, const unsigned char *stage_g) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  const int P = p.T * p.k;
+  if (u1 <= u0) return true;
+  for (long long it = u0 / ph.UPI; it * ph.UPI < u1; ++it) {
+    const int ua = (int)(max(u0, it * ph.UPI) - it * ph.UPI);
+    const int ub = (int)(min(u1, (it + 1) * ph.UPI) - it * ph.UPI);
+    const int job = (int)(it / ph.RB), rb = (int)(it - (long long)job * ph.RB);
+    const int n = s_jn[job], beg = s_jbeg[job];
+    BRows br;
+    int epair[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      br.row[nt] = nullptr;
+      epair[nt][0] = epair[nt][1] = -1;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTM; ++nt) {
+      const int ni = nt * 8 + g;
+      if (ni < n) {
+        const int pair = s_plist[beg + ni];
+        const int tok = pair < P ? pair / p.k : pair - P;
+        br.row[nt] = reinterpret_cast<const uint16_t *>(stage_g + (size_t)tok * p.sm.rsh);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int nc = nt * 8 + 2 * tig + c;
+        epair[nt][c] = nc < n ? s_plist[beg + nc] : -1;
+      }
+    }
+    const bool ok =
+        (NTM == 1 || n <= 8)
+            ? sk_item<FMT, true, 1>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr)
+            : sk_item<FMT, true, NTM>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr);
+    if (!ok) return false;
+  }
+  return true;
+}
+
+// Down pass over this warp's units.  B rows are rows of a: the CTA's first
+// jobs are staged in shared memory at stage_g (nst jobs; job jfirst + i
+// starts at staged row row0 of lane i), later ones are read from global
+// memory.
+template <int FMT, int NTM>
+MOE_DEV bool decode_down(WarpRing &r, const Phase &ph, const SKCtx &sk, long long u0, long long u1,
+                         const DecodeParams &p, const int *s_plist, const int *s_jbeg,
+                         const int *s_jn, const unsigned char *stage_g, uint32_t st_bar, int jfirst,
+                         int nst, int row0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  bool staged_ready = false;
+  if (u1 <= u0) return true;
+  for (long long it = u0 / ph.UPI; it * ph.UPI < u1; ++it) {
+    const int ua = (int)(max(u0, it * ph.UPI) - it * ph.UPI);
+    const int ub = (int)(min(u1, (it + 1) * ph.UPI) - it * ph.UPI);
+    const int job = (int)(it / ph.RB), rb = (int)(it - (long long)job * ph.RB);
+    const int n = s_jn[job], beg = s_jbeg[job];
+    const int sj = job - jfirst;
+    const bool staged = sj >= 0 && sj < nst;
+    const int jrow0 = __shfl_sync(0xffffffffu, row0, staged ? sj : 0);
+    if (staged && !staged_ready) {
+      if (__any_sync(0xffffffffu, !mbar_wait_bounded(st_bar, 0))) return false;
+      staged_ready = true;
+    }
+    BRows br;
+    int epair[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      br.row[nt] = nullptr;
+      epair[nt][0] = epair[nt][1] = -1;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTM; ++nt) {
+      const int ni = nt * 8 + g;
+      if (ni < n)
+        br.row[nt] = staged ? reinterpret_cast<const uint16_t *>(stage_g + (size_t)(jrow0 + ni) * p.sm.rsa)
+                            : p.abuf + (long long)s_plist[beg + ni] * p.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int nc = nt * 8 + 2 * tig + c;
+        epair[nt][c] = nc < n ? s_plist[beg + nc] : -1;
+      }
+    }
+    const bool ok =
+        (NTM == 1 || n <= 8)
+            ? sk_item<FMT, false, 1>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf)
+            : sk_item<FMT, false, NTM>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf);
+    if (!ok) return false;
+  }
+  return true;
+}
+
+// dot of one 128-column chunk of a router row (w: this lane's 4 columns)
+// with up to 8 staged token rows
+MOE_DEV void dot8(float (&acc)[8], const float4 w, uint32_t hcol, int t0, int T, int rsh) {
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    if (t0 + tt < T) {
+      const uint2 v = lds_u2(hcol + (uint32_t)(t0 + tt) * rsh);
+      acc[tt] = fmaf(w.x, __uint_as_float(v.x << 16), acc[tt]);
+      acc[tt] = fmaf(w.y, __uint_as_float(v.x & 0xFFFF0000u), acc[tt]);
+      acc[tt] = fmaf(w.z, __uint_as_float(v.y << 16), acc[tt]);
+      acc[tt] = fmaf(w.w, __uint_as_float(v.y & 0xFFFF0000u), acc[tt]);
+    }
+  }
+}
+
+// The decode kernel.  NTM = 8-token column tiles per job (jobs of <= 8 NTM
+// tokens); one CTA per SM.
+template <int FMT, int NTM>
+__global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
+    decode_kernel(DecodeParams p) {
+  using CG = GemvCfg<FMT, true, NTM>;
+  using CD = GemvCfg<FMT, false, NTM>;
+  constexpr int WARPS = CG::WARPS;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_njobs;
+  __shared__ unsigned long long s_bar0;  // grid barrier counter at launch
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int T = p.T, d = p.d, f = p.f, E = p.E, k = p.k;
+  const DecSmem &L = p.sm;
+  int *s_slot = reinterpret_cast<int *>(smem + L.slot);
+  unsigned *s_mask = reinterpret_cast<unsigned *>(smem + L.mask);
+  int *s_cnt = reinterpret_cast<int *>(smem + L.cnt);
+  int *s_idx = reinterpret_cast<int *>(smem + L.idx);
+  float *s_w = reinterpret_cast<float *>(smem + L.w);
+  int *s_plist = reinterpret_cast<int *>(smem + L.plist);
+  unsigned long long *s_jptr = reinterpret_cast<unsigned long long *>(smem + L.jptr);
+  int *s_jbeg = reinterpret_cast<int *>(smem + L.jbeg);
+  int *s_jn = reinterpret_cast<int *>(smem + L.jn);
+  float *s_part = reinterpret_cast<float *>(smem + L.part);
+  const uint32_t stage_s = smem_addr(smem + L.stage);
+  const unsigned char *stage_g = smem + L.stage;
+  const uint32_t bars = smem_addr(smem + L.bars);
+  const uint32_t h_bar = bars + WARPS * kRingD * 8, st_bar = h_bar + 8;
+
+  MOE_TRACE(kTrRouteStart);
+  WarpRing r;
+  ring_init(r, smem_addr(smem) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT);
+  if (lane == 0) {
+    for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, 1);
+    if (wid == 0) {
+      mbar_init(h_bar, 1);
+      mbar_init(st_bar, 1);
+    }
+    fence_mbar_init();
+  }
+  // Router rows of this CTA: rpc rows, each dotted in qp parts of cpp
+  // 128-column chunks by one warp per (row, part).  The first task's row
+  // part goes into registers before the dependency wait (the router weights
+  // do not depend on earlier kernels).
+  const int RPC = L.rpc, QP = L.qp, CPP = (d / 128) / QP, ntask = RPC * QP;
+  float4 wv[kDecWv];
+  {
+    const int rr = wid / QP, q = wid - rr * QP, e = blockIdx.x * RPC + rr;
+    const bool has = wid < ntask && e < E;
+    const float4 *wr = reinterpret_cast<const float4 *>(p.W + (long long)(has ? e : 0) * d) +
+                       q * CPP * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < kDecWv; ++i)
+      wv[i] = (has && i < CPP) ? __ldg(wr + 32 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int e = tid; e < E; e += blockDim.x) {
+    s_slot[e] = p.slot_of ? p.slot_of[(long long)p.layer * E + e] : -1;
+    s_mask[e] = 0u;
+  }
+  __syncthreads();
+  pdl_wait();
+  MOE_TRACE(kTrRouteWaited);
+  if (tid == 0) s_bar0 = ld_acquire_u64(p.bar);  // read by all after the next barrier
+
+  // ---------------- phase 1: the window, RMSNorm, router logits
+  if (tid == 0) {
+    mbar_expect_tx(h_bar, (uint32_t)T * d * 2);
+    for (int t = 0; t < T; ++t)
+      bulk_g2s(stage_s + (uint32_t)t * L.rsh, p.x + (long long)t * d, (uint32_t)d * 2, h_bar);
+  }
+  if (__syncthreads_or(!mbar_wait_bounded(h_bar, 0))) {
+    if (tid == 0) atomicOr(p.status, kErrTimeout);
+    return;
+  }
+  if (p.use_norm) {  // fp32 sum of squares, IEEE sqrt and divide, bf16 RNE
+    for (int t = wid; t < T; t += WARPS) {
+      uint16_t *hr = reinterpret_cast<uint16_t *>(smem + L.stage + (long long)t * L.rsh);
+      float ss = 0.f;
+      for (int i = lane * 4; i < d; i += 128) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(hr + i);
+        const float a0 = __uint_as_float(v.x << 16), a1 = __uint_as_float(v.x & 0xFFFF0000u);
+        const float a2 = __uint_as_float(v.y << 16), a3 = __uint_as_float(v.y & 0xFFFF0000u);
+        ss += a0 * a0 + a1 * a1 + a2 * a2 + a3 * a3;
+      }
+      ss = warp_sum(ss);
+      const float inv = 1.0f / sqrtf(ss / (float)d + p.eps);
+      for (int i = lane * 4; i < d; i += 128) {
+        uint2 v = *reinterpret_cast<const uint2 *>(hr + i);
+        const float in[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                             __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u)};
+        unsigned short o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float rv = in[j] * inv;
+          if (p.gamma) rv *= p.gamma[i + j];
+          o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(rv));
+        }
+        v.x = o[0] | ((uint32_t)o[1] << 16);
+        v.y = o[2] | ((uint32_t)o[3] << 16);
+        *reinterpret_cast<uint2 *>(hr + i) = v;
+      }
+    }
+    __syncthreads();
+  }
+  for (int task = wid, it = 0; task < ntask; task += WARPS, ++it) {
+    const int rr = task / QP, q = task - rr * QP, e = blockIdx.x * RPC + rr;
+    if (e >= E) continue;
+    const float4 *wr = reinterpret_cast<const float4 *>(p.W + (long long)e * d) + q * CPP * 32 + lane;
+    const uint32_t hcol = stage_s + 2u * (uint32_t)(q * CPP * 128 + lane * 4);
+    for (int t0 = 0; t0 < T; t0 += 8) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kDecWv; ++i)
+        if (i < CPP) dot8(acc, it == 0 ? wv[i] : __ldg(wr + 32 * i), hcol + 256u * i, t0, T, L.rsh);
+      for (int i = kDecWv; i < CPP; ++i) dot8(acc, __ldg(wr + 32 * i), hcol + 256u * i, t0, T, L.rsh);
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt) {
+        if (t0 + tt >= T) break;
+        const float v = warp_sum(acc[tt]);
+        if (lane == tt) s_part[task * T + t0 + tt] = v;
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < RPC * T; i += blockDim.x) {
+    const int rr = i / T, t = i - rr * T, e = blockIdx.x * RPC + rr;
+    if (e < E) {
+      float s = 0.f;
+      for (int q = 0; q < QP; ++q) s += s_part[(rr * QP + q) * T + t];
+      if (p.bias) s += p.bias[e];
+      p.logits[(long long)t * E + e] = s;
+    }
+  }
+  MOE_TRACE(kTrRouteLogits);
+  const unsigned long long G = gridDim.x, ep0 = s_bar0 / G;
+  const unsigned long long ep1 = ep0 + 1;
+  if (!grid_sync(p.bar, ep1 * G)) {
+    if (tid == 0) atomicOr(p.status, kErrTimeout);
+    return;
+  }
+  MOE_TRACE(kTrRouteLastStart);
+
+  // ---------------- phase 2: routing (every CTA, redundantly)
+  unsigned long long *near = blockIdx.x == 0 ? &p.stats[4] : nullptr;
+  if (L.npl == 4) decode_topk<4>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  else if (L.npl == 16) decode_topk<16>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  else decode_topk<32>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  __syncthreads();
+  MOE_TRACE(kTrRouteTopk);
+  {
+    const int nj = decode_jobs(p, s_slot, s_mask, s_idx, s_cnt, s_plist, s_jptr, s_jbeg, s_jn);
+    if (tid == 0) s_njobs = nj;
+  }
+  __syncthreads();
+  MOE_TRACE(kTrRouteEnd);
+  const int n_jobs = s_njobs;
+  const int W = gridDim.x * WARPS, gw = blockIdx.x * WARPS + wid;
+
+  // ---------------- phase 3: gate/up
+  const Phase ph1 = make_phase(s_jptr, f, d, CG::TK, CG::STRIDE, 0);
+  SKCtx sk1{(long long)n_jobs * ph1.RB * ph1.UPI, W, gw, ep1, p.ws, p.flags};
+  {
+    const long long u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1);
+    ring_start(r, ph1, u0 / ph1.UPI, (int)(u0 % ph1.UPI), u1 - u0, 1);
+    if (lane == 0) ring_prologue(r, ph1);
+    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g)) {
+      if (lane == 0) atomicOr(p.status, kErrTimeout);
+      ring_drain(r);
+    }
+  }
+  if (lane == 0) trace_point(kTrGateEnd);
+
+  // ---------------- phase 4: down projection
+  const Phase ph2 = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes);
+  SKCtx sk2{(long long)n_jobs * ph2.RB * ph2.UPI, W, gw, ep0 + 2, p.ws, p.flags + W};
+  const long long v0 = sk_start(sk2, gw), v1 = sk_start(sk2, gw + 1);
+  ring_start(r, ph2, v0 / ph2.UPI, (int)(v0 % ph2.UPI), v1 - v0, 1);
+  if (lane == 0) ring_prologue(r, ph2);  // weights stream in while the grid syncs
+  if (!grid_sync(p.bar, sk2.epoch * G)) {
+    ring_drain(r);
+    if (tid == 0) atomicOr(p.status, kErrTimeout);
+    return;
+  }
+  MOE_TRACE(kTrDownWaited);
+  // Stage the a rows of this CTA's first down jobs (whole jobs, at most
+  // kMaxStagedJobs, as many as fit).  Every warp derives the same plan; lane
+  // i describes job jfirst + i.
+  int jfirst = 0, njobs_cta = 0;
+  {
+    const long long c0 = sk_start(sk2, blockIdx.x * WARPS), c1 = sk_start(sk2, (blockIdx.x + 1) * WARPS);
+    if (c1 > c0) {
+      jfirst = (int)(c0 / ph2.UPI / ph2.RB);
+      njobs_cta = (int)((c1 - 1) / ph2.UPI / ph2.RB) - jfirst + 1;
+    }
+  }
+  int pn = 0, pbeg = 0;
+  if (lane < njobs_cta && lane < kMaxStagedJobs) {
+    pn = s_jn[jfirst + lane];
+    pbeg = s_jbeg[jfirst + lane];
+  }
+  int incl = pn;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int row0 = incl - pn;
+  const int cap = L.stage_bytes / L.rsa;
+  const int nst = __popc(__ballot_sync(0xffffffffu, pn > 0 && incl <= cap));
+  const int used = nst ? __shfl_sync(0xffffffffu, incl, nst - 1) : 0;
+  if (wid == 0) {
+    // a was written by other CTAs' generic stores before the barrier; the
+    // window rows in the staging area were last read before it
+    fence_proxy_async_global();
+    fence_proxy_async_smem();
+    if (lane == 0) mbar_expect_tx(st_bar, (uint32_t)used * f * 2);
+    __syncwarp();
+    for (int r0 = 0; r0 < used; r0 += 32) {
+      const int rr = r0 + lane;
+      int sj = 0;
+      for (int q = 1; q < nst; ++q) sj += rr >= __shfl_sync(0xffffffffu, row0, q) ? 1 : 0;
+      const int beg = __shfl_sync(0xffffffffu, pbeg, sj);
+      const int rj = rr - __shfl_sync(0xffffffffu, row0, sj);
+      if (rr < used)
+        bulk_g2s(stage_s + (uint32_t)rr * L.rsa, p.abuf + (long long)s_plist[beg + rj] * f,
+                 (uint32_t)f * 2, st_bar);
+    }
+  }
+  if (!decode_down<FMT, NTM>(r, ph2, sk2, v0, v1, p, s_plist, s_jbeg, s_jn, stage_g, st_bar, jfirst,
+                             nst, row0)) {
+    if (lane == 0) atomicOr(p.status, kErrTimeout);
+    ring_drain(r);
+  }
+  if (lane == 0) trace_point(kTrDownEnd);
+  // the staged rows must have landed before the CTA exits
+  if (wid == 0 && used > 0 && nst > 0) (void)mbar_wait_bounded(st_bar, 0);
+  if (!grid_sync(p.bar, (ep0 + 3) * G)) {
+    if (tid == 0) atomicOr(p.status, kErrTimeout);
+    return;
+  }
+  pdl_launch_dependents();
+
+  // ---------------- phase 5: combine + residual
+  MOE_TRACE(kTrCombStart);
+  const int P = T * k, per_t = d / 4;
+  for (int i = blockIdx.x * blockDim.x + tid; i < T * per_t; i += gridDim.x * blockDim.x) {
+    const int t = i / per_t, o = (i - t * per_t) * 4;
+    const float4 sh = p.shared ? ldcg_f4(p.ybuf + ((long long)P + t) * d + o) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int j0 = 0; j0 < k; j0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (j0 + q < k) v[q] = ldcg_f4(p.ybuf + ((long long)t * k + j0 + q) * d + o);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (j0 + q < k) {
+          const float wj = s_w[t * k + j0 + q];
+          a0 = fmaf(wj, v[q].x, a0);
+          a1 = fmaf(wj, v[q].y, a1);
+          a2 = fmaf(wj, v[q].z, a2);
+          a3 = fmaf(wj, v[q].w, a3);
+        }
+      }
+    }
+    a0 += sh.x;
+    a1 += sh.y;
+    a2 += sh.z;
+    a3 += sh.w;
+    if (p.delta) {
+      *reinterpret_cast<float4 *>(p.delta + (long long)t * d + o) = make_float4(a0, a1, a2, a3);
+    } else {
+      uint16_t *xr = p.x + (long long)t * d + o;
+      const uint2 xv = *reinterpret_cast<const uint2 *>(xr);
+      uint2 o2;
+      o2.x = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.x << 16) + a0)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.x & 0xFFFF0000u) + a1)) << 16);
+      o2.y = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.y << 16) + a2)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.y & 0xFFFF0000u) + a3)) << 16);
+      *reinterpret_cast<uint2 *>(xr) = o2;
+    }
+  }
+  if (lane == 0) trace_point(kTrCombEnd);
+}
+
+}  // namespace moe

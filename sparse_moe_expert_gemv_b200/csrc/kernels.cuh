@@ -31,6 +31,14 @@ struct RepackParams {
   Layout L;
 };
 
+// First reduction column of k-step `st` held by lane quad position `tig`:
+// within each 32-column block, lane tig owns columns [8 tig, 8 tig + 8): the
+// first four feed k-step 2q (fragment columns 2tig, 2tig+1, 2tig+8, 2tig+9
+// in that order), the next four k-step 2q+1.  The same permutation of the
+// reduction applies to the codes and to the B operand, so one 16-byte load
+// of a B row gives a lane both fragments of two consecutive k-steps.
+MOE_HOST_DEV_INLINE int kb_step(int st, int tig) { return 32 * (st >> 1) + 8 * tig + 4 * (st & 1); }
+
 // One thread per 32-bit code word of the device layout, then one per scale
 // entry.  Canonical layout: per expert Wg [f,d], Wu [f,d], Wd [d,f] codes
 // back to back (Q4: 2 per byte, low nibble first; Q2: 4 per byte, element i
@@ -77,7 +85,7 @@ __global__ void repack_kernel(RepackParams p) {
       const int r0 = rb * 16 + g, r1 = r0 + 8;
       uint32_t v = 0;
       if (q4) {
-        const int kb = t * 64 + 16 * word + 4 * tig;
+        const int kb = t * 64 + kb_step(word, tig);
         for (int fr = 0; fr < 4; ++fr) {
           const int row = (fr & 1) ? r1 : r0, col = kb + ((fr & 2) ? 2 : 0);
           const uint32_t lo = (src[(long long)row * (K / 2) + col / 2] >> (4 * (col & 1))) & 0xF;
@@ -88,7 +96,7 @@ __global__ void repack_kernel(RepackParams p) {
       } else {
         for (int r = 0; r < 8; ++r) {
           const int st = 2 * word + (r >> 2), fr = r & 3;
-          const int kb = t * 128 + 16 * st + 4 * tig;
+          const int kb = t * 128 + kb_step(st, tig);
           const int row = (fr & 1) ? r1 : r0, col = kb + ((fr & 2) ? 2 : 0);
           const uint32_t lo = (src[(long long)row * (K / 4) + col / 4] >> (2 * (col & 3))) & 3;
           const uint32_t hi = (src[(long long)row * (K / 4) + (col + 1) / 4] >> (2 * ((col + 1) & 3))) & 3;

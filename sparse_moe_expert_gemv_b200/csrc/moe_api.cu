@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "../../include/moe.h"
+#include "decode.cuh"
 #include "kernels.cuh"
 
 using namespace moe;
@@ -58,6 +59,11 @@ struct moe_ctx {
   uint16_t *hbuf = nullptr, *abuf = nullptr;
   int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
   unsigned int *ticket = nullptr;    // fused-routing CTA counter
+  // single-launch decode kernel: grid barrier counter, hand-over flags and
+  // partial sums (one slot per warp of the grid)
+  unsigned long long *dec_bar = nullptr, *dec_flags = nullptr;
+  float *dec_ws = nullptr;
+  size_t dec_sync_bytes = 0;  // bytes of the counter + flags block (cleared after a timeout)
   unsigned long long *trace = nullptr;  // moe_set_trace buffer
   unsigned long long *stats = nullptr;
   std::vector<int32_t> host_counts;
@@ -186,6 +192,9 @@ moe_status do_configure(moe_ctx *c) {
     return at;
   };
   const size_t o_status = carve(sizeof(int)), o_ticket = carve(sizeof(unsigned int));
+  const size_t dec_warps = (size_t)c->n_sm * 16;
+  const size_t o_dbar = carve(sizeof(unsigned long long) * (1 + 2 * dec_warps));
+  const size_t o_dws = carve(sizeof(float) * dec_warps * 32 * 16);
   const size_t o_njobs = carve(sizeof(int)), o_last = carve(4 * sizeof(int));
   const size_t o_stats = carve(8 * sizeof(unsigned long long));
   const size_t o_jptr = carve((size_t)c->max_jobs * sizeof(unsigned long long));
@@ -202,6 +211,10 @@ moe_status do_configure(moe_ctx *c) {
   uint8_t *b = c->scratch;
   c->status = (int *)(b + o_status);
   c->ticket = (unsigned int *)(b + o_ticket);
+  c->dec_bar = (unsigned long long *)(b + o_dbar);
+  c->dec_flags = c->dec_bar + 1;
+  c->dec_sync_bytes = sizeof(unsigned long long) * (1 + 2 * dec_warps);
+  c->dec_ws = (float *)(b + o_dws);
   c->n_jobs = (int *)(b + o_njobs);
   c->last = (int *)(b + o_last);
   c->stats = (unsigned long long *)(b + o_stats);
@@ -298,6 +311,47 @@ cudaError_t setup_finish() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
   return e;
+}
+
+cudaError_t setup_decode() {
+  cudaError_t e = cudaSuccess;
+  void (*ks[])(DecodeParams) = {decode_kernel<1, 1>, decode_kernel<1, 2>, decode_kernel<2, 1>,
+                                decode_kernel<2, 2>};
+  for (auto k : ks)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+  return e;
+}
+
+// Shared-memory carve of the decode kernel for a window of T tokens.
+DecSmem decode_layout(const moe_ctx *c, int T) {
+  const int ntm = T <= 8 ? 1 : 2;
+  int ring, warps;
+  if (c->fmt == MOE_Q4_SYM_G32_F16) {
+    ring = ntm == 1 ? GemvCfg<1, true, 1>::RING : GemvCfg<1, true, 2>::RING;
+    warps = ntm == 1 ? GemvCfg<1, true, 1>::WARPS : GemvCfg<1, true, 2>::WARPS;
+  } else {
+    ring = ntm == 1 ? GemvCfg<2, true, 1>::RING : GemvCfg<2, true, 2>::RING;
+    warps = ntm == 1 ? GemvCfg<2, true, 1>::WARPS : GemvCfg<2, true, 2>::WARPS;
+  }
+  return dec_layout(ring, warps, 8 * ntm, T, c->d, c->f, c->E, c->k, c->n_sm);
+}
+
+// Windows the single-launch decode kernel serves: token sets fit a 32-bit
+// mask, the pairs and the window fit its shared memory.
+bool use_decode_kernel(const moe_ctx *c, int T) {
+  if (T < 1 || T > kDecMaxT || T * c->k > kDecMaxPairs || c->E > kDecMaxE || c->k > kDecMaxK)
+    return false;
+  const DecSmem L = decode_layout(c, T);
+  return L.stage_bytes > 0 && (long long)T * L.rsh <= L.stage_bytes && L.rsa <= L.stage_bytes;
+}
+
+cudaError_t launch_decode(moe_ctx *c, cudaStream_t s, const DecodeParams &dp) {
+  const bool q4 = c->fmt == MOE_Q4_SYM_G32_F16, one = dp.T <= 8;
+  const int warps = one ? 16 : 8;
+  void (*k)(DecodeParams) = q4 ? (one ? decode_kernel<1, 1> : decode_kernel<1, 2>)
+                               : (one ? decode_kernel<2, 1> : decode_kernel<2, 2>);
+  return launch(k, dim3(c->n_sm), dim3(warps * 32), kDecSmem, s, dp);
 }
 
 cudaError_t launch_router(moe_ctx *c, cudaStream_t s, const RouterParams &rp) {
@@ -425,6 +479,51 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
 // gated expert GEMV, the down GEMV and the combine + residual.
 moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta, cudaStream_t s) {
   CUDA_TRY(c, prof_mark(c, 0, s));
+  if (use_decode_kernel(c, T)) {
+    DecodeParams dp{};
+    dp.x = x;
+    dp.delta = delta;
+    dp.gamma = c->has_gamma[layer] ? c->d_gamma + (size_t)layer * c->d : nullptr;
+    dp.eps = c->eps[layer];
+    dp.use_norm = c->has_norm[layer];
+    dp.W = c->d_router + (size_t)layer * c->E * c->d;
+    dp.bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr;
+    dp.T = T;
+    dp.d = c->d;
+    dp.f = c->f;
+    dp.E = c->E;
+    dp.k = c->k;
+    dp.layer = layer;
+    dp.chunk = T <= 8 ? 8 : 16;
+    dp.slot_of = c->d_slot_of;
+    dp.n_slots = c->n_slots;
+    dp.arena = c->arena;
+    dp.pool = c->pool;
+    dp.shared = c->n_shared ? c->shared + (size_t)layer * c->lay.expert_bytes : nullptr;
+    dp.expert_bytes = c->lay.expert_bytes;
+    dp.p1_bytes = c->lay.p1_bytes;
+    dp.logits = c->logits;
+    dp.abuf = c->abuf;
+    dp.ybuf = c->ybuf;
+    dp.ws = c->dec_ws;
+    dp.flags = c->dec_flags;
+    dp.bar = c->dec_bar;
+    dp.cnt_out = c->cnt_out;
+    dp.stats = c->stats;
+    dp.last = c->last;
+    dp.status = c->status;
+    dp.sm = decode_layout(c, T);
+    CUDA_TRY(c, launch_decode(c, s, dp));
+    // one kernel: the profile's route / experts / combine marks coincide
+    CUDA_TRY(c, prof_mark(c, 1, s));
+    CUDA_TRY(c, prof_mark(c, 2, s));
+    CUDA_TRY(c, prof_mark(c, 3, s));
+    if (c->profiling) {
+      c->prof_next = (c->prof_next + 1) % kProfSlots;
+      c->prof_pending = std::min(c->prof_pending + 1, kProfSlots);
+    }
+    return MOE_OK;
+  }
   FinishParams fp = finish_params(c, layer, T);
   fp.build_jobs = 1;
   const uint16_t *h = nullptr;
@@ -571,6 +670,7 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = setup_route_fused();
   if (e == cudaSuccess) e = setup_finish();
+  if (e == cudaSuccess) e = setup_decode();
   if (e == cudaSuccess) e = setup_gemv<1, true, 1>(c->n_sm, &c->gemv_blocks[0][1][0]);
   if (e == cudaSuccess) e = setup_gemv<1, false, 1>(c->n_sm, &c->gemv_blocks[0][0][0]);
   if (e == cudaSuccess) e = setup_gemv<2, true, 1>(c->n_sm, &c->gemv_blocks[1][1][0]);
@@ -844,6 +944,9 @@ moe_status moe_sync(moe_ctx *c, int timeout_ms) {
   int st = 0;
   CUDA_TRY(c, cudaMemcpyAsync(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost, c->io));
   CUDA_TRY(c, cudaMemsetAsync(c->status, 0, sizeof(int), c->io));
+  // a decode kernel that gave up a wait may have left its grid barrier
+  // counter mid-count: start it (and the hand-over flags) again from zero
+  if (st & kErrTimeout) CUDA_TRY(c, cudaMemsetAsync(c->dec_bar, 0, c->dec_sync_bytes, c->io));
   CUDA_TRY(c, cudaStreamSynchronize(c->io));
   if (st & kErrBadSlot) return fail(c, MOE_ERR_BAD_SLOT, "device status 0x%x: bad slot", st);
   if (st) return fail(c, MOE_ERR_DEVICE, "device status 0x%x", st);

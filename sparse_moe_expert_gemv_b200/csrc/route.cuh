@@ -115,6 +115,58 @@ MOE_DEV unsigned long long tournament_max(const unsigned long long (&v)[N]) {
   return m[0];
 }
 
+// Top-k + renormalised softmax of one token by one warp (Strata engine
+// analysis article "93 token/s on one 8 GB card", section "Architecture
+// overview": the router picks the top 10 of 512 experts per token).  A lane
+// holds logits lane + 32 i as 64-bit (order-preserving key << 32 | ~expert)
+// values, so the larger value is the larger logit and equal logits favour
+// the lower id.  Each selection round: a register tournament gives every
+// lane its best, one redux.max over the warp gives the winning key and a
+// second one the lowest id holding it; the winner's entry is cleared.  Lane
+// j < k returns the j-th selection (descending logit) and its weight
+// exp(l_j - l_0) / sum_j' exp(l_j' - l_0).  When near_ties is non-null, a
+// (k+1)-th logit within 1e-5 of the k-th counts one near tie.
+template <int NPL>
+MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int &sel_e,
+                       float &sel_w, unsigned long long *near_ties) {
+  unsigned long long pk[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    pk[i] = e < E ? ((unsigned long long)order_key(__ldcg(lr + e)) << 32) | (uint32_t)~e : 0ull;
+  }
+  if (trace && lane == 0 && pk[0] != 1ull) trace_point(kTrRouteLoaded);
+  uint32_t my_key = 0, k0 = 0, kk = 0;
+  int my_i = 0;
+  for (int j = 0; j <= k; ++j) {
+    if (j == k && k == E) break;
+    const unsigned long long best = tournament_max<NPL>(pk);
+    const uint32_t hi = (uint32_t)(best >> 32);
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, hi == wmax ? (uint32_t)best : 0u);
+    const int wi = (int)~wlo;
+    if (j == k) {  // the (k+1)-th logit: near-tie count only
+      if (near_ties && lane == 0 && key_to_float(kk) - key_to_float(wmax) < 1e-5f)
+        atomicAdd(near_ties, 1ULL);
+      break;
+    }
+    const bool mine = (wi & 31) == lane;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) pk[i] = (mine && (wi >> 5) == i) ? 0ull : pk[i];
+    if (lane == j) {
+      my_key = wmax;
+      my_i = wi;
+    }
+    if (j == 0) k0 = wmax;
+    kk = wmax;
+  }
+  if (trace && lane == 0) trace_point(kTrRouteSelected);
+  const float ex = lane < k ? expf(key_to_float(my_key) - key_to_float(k0)) : 0.f;
+  const float den = warp_sum(ex);
+  sel_e = my_i;
+  sel_w = ex / den;
+}
+
 // Shared-memory words the body needs (dynamic smem of the finish kernel;
 // the fused kernel reuses its staging area).
 MOE_HOST_DEV_INLINE int finish_smem_ints(int E, int P) {
@@ -122,13 +174,7 @@ MOE_HOST_DEV_INLINE int finish_smem_ints(int E, int P) {
 }
 
 // The routing body, run by one CTA after the logits exist.
-//  Phase A: one warp per token selects the k largest logits.  A lane holds
-//    its logits as 64-bit (order-preserving key, ~expert id) values, so the
-//    larger value is the larger logit and equal logits favour the lower id.
-//    Each selection round: a register tournament gives every lane its best,
-//    one redux.max over the warp gives the winning key and a second one the
-//    lowest id holding it; the winner's entry is cleared.  Then the softmax
-//    over the selected k.
+//  Phase A: one warp per token selects the k largest logits (warp_topk).
 //  Phase B: counting sort of the T*k pairs by expert (histogram, exclusive
 //    scan, stable scatter with ascending t).
 //  Phase C: the residency lookup (slot table -> slot pool or backing arena)
@@ -151,47 +197,13 @@ MOE_DEV void finish_body(const FinishParams &p, int *sm, const int (&slot_pref)[
   // ---------------- phase A: top-k + softmax
   if (p.logits) {
     for (int t = wid; t < T; t += nw) {
-      // lane holds logits lane + 32 i as (order key << 32 | ~expert): the
-      // larger packed value is the larger logit, equal logits -> lower id
-      unsigned long long pk[NPL];
-      const float *lr = p.logits + (long long)t * E;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        pk[i] = e < E ? ((unsigned long long)order_key(__ldcg(lr + e)) << 32) | (uint32_t)~e : 0ull;
-      }
-      if (t == 0 && lane == 0 && pk[0] != 1ull) trace_point(kTrRouteLoaded);
-      uint32_t my_key = 0, k0 = 0, kk = 0;
-      int my_i = 0;
-      for (int j = 0; j <= k; ++j) {
-        if (j == k && k == E) break;
-        unsigned long long best = tournament_max<NPL>(pk);
-        const uint32_t hi = (uint32_t)(best >> 32);
-        const uint32_t wmax = __reduce_max_sync(0xffffffffu, hi);
-        const uint32_t wlo = __reduce_max_sync(0xffffffffu, hi == wmax ? (uint32_t)best : 0u);
-        const int wi = (int)~wlo;
-        if (j == k) {  // the (k+1)-th logit: near-tie count only
-          if (lane == 0 && key_to_float(kk) - key_to_float(wmax) < 1e-5f)
-            atomicAdd(&p.stats[4], 1ULL);
-          break;
-        }
-        const bool mine = (wi & 31) == lane;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) pk[i] = (mine && (wi >> 5) == i) ? 0ull : pk[i];
-        if (lane == j) {
-          my_key = wmax;
-          my_i = wi;
-        }
-        if (j == 0) k0 = wmax;
-        kk = wmax;
-      }
-      if (t == 0 && lane == 0) trace_point(kTrRouteSelected);
-      const float ex = lane < k ? expf(key_to_float(my_key) - key_to_float(k0)) : 0.f;
-      const float den = warp_sum(ex);
+      int sel_e;
+      float sel_w;
+      warp_topk<NPL>(p.logits + (long long)t * E, E, k, lane, t == 0, sel_e, sel_w, &p.stats[4]);
       if (lane < k) {
-        p.idx[(long long)t * k + lane] = my_i;
-        p.w[(long long)t * k + lane] = ex / den;
-        if (smem_pairs) sidx[t * k + lane] = my_i;
+        p.idx[(long long)t * k + lane] = sel_e;
+        p.w[(long long)t * k + lane] = sel_w;
+        if (smem_pairs) sidx[t * k + lane] = sel_e;
       }
     }
   } else if (smem_pairs) {
