@@ -38,8 +38,9 @@ constexpr int kDecMaxT = 32;        // tokens per window (token sets are 32-bit 
 constexpr int kDecMaxPairs = 512;   // T * k
 constexpr int kDecMaxE = 1024;      // experts (top-k holds <= 32 logits per lane)
 constexpr int kDecMaxK = 32;        // lane j of the top-k warp returns selection j
-constexpr int kDecSmem = 224 * 1024;
+constexpr int kDecSmem = 226 * 1024;
 constexpr int kDecWv = 8;           // router-row float4s per lane held in registers
+constexpr int kHandFloats = 8;      // partial-sum floats per lane (2 matrices x 4)
 
 // ------------------------------------------------ memory-model helpers
 MOE_DEV unsigned long long ld_acquire_u64(const unsigned long long *p) {
@@ -99,6 +100,10 @@ struct DecSmem {
   int plist;         // int [T*k + T] pair ids in job order
   int jptr, jbeg, jn;  // job list: u64 expert address, first pair, tokens
   int part;          // float [rpc * qp * T] router partial dots
+  int hg, ngd;       // float [T][ngd]   group sums of the window rows (gate/up B)
+  int hd, ngf;       // float [rows][ngf] group sums of the staged a rows (down B)
+  int hd_rows;
+  int hand, hflag;   // partial sums handed to a warp of the same CTA: float [warps][32][8], u64 [warps]
   int stage;         // window rows (phase 1-3), then down-projection B rows
   int stage_bytes;
   int rsh, rsa;      // padded row strides (bytes) of staged h and a rows
@@ -112,7 +117,7 @@ MOE_HOST_DEV_INLINE int dec_align(int x, int a) { return (x + a - 1) / a * a; }
 // The carve for one launch shape; ring = bytes of the warps' rings.  The
 // caller checks T * rsh <= stage_bytes.
 inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, int E, int k,
-                          int grid) {
+                          int grid, int group) {
   DecSmem L{};
   int off = ring;
   auto carve = [&](int bytes, int align) {
@@ -138,6 +143,13 @@ inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, i
   L.qp = 1;
   while (L.rpc * L.qp * 2 <= warps && nch % (L.qp * 2) == 0) L.qp *= 2;
   L.part = carve(L.rpc * L.qp * T * 4, 16);
+  L.ngd = d / group;
+  L.ngf = f / group;
+  L.hg = carve(T * L.ngd * 4, 16);
+  L.hd_rows = kMaxStagedJobs * chunk;
+  L.hd = carve(L.hd_rows * L.ngf * 4, 16);
+  L.hand = carve(warps * 32 * kHandFloats * 4, 16);
+  L.hflag = carve(warps * 8, 8);
   L.stage = carve(0, 128);
   L.stage_bytes = kDecSmem - L.stage;
   L.rsh = 2 * d + 64;
@@ -171,6 +183,29 @@ struct DecodeParams {
   int *status;
   DecSmem sm;
 };
+
+// Group sums of staged bf16 rows: tab[r][q] = scale * sum of the G entries
+// of group q of row r (fp32, in order), for r < rows.  All threads.
+MOE_DEV void group_sums(const unsigned char *rows_g, int rs, int rows, int ng, int G, float scale,
+                        float *tab) {
+  for (int i = threadIdx.x; i < rows * ng; i += blockDim.x) {
+    const int r = i / ng, q = i - r * ng;
+    const uint4 *src = reinterpret_cast<const uint4 *>(rows_g + (size_t)r * rs + (size_t)q * G * 2);
+    float acc = 0.f;
+    for (int j = 0; j < G / 8; ++j) {
+      const uint4 v = src[j];
+      acc += __uint_as_float(v.x << 16);
+      acc += __uint_as_float(v.x & 0xFFFF0000u);
+      acc += __uint_as_float(v.y << 16);
+      acc += __uint_as_float(v.y & 0xFFFF0000u);
+      acc += __uint_as_float(v.z << 16);
+      acc += __uint_as_float(v.z & 0xFFFF0000u);
+      acc += __uint_as_float(v.w << 16);
+      acc += __uint_as_float(v.w & 0xFFFF0000u);
+    }
+    tab[i] = scale * acc;
+  }
+}
 
 // ------------------------------------------------ phase 2: routing
 // Top-k of every token, one warp per token; selections and weights into
@@ -276,31 +311,50 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
 // The phase's U weight units (job-major, then row block, then unit) are
 // split over the W warps of the grid: warp w owns [U w / W, U (w+1) / W).
 struct SKCtx {
-  long long U;
-  int W, gw;
+  int U, W, gw;
+  int q, rm;                  // U = q W + rm: start(w) = q w + (rm w) / W in 32 bits
   unsigned long long epoch;   // this phase's barrier number
-  float *ws;                  // [W][32 lanes][16] partial sums
-  unsigned long long *flags;  // [W] this phase's hand-over flags
+  float *ws;                  // [W][32 lanes][16] partial sums (hand-over between CTAs)
+  unsigned long long *flags;  // [W] this phase's hand-over flags (between CTAs)
+  float *s_hand;              // [warps][32][kHandFloats] same hand-over within the CTA
+  unsigned long long *s_flag; // [warps]
+  int warps;                  // warps per CTA
+  int cta_start;              // first unit of this CTA's range
 };
 
-MOE_DEV long long sk_start(const SKCtx &sk, int w) { return sk.U * w / sk.W; }
+MOE_DEV SKCtx sk_make(int U, int W, int gw, unsigned long long epoch, float *ws,
+                      unsigned long long *flags, float *s_hand, unsigned long long *s_flag,
+                      int warps) {
+  SKCtx sk{U, W, gw, U / W, U % W, epoch, ws, flags, s_hand, s_flag, warps, 0};
+  sk.cta_start = sk.q * (gw - gw % warps) + (sk.rm * (gw - gw % warps)) / W;
+  return sk;
+}
+
+// First unit of warp w's range (= floor(U w / W)).
+MOE_DEV int sk_start(const SKCtx &sk, int w) { return sk.q * w + (sk.rm * w) / sk.W; }
 
 // One item of the warp's range: units [ua, ub) of item `it`.
 //  ua > 0   the item began in an earlier warp's range: publish the partial
-//           sum (ws[gw], then flags[gw] = epoch) for that warp to add;
+//           sum for that warp to add -- in shared memory when it runs in
+//           this CTA, else in ws[gw] with flags[gw] = epoch;
 //  ub < UPI the item continues in later warps' ranges: add their partial
 //           sums in warp order, then store;
 //  else     the whole item is here: store.
-template <int FMT, bool GATED, int NTA>
-MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, long long it, int ua, int ub,
+template <int FMT, bool GATED, int NTA, bool HTAB>
+MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, int ubase, int ua, int ub,
                      int lane, int rb, const BRows &br, const int (&epair)[2][2], int R,
                      uint16_t *out_a, float *out_y) {
-  using Run = ItemRun<FMT, GATED, NTA>;
+  using Run = ItemRun<FMT, GATED, NTA, HTAB>;
   constexpr int NM = Run::C::NM;
   float acc[NM][NTA][4];
   if (!Run::run(r, ph, lane, ua, ub, br, acc)) return false;
+  static_assert(NM * NTA * 4 <= kHandFloats || NTA > 1, "hand-over slot too small");
+  const int cta_w0 = sk.gw - sk.gw % sk.warps;  // first warp of this CTA
   if (ua > 0) {
-    float4 *mine = reinterpret_cast<float4 *>(sk.ws + ((long long)sk.gw * 32 + lane) * 16);
+    // the item's first unit (ubase) lies in this CTA's range iff its owner runs here
+    const bool local = NM * NTA * 4 <= kHandFloats && ubase >= sk.cta_start;
+    float4 *mine = local ? reinterpret_cast<float4 *>(sk.s_hand + ((sk.gw - cta_w0) * 32 + lane) * kHandFloats)
+                         : reinterpret_cast<float4 *>(sk.ws + ((long long)sk.gw * 32 + lane) * 16);
 #pragma unroll
     for (int m = 0; m < NM; ++m)
 #pragma unroll
@@ -308,24 +362,47 @@ MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, long long it
         mine[m * NTA + nt] = make_float4(acc[m][nt][0], acc[m][nt][1], acc[m][nt][2], acc[m][nt][3]);
     __syncwarp();
     if (lane == 0) {
-      __threadfence();
-      st_release_u64(sk.flags + sk.gw, sk.epoch);
+      if (local) {
+        __threadfence_block();
+        *reinterpret_cast<volatile unsigned long long *>(sk.s_flag + (sk.gw - cta_w0)) = sk.epoch;
+      } else {
+        __threadfence();
+        st_release_u64(sk.flags + sk.gw, sk.epoch);
+      }
     }
     return true;
   }
   if (ub < ph.UPI) {
-    const long long iend = (it + 1) * ph.UPI;
+    const int iend = ubase + ph.UPI;
     for (int w2 = sk.gw + 1; w2 < sk.W; ++w2) {
-      const long long s2 = sk_start(sk, w2);
+      const int s2 = sk_start(sk, w2);
       if (s2 >= iend) break;
       if (sk_start(sk, w2 + 1) == s2) continue;  // empty range: nothing to add
-      if (__any_sync(0xffffffffu, !wait_flag(sk.flags + w2, sk.epoch))) return false;
-      const float *src = sk.ws + ((long long)w2 * 32 + lane) * 16;
+      const bool local = NM * NTA * 4 <= kHandFloats && w2 < cta_w0 + sk.warps;
+      const float *src;
+      if (local) {
+        bool ok = false;
+        for (uint32_t i = 0; !ok && i < (1u << 24); ++i)
+          ok = *reinterpret_cast<volatile unsigned long long *>(sk.s_flag + (w2 - cta_w0)) == sk.epoch;
+        if (__any_sync(0xffffffffu, !ok)) return false;
+        __threadfence_block();
+        src = sk.s_hand + ((w2 - cta_w0) * 32 + lane) * kHandFloats;
+      } else {
+        if (__any_sync(0xffffffffu, !wait_flag(sk.flags + w2, sk.epoch))) return false;
+        src = sk.ws + ((long long)w2 * 32 + lane) * 16;
+      }
 #pragma unroll
       for (int m = 0; m < NM; ++m)
 #pragma unroll
         for (int nt = 0; nt < NTA; ++nt) {
-          const float4 v = ldcg_f4(src + 4 * (m * NTA + nt));
+          float4 v;
+          if (local) {  // asm load: not moved above the fence
+            const uint4 q = ld_v4(src + 4 * (m * NTA + nt));
+            v = make_float4(__uint_as_float(q.x), __uint_as_float(q.y), __uint_as_float(q.z),
+                            __uint_as_float(q.w));
+          } else {
+            v = ldcg_f4(src + 4 * (m * NTA + nt));
+          }
           acc[m][nt][0] += v.x;
           acc[m][nt][1] += v.y;
           acc[m][nt][2] += v.z;
@@ -340,22 +417,23 @@ MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, long long it
 // Gate/up pass over this warp's units.  B rows are the window's token rows,
 // all staged in shared memory (row stride rsh) at stage_g.
 template <int FMT, int NTM>
-MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, long long u0, long long u1,
+MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, int u0, int u1,
                           const DecodeParams &p, const int *s_plist, const int *s_jbeg,
-                          const int *s_jn, const unsigned char *stage_g) {
+                          const int *s_jn, const unsigned char *stage_g, const float *s_hg) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
   const int P = p.T * p.k;
   if (u1 <= u0) return true;
-  for (long long it = u0 / ph.UPI; it * ph.UPI < u1; ++it) {
-    const int ua = (int)(max(u0, it * ph.UPI) - it * ph.UPI);
-    const int ub = (int)(min(u1, (it + 1) * ph.UPI) - it * ph.UPI);
-    const int job = (int)(it / ph.RB), rb = (int)(it - (long long)job * ph.RB);
+  const int it0 = u0 / ph.UPI;
+  int job = it0 / ph.RB, rb = it0 - job * ph.RB;
+  for (int ubase = it0 * ph.UPI; ubase < u1; ubase += ph.UPI) {
+    const int ua = max(u0, ubase) - ubase, ub = min(u1, ubase + ph.UPI) - ubase;
     const int n = s_jn[job], beg = s_jbeg[job];
     BRows br;
     int epair[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       br.row[nt] = nullptr;
+      br.hc[nt][0] = br.hc[nt][1] = nullptr;
       epair[nt][0] = epair[nt][1] = -1;
     }
 #pragma unroll
@@ -370,13 +448,21 @@ MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, long lo
       for (int c = 0; c < 2; ++c) {
         const int nc = nt * 8 + 2 * tig + c;
         epair[nt][c] = nc < n ? s_plist[beg + nc] : -1;
+        if (nc < n) {
+          const int pc = epair[nt][c];
+          br.hc[nt][c] = s_hg + (pc < P ? pc / p.k : pc - P) * p.sm.ngd;
+        }
       }
     }
     const bool ok =
         (NTM == 1 || n <= 8)
-            ? sk_item<FMT, true, 1>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr)
-            : sk_item<FMT, true, NTM>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr);
+            ? sk_item<FMT, true, 1, true>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr)
+            : sk_item<FMT, true, NTM, true>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.f, p.abuf, nullptr);
     if (!ok) return false;
+    if (++rb == ph.RB) {
+      rb = 0;
+      ++job;
+    }
   }
   return true;
 }
@@ -386,30 +472,26 @@ MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, long lo
 // starts at staged row row0 of lane i), later ones are read from global
 // memory.
 template <int FMT, int NTM>
-MOE_DEV bool decode_down(WarpRing &r, const Phase &ph, const SKCtx &sk, long long u0, long long u1,
+MOE_DEV bool decode_down(WarpRing &r, const Phase &ph, const SKCtx &sk, int u0, int u1,
                          const DecodeParams &p, const int *s_plist, const int *s_jbeg,
-                         const int *s_jn, const unsigned char *stage_g, uint32_t st_bar, int jfirst,
+                         const int *s_jn, const unsigned char *stage_g, const float *s_hd, int jfirst,
                          int nst, int row0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
-  bool staged_ready = false;
   if (u1 <= u0) return true;
-  for (long long it = u0 / ph.UPI; it * ph.UPI < u1; ++it) {
-    const int ua = (int)(max(u0, it * ph.UPI) - it * ph.UPI);
-    const int ub = (int)(min(u1, (it + 1) * ph.UPI) - it * ph.UPI);
-    const int job = (int)(it / ph.RB), rb = (int)(it - (long long)job * ph.RB);
+  const int it0 = u0 / ph.UPI;
+  int job = it0 / ph.RB, rb = it0 - job * ph.RB;
+  for (int ubase = it0 * ph.UPI; ubase < u1; ubase += ph.UPI) {
+    const int ua = max(u0, ubase) - ubase, ub = min(u1, ubase + ph.UPI) - ubase;
     const int n = s_jn[job], beg = s_jbeg[job];
     const int sj = job - jfirst;
     const bool staged = sj >= 0 && sj < nst;
     const int jrow0 = __shfl_sync(0xffffffffu, row0, staged ? sj : 0);
-    if (staged && !staged_ready) {
-      if (__any_sync(0xffffffffu, !mbar_wait_bounded(st_bar, 0))) return false;
-      staged_ready = true;
-    }
     BRows br;
     int epair[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       br.row[nt] = nullptr;
+      br.hc[nt][0] = br.hc[nt][1] = nullptr;
       epair[nt][0] = epair[nt][1] = -1;
     }
 #pragma unroll
@@ -422,13 +504,23 @@ MOE_DEV bool decode_down(WarpRing &r, const Phase &ph, const SKCtx &sk, long lon
       for (int c = 0; c < 2; ++c) {
         const int nc = nt * 8 + 2 * tig + c;
         epair[nt][c] = nc < n ? s_plist[beg + nc] : -1;
+        if (staged && nc < n) br.hc[nt][c] = s_hd + (jrow0 + nc) * p.sm.ngf;
       }
     }
-    const bool ok =
-        (NTM == 1 || n <= 8)
-            ? sk_item<FMT, false, 1>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf)
-            : sk_item<FMT, false, NTM>(r, ph, sk, it, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf);
+    bool ok;
+    if (staged)
+      ok = (NTM == 1 || n <= 8)
+               ? sk_item<FMT, false, 1, true>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf)
+               : sk_item<FMT, false, NTM, true>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf);
+    else  // rows read from global memory: group sums from the tensor core
+      ok = (NTM == 1 || n <= 8)
+               ? sk_item<FMT, false, 1, false>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf)
+               : sk_item<FMT, false, NTM, false>(r, ph, sk, ubase, ua, ub, lane, rb, br, epair, p.d, nullptr, p.ybuf);
     if (!ok) return false;
+    if (++rb == ph.RB) {
+      rb = 0;
+      ++job;
+    }
   }
   return true;
 }
@@ -472,6 +564,12 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   int *s_jbeg = reinterpret_cast<int *>(smem + L.jbeg);
   int *s_jn = reinterpret_cast<int *>(smem + L.jn);
   float *s_part = reinterpret_cast<float *>(smem + L.part);
+  float *s_hg = reinterpret_cast<float *>(smem + L.hg);
+  float *s_hd = reinterpret_cast<float *>(smem + L.hd);
+  float *s_hand = reinterpret_cast<float *>(smem + L.hand);
+  unsigned long long *s_hflag = reinterpret_cast<unsigned long long *>(smem + L.hflag);
+  constexpr int GQ = FMT == 1 ? 32 : 64;            // quantisation group
+  constexpr float kSumScale = FMT == 1 ? -136.f : 1.f;  // see ItemRun::tile
   const uint32_t stage_s = smem_addr(smem + L.stage);
   const unsigned char *stage_g = smem + L.stage;
   const uint32_t bars = smem_addr(smem + L.bars);
@@ -507,6 +605,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     s_slot[e] = p.slot_of ? p.slot_of[(long long)p.layer * E + e] : -1;
     s_mask[e] = 0u;
   }
+  if (tid < WARPS) s_hflag[tid] = 0ull;  // epochs start at 1
   __syncthreads();
   pdl_wait();
   MOE_TRACE(kTrRouteWaited);
@@ -552,6 +651,9 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     }
     __syncthreads();
   }
+  // group sums of the window rows for the gate/up pass (read after the
+  // barriers below)
+  group_sums(stage_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
   for (int task = wid, it = 0; task < ntask; task += WARPS, ++it) {
     const int rr = task / QP, q = task - rr * QP, e = blockIdx.x * RPC + rr;
     if (e >= E) continue;
@@ -608,12 +710,12 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
 
   // ---------------- phase 3: gate/up
   const Phase ph1 = make_phase(s_jptr, f, d, CG::TK, CG::STRIDE, 0);
-  SKCtx sk1{(long long)n_jobs * ph1.RB * ph1.UPI, W, gw, ep1, p.ws, p.flags};
+  const SKCtx sk1 = sk_make(n_jobs * ph1.RB * ph1.UPI, W, gw, ep1, p.ws, p.flags, s_hand, s_hflag, WARPS);
   {
-    const long long u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1);
-    ring_start(r, ph1, u0 / ph1.UPI, (int)(u0 % ph1.UPI), u1 - u0, 1);
+    const int u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1), i0 = u0 / ph1.UPI;
+    ring_start(r, ph1, i0 / ph1.RB, i0 % ph1.RB, u0 - i0 * ph1.UPI, u1 - u0, 1);
     if (lane == 0) ring_prologue(r, ph1);
-    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g)) {
+    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg)) {
       if (lane == 0) atomicOr(p.status, kErrTimeout);
       ring_drain(r);
     }
@@ -622,11 +724,15 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
 
   // ---------------- phase 4: down projection
   const Phase ph2 = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes);
-  SKCtx sk2{(long long)n_jobs * ph2.RB * ph2.UPI, W, gw, ep0 + 2, p.ws, p.flags + W};
-  const long long v0 = sk_start(sk2, gw), v1 = sk_start(sk2, gw + 1);
-  ring_start(r, ph2, v0 / ph2.UPI, (int)(v0 % ph2.UPI), v1 - v0, 1);
+  const SKCtx sk2 = sk_make(n_jobs * ph2.RB * ph2.UPI, W, gw, ep0 + 2, p.ws, p.flags + W, s_hand,
+                            s_hflag, WARPS);
+  const int v0 = sk_start(sk2, gw), v1 = sk_start(sk2, gw + 1);
+  {
+    const int i0 = v0 / ph2.UPI;
+    ring_start(r, ph2, i0 / ph2.RB, i0 % ph2.RB, v0 - i0 * ph2.UPI, v1 - v0, 1);
+  }
   if (lane == 0) ring_prologue(r, ph2);  // weights stream in while the grid syncs
-  if (!grid_sync(p.bar, sk2.epoch * G)) {
+  if (!grid_sync(p.bar, (ep0 + 2) * G)) {
     ring_drain(r);
     if (tid == 0) atomicOr(p.status, kErrTimeout);
     return;
@@ -637,10 +743,10 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   // i describes job jfirst + i.
   int jfirst = 0, njobs_cta = 0;
   {
-    const long long c0 = sk_start(sk2, blockIdx.x * WARPS), c1 = sk_start(sk2, (blockIdx.x + 1) * WARPS);
+    const int c0 = sk_start(sk2, blockIdx.x * WARPS), c1 = sk_start(sk2, (blockIdx.x + 1) * WARPS);
     if (c1 > c0) {
-      jfirst = (int)(c0 / ph2.UPI / ph2.RB);
-      njobs_cta = (int)((c1 - 1) / ph2.UPI / ph2.RB) - jfirst + 1;
+      jfirst = c0 / ph2.UPI / ph2.RB;
+      njobs_cta = (c1 - 1) / ph2.UPI / ph2.RB - jfirst + 1;
     }
   }
   int pn = 0, pbeg = 0;
@@ -656,7 +762,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   }
   const int row0 = incl - pn;
   const int cap = L.stage_bytes / L.rsa;
-  const int nst = __popc(__ballot_sync(0xffffffffu, pn > 0 && incl <= cap));
+  const int nst = __popc(__ballot_sync(0xffffffffu, pn > 0 && incl <= cap && incl <= L.hd_rows));
   const int used = nst ? __shfl_sync(0xffffffffu, incl, nst - 1) : 0;
   if (wid == 0) {
     // a was written by other CTAs' generic stores before the barrier; the
@@ -676,14 +782,20 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
                  (uint32_t)f * 2, st_bar);
     }
   }
-  if (!decode_down<FMT, NTM>(r, ph2, sk2, v0, v1, p, s_plist, s_jbeg, s_jn, stage_g, st_bar, jfirst,
+  // every thread: the staged rows, then their group sums
+  if (__syncthreads_or(!mbar_wait_bounded(st_bar, 0))) {
+    ring_drain(r);
+    if (tid == 0) atomicOr(p.status, kErrTimeout);
+    return;
+  }
+  group_sums(stage_g, L.rsa, used, L.ngf, GQ, kSumScale, s_hd);
+  __syncthreads();
+  if (!decode_down<FMT, NTM>(r, ph2, sk2, v0, v1, p, s_plist, s_jbeg, s_jn, stage_g, s_hd, jfirst,
                              nst, row0)) {
     if (lane == 0) atomicOr(p.status, kErrTimeout);
     ring_drain(r);
   }
   if (lane == 0) trace_point(kTrDownEnd);
-  // the staged rows must have landed before the CTA exits
-  if (wid == 0 && used > 0 && nst > 0) (void)mbar_wait_bounded(st_bar, 0);
   if (!grid_sync(p.bar, (ep0 + 3) * G)) {
     if (tid == 0) atomicOr(p.status, kErrTimeout);
     return;

@@ -95,26 +95,26 @@ MOE_DEV Phase make_phase(const unsigned long long *job_ptr, int R, int K, int TK
   return ph;
 }
 
-MOE_DEV const unsigned char *unit_addr(const Phase &ph, long long item, int unit) {
-  const long long job = item / ph.RB;
-  const int rb = (int)(item - job * ph.RB);
+// First byte of item (job, rb) of the pass.
+MOE_DEV const unsigned char *item_base(const Phase &ph, int job, int rb) {
   return reinterpret_cast<const unsigned char *>(ph.job_ptr[job]) + ph.region_off +
-         ((long long)rb * ph.NTILE + (long long)unit * ph.tps) * ph.stride;
+         (long long)rb * ph.NTILE * ph.stride;
 }
 
-// A walk over consecutive weight units: n units from (item, unit), items
-// istep apart.
+// A walk over consecutive weight units: n units from unit `unit` of item
+// (job, rb); the next item is istep row blocks further.  Only increments and
+// compares: no division per unit or item.
 struct UnitCursor {
-  long long rem, item;
-  int unit;
+  int rem, job, rb, unit;
   const unsigned char *addr;
 };
 
-MOE_DEV void cursor_start(UnitCursor &c, const Phase &ph, long long item, int unit, long long n) {
+MOE_DEV void cursor_start(UnitCursor &c, const Phase &ph, int job, int rb, int unit, int n) {
   c.rem = n;
-  c.item = item;
+  c.job = job;
+  c.rb = rb;
   c.unit = unit;
-  c.addr = n > 0 ? unit_addr(ph, item, unit) : nullptr;
+  c.addr = n > 0 ? item_base(ph, job, rb) + (long long)unit * ph.tps * ph.stride : nullptr;
 }
 
 MOE_DEV void cursor_advance(UnitCursor &c, const Phase &ph, int istep) {
@@ -122,8 +122,12 @@ MOE_DEV void cursor_advance(UnitCursor &c, const Phase &ph, int istep) {
   c.addr += ph.tps * ph.stride;
   if (++c.unit == ph.UPI) {
     c.unit = 0;
-    c.item += istep;
-    if (c.rem > 0) c.addr = unit_addr(ph, c.item, 0);
+    c.rb += istep;
+    while (c.rb >= ph.RB) {
+      c.rb -= ph.RB;
+      ++c.job;
+    }
+    if (c.rem > 0) c.addr = item_base(ph, c.job, c.rb);
   }
 }
 
@@ -153,20 +157,21 @@ MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t sl
   r.policy = l2_evict_first();
 }
 
-// Point the producer at n units starting at (item, unit); consecutive items
-// are istep apart.
-MOE_DEV void ring_start(WarpRing &r, const Phase &ph, long long item, int unit, long long n,
-                        int istep) {
+// Point the producer at n units starting at unit `unit` of item (job, rb);
+// consecutive items are istep row blocks apart.
+MOE_DEV void ring_start(WarpRing &r, const Phase &ph, int job, int rb, int unit, int n, int istep) {
   r.istep = istep;
-  cursor_start(r.ld, ph, item, unit, n);
+  cursor_start(r.ld, ph, job, rb, unit, n);
 }
 
-// lane 0: issue the producer's next unit into slot `slot`
+// lane 0: issue the producer's next unit into slot `slot`.  The slot's
+// previous unit was read with ld.shared by every lane, and those reads are
+// ordered before this copy by the __syncwarp that precedes the call (the
+// values were consumed by then), as in a TMA pipeline's consumer release.
 MOE_DEV void ring_issue(WarpRing &r, const Phase &ph, int slot) {
   if (r.ld.rem <= 0) return;
   const uint32_t bytes = (uint32_t)(ph.tps * ph.stride);
   const uint32_t bar = r.bar_s + 8 * slot;
-  fence_proxy_async_smem();
   mbar_expect_tx(bar, bytes);
   bulk_g2s_hint(r.data_s + slot * r.slot_stride, r.ld.addr, bytes, bar, r.policy);
   ++r.inflight;
@@ -196,10 +201,19 @@ MOE_DEV void ring_drain(WarpRing &r) {
 
 // The lane's B rows for the current item (its token column g of each 8-token
 // column tile): generic addresses of rows staged in shared memory or of rows
-// in global memory; null = no token.
+// in global memory; null = no token.  With a sum table (HTAB), hc[nt][c] is
+// the table row of the token in accumulator column 2 tig + c: one float per
+// quantisation group of the reduction (see ItemRun::tile); null = no token.
 struct BRows {
   const uint16_t *row[2];
+  const float *hc[2][2];
 };
+
+MOE_DEV float2 ld_f2(const float *p) {
+  float2 r;
+  asm volatile("ld.v2.f32 {%0,%1}, [%2];" : "=f"(r.x), "=f"(r.y) : "l"(p));
+  return r;
+}
 
 MOE_DEV uint4 ld_v4(const void *p) {
   uint4 r;
@@ -208,27 +222,39 @@ MOE_DEV uint4 ld_v4(const void *p) {
 }
 
 // One item (16 output rows of one job) of the streaming GEMV; NTA = 8-token
-// column tiles of the job (1 or 2).
-template <int FMT, bool GATED, int NTA>
+// column tiles of the job (1 or 2).  The per-group sums of the B rows that
+// the tile math needs come either from a table (HTAB: -136 sum(h) for Q4,
+// sum(h) for Q2, per row and group, computed once per call) or from an mma
+// of the B fragments against ones.
+template <int FMT, bool GATED, int NTA, bool HTAB = false>
 struct ItemRun {
   using C = GemvCfg<FMT, GATED>;  // tile geometry does not depend on NTM or WARPS
   static constexpr int NB = C::STEPS / 2;  // 16-byte B loads per tile and column tile
 
-  // B fragments of tile t: b[nt][q] holds k-steps 2q (x, y) and 2q+1 (z, w)
-  static MOE_DEV void load_b(uint4 (&b)[NTA][NB], const BRows &br, int t, int tig) {
+  // B fragments of tile t: b[nt][q] holds k-steps 2q (x, y) and 2q+1 (z, w);
+  // with HTAB, hv[nt][c] = the table entries of the tile's groups 2t, 2t+1
+  // for accumulator column 2 tig + c
+  static MOE_DEV void load_b(uint4 (&b)[NTA][NB], float2 (&hv)[NTA][2], const BRows &br, int t,
+                             int tig) {
 #pragma unroll
-    for (int nt = 0; nt < NTA; ++nt)
+    for (int nt = 0; nt < NTA; ++nt) {
 #pragma unroll
       for (int q = 0; q < NB; ++q) {
         const int col = t * C::TK + 32 * q + 8 * tig;
         b[nt][q] = br.row[nt] ? ld_v4(br.row[nt] + col) : make_uint4(0u, 0u, 0u, 0u);
       }
+      if constexpr (HTAB) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          hv[nt][c] = br.hc[nt][c] ? ld_f2(br.hc[nt][c] + 2 * t) : make_float2(0.f, 0.f);
+      }
+    }
   }
 
   // acc += this tile's contribution.  c runs over the accumulator entries:
   // (row g, col 2tig), (row g, col 2tig+1), (row g+8, col 2tig), (row g+8, col 2tig+1).
   static MOE_DEV void tile(uint32_t tile_s, int lane, const uint4 (&b)[NTA][NB],
-                           float (&acc)[C::NM][NTA][4]) {
+                           const float2 (&hv)[NTA][2], float (&acc)[C::NM][NTA][4]) {
     const int g = lane >> 2;
     const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
     uint4 cw[C::NM];
@@ -253,10 +279,20 @@ struct ItemRun {
 #pragma unroll
         for (int nt = 0; nt < NTA; ++nt) {
           const uint4 bb = b[nt][grp];
-          float hs[4];
-          mma_bf16_acc(hs, ones, bb.x, bb.y, true);
-          mma_bf16_16816(hs, ones, bb.z, bb.w, hs);
-          const float ci[4] = {-136.f * hs[0], -136.f * hs[1], -136.f * hs[2], -136.f * hs[3]};
+          float ci[4];
+          if constexpr (HTAB) {
+            const float h0 = grp ? hv[nt][0].y : hv[nt][0].x, h1 = grp ? hv[nt][1].y : hv[nt][1].x;
+            ci[0] = h0;
+            ci[1] = h1;
+            ci[2] = h0;
+            ci[3] = h1;
+          } else {
+            float hs[4];
+            mma_bf16_acc(hs, ones, bb.x, bb.y, true);
+            mma_bf16_16816(hs, ones, bb.z, bb.w, hs);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ci[c] = -136.f * hs[c];
+          }
 #pragma unroll
           for (int m = 0; m < C::NM; ++m) {
             float tmp[4];
@@ -296,7 +332,7 @@ struct ItemRun {
             for (int hs2 = 0; hs2 < 2; ++hs2) {
               const bool first = wv == 0 && hs2 == 0;
               const uint32_t b0 = hs2 ? bb.z : bb.x, b1 = hs2 ? bb.w : bb.y;
-              mma_bf16_acc(hs[nt], ones, b0, b1, first);
+              if constexpr (!HTAB) mma_bf16_acc(hs[nt], ones, b0, b1, first);
 #pragma unroll
               for (int m = 0; m < C::NM; ++m) {
                 const uint32_t af[4] = {a8[m][4 * hs2], a8[m][4 * hs2 + 1], a8[m][4 * hs2 + 2],
@@ -304,6 +340,16 @@ struct ItemRun {
                 mma_bf16_acc(tmp[m][nt], af, b0, b1, first);
               }
             }
+          }
+        }
+        if constexpr (HTAB) {
+#pragma unroll
+          for (int nt = 0; nt < NTA; ++nt) {
+            const float h0 = grp ? hv[nt][0].y : hv[nt][0].x, h1 = grp ? hv[nt][1].y : hv[nt][1].x;
+            hs[nt][0] = h0;
+            hs[nt][1] = h1;
+            hs[nt][2] = h0;
+            hs[nt][3] = h1;
           }
         }
 #pragma unroll
@@ -339,8 +385,9 @@ struct ItemRun {
       const uint32_t slot_s = r.data_s + r.u * r.slot_stride;
       for (int tt = 0; tt < ph.tps; ++tt) {
         uint4 b[NTA][NB];
-        load_b(b, br, u * ph.tps + tt, tig);
-        tile(slot_s + tt * C::STRIDE, lane, b, acc);
+        float2 hv[NTA][2];
+        load_b(b, hv, br, u * ph.tps + tt, tig);
+        tile(slot_s + tt * C::STRIDE, lane, b, hv, acc);
       }
       __syncwarp();
       if (lane == 0) {
@@ -432,7 +479,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, GATED, NTM>::WARPS * 32, 1)
   // weight stream: kRingD units in flight per warp (weights do not depend on
   // the previous kernel, so the down projection starts streaming before its
   // wait)
-  ring_start(r, ph, first, 0, (long long)my_items * ph.UPI, C::WARPS);
+  ring_start(r, ph, first / RB, first % RB, 0, my_items * ph.UPI, C::WARPS);
   if (lane == 0) ring_prologue(r, ph);
   if (!GATED) {
     pdl_wait();
@@ -499,6 +546,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, GATED, NTM>::WARPS * 32, 1)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       br.row[nt] = nullptr;
+      br.hc[nt][0] = br.hc[nt][1] = nullptr;
       epair[nt][0] = epair[nt][1] = -1;
     }
 #pragma unroll

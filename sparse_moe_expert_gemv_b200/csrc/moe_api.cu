@@ -315,26 +315,22 @@ cudaError_t setup_finish() {
 
 cudaError_t setup_decode() {
   cudaError_t e = cudaSuccess;
-  void (*ks[])(DecodeParams) = {decode_kernel<1, 1>, decode_kernel<1, 2>, decode_kernel<2, 1>,
-                                decode_kernel<2, 2>};
+  void (*ks[])(DecodeParams) = {decode_kernel<1, 1>, decode_kernel<2, 1>};
   for (auto k : ks)
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   return e;
 }
 
-// Shared-memory carve of the decode kernel for a window of T tokens.
+// Shared-memory carve of the decode kernel for a window of T tokens.  The
+// decode kernel always runs 16 warps with jobs of <= 8 tokens: a window of
+// up to 32 tokens rarely puts more than 8 on one expert, and 16 warps hide
+// the GEMV's latency better than 8 warps with two column tiles.
 DecSmem decode_layout(const moe_ctx *c, int T) {
-  const int ntm = T <= 8 ? 1 : 2;
-  int ring, warps;
-  if (c->fmt == MOE_Q4_SYM_G32_F16) {
-    ring = ntm == 1 ? GemvCfg<1, true, 1>::RING : GemvCfg<1, true, 2>::RING;
-    warps = ntm == 1 ? GemvCfg<1, true, 1>::WARPS : GemvCfg<1, true, 2>::WARPS;
-  } else {
-    ring = ntm == 1 ? GemvCfg<2, true, 1>::RING : GemvCfg<2, true, 2>::RING;
-    warps = ntm == 1 ? GemvCfg<2, true, 1>::WARPS : GemvCfg<2, true, 2>::WARPS;
-  }
-  return dec_layout(ring, warps, 8 * ntm, T, c->d, c->f, c->E, c->k, c->n_sm);
+  const bool q4 = c->fmt == MOE_Q4_SYM_G32_F16;
+  const int ring = q4 ? GemvCfg<1, true, 1>::RING : GemvCfg<2, true, 1>::RING;
+  return dec_layout(ring, GemvCfg<1, true, 1>::WARPS, 8, T, c->d, c->f, c->E, c->k, c->n_sm,
+                    c->lay.G);
 }
 
 // Windows the single-launch decode kernel serves: token sets fit a 32-bit
@@ -347,11 +343,8 @@ bool use_decode_kernel(const moe_ctx *c, int T) {
 }
 
 cudaError_t launch_decode(moe_ctx *c, cudaStream_t s, const DecodeParams &dp) {
-  const bool q4 = c->fmt == MOE_Q4_SYM_G32_F16, one = dp.T <= 8;
-  const int warps = one ? 16 : 8;
-  void (*k)(DecodeParams) = q4 ? (one ? decode_kernel<1, 1> : decode_kernel<1, 2>)
-                               : (one ? decode_kernel<2, 1> : decode_kernel<2, 2>);
-  return launch(k, dim3(c->n_sm), dim3(warps * 32), kDecSmem, s, dp);
+  void (*k)(DecodeParams) = c->fmt == MOE_Q4_SYM_G32_F16 ? decode_kernel<1, 1> : decode_kernel<2, 1>;
+  return launch(k, dim3(c->n_sm), dim3(GemvCfg<1, true, 1>::WARPS * 32), kDecSmem, s, dp);
 }
 
 cudaError_t launch_router(moe_ctx *c, cudaStream_t s, const RouterParams &rp) {
@@ -494,7 +487,7 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.E = c->E;
     dp.k = c->k;
     dp.layer = layer;
-    dp.chunk = T <= 8 ? 8 : 16;
+    dp.chunk = 8;
     dp.slot_of = c->d_slot_of;
     dp.n_slots = c->n_slots;
     dp.arena = c->arena;
