@@ -53,6 +53,26 @@ def parse():
 
 
 # ----------------------------------------------------------------- helpers
+def kernel_traffic(kernel_bytes_per_launch):
+    """Per-launch DRAM traffic of decode_kernel from the committed ncu record,
+    scaled to this run's algorithmic bytes per launch (the record's launch
+    routed a different window).  None when the kernel sources changed since
+    the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        rec = json.load(fh)
+    h = hashlib.sha256()
+    for s in rec["sources"]:
+        with open(os.path.join(ROOT, s), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["traffic_over_algorithmic"] * kernel_bytes_per_launch
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -331,7 +351,7 @@ def run_native(args, world, rank, local):
             "unit": "GB/s",
             "frac": (kern_gbs / hbm) if kern_gbs else None,
             "launch_us": kern_ms / max(ncalls, 1) * 1e3,
-            "traffic": None,
+            "traffic": kernel_traffic(kern_bytes / K) if single else None,
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                            else "fallback 6650 GB/s",
             "per_unit": per_unit,
