@@ -189,10 +189,23 @@ MOE_API moe_status moe_forward_delta(moe_ctx *ctx, int layer, const void *x_dev,
 MOE_API moe_status moe_forward_stack(moe_ctx *ctx, void *x_dev, int T, void *stream);
 
 /* moe_prefill: a prefill chunk of N tokens (N <= max_tokens) through
- * `layer`, in place (x <- x + MoE(norm(x))), using the tensor-core grouped
- * GEMM path for experts that receive many tokens. */
+ * `layer`, in place (x <- x + MoE(norm(x))).  The engine article "93 token/s
+ * on one 8 GB card", section "Architecture overview", runs prefill in chunks
+ * of up to 8192 tokens; per expert such a chunk is a dense contraction.  For
+ * Q4 experts and N > 32 the experts run as a grouped GEMM on the tensor
+ * cores (tcgen05): tokens sorted by expert, 128-token tiles, weights
+ * dequantised to fp16 tile by tile in shared memory, fp32 accumulation in
+ * tensor memory.  Activations enter as fp16 (exact for |h| < 65504; larger
+ * values saturate).  Q2 experts and N <= 32 take the moe_forward path.
+ * Requires a context configured with max_tokens >= N.  Errors: INVALID_ARG,
+ * STATE; device faults through moe_sync. */
 MOE_API moe_status moe_prefill(moe_ctx *ctx, int layer, void *x_dev, int N,
                        void *stream);
+
+/* moe_prefill_delta: as moe_prefill but leaves x unchanged and writes the
+ * fp32 MoE output delta_dev [N, d]. */
+MOE_API moe_status moe_prefill_delta(moe_ctx *ctx, int layer, const void *x_dev, int N,
+                                     float *delta_dev, void *stream);
 
 /* moe_sync: wait (polling cudaEventQuery, at most timeout_ms; < 0 = no
  * limit) until the work queued by this context has finished, then read and

@@ -30,7 +30,7 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_forward_stack", "moe_prefill", "moe_sync", "moe_get_stats",
            "moe_last_error", "moe_status_string", "moe_expert_bytes",
            "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
-           "moe_set_trace", "moe_read_trace", "moe_route_static")
+           "moe_set_trace", "moe_read_trace", "moe_route_static", "moe_prefill_delta")
 
 
 class MoeError(RuntimeError):
@@ -68,6 +68,7 @@ def _load():
         "moe_forward_delta": [P, I, P, I, P, P],
         "moe_forward_stack": [P, P, I, P],
         "moe_prefill": [P, I, P, I, P],
+        "moe_prefill_delta": [P, I, P, I, P, P],
         "moe_sync": [P, I],
         "moe_get_stats": [P, ctypes.POINTER(MoeStats)],
         "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
@@ -198,6 +199,10 @@ def moe_forward_stack(ctx, x, T, stream=None):
 
 def moe_prefill(ctx, layer, x, N, stream=None):
     _check(ctx, _lib.moe_prefill(ctx, layer, _ptr(x), N, _stream(stream)))
+
+
+def moe_prefill_delta(ctx, layer, x, N, delta, stream=None):
+    _check(ctx, _lib.moe_prefill_delta(ctx, layer, _ptr(x), N, _ptr(delta), _stream(stream)))
 
 
 def moe_sync(ctx, timeout_ms=-1):

@@ -26,6 +26,7 @@
 #include "../../include/moe.h"
 #include "decode.cuh"
 #include "kernels.cuh"
+#include "prefill.cuh"
 
 using namespace moe;
 
@@ -64,6 +65,15 @@ struct moe_ctx {
   unsigned long long *dec_bar = nullptr, *dec_flags = nullptr;
   float *dec_ws = nullptr;
   size_t dec_sync_bytes = 0;  // bytes of the counter + flags block (cleared after a timeout)
+  // prefill (grouped GEMM) buffers, present when max_tokens > kDecMaxT
+  uint8_t *pf = nullptr;
+  __half *pf_hg = nullptr;              // grouped A rows, fp16 [rows][d]
+  int *pf_row_of = nullptr, *pf_boff = nullptr, *pf_eoff = nullptr, *pf_ntiles = nullptr;
+  unsigned short *pf_bmask = nullptr;
+  PfTile *pf_tiles = nullptr;
+  int pf_max_tiles = 0, pf_rows = 0;
+  CUtensorMap pf_map_h{}, pf_map_a{};   // TMA maps of the grouped A matrices
+  bool pf_maps = false;
   unsigned long long *trace = nullptr;  // moe_set_trace buffer
   unsigned long long *stats = nullptr;
   std::vector<int32_t> host_counts;
@@ -231,6 +241,31 @@ moe_status do_configure(moe_ctx *c) {
   c->hbuf = (uint16_t *)(b + o_h);
   c->abuf = (uint16_t *)(b + o_a);
   c->ybuf = (float *)(b + o_y);
+  if (T > kDecMaxT) {  // prefill-capable: grouped-GEMM buffers
+    const long long rows = Ptot;
+    const int blocks = (T + kPfTok - 1) / kPfTok;
+    c->pf_rows = (int)rows;
+    c->pf_max_tiles = (int)((P + kPfBM - 1) / kPfBM + E + (T + kPfBM - 1) / kPfBM + 4);
+    size_t po = 0;
+    auto pcarve = [&](size_t bytes) {
+      const size_t at = po;
+      po += (bytes + 1023) / 1024 * 1024;
+      return at;
+    };
+    const size_t o_hg = pcarve((size_t)rows * d * 2), o_row = pcarve((size_t)rows * 4);
+    const size_t o_bm = pcarve((size_t)blocks * E * 2), o_bo = pcarve((size_t)blocks * E * 4);
+    const size_t o_eo = pcarve((size_t)(E + 1) * 4), o_nt = pcarve(4);
+    const size_t o_tl = pcarve((size_t)c->pf_max_tiles * sizeof(PfTile));
+    CUDA_TRY(c, cudaMalloc(&c->pf, po));
+    CUDA_TRY(c, cudaMemset(c->pf, 0, po));
+    c->pf_hg = (__half *)(c->pf + o_hg);
+    c->pf_row_of = (int *)(c->pf + o_row);
+    c->pf_bmask = (unsigned short *)(c->pf + o_bm);
+    c->pf_boff = (int *)(c->pf + o_bo);
+    c->pf_eoff = (int *)(c->pf + o_eo);
+    c->pf_ntiles = (int *)(c->pf + o_nt);
+    c->pf_tiles = (PfTile *)(c->pf + o_tl);
+  }
   c->has_router.assign(c->L, 0);
   c->has_bias.assign(c->L, 0);
   c->has_norm.assign(c->L, 0);
@@ -467,6 +502,141 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
   return MOE_OK;
 }
 
+// 2-D TMA map of a row-major fp16 matrix [rows][cols]: boxes of 64 columns x
+// 128 rows, 128-byte swizzle (the layout the tcgen05 descriptors expect).
+// The driver's tensor-map encoder, looked up through the runtime so the
+// library has no link-time dependency on the driver library.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kPfBK, (cuuint32_t)kPfBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t setup_prefill() {
+  cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kPfStagesG * (kPfBM * kPfBK * 2 + 2 * kPfBN * kPfBK * 2) + 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPfStagesD * (kPfBM * kPfBK * 2 + kPfBN * kPfBK * 2) + 1024);
+  return e;
+}
+
+// Prefill through the grouped tcgen05 GEMM: Q4 experts, more tokens than a
+// decode window, f and d multiples of the 128-column GEMM slice.
+bool use_prefill_gemm(const moe_ctx *c, int N) {
+  return c->pf && c->fmt == MOE_Q4_SYM_G32_F16 && N > kDecMaxT && c->d % kPfBN == 0 &&
+         c->f % kPfBN == 0 && c->E <= kPfMaxE;
+}
+
+moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta, cudaStream_t s) {
+  const int E = c->E, k = c->k, d = c->d, f = c->f;
+  if (!c->pf_maps) {
+    if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
+        !encode_map_f16(&c->pf_map_a, c->abuf, c->pf_rows, f))
+      return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    c->pf_maps = true;
+  }
+  CUDA_TRY(c, prof_mark(c, 0, s));
+  cudaError_t e = cudaSuccess;
+  const uint16_t *h = router_input(c, layer, x, N, s, &e);
+  CUDA_TRY(c, e);
+  RouterParams rp{h, c->d_router + (size_t)layer * E * d,
+                  c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E, c->logits};
+  CUDA_TRY(c, launch_router(c, s, rp));
+  const int blocks = (N + kPfTok - 1) / kPfTok;
+  PfRouteParams tp{c->logits, N, E, k, c->idx, c->w, c->pf_bmask, &c->stats[4]};
+  const dim3 tg(blocks), tb(kPfTok * 32);
+  if (E <= 128) CUDA_TRY(c, launch(prefill_topk_kernel<4>, tg, tb, 0, s, tp));
+  else if (E <= 512) CUDA_TRY(c, launch(prefill_topk_kernel<16>, tg, tb, 0, s, tp));
+  else CUDA_TRY(c, launch(prefill_topk_kernel<32>, tg, tb, 0, s, tp));
+  PfScanParams sp{};
+  sp.bmask = c->pf_bmask;
+  sp.blocks = blocks;
+  sp.E = E;
+  sp.T = N;
+  sp.k = k;
+  sp.boff = c->pf_boff;
+  sp.eoff = c->pf_eoff;
+  sp.slot_of = c->d_slot_of;
+  sp.n_slots = c->n_slots;
+  sp.layer = layer;
+  sp.arena = c->arena;
+  sp.pool = c->pool;
+  sp.shared = c->n_shared ? c->shared + (size_t)layer * c->lay.expert_bytes : nullptr;
+  sp.expert_bytes = c->lay.expert_bytes;
+  sp.tiles = c->pf_tiles;
+  sp.n_tiles = c->pf_ntiles;
+  sp.max_tiles = c->pf_max_tiles;
+  sp.cnt_out = c->cnt_out;
+  sp.stats = c->stats;
+  sp.last = c->last;
+  sp.status = c->status;
+  CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
+  PfScatterParams cp{c->idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
+                     c->pf_row_of, c->pf_hg};
+  CUDA_TRY(c, launch(prefill_scatter_kernel, tg, tb, 0, s, cp));
+  CUDA_TRY(c, prof_mark(c, 1, s));
+  PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
+                  nullptr, c->status};
+  const int smem1 = kPfStagesG * (kPfBM * kPfBK * 2 + 2 * kPfBN * kPfBK * 2) + 1024;
+  const int smem2 = kPfStagesD * (kPfBM * kPfBK * 2 + kPfBN * kPfBK * 2) + 1024;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c->n_sm);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = smem1;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<true>, c->pf_map_h, g1));
+    PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / 64, c->lay.p1_bytes, nullptr, c->ybuf,
+                    c->status};
+    cfg.dynamicSmemBytes = smem2;
+    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<false>, c->pf_map_a, g2));
+  }
+  CUDA_TRY(c, prof_mark(c, 2, s));
+  PfCombineParams mp{c->ybuf, c->w, c->pf_row_of, N, k, d, c->n_shared, x, delta};
+  const long long n4 = (long long)N * d / 4;
+  const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
+  CUDA_TRY(c, launch(prefill_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));
+  CUDA_TRY(c, prof_mark(c, 3, s));
+  if (c->profiling) {
+    c->prof_next = (c->prof_next + 1) % kProfSlots;
+    c->prof_pending = std::min(c->prof_pending + 1, kProfSlots);
+  }
+  return MOE_OK;
+}
+
 // The whole decode chain for one layer.  delta == nullptr: residual mode.
 // Windows of <= kFusedMaxT tokens take four launches: fused routing, the
 // gated expert GEMV, the down GEMV and the combine + residual.
@@ -664,6 +834,7 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   if (e == cudaSuccess) e = setup_route_fused();
   if (e == cudaSuccess) e = setup_finish();
   if (e == cudaSuccess) e = setup_decode();
+  if (e == cudaSuccess) e = setup_prefill();
   if (e == cudaSuccess) e = setup_gemv<1, true, 1>(c->n_sm, &c->gemv_blocks[0][1][0]);
   if (e == cudaSuccess) e = setup_gemv<1, false, 1>(c->n_sm, &c->gemv_blocks[0][0][0]);
   if (e == cudaSuccess) e = setup_gemv<2, true, 1>(c->n_sm, &c->gemv_blocks[1][1][0]);
@@ -699,6 +870,7 @@ moe_status moe_destroy(moe_ctx *c) {
   cudaDeviceSynchronize();
   for (auto &kv : c->stack_graphs) cudaGraphExecDestroy(kv.second);
   for (cudaEvent_t ev : c->prof_ev) cudaEventDestroy(ev);
+  dfree(c->pf);
   dfree(c->arena);
   dfree(c->shared);
   dfree(c->pool);
@@ -915,9 +1087,32 @@ moe_status moe_forward_stack(moe_ctx *c, void *x, int T, void *stream) {
 }
 
 moe_status moe_prefill(moe_ctx *c, int layer, void *x, int N, void *stream) {
-  // A prefill chunk computes the same layer function as a decode window; the
-  // grouped expert kernels split each expert's tokens into jobs.
-  return moe_forward(c, layer, x, N, stream);
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !x || N < 1 || N > c->max_tokens || !aligned16(x))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_prefill: bad arguments (N=%d max=%d)", N,
+                c->max_tokens);
+  moe_status st = check_ready(c, layer);
+  if (st) return st;
+  c->last_stream = (cudaStream_t)stream;
+  if (!use_prefill_gemm(c, N))
+    return forward_impl(c, layer, (uint16_t *)x, N, nullptr, (cudaStream_t)stream);
+  return prefill_impl(c, layer, (uint16_t *)x, N, nullptr, (cudaStream_t)stream);
+}
+
+moe_status moe_prefill_delta(moe_ctx *c, int layer, const void *x, int N, float *delta,
+                             void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !x || !delta || N < 1 || N > c->max_tokens || !aligned16(x) ||
+      !aligned16(delta))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_prefill_delta: bad arguments");
+  moe_status st = check_ready(c, layer);
+  if (st) return st;
+  c->last_stream = (cudaStream_t)stream;
+  uint16_t *xp = (uint16_t *)const_cast<void *>(x);
+  if (!use_prefill_gemm(c, N)) return forward_impl(c, layer, xp, N, delta, (cudaStream_t)stream);
+  return prefill_impl(c, layer, xp, N, delta, (cudaStream_t)stream);
 }
 
 moe_status moe_sync(moe_ctx *c, int timeout_ms) {

@@ -1,0 +1,546 @@
+// prefill.cuh -- the MoE layer for a prefill chunk of up to 8192 tokens
+// (sm_100a).
+//
+// A chunk is a real dense contraction per expert (the engine article "93
+// token/s on one 8 GB card", section "Architecture overview": prefill runs
+// in chunks of up to 8192 tokens), so the experts run as a grouped GEMM on
+// the 5th-generation tensor cores:
+//
+//   prefill_topk_kernel     one warp per token: top-k + softmax; per block of
+//                           16 tokens, each expert's token set (a bitmask)
+//   prefill_scan_kernel     per expert: tokens per block of 16 (column scan),
+//                           the expert's first row in grouped order, and the
+//                           list of 128-row tiles (expert, first row, rows)
+//   prefill_scatter_kernel  pair -> row in grouped order (stable: ascending t
+//                           within an expert) and the gather of every pair's
+//                           token row into the grouped A matrix (fp16)
+//   prefill_gemm_kernel     A tile (TMA, 128B swizzle) x dequantised weight
+//                           tile (written by the CTA's warps straight into
+//                           the swizzled fp16 layout) -> tcgen05.mma, fp32
+//                           accumulators in TMEM; gate/up pass writes
+//                           SiLU(G) * U (fp16), down pass writes y (fp32)
+//   prefill_combine_kernel  x += sum_j w_j y[row(t, j)] + y_shared[t]
+//
+// Operands are fp16: a Q4 weight s*(c-8) with its fp16 scale is one
+// rounding away from exact in fp16, and bf16 activations convert to fp16
+// exactly in fp16's normal range (values beyond +-65504 saturate).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "route.cuh"
+
+namespace moe {
+
+constexpr int kPfTok = 16;       // tokens per block of the top-k / scatter kernels (one warp each)
+constexpr int kPfBM = 128;       // GEMM tile rows (tokens of one expert)
+constexpr int kPfBN = 128;       // GEMM tile columns (output features)
+constexpr int kPfBK = 64;        // reduction per stage (one 128-byte swizzle row of fp16)
+constexpr int kPfThreads = 256;  // GEMM CTA: 8 warps dequantise, warp 0 lane 0 issues
+constexpr int kPfStagesG = 3, kPfStagesD = 4;
+constexpr int kPfMaxE = 1024;
+
+struct PfTile {                  // one 128-row tile of one expert
+  const uint8_t *w;              // expert base (repacked layout)
+  int row0, rows;                // first row in grouped order, rows <= 128
+};
+
+struct PfRouteParams {
+  const float *logits;  // [T, E]
+  int T, E, k;
+  int *idx;             // [T, k]
+  float *w;             // [T, k]
+  unsigned short *bmask;  // [blocks][E]: bit i = token 16 b + i selected the expert
+  unsigned long long *near_ties;
+};
+
+// One warp per token; then the block's per-expert token sets.
+template <int NPL>
+__global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams p) {
+  __shared__ unsigned s_mask[kPfMaxE];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  pdl_wait();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_mask[e] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kPfTok + wid;
+  if (t < p.T) {
+    int e;
+    float w;
+    warp_topk<NPL>(p.logits + (long long)t * p.E, p.E, p.k, lane, false, e, w, p.near_ties);
+    if (lane < p.k) {
+      p.idx[(long long)t * p.k + lane] = e;
+      p.w[(long long)t * p.k + lane] = w;
+      atomicOr(&s_mask[e], 1u << wid);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+    p.bmask[(long long)blockIdx.x * p.E + e] = (unsigned short)s_mask[e];
+  pdl_launch_dependents();
+}
+
+struct PfScanParams {
+  const unsigned short *bmask;  // [blocks][E]
+  int blocks, E, T, k;
+  int *boff;                    // [blocks][E] first row of (block, expert) in grouped order
+  int *eoff;                    // [E + 1]
+  const int *slot_of;           // residency table [L*E]
+  int n_slots, layer;
+  const uint8_t *arena, *pool, *shared;
+  long long expert_bytes;
+  PfTile *tiles;                // [max_tiles]
+  int *n_tiles;
+  int max_tiles;
+  int *cnt_out;                 // [E] statistics
+  unsigned long long *stats;
+  int *last;
+  int *status;
+};
+
+// One CTA of 1024 threads.  Thread e walks its expert's column of block
+// masks (block order = token order, so rows stay in ascending t), then one
+// block scan gives the experts' first rows and first tiles.
+__global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
+  __shared__ int s_cnt[2 * kPfMaxE + 2];
+  __shared__ int s_red[32];
+  __shared__ unsigned long long s_hm[3];
+  pdl_wait();
+  const int tid = threadIdx.x;
+  int *cnt = s_cnt, *tl = s_cnt + kPfMaxE + 1;
+  if (tid < 3) s_hm[tid] = 0;
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < p.blocks; ++b) {
+      p.boff[(long long)b * p.E + e] = run;  // relative to the expert's first row
+      run += __popc(p.bmask[(long long)b * p.E + e]);
+    }
+    cnt[e] = run;
+    tl[e] = (run + kPfBM - 1) / kPfBM;
+  }
+  block_exclusive_scan(cnt, cnt, p.E, s_red);
+  block_exclusive_scan(tl, tl, p.E, s_red);
+  const int routed_tiles = tl[p.E], P = cnt[p.E];
+  const int shared_tiles = p.shared ? (p.T + kPfBM - 1) / kPfBM : 0;
+  if (routed_tiles + shared_tiles > p.max_tiles) {
+    if (tid == 0) {
+      atomicOr(p.status, kErrJobOverflow);
+      *p.n_tiles = 0;
+    }
+    return;
+  }
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    p.eoff[e] = cnt[e];
+    const int n = cnt[e + 1] - cnt[e];
+    p.cnt_out[e] = n;
+    if (!n) continue;
+    const int slot = p.slot_of ? p.slot_of[(long long)p.layer * p.E + e] : -1;
+    const bool hit = slot >= 0 && slot < p.n_slots;
+    if (!hit && slot >= p.n_slots) atomicOr(p.status, kErrBadSlot);
+    const uint8_t *ptr = hit ? p.pool + (long long)slot * p.expert_bytes
+                             : p.arena + ((long long)p.layer * p.E + e) * p.expert_bytes;
+    atomicAdd(&s_hm[hit ? 0 : 1], (unsigned long long)n);
+    atomicAdd(&s_hm[2], 1ull);
+    for (int m = 0, ti = tl[e]; m < n; m += kPfBM, ++ti) {
+      p.tiles[ti].w = ptr;
+      p.tiles[ti].row0 = cnt[e] + m;
+      p.tiles[ti].rows = min(kPfBM, n - m);
+    }
+  }
+  if (tid == 0) p.eoff[p.E] = P;
+  for (int q = tid; q < shared_tiles; q += blockDim.x) {
+    p.tiles[routed_tiles + q].w = p.shared;
+    p.tiles[routed_tiles + q].row0 = P + q * kPfBM;
+    p.tiles[routed_tiles + q].rows = min(kPfBM, p.T - q * kPfBM);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    *p.n_tiles = routed_tiles + shared_tiles;
+    atomicAdd(&p.stats[0], 1ULL);
+    atomicAdd(&p.stats[1], (unsigned long long)p.T);
+    atomicAdd(&p.stats[2], s_hm[0]);
+    atomicAdd(&p.stats[3], s_hm[1]);
+    p.last[0] = p.T;
+    p.last[1] = (int)s_hm[2];
+    p.last[2] = p.layer;
+  }
+  pdl_launch_dependents();
+}
+
+struct PfScatterParams {
+  const int *idx;               // [T, k]
+  const unsigned short *bmask;  // [blocks][E]
+  const int *boff, *eoff;
+  const uint16_t *h;            // bf16 [T, d]
+  int T, E, k, d, has_shared;
+  int *row_of;                  // [T*k + T]: grouped row of pair (shared pair P + t)
+  __half *hg;                   // fp16 [rows][d] grouped A matrix
+};
+
+// One warp per token: its k pairs (and its shared-expert pair) get their
+// grouped rows, and the token's row is copied (fp16, saturating) to each.
+__global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterParams p) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  pdl_wait();
+  const int t = blockIdx.x * kPfTok + wid;
+  if (t >= p.T) return;
+  const int P = p.T * p.k;
+  int rows[33];
+  const int nr = p.k + (p.has_shared ? 1 : 0);
+  for (int j = 0; j < p.k; ++j) {
+    const int e = __ldg(p.idx + (long long)t * p.k + j);
+    const unsigned m = p.bmask[(long long)blockIdx.x * p.E + e];
+    const int rank = __popc(m & ((1u << wid) - 1u));
+    rows[j] = p.eoff[e] + p.boff[(long long)blockIdx.x * p.E + e] + rank;
+  }
+  if (p.has_shared) rows[p.k] = P + t;
+  if (lane < p.k) p.row_of[(long long)t * p.k + lane] = rows[lane];
+  if (lane == 0 && p.has_shared) p.row_of[P + t] = P + t;
+  // copy the token row to every destination, 8 elements per lane per step
+  const uint4 *src = reinterpret_cast<const uint4 *>(p.h + (long long)t * p.d);
+  for (int i = lane; i < p.d / 8; i += 32) {
+    const uint4 v = __ldg(src + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(in[q] << 16), hi = __uint_as_float(in[q] & 0xFFFF0000u);
+      uint32_t r;
+      asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+      out[q] = r;
+    }
+    const uint4 o = make_uint4(out[0], out[1], out[2], out[3]);
+    for (int j = 0; j < nr; ++j) reinterpret_cast<uint4 *>(p.hg + (long long)rows[j] * p.d)[i] = o;
+  }
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------- tcgen05 helpers
+// Shared-memory matrix descriptor (sm_100): start address >> 4 in bits
+// [0,14), leading byte offset >> 4 in [16,30), stride byte offset >> 4 in
+// [32,46), descriptor version 1 in [46,48), layout in [61,64) (2 = 128-byte
+// swizzle).  A K-major tile of rows x 64 fp16 with 128-byte swizzle: rows of
+// 128 B, 8-row groups 1024 B apart (SBO); LBO is unused.
+MOE_DEV uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: D fp32 (bits 4-5 = 1), A and B fp16
+// (bits 7-9, 10-12 = 0), both K-major, N >> 3 in [17,23), M >> 4 in [24,29).
+constexpr uint32_t umma_idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+MOE_DEV void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+// Arrive on an mbarrier once every tcgen05 operation this thread issued so far
+// has completed.
+MOE_DEV void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+MOE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MOE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 TMEM columns of this warp's 32 lanes (thread i = lane 32 (warp % 4) + i)
+MOE_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2-D TMA tile load (x = element offset along the contiguous dimension, y = row)
+MOE_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+MOE_DEV uint32_t h2_dup(uint32_t v, bool hi) {  // (h, h) from one fp16 half of v
+  const uint32_t h = hi ? (v >> 16) : (v & 0xFFFFu);
+  return h | (h << 16);
+}
+MOE_DEV uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+MOE_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Dequantise one 32-bit code word of a repacked Q4 tile into the swizzled
+// fp16 B tile.  The word of lane (g, tig), k-step st holds rows r0 = 16 rb +
+// g and r1 = r0 + 8, reduction columns kb .. kb+3 (kb = kb_step(st, tig)):
+// nibbles at bits 0/16 and 8/24 are row r0's columns (kb, kb+1) and
+// (kb+2, kb+3), bits 4/20 and 12/28 row r1's.  A nibble at bit 0 of an fp16
+// half over 0x6400 is 1024 + c; at bit 4 over 0x5400 it is 64 + c; one
+// subtraction gives c - 8 exactly and one multiplication by the group's
+// fp16 scale rounds once.
+MOE_DEV void dequant_q4_word(uint32_t w, uint32_t s0, uint32_t s1, uint32_t dst_s, int r0, int kb) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t c1032 = 0x64086408u, c72 = 0x54805480u;  // fp16 1032.0, 72.0
+  const uint32_t a0 = hmul2(hsub2(lop3_and_or(w, 0x000F000Fu, 0x64006400u), c1032), s0);
+  const uint32_t a2 = hmul2(hsub2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), c1032), s0);
+  const uint32_t b0 = hmul2(hsub2(lop3_and_or(w, 0x00F000F0u, 0x54005400u), c72), s1);
+  const uint32_t b2 = hmul2(hsub2(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), c72), s1);
+  // 128-byte swizzle: row r at (r / 8) * 1024 + (r % 8) * 128, 16-byte chunk c -> c ^ (r % 8)
+  const int r1 = r0 + 8;
+  const uint32_t ch = (uint32_t)(kb >> 3), sub = (uint32_t)(kb & 7) * 2;
+  const uint32_t o0 = (uint32_t)(r0 >> 3) * 1024 + (uint32_t)(r0 & 7) * 128 + ((ch ^ (r0 & 7)) << 4) + sub;
+  const uint32_t o1 = (uint32_t)(r1 >> 3) * 1024 + (uint32_t)(r1 & 7) * 128 + ((ch ^ (r1 & 7)) << 4) + sub;
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst_s + o0), "r"(a0), "r"(a2) : "memory");
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst_s + o1), "r"(b0), "r"(b2) : "memory");
+}
+
+struct PfGemmParams {
+  const PfTile *tiles;
+  const int *n_tiles;
+  int K;                 // reduction (d for gate/up, f for down)
+  int N;                 // output features (f for gate/up, d for down)
+  int ntile_k;           // repacked tiles along K: K / 64
+  long long region_off;  // 0 (gate/up) or the down region's offset
+  __half *out_a;         // gate/up: SiLU(G) * U, fp16 [rows][N]
+  float *out_y;          // down: fp32 [rows][N]
+  int *status;
+};
+
+// Grouped GEMM over the tile list.  Work item = (128-row tile, 128-column
+// slice); persistent CTAs walk items blockIdx.x, + gridDim.x, ...  Per item:
+// for every 64-column step of the reduction, warp 0 lane 0 TMA-loads the A
+// tile into the stage, all eight warps dequantise the weight tiles (two
+// matrices for gate/up) into the stage, and warp 0 lane 0 issues four
+// m128n128k16 MMAs per matrix and commits them to the stage's empty barrier,
+// so dequantising the next stage overlaps the tensor core.  After the last
+// step the accumulators (TMEM) are read back by all warps: lanes = rows,
+// each warp a quarter of the rows and half of the columns.
+template <bool GATED>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
+  constexpr int NM = GATED ? 2 : 1;
+  constexpr int S = GATED ? kPfStagesG : kPfStagesD;
+  constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;  // 16 KB per matrix
+  constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;  // 16 KB
+  constexpr uint32_t STAGE = TILE_A + NM * TILE_B;
+  extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
+  __shared__ __align__(8) unsigned long long s_full[S], s_empty[S], s_acc;
+  __shared__ uint32_t s_tmem;
+  const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+  const uint32_t base = smem_addr(pf_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_addr(&s_full[i]), 1);
+      mbar_init(smem_addr(&s_empty[i]), 1);
+    }
+    mbar_init(smem_addr(&s_acc), 1);
+    fence_mbar_init();
+  }
+  if (wid == 0) {  // 256 columns: G and U (or D) accumulators of 128 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_addr(&s_tmem)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  pdl_wait();
+  const int ntiles = ldcg_i32(p.n_tiles);
+  const int nslices = p.N / kPfBN, nsteps = p.K / kPfBK;
+  const long long items = (long long)ntiles * nslices;
+  constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, kPfBN);
+  uint32_t it = 0;      // stage counter over all items of this CTA
+  uint32_t acc_ph = 0;  // parity of the accumulator barrier
+  bool ok = true;
+  for (long long item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    const PfTile tile = p.tiles[item / nslices];
+    const int n0 = (int)(item % nslices) * kPfBN;
+    const uint8_t *wbase = tile.w + p.region_off;
+    for (int ks = 0; ks < nsteps; ++ks, ++it) {
+      const uint32_t st = it % S, use = it / S;
+      const uint32_t sa = stage0 + st * STAGE, sb = sa + TILE_A;
+      // the stage's previous MMAs must be done before it is overwritten
+      if (use > 0 && __syncthreads_or(!mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      if (tid == 0) {
+        mbar_expect_tx(smem_addr(&s_full[st]), TILE_A);
+        tma_load_2d(sa, &amap, ks * kPfBK, tile.row0, smem_addr(&s_full[st]));
+      }
+      // dequantise: 8 row blocks x NM matrices of 128 code words; thread ->
+      // one (row block, matrix) quarter-tile of 32 words... 8 (gated) or 4 words
+      {
+        constexpr int WPT = 8 * NM * 128 / kPfThreads;  // words per thread
+        const int q = tid / (128 / WPT);                 // (row block, matrix) tile of this thread
+        const int rbl = q / NM, m = q % NM;
+        const int w0 = (tid % (128 / WPT)) * WPT;        // first word (lane * 4 + word)
+        const int rb = n0 / 16 + rbl;
+        const uint8_t *tp = wbase + ((long long)(rb * p.ntile_k + ks) * NM + m) * 576;
+        uint32_t wv[WPT];
+#pragma unroll
+        for (int v = 0; v < WPT; v += 4) {
+          const uint4 x = __ldg(reinterpret_cast<const uint4 *>(tp) + (w0 + v) / 4);
+          wv[v] = x.x;
+          wv[v + 1] = x.y;
+          wv[v + 2] = x.z;
+          wv[v + 3] = x.w;
+        }
+        const uint32_t dst = sb + m * TILE_B;
+#pragma unroll
+        for (int v = 0; v < WPT; ++v) {
+          const int wi = w0 + v, ln = wi >> 2, word = wi & 3;
+          const int g = ln >> 2, tig = ln & 3;
+          const uint2 sc = __ldg(reinterpret_cast<const uint2 *>(tp + 512) + g);
+          const uint32_t sv = (word >> 1) ? sc.y : sc.x;  // group of this k-step
+          dequant_q4_word(wv[v], h2_dup(sv, false), h2_dup(sv, true), dst, rbl * 16 + g,
+                          kb_step(word, tig));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        if (!mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
+          atomicOr(p.status, kErrTimeout);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kPfBK / 16; ++kk) {
+            const uint64_t da = umma_desc_sw128(sa + kk * 32);
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+              umma_f16(tmem + m * 128, da, umma_desc_sw128(sb + m * TILE_B + kk * 32), IDESC,
+                       (ks | kk) != 0);
+          }
+        }
+        umma_commit(smem_addr(&s_empty[st]));
+        if (ks == nsteps - 1) umma_commit(smem_addr(&s_acc));
+      }
+    }
+    if (!ok) break;
+    // epilogue: accumulators -> registers -> global
+    if (__syncthreads_or(!mbar_wait_bounded(smem_addr(&s_acc), acc_ph))) {
+      ok = false;
+      break;
+    }
+    acc_ph ^= 1u;
+    tc_fence_after();
+    {
+      const int quarter = wid & 3, half = wid >> 2;
+      const int r = quarter * 32 + lane;  // tile row = TMEM lane
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+        float g[32];
+        tmem_ld32(lane_addr + c0, g);
+        if constexpr (GATED) {
+          float u[32];
+          tmem_ld32(lane_addr + 128 + c0, u);
+          if (r < tile.rows) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int i = v * 8 + q * 2;
+                const float a0 = g[i] / (1.0f + __expf(-g[i])) * u[i];
+                const float a1 = g[i + 1] / (1.0f + __expf(-g[i + 1])) * u[i + 1];
+                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
+              }
+              dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        } else {
+          if (r < tile.rows) {
+            float4 *dst = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) dst[v] = make_float4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM read before the next item's first MMA overwrites it
+    tc_fence_after();
+  }
+  if (!ok && tid == 0) atomicOr(p.status, kErrTimeout);
+  // drain: every committed MMA group must be complete before TMEM is freed
+  if (tid == 0 && it > 0) {
+    const uint32_t last = it - 1;
+    (void)mbar_wait_bounded(smem_addr(&s_empty[last % S]), (last / S) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (wid == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+  pdl_launch_dependents();
+}
+
+struct PfCombineParams {
+  const float *y;     // [rows][d] grouped order
+  const float *w;     // [T][k]
+  const int *row_of;  // [T*k + T]
+  int T, k, d, has_shared;
+  uint16_t *x;        // bf16 [T][d] residual (mode 0)
+  float *delta;       // fp32 [T][d] (mode 1)
+};
+
+// x[t] <- bf16(x[t] + sum_j w[t,j] y[row(t,j)] + y[row(shared, t)]), j in order.
+__global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p) {
+  pdl_wait();
+  const int per_t = p.d / 4, P = p.T * p.k;
+  const long long n = (long long)p.T * per_t;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / per_t), o = (int)(i - (long long)t * per_t) * 4;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int j = 0; j < p.k; ++j) {
+      const float wj = __ldg(p.w + (long long)t * p.k + j);
+      const float4 v = ldcg_f4(p.y + (long long)__ldg(p.row_of + (long long)t * p.k + j) * p.d + o);
+      a0 = fmaf(wj, v.x, a0);
+      a1 = fmaf(wj, v.y, a1);
+      a2 = fmaf(wj, v.z, a2);
+      a3 = fmaf(wj, v.w, a3);
+    }
+    if (p.has_shared) {
+      const float4 sh = ldcg_f4(p.y + (long long)(P + t) * p.d + o);
+      a0 += sh.x;
+      a1 += sh.y;
+      a2 += sh.z;
+      a3 += sh.w;
+    }
+    if (p.delta) {
+      *reinterpret_cast<float4 *>(p.delta + (long long)t * p.d + o) = make_float4(a0, a1, a2, a3);
+    } else {
+      uint16_t *xr = p.x + (long long)t * p.d + o;
+      const uint2 xv = *reinterpret_cast<const uint2 *>(xr);
+      uint2 o2;
+      o2.x = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.x << 16) + a0)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.x & 0xFFFF0000u) + a1)) << 16);
+      o2.y = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.y << 16) + a2)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(xv.y & 0xFFFF0000u) + a3)) << 16);
+      *reinterpret_cast<uint2 *>(xr) = o2;
+    }
+  }
+}
+
+}  // namespace moe
