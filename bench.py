@@ -39,8 +39,10 @@ D, F, E, K_TOP = 2048, 768, 512, 10
 
 def parse():
     ap = argparse.ArgumentParser()
+    # (defaults that depend on the workload are filled in below)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 200 decode windows, 20 prefill chunks)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="decode", choices=["decode", "q2", "prefill"])
@@ -49,7 +51,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seed", type=int, default=0)
-    return ap.parse_args()
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = 20 if a.workload == "prefill" else 200
+    return a
 
 
 # ----------------------------------------------------------------- helpers
@@ -240,14 +245,16 @@ def run_native(args, world, rank, local):
     total_bytes = expert_bytes + router_bytes + act_bytes
 
     stream = torch.cuda.current_stream()
+    prefill = args.workload == "prefill"
+    call = B.moe_prefill if prefill else B.moe_forward  # the public call a step makes
     # warm-up (eager), then capture the K timed steps as one CUDA graph
     for i in range(W):
-        B.moe_forward(ctx, layer_of[i], x_work[i], T)
+        call(ctx, layer_of[i], x_work[i], T)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(W, n_win):
-            B.moe_forward(ctx, layer_of[i], x_work[i], T)
+            call(ctx, layer_of[i], x_work[i], T)
     torch.cuda.synchronize()
     x_work.copy_(x_dev0)
     torch.cuda.synchronize()
@@ -274,7 +281,7 @@ def run_native(args, world, rank, local):
     gp = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gp):
         for i in range(W, n_win):
-            B.moe_forward(ctx, layer_of[i], x_work[i], T)
+            call(ctx, layer_of[i], x_work[i], T)
     x_work.copy_(x_dev0)
     torch.cuda.synchronize()
     gp.replay()
@@ -286,14 +293,14 @@ def run_native(args, world, rank, local):
     xbuf = torch.empty((T, D), dtype=torch.int16, device="cuda")
     for i in range(min(W, 3)):
         xbuf.copy_(x_host[i], non_blocking=True)
-        B.moe_forward(ctx, layer_of[i], xbuf, T)
+        call(ctx, layer_of[i], xbuf, T)
         out_host[i].copy_(xbuf, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
     e0.record(stream)
     for i in range(W, n_win):
         xbuf.copy_(x_host[i], non_blocking=True)
-        B.moe_forward(ctx, layer_of[i], xbuf, T)
+        call(ctx, layer_of[i], xbuf, T)
         out_host[i].copy_(xbuf, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -306,6 +313,10 @@ def run_native(args, world, rank, local):
     # profile's three segments are then one kernel); larger ones as five
     # launches, of which the two expert GEMV launches dominate
     single = T <= 32
+    flops = 6.0 * D * F * (T * K_TOP + T)  # per call: gate, up, down GEMMs, routed + shared rows
+    if prefill:
+        gemm_ms = exp_ms / max(ncalls, 1)  # the two grouped GEMM launches of one call
+        gemm_tf = flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     if single:
         kern_ms = route_ms + exp_ms + comb_ms
         kern_bytes = expert_bytes + router_bytes
@@ -329,8 +340,10 @@ def run_native(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "q4-g32 weights, bf16 activations, fp32 accumulate" if spec["fmt"] == I.Q4
-                 else "q2-g64 weights, bf16 activations, fp32 accumulate",
+        "dtype": ("q4-g32 weights dequantised to fp16 per tile, fp16 activations, fp32 accumulate"
+                  if prefill else
+                  "q4-g32 weights, bf16 activations, fp32 accumulate" if spec["fmt"] == I.Q4
+                  else "q2-g64 weights, bf16 activations, fp32 accumulate"),
         "data": "synthetic (seeded generator; random-init weights of the layer's shape)",
         "config": {"workload": spec["name"], "tokens_per_step": T, "layers_rotated": n_rot,
                    "l2": f"no flush: each step reads a different layer copy "
@@ -344,6 +357,19 @@ def run_native(args, world, rank, local):
                                  "experts": exp_ms / max(ncalls, 1),
                                  "combine": comb_ms / max(ncalls, 1)},
         "roofline": {
+            "bound": "tensor",
+            "kernel": "prefill_gemm_kernel (gate/up + down grouped GEMMs of one call, tcgen05 fp16)",
+            "achieved": gemm_tf,
+            "peak": tflops,
+            "unit": "TFLOP/s",
+            "frac": (gemm_tf / tflops) if gemm_tf else None,
+            "launch_us": gemm_ms * 1e3,
+            "traffic": None,
+            "peak_source": (f"{peak_kind} bf16_tflops (MEASURED_PEAKS.json); fp16 dense rate = bf16 "
+                            "rate (nominal ratio 1:1)"),
+            "per_unit": f"6 d f = {6 * D * F} FLOP per (token, expert) row; "
+                        f"{T * K_TOP + T} rows per call",
+        } if prefill else {
             "bound": "hbm",
             "kernel": kern_name,
             "achieved": kern_gbs,
@@ -358,7 +384,7 @@ def run_native(args, world, rank, local):
         },
         "e2e": {"value": world * tok / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": K * (1 if single else 5),
+        "gpu_launches": K * (1 if single else (7 if prefill else 5)),
         "clocks": clocks,
     }
     B.moe_destroy(ctx)

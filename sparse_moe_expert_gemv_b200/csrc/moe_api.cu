@@ -540,11 +540,10 @@ bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
 
 cudaError_t setup_prefill() {
   cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kPfStagesG * (kPfBM * kPfBK * 2 + 2 * kPfBN * kPfBK * 2) + 1024);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg<true>::SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(prefill_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPfStagesD * (kPfBM * kPfBK * 2 + kPfBN * kPfBK * 2) + 1024);
+                             PfCfg<false>::SMEM);
   return e;
 }
 
@@ -567,9 +566,11 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   cudaError_t e = cudaSuccess;
   const uint16_t *h = router_input(c, layer, x, N, s, &e);
   CUDA_TRY(c, e);
-  RouterParams rp{h, c->d_router + (size_t)layer * E * d,
-                  c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E, c->logits};
-  CUDA_TRY(c, launch_router(c, s, rp));
+  RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d,
+                      c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E,
+                      c->logits};
+  CUDA_TRY(c, launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN),
+                     dim3(256), 0, s, rp));
   const int blocks = (N + kPfTok - 1) / kPfTok;
   PfRouteParams tp{c->logits, N, E, k, c->idx, c->w, c->pf_bmask, &c->stats[4]};
   const dim3 tg(blocks), tb(kPfTok * 32);
@@ -605,12 +606,11 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   CUDA_TRY(c, prof_mark(c, 1, s));
   PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
                   nullptr, c->status};
-  const int smem1 = kPfStagesG * (kPfBM * kPfBK * 2 + 2 * kPfBN * kPfBK * 2) + 1024;
-  const int smem2 = kPfStagesD * (kPfBM * kPfBK * 2 + kPfBN * kPfBK * 2) + 1024;
+  const int smem1 = PfCfg<true>::SMEM, smem2 = PfCfg<false>::SMEM;
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(c->n_sm);
-    cfg.blockDim = dim3(kPfThreads);
+    cfg.blockDim = dim3(kPfGemmThreads);
     cfg.dynamicSmemBytes = smem1;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

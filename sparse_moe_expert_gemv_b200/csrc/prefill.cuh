@@ -37,8 +37,6 @@ constexpr int kPfTok = 16;       // tokens per block of the top-k / scatter kern
 constexpr int kPfBM = 128;       // GEMM tile rows (tokens of one expert)
 constexpr int kPfBN = 128;       // GEMM tile columns (output features)
 constexpr int kPfBK = 64;        // reduction per stage (one 128-byte swizzle row of fp16)
-constexpr int kPfThreads = 256;  // GEMM CTA: 8 warps dequantise, warp 0 lane 0 issues
-constexpr int kPfStagesG = 3, kPfStagesD = 4;
 constexpr int kPfMaxE = 1024;
 
 struct PfTile {                  // one 128-row tile of one expert
@@ -215,6 +213,96 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
   pdl_launch_dependents();
 }
 
+// ------------------------------------------------------------ router GEMM
+// logits[t, e] = sum_i W[e, i] h[t, i] (+ b[e]) for a whole chunk, fp32 FMA
+// (routing decisions are compared bit-exactly, so no reduced-precision
+// tensor-core path).  CTA tile: 128 tokens x 128 experts, 256 threads, each
+// an 8 x 8 block of outputs; the reduction walks i in order, 16 at a time
+// through shared memory (h converted from bf16 on the way in).
+struct RouterGemmParams {
+  const uint16_t *h;   // bf16 [T, d]
+  const float *W;      // fp32 [E, d]
+  const float *bias;   // [E] or null
+  int T, d, E;
+  float *logits;       // [T, E]
+};
+
+constexpr int kRgBM = 128, kRgBN = 128, kRgBK = 16;
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
+  __shared__ __align__(16) float As[2][kRgBK][kRgBM + 4];
+  __shared__ __align__(16) float Ws[2][kRgBK][kRgBN + 4];
+  pdl_wait();
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int t0 = blockIdx.x * kRgBM, e0 = blockIdx.y * kRgBN;
+  // loaders: thread -> (row = tid / 2, 8 columns at (tid % 2) * 8)
+  const int lr = tid >> 1, lc = (tid & 1) * 8;
+  const int ta = t0 + lr, ew = e0 + lr;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  auto load = [&](int k0, uint4 &hv, float4 &w0, float4 &w1) {
+    hv = ta < p.T ? __ldg(reinterpret_cast<const uint4 *>(p.h + (long long)ta * p.d + k0 + lc))
+                  : make_uint4(0u, 0u, 0u, 0u);
+    if (ew < p.E) {
+      const float4 *wp = reinterpret_cast<const float4 *>(p.W + (long long)ew * p.d + k0 + lc);
+      w0 = __ldg(wp);
+      w1 = __ldg(wp + 1);
+    } else {
+      w0 = w1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store = [&](int buf, const uint4 &hv, const float4 &w0, const float4 &w1) {
+    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      As[buf][lc + 2 * q][lr] = __uint_as_float(hw[q] << 16);
+      As[buf][lc + 2 * q + 1][lr] = __uint_as_float(hw[q] & 0xFFFF0000u);
+    }
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) Ws[buf][lc + q][lr] = wv[q];
+  };
+  uint4 hv;
+  float4 w0, w1;
+  load(0, hv, w0, w1);
+  store(0, hv, w0, w1);
+  __syncthreads();
+  const int nk = p.d / kRgBK;
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) load((kt + 1) * kRgBK, hv, w0, w1);
+#pragma unroll
+    for (int k = 0; k < kRgBK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Ws[buf][k][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Ws[buf][k][tx * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (kt + 1 < nk) store(buf ^ 1, hv, w0, w1);
+    __syncthreads();
+  }
+  pdl_launch_dependents();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + ty * 8 + i;
+    if (t >= p.T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + tx * 8 + j;
+      if (e < p.E) p.logits[(long long)t * p.E + e] = acc[i][j] + (p.bias ? p.bias[e] : 0.f);
+    }
+  }
+}
+
 // ---------------------------------------------------------- tcgen05 helpers
 // Shared-memory matrix descriptor (sm_100): start address >> 4 in bits
 // [0,14), leading byte offset >> 4 in [16,30), stride byte offset >> 4 in
@@ -324,38 +412,65 @@ struct PfGemmParams {
   int *status;
 };
 
-// Grouped GEMM over the tile list.  Work item = (128-row tile, 128-column
-// slice); persistent CTAs walk items blockIdx.x, + gridDim.x, ...  Per item:
-// for every 64-column step of the reduction, warp 0 lane 0 TMA-loads the A
-// tile into the stage, all eight warps dequantise the weight tiles (two
-// matrices for gate/up) into the stage, and warp 0 lane 0 issues four
-// m128n128k16 MMAs per matrix and commits them to the stage's empty barrier,
-// so dequantising the next stage overlaps the tensor core.  After the last
-// step the accumulators (TMEM) are read back by all warps: lanes = rows,
-// each warp a quarter of the rows and half of the columns.
+constexpr int kPfGemmThreads = 512;  // 16 warps
+constexpr int kPfDeqWarp0 = 8;       // warps 8..15 dequantise
+constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM lane quarters 0..3)
+
 template <bool GATED>
-__global__ void __launch_bounds__(kPfThreads, 1)
+struct PfCfg {
+  static constexpr int NM = GATED ? 2 : 1;
+  static constexpr int S = GATED ? 3 : 5;                   // pipeline stages
+  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB
+  static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per matrix
+  static constexpr uint32_t CODES = 8 * NM * 576;           // 8 row blocks of repacked tiles
+  static constexpr uint32_t STAGE = TILE_A + NM * TILE_B + CODES;
+  static constexpr uint32_t STAGE_AL = (STAGE + 1023) / 1024 * 1024;
+  static constexpr uint32_t SMEM = S * STAGE_AL + 1024;     // + alignment slack
+  static constexpr uint32_t ACC_COLS = NM * kPfBN;          // TMEM columns per accumulator buffer
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered (256 or 512)
+};
+
+// Grouped GEMM over the tile list, warp-specialised.  Work item = (128-row
+// tile, 128-column slice); persistent CTAs walk items blockIdx.x, +gridDim.x.
+//  warp 0 lane 0   producer: per 64-column reduction step, the A tile (2-D
+//                  TMA, 128-byte swizzle) and the 8 repacked code tiles of
+//                  the slice (1-D bulk copies) into a free stage
+//  warps 8..15     dequantise the stage's codes into the swizzled fp16 B
+//                  tile(s), then arrive on the stage's B barrier
+//  warp 1 lane 0   issues the MMAs (m128n128k16, A and B from shared memory,
+//                  fp32 accumulator in TMEM) and commits each stage's
+//                  release; accumulators alternate between two TMEM buffers
+//  warps 4..7      drain an accumulator buffer (TMEM lanes = tile rows) while
+//                  the next item accumulates into the other one
+// Every wait is bounded; a timeout raises kErrTimeout and every role stops.
+template <bool GATED>
+__global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
-  constexpr int NM = GATED ? 2 : 1;
-  constexpr int S = GATED ? kPfStagesG : kPfStagesD;
-  constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;  // 16 KB per matrix
-  constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;  // 16 KB
-  constexpr uint32_t STAGE = TILE_A + NM * TILE_B;
+  using C = PfCfg<GATED>;
+  constexpr int S = C::S, NM = C::NM;
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
-  __shared__ __align__(8) unsigned long long s_full[S], s_empty[S], s_acc;
+  __shared__ __align__(8) unsigned long long s_full[S], s_deq[S], s_empty[S], s_accf[2], s_acce[2];
   __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
   const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
   const uint32_t base = smem_addr(pf_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(smem_addr(&s_full[i]), 1);
+      mbar_init(smem_addr(&s_deq[i]), 256);
       mbar_init(smem_addr(&s_empty[i]), 1);
     }
-    mbar_init(smem_addr(&s_acc), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_addr(&s_accf[b]), 1);
+      mbar_init(smem_addr(&s_acce[b]), 128);
+    }
+    s_abort = 0;
     fence_mbar_init();
   }
-  if (wid == 0) {  // 256 columns: G and U (or D) accumulators of 128 columns
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_addr(&s_tmem)));
+  if (wid == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&s_tmem)),
+                 "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -365,95 +480,100 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   pdl_wait();
   const int ntiles = ldcg_i32(p.n_tiles);
   const int nslices = p.N / kPfBN, nsteps = p.K / kPfBK;
-  const long long items = (long long)ntiles * nslices;
-  constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, kPfBN);
-  uint32_t it = 0;      // stage counter over all items of this CTA
-  uint32_t acc_ph = 0;  // parity of the accumulator barrier
-  bool ok = true;
-  for (long long item = blockIdx.x; item < items && ok; item += gridDim.x) {
-    const PfTile tile = p.tiles[item / nslices];
-    const int n0 = (int)(item % nslices) * kPfBN;
-    const uint8_t *wbase = tile.w + p.region_off;
-    for (int ks = 0; ks < nsteps; ++ks, ++it) {
-      const uint32_t st = it % S, use = it / S;
-      const uint32_t sa = stage0 + st * STAGE, sb = sa + TILE_A;
-      // the stage's previous MMAs must be done before it is overwritten
-      if (use > 0 && __syncthreads_or(!mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1))) {
-        ok = false;
-        break;
-      }
-      if (tid == 0) {
-        mbar_expect_tx(smem_addr(&s_full[st]), TILE_A);
-        tma_load_2d(sa, &amap, ks * kPfBK, tile.row0, smem_addr(&s_full[st]));
-      }
-      // dequantise: 8 row blocks x NM matrices of 128 code words; thread ->
-      // one (row block, matrix) quarter-tile of 32 words... 8 (gated) or 4 words
-      {
-        constexpr int WPT = 8 * NM * 128 / kPfThreads;  // words per thread
-        const int q = tid / (128 / WPT);                 // (row block, matrix) tile of this thread
-        const int rbl = q / NM, m = q % NM;
-        const int w0 = (tid % (128 / WPT)) * WPT;        // first word (lane * 4 + word)
-        const int rb = n0 / 16 + rbl;
-        const uint8_t *tp = wbase + ((long long)(rb * p.ntile_k + ks) * NM + m) * 576;
-        uint32_t wv[WPT];
-#pragma unroll
-        for (int v = 0; v < WPT; v += 4) {
-          const uint4 x = __ldg(reinterpret_cast<const uint4 *>(tp) + (w0 + v) / 4);
-          wv[v] = x.x;
-          wv[v + 1] = x.y;
-          wv[v + 2] = x.z;
-          wv[v + 3] = x.w;
-        }
-        const uint32_t dst = sb + m * TILE_B;
-#pragma unroll
-        for (int v = 0; v < WPT; ++v) {
-          const int wi = w0 + v, ln = wi >> 2, word = wi & 3;
-          const int g = ln >> 2, tig = ln & 3;
-          const uint2 sc = __ldg(reinterpret_cast<const uint2 *>(tp + 512) + g);
-          const uint32_t sv = (word >> 1) ? sc.y : sc.x;  // group of this k-step
-          dequant_q4_word(wv[v], h2_dup(sv, false), h2_dup(sv, true), dst, rbl * 16 + g,
-                          kb_step(word, tig));
+  const int items = ntiles * nslices;
+  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_AL; };
+  auto stage_b = [&](uint32_t st) { return stage0 + st * C::STAGE_AL + C::TILE_A; };
+  auto stage_c = [&](uint32_t st) { return stage0 + st * C::STAGE_AL + C::TILE_A + NM * C::TILE_B; };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
+  auto give_up = [&]() {
+    *reinterpret_cast<volatile int *>(&s_abort) = 1;
+    atomicOr(p.status, kErrTimeout);
+  };
+
+  if (wid == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x) {
+        const PfTile tile = p.tiles[item / nslices];
+        const int rb0 = (item % nslices) * (kPfBN / 16);
+        const uint8_t *wbase = tile.w + p.region_off;
+        for (int ks = 0; ks < nsteps; ++ks, ++it) {
+          const uint32_t st = it % S, use = it / S;
+          if (use > 0 && !mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1)) {
+            give_up();
+            break;
+          }
+          const uint32_t bar = smem_addr(&s_full[st]);
+          mbar_expect_tx(bar, C::TILE_A + C::CODES);
+          tma_load_2d(stage_a(st), &amap, ks * kPfBK, tile.row0, bar);
+          for (int r = 0; r < 8; ++r)
+            bulk_g2s(stage_c(st) + r * NM * 576,
+                     wbase + ((long long)(rb0 + r) * p.ntile_k + ks) * NM * 576, NM * 576, bar);
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
+    }
+  } else if (wid == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, kPfBN);
+      uint32_t it = 0, ii = 0;
+      for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x, ++ii) {
+        const uint32_t buf = ii & 1, acc = tmem + buf * C::ACC_COLS;
+        if (ii >= 2 && !mbar_wait_bounded(smem_addr(&s_acce[buf]), ((ii >> 1) - 1) & 1)) {
+          give_up();
+          break;
+        }
         tc_fence_after();
-        if (!mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
-          atomicOr(p.status, kErrTimeout);
-        } else {
+        bool ok = true;
+        for (int ks = 0; ks < nsteps; ++ks, ++it) {
+          const uint32_t st = it % S, use = it / S;
+          if (!mbar_wait_bounded(smem_addr(&s_deq[st]), use & 1) ||
+              !mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kPfBK / 16; ++kk) {
-            const uint64_t da = umma_desc_sw128(sa + kk * 32);
+            const uint64_t da = umma_desc_sw128(stage_a(st) + kk * 32);
 #pragma unroll
             for (int m = 0; m < NM; ++m)
-              umma_f16(tmem + m * 128, da, umma_desc_sw128(sb + m * TILE_B + kk * 32), IDESC,
-                       (ks | kk) != 0);
+              umma_f16(acc + m * kPfBN, da, umma_desc_sw128(stage_b(st) + m * C::TILE_B + kk * 32),
+                       IDESC, (ks | kk) != 0);
           }
+          umma_commit(smem_addr(&s_empty[st]));
         }
-        umma_commit(smem_addr(&s_empty[st]));
-        if (ks == nsteps - 1) umma_commit(smem_addr(&s_acc));
+        if (!ok) {
+          give_up();
+          break;
+        }
+        umma_commit(smem_addr(&s_accf[buf]));
       }
+      // every committed MMA must be complete before TMEM is released
+      if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_empty[(it - 1) % S]), ((it - 1) / S) & 1);
     }
-    if (!ok) break;
-    // epilogue: accumulators -> registers -> global
-    if (__syncthreads_or(!mbar_wait_bounded(smem_addr(&s_acc), acc_ph))) {
-      ok = false;
-      break;
-    }
-    acc_ph ^= 1u;
-    tc_fence_after();
-    {
-      const int quarter = wid & 3, half = wid >> 2;
-      const int r = quarter * 32 + lane;  // tile row = TMEM lane
-      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+  } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = wid & 3, r = quarter * 32 + lane;  // tile row = TMEM lane
+    uint32_t ii = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++ii) {
+      const uint32_t buf = ii & 1;
+      const bool ok = mbar_wait_bounded(smem_addr(&s_accf[buf]), (ii >> 1) & 1);
+      if (__any_sync(0xffffffffu, !ok) || aborted()) {
+        if (lane == 0) give_up();
+        break;
+      }
+      tc_fence_after();
+      const PfTile tile = p.tiles[item / nslices];
+      const int n0 = (item % nslices) * kPfBN;
+      const uint32_t lane_addr = tmem + buf * C::ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+      for (int c0 = 0; c0 < kPfBN; c0 += 32) {
         float g[32];
         tmem_ld32(lane_addr + c0, g);
         if constexpr (GATED) {
           float u[32];
-          tmem_ld32(lane_addr + 128 + c0, u);
+          tmem_ld32(lane_addr + kPfBN + c0, u);
           if (r < tile.rows) {
             uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
 #pragma unroll
@@ -477,21 +597,57 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(smem_addr(&s_acce[buf]));
     }
-    tc_fence_before();
-    __syncthreads();  // TMEM read before the next item's first MMA overwrites it
-    tc_fence_after();
-  }
-  if (!ok && tid == 0) atomicOr(p.status, kErrTimeout);
-  // drain: every committed MMA group must be complete before TMEM is freed
-  if (tid == 0 && it > 0) {
-    const uint32_t last = it - 1;
-    (void)mbar_wait_bounded(smem_addr(&s_empty[last % S]), (last / S) & 1);
+  } else if (wid >= kPfDeqWarp0) {
+    // ------------------------------------------------------------ dequantise
+    const int dt = tid - kPfDeqWarp0 * 32;  // 0..255
+    constexpr int WPT = 8 * NM * 128 / 256;  // code words per thread
+    const int q = dt / (128 / WPT);          // (row block, matrix) tile of this thread
+    const int rbl = q / NM, m = q % NM;
+    const int w0 = (dt % (128 / WPT)) * WPT; // first word (lane * 4 + word)
+    uint32_t it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      for (int ks = 0; ks < nsteps; ++ks, ++it) {
+        const uint32_t st = it % S, use = it / S;
+        const bool got = mbar_wait_bounded(smem_addr(&s_full[st]), use & 1);
+        if (__any_sync(0xffffffffu, !got) || aborted()) {
+          if (lane == 0) give_up();
+          ok = false;
+          break;
+        }
+        const uint32_t tsm = stage_c(st) + (rbl * NM + m) * 576;  // this thread's code tile
+        uint32_t wv[WPT];
+#pragma unroll
+        for (int v = 0; v < WPT; v += 4) {
+          const uint4 x = lds_u4(tsm + (w0 + v) * 4);
+          wv[v] = x.x;
+          wv[v + 1] = x.y;
+          wv[v + 2] = x.z;
+          wv[v + 3] = x.w;
+        }
+        const uint32_t dst = stage_b(st) + m * C::TILE_B;
+#pragma unroll
+        for (int v = 0; v < WPT; ++v) {
+          const int wi = w0 + v, ln = wi >> 2, word = wi & 3;
+          const int g = ln >> 2, tig = ln & 3;
+          const uint2 sc = lds_u2(tsm + 512 + g * 8);
+          const uint32_t sv = (word >> 1) ? sc.y : sc.x;  // group of this k-step
+          dequant_q4_word(wv[v], h2_dup(sv, false), h2_dup(sv, true), dst, rbl * 16 + g,
+                          kb_step(word, tig));
+        }
+        fence_proxy_async_smem();  // the tensor core reads B through the async proxy
+        mbar_arrive(smem_addr(&s_deq[st]));
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (wid == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+  if (wid == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
   pdl_launch_dependents();
 }
 
