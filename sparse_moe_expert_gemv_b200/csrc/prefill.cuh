@@ -376,28 +376,48 @@ MOE_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
   return r;
 }
 
-// Dequantise one 32-bit code word of a repacked Q4 tile into the swizzled
-// fp16 B tile.  The word of lane (g, tig), k-step st holds rows r0 = 16 rb +
-// g and r1 = r0 + 8, reduction columns kb .. kb+3 (kb = kb_step(st, tig)):
-// nibbles at bits 0/16 and 8/24 are row r0's columns (kb, kb+1) and
-// (kb+2, kb+3), bits 4/20 and 12/28 row r1's.  A nibble at bit 0 of an fp16
-// half over 0x6400 is 1024 + c; at bit 4 over 0x5400 it is 64 + c; one
-// subtraction gives c - 8 exactly and one multiplication by the group's
-// fp16 scale rounds once.
-MOE_DEV void dequant_q4_word(uint32_t w, uint32_t s0, uint32_t s1, uint32_t dst_s, int r0, int kb) {
-  const uint32_t w8 = w >> 8;
+// One code-word pair of a k-step pair: rows r0 (fp16 halves at nibble bits
+// 0/16 and 8/24) and r1 (bits 4/20 and 12/28), columns kb .. kb+7 from words
+// wa (kb .. kb+3) and wb (kb+4 .. kb+7).
+MOE_DEV void dq_pair(uint32_t wa, uint32_t wb, uint32_t s0, uint32_t s1, uint4 &row0, uint4 &row1) {
   const uint32_t c1032 = 0x64086408u, c72 = 0x54805480u;  // fp16 1032.0, 72.0
-  const uint32_t a0 = hmul2(hsub2(lop3_and_or(w, 0x000F000Fu, 0x64006400u), c1032), s0);
-  const uint32_t a2 = hmul2(hsub2(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), c1032), s0);
-  const uint32_t b0 = hmul2(hsub2(lop3_and_or(w, 0x00F000F0u, 0x54005400u), c72), s1);
-  const uint32_t b2 = hmul2(hsub2(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), c72), s1);
-  // 128-byte swizzle: row r at (r / 8) * 1024 + (r % 8) * 128, 16-byte chunk c -> c ^ (r % 8)
+  const uint32_t a8 = wa >> 8, b8 = wb >> 8;
+  row0.x = hmul2(hsub2(lop3_and_or(wa, 0x000F000Fu, 0x64006400u), c1032), s0);
+  row0.y = hmul2(hsub2(lop3_and_or(a8, 0x000F000Fu, 0x64006400u), c1032), s0);
+  row0.z = hmul2(hsub2(lop3_and_or(wb, 0x000F000Fu, 0x64006400u), c1032), s0);
+  row0.w = hmul2(hsub2(lop3_and_or(b8, 0x000F000Fu, 0x64006400u), c1032), s0);
+  row1.x = hmul2(hsub2(lop3_and_or(wa, 0x00F000F0u, 0x54005400u), c72), s1);
+  row1.y = hmul2(hsub2(lop3_and_or(a8, 0x00F000F0u, 0x54005400u), c72), s1);
+  row1.z = hmul2(hsub2(lop3_and_or(wb, 0x00F000F0u, 0x54005400u), c72), s1);
+  row1.w = hmul2(hsub2(lop3_and_or(b8, 0x00F000F0u, 0x54005400u), c72), s1);
+}
+
+// Dequantise the four code words of one lane (g, tig) of a repacked Q4 tile
+// into the swizzled fp16 B tile.  Word st of the lane holds reduction columns
+// kb_step(st, tig) .. +3 of rows r0 = 16 rb + g and r0 + 8, so words 0 and 1
+// fill 16-byte chunk tig of both rows (group 0) and words 2 and 3 chunk
+// 4 + tig (group 1); sc holds the rows' scales of the two groups.  Lanes
+// with odd g store their group-1 chunk first: in each store instruction the
+// eight lanes of a wavefront (rows g, g+1 of one tile, tig 0..3) then cover
+// all eight swizzled 16-byte positions of the 128-byte bank window.
+MOE_DEV void dequant_q4_lane(uint4 w, uint2 sc, uint32_t dst_s, int r0, int g, int tig) {
   const int r1 = r0 + 8;
-  const uint32_t ch = (uint32_t)(kb >> 3), sub = (uint32_t)(kb & 7) * 2;
-  const uint32_t o0 = (uint32_t)(r0 >> 3) * 1024 + (uint32_t)(r0 & 7) * 128 + ((ch ^ (r0 & 7)) << 4) + sub;
-  const uint32_t o1 = (uint32_t)(r1 >> 3) * 1024 + (uint32_t)(r1 & 7) * 128 + ((ch ^ (r1 & 7)) << 4) + sub;
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst_s + o0), "r"(a0), "r"(a2) : "memory");
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst_s + o1), "r"(b0), "r"(b2) : "memory");
+  const uint32_t base0 = dst_s + (uint32_t)(r0 >> 3) * 1024 + (uint32_t)(r0 & 7) * 128;
+  const uint32_t base1 = dst_s + (uint32_t)(r1 >> 3) * 1024 + (uint32_t)(r1 & 7) * 128;
+  uint4 a0, b0, a1, b1;
+  dq_pair(w.x, w.y, h2_dup(sc.x, false), h2_dup(sc.x, true), a0, b0);  // group 0
+  dq_pair(w.z, w.w, h2_dup(sc.y, false), h2_dup(sc.y, true), a1, b1);  // group 1
+  const bool odd = g & 1;
+  const uint32_t cf = (uint32_t)((odd ? 4 : 0) + tig), cs = (uint32_t)((odd ? 0 : 4) + tig);
+  const uint4 f0 = odd ? a1 : a0, s0 = odd ? a0 : a1, f1 = odd ? b1 : b0, s1 = odd ? b0 : b1;
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base0 + ((cf ^ (r0 & 7)) << 4)),
+               "r"(f0.x), "r"(f0.y), "r"(f0.z), "r"(f0.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base0 + ((cs ^ (r0 & 7)) << 4)),
+               "r"(s0.x), "r"(s0.y), "r"(s0.z), "r"(s0.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base1 + ((cf ^ (r1 & 7)) << 4)),
+               "r"(f1.x), "r"(f1.y), "r"(f1.z), "r"(f1.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base1 + ((cs ^ (r1 & 7)) << 4)),
+               "r"(s1.x), "r"(s1.y), "r"(s1.z), "r"(s1.w) : "memory");
 }
 
 struct PfGemmParams {
@@ -602,11 +622,11 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     }
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
-    const int dt = tid - kPfDeqWarp0 * 32;  // 0..255
-    constexpr int WPT = 8 * NM * 128 / 256;  // code words per thread
-    const int q = dt / (128 / WPT);          // (row block, matrix) tile of this thread
-    const int rbl = q / NM, m = q % NM;
-    const int w0 = (dt % (128 / WPT)) * WPT; // first word (lane * 4 + word)
+    // warp -> TPT (row block, matrix) code tiles, lane -> the tile's lane:
+    // contiguous 16-byte code reads, conflict-free stores (dequant_q4_lane)
+    const int dw = wid - kPfDeqWarp0;        // 0..7
+    constexpr int TPT = 8 * NM / 8;          // tiles per warp: 2 (gate/up) or 1 (down)
+    const int g = lane >> 2, tig = lane & 3;
     uint32_t it = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
@@ -618,25 +638,12 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t tsm = stage_c(st) + (rbl * NM + m) * 576;  // this thread's code tile
-        uint32_t wv[WPT];
 #pragma unroll
-        for (int v = 0; v < WPT; v += 4) {
-          const uint4 x = lds_u4(tsm + (w0 + v) * 4);
-          wv[v] = x.x;
-          wv[v + 1] = x.y;
-          wv[v + 2] = x.z;
-          wv[v + 3] = x.w;
-        }
-        const uint32_t dst = stage_b(st) + m * C::TILE_B;
-#pragma unroll
-        for (int v = 0; v < WPT; ++v) {
-          const int wi = w0 + v, ln = wi >> 2, word = wi & 3;
-          const int g = ln >> 2, tig = ln & 3;
-          const uint2 sc = lds_u2(tsm + 512 + g * 8);
-          const uint32_t sv = (word >> 1) ? sc.y : sc.x;  // group of this k-step
-          dequant_q4_word(wv[v], h2_dup(sv, false), h2_dup(sv, true), dst, rbl * 16 + g,
-                          kb_step(word, tig));
+        for (int l = 0; l < TPT; ++l) {
+          const int q = dw * TPT + l, rbl = q / NM, m = q % NM;   // (row block, matrix) tile
+          const uint32_t tsm = stage_c(st) + q * 576;
+          dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8),
+                          stage_b(st) + m * C::TILE_B, rbl * 16 + g, g, tig);
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
         mbar_arrive(smem_addr(&s_deq[st]));
