@@ -89,10 +89,15 @@ MOE_DEV bool wait_flag(const unsigned long long *f, unsigned long long epoch) {
 }
 
 // ------------------------------------------------ shared-memory carve
-// Byte offsets from the dynamic shared-memory base.  The weight ring of
-// every warp comes first (offset 0).
+// Byte offsets from the dynamic shared-memory base: tables first, then the
+// warps' weight rings, then the staging area (contiguous with the rings, so
+// a wide window can span both while the rings are still idle).
 struct DecSmem {
-  int bars;          // ring mbarriers of every warp, then the window and staging barriers
+  int ring;          // the warps' weight rings (directly before the staging area)
+  int win;           // phase 1 window rows: the staging area, or ring + staging for wide windows
+  int restage;       // 1: after routing each CTA re-stages only its gate/up jobs' token rows
+  int rowmap;        // int [T]: staging row of token t for the gate/up pass, or -1 (global)
+  int bars;          // ring mbarriers of every warp, then the window, staging and restage barriers
   int slot;          // int [E]      residency slots of this layer
   int mask;          // u32 [E]      token set of every expert
   int cnt;           // int [E+1]    per expert (jobs << 16 | tokens), then its exclusive scan
@@ -115,11 +120,11 @@ struct DecSmem {
 MOE_HOST_DEV_INLINE int dec_align(int x, int a) { return (x + a - 1) / a * a; }
 
 // The carve for one launch shape; ring = bytes of the warps' rings.  The
-// caller checks T * rsh <= stage_bytes.
+// caller checks T * rsh <= kDecSmem - win.
 inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, int E, int k,
                           int grid, int group) {
   DecSmem L{};
-  int off = ring;
+  int off = 0;
   auto carve = [&](int bytes, int align) {
     off = dec_align(off, align);
     const int at = off;
@@ -128,7 +133,8 @@ inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, i
   };
   const int P = T * k;
   L.max_jobs = P + (T + chunk - 1) / chunk;
-  L.bars = carve((warps * kRingD + 2) * 8, 8);
+  L.bars = carve((warps * kRingD + 3) * 8, 8);
+  L.rowmap = carve(T * 4, 16);
   L.slot = carve(E * 4, 16);
   L.mask = carve(E * 4, 16);
   L.cnt = carve((E + 1) * 4, 16);
@@ -150,10 +156,13 @@ inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, i
   L.hd = carve(L.hd_rows * L.ngf * 4, 16);
   L.hand = carve(warps * 32 * kHandFloats * 4, 16);
   L.hflag = carve(warps * 8, 8);
+  L.ring = carve(ring, 128);
   L.stage = carve(0, 128);
   L.stage_bytes = kDecSmem - L.stage;
   L.rsh = 2 * d + 64;
   L.rsa = 2 * f + 64;
+  L.restage = T * L.rsh > L.stage_bytes;
+  L.win = L.restage ? L.ring : L.stage;
   L.npl = E <= 128 ? 4 : E <= 512 ? 16 : 32;
   return L;
 }
@@ -172,6 +181,7 @@ struct DecodeParams {
   const uint8_t *arena, *pool, *shared;
   long long expert_bytes, p1_bytes;
   float *logits;        // [T, E]
+  uint16_t *hbuf;       // bf16 [T, d]: the normalised window (wide windows with RMSNorm)
   uint16_t *abuf;       // bf16 [T*k + T, f]
   float *ybuf;          // fp32 [T*k + T, d]
   float *ws;            // stream-K partial sums [warps of the grid][32][16]
@@ -414,12 +424,14 @@ MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, int ubase, i
   return true;
 }
 
-// Gate/up pass over this warp's units.  B rows are the window's token rows,
-// all staged in shared memory (row stride rsh) at stage_g.
+// Gate/up pass over this warp's units.  B rows are the window's token rows:
+// token t at staging row s_rowmap[t] (row stride rsh) at stage_g, or in
+// global memory (gsrc) when s_rowmap[t] < 0.
 template <int FMT, int NTM>
 MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, int u0, int u1,
                           const DecodeParams &p, const int *s_plist, const int *s_jbeg,
-                          const int *s_jn, const unsigned char *stage_g, const float *s_hg) {
+                          const int *s_jn, const unsigned char *stage_g, const float *s_hg,
+                          const int *s_rowmap, const uint16_t *gsrc) {
   const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
   const int P = p.T * p.k;
   if (u1 <= u0) return true;
@@ -442,7 +454,9 @@ MOE_DEV bool decode_gated(WarpRing &r, const Phase &ph, const SKCtx &sk, int u0,
       if (ni < n) {
         const int pair = s_plist[beg + ni];
         const int tok = pair < P ? pair / p.k : pair - P;
-        br.row[nt] = reinterpret_cast<const uint16_t *>(stage_g + (size_t)tok * p.sm.rsh);
+        const int sr = s_rowmap[tok];
+        br.row[nt] = sr >= 0 ? reinterpret_cast<const uint16_t *>(stage_g + (size_t)sr * p.sm.rsh)
+                             : gsrc + (long long)tok * p.d;
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -572,17 +586,21 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   constexpr float kSumScale = FMT == 1 ? -136.f : 1.f;  // see ItemRun::tile
   const uint32_t stage_s = smem_addr(smem + L.stage);
   const unsigned char *stage_g = smem + L.stage;
+  const uint32_t win_s = smem_addr(smem + L.win);
+  unsigned char *win_g = smem + L.win;
+  int *s_rowmap = reinterpret_cast<int *>(smem + L.rowmap);
   const uint32_t bars = smem_addr(smem + L.bars);
-  const uint32_t h_bar = bars + WARPS * kRingD * 8, st_bar = h_bar + 8;
+  const uint32_t h_bar = bars + WARPS * kRingD * 8, st_bar = h_bar + 8, rs_bar = h_bar + 16;
 
   MOE_TRACE(kTrRouteStart);
   WarpRing r;
-  ring_init(r, smem_addr(smem) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT);
+  ring_init(r, smem_addr(smem + L.ring) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT);
   if (lane == 0) {
     for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, 1);
     if (wid == 0) {
       mbar_init(h_bar, 1);
       mbar_init(st_bar, 1);
+      mbar_init(rs_bar, 1);
     }
     fence_mbar_init();
   }
@@ -615,7 +633,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   if (tid == 0) {
     mbar_expect_tx(h_bar, (uint32_t)T * d * 2);
     for (int t = 0; t < T; ++t)
-      bulk_g2s(stage_s + (uint32_t)t * L.rsh, p.x + (long long)t * d, (uint32_t)d * 2, h_bar);
+      bulk_g2s(win_s + (uint32_t)t * L.rsh, p.x + (long long)t * d, (uint32_t)d * 2, h_bar);
   }
   if (__syncthreads_or(!mbar_wait_bounded(h_bar, 0))) {
     if (tid == 0) atomicOr(p.status, kErrTimeout);
@@ -623,7 +641,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   }
   if (p.use_norm) {  // fp32 sum of squares, IEEE sqrt and divide, bf16 RNE
     for (int t = wid; t < T; t += WARPS) {
-      uint16_t *hr = reinterpret_cast<uint16_t *>(smem + L.stage + (long long)t * L.rsh);
+      uint16_t *hr = reinterpret_cast<uint16_t *>(win_g + (long long)t * L.rsh);
       float ss = 0.f;
       for (int i = lane * 4; i < d; i += 128) {
         const uint2 v = *reinterpret_cast<const uint2 *>(hr + i);
@@ -647,18 +665,21 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
         v.x = o[0] | ((uint32_t)o[1] << 16);
         v.y = o[2] | ((uint32_t)o[3] << 16);
         *reinterpret_cast<uint2 *>(hr + i) = v;
+        // wide windows re-stage rows after routing: CTA 0 publishes the
+        // normalised rows (visible to every CTA after the first barrier)
+        if (L.restage && blockIdx.x == 0) *reinterpret_cast<uint2 *>(p.hbuf + (long long)t * d + i) = v;
       }
     }
     __syncthreads();
   }
   // group sums of the window rows for the gate/up pass (read after the
   // barriers below)
-  group_sums(stage_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
+  group_sums(win_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
   for (int task = wid, it = 0; task < ntask; task += WARPS, ++it) {
     const int rr = task / QP, q = task - rr * QP, e = blockIdx.x * RPC + rr;
     if (e >= E) continue;
     const float4 *wr = reinterpret_cast<const float4 *>(p.W + (long long)e * d) + q * CPP * 32 + lane;
-    const uint32_t hcol = stage_s + 2u * (uint32_t)(q * CPP * 128 + lane * 4);
+    const uint32_t hcol = win_s + 2u * (uint32_t)(q * CPP * 128 + lane * 4);
     for (int t0 = 0; t0 < T; t0 += 8) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -711,11 +732,54 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   // ---------------- phase 3: gate/up
   const Phase ph1 = make_phase(s_jptr, f, d, CG::TK, CG::STRIDE, 0);
   const SKCtx sk1 = sk_make(n_jobs * ph1.RB * ph1.UPI, W, gw, ep1, p.ws, p.flags, s_hand, s_hflag, WARPS);
+  // Token rows for the gate/up B operand.  A window that fits the staging
+  // area stays there (row t at staging row t).  A wide window was staged
+  // over the rings and the staging area; now that the rings are needed, the
+  // CTA copies only the tokens of its own gate/up jobs into the staging
+  // area (as many as fit), and reads any others from global memory.
+  const uint16_t *gsrc = p.use_norm ? p.hbuf : p.x;
+  if (!L.restage) {
+    for (int t = tid; t < T; t += blockDim.x) s_rowmap[t] = t;
+  } else {
+    for (int t = tid; t < T; t += blockDim.x) s_rowmap[t] = -1;
+    __syncthreads();
+    if (tid == 0) {
+      const int c0 = sk_start(sk1, blockIdx.x * WARPS), c1 = sk_start(sk1, (blockIdx.x + 1) * WARPS);
+      const int cap = L.stage_bytes / L.rsh, P = T * k;
+      int rows = 0;
+      if (c1 > c0) {
+        const int jf = c0 / ph1.UPI / ph1.RB, jl = (c1 - 1) / ph1.UPI / ph1.RB;
+        for (int j = jf; j <= jl; ++j)
+          for (int i = 0; i < s_jn[j]; ++i) {
+            const int pr = s_plist[s_jbeg[j] + i], tok = pr < P ? pr / k : pr - P;
+            if (s_rowmap[tok] < 0 && rows < cap) s_rowmap[tok] = rows++;
+          }
+      }
+      // the normalised rows came from generic stores before the first barrier;
+      // the window area was last read by this CTA's generic loads
+      fence_proxy_async_global();
+      fence_proxy_async_smem();
+      mbar_expect_tx(rs_bar, (uint32_t)rows * d * 2);
+      for (int t = 0; t < T; ++t)
+        if (s_rowmap[t] >= 0)
+          bulk_g2s(stage_s + (uint32_t)s_rowmap[t] * L.rsh, gsrc + (long long)t * d, (uint32_t)d * 2,
+                   rs_bar);
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(rs_bar, 0))) {
+      if (tid == 0) atomicOr(p.status, kErrTimeout);
+      return;
+    }
+  }
+  __syncthreads();
   {
     const int u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1), i0 = u0 / ph1.UPI;
     ring_start(r, ph1, i0 / ph1.RB, i0 % ph1.RB, u0 - i0 * ph1.UPI, u1 - u0, 1);
-    if (lane == 0) ring_prologue(r, ph1);
-    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg)) {
+    if (lane == 0) {
+      fence_proxy_async_smem();  // a wide window occupied the rings until now
+      ring_prologue(r, ph1);
+    }
+    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg, s_rowmap,
+                                gsrc)) {
       if (lane == 0) atomicOr(p.status, kErrTimeout);
       ring_drain(r);
     }

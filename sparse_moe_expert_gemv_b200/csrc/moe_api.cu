@@ -374,7 +374,8 @@ bool use_decode_kernel(const moe_ctx *c, int T) {
   if (T < 1 || T > kDecMaxT || T * c->k > kDecMaxPairs || c->E > kDecMaxE || c->k > kDecMaxK)
     return false;
   const DecSmem L = decode_layout(c, T);
-  return L.stage_bytes > 0 && (long long)T * L.rsh <= L.stage_bytes && L.rsa <= L.stage_bytes;
+  return L.stage_bytes >= L.rsh && (long long)T * L.rsh <= kDecSmem - L.win &&
+         L.rsa <= L.stage_bytes;
 }
 
 cudaError_t launch_decode(moe_ctx *c, cudaStream_t s, const DecodeParams &dp) {
@@ -666,6 +667,7 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.expert_bytes = c->lay.expert_bytes;
     dp.p1_bytes = c->lay.p1_bytes;
     dp.logits = c->logits;
+    dp.hbuf = c->hbuf;
     dp.abuf = c->abuf;
     dp.ybuf = c->ybuf;
     dp.ws = c->dec_ws;

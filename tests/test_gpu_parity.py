@@ -138,6 +138,19 @@ def test_decode_q4_full_max_tokens(B, decode_q4):
     check(out, oracle_for(spec, x, sample), spec, sample)
 
 
+@pytest.mark.parametrize("T", [16, 32])
+def test_decode_q4_wide_windows(B, decode_q4, T):
+    """Windows of 16 and 32 tokens: the 32-token window no longer fits the
+    single-launch kernel's staging area next to the weight rings, so each
+    CTA re-stages only its own jobs' token rows after routing."""
+    ctx, spec = decode_q4
+    x = I.hidden_np(0, T, 2048, window=300 + T)
+    out = run(B, ctx, spec, x)
+    sample = np.array([0, T // 2, T - 1])
+    rel, ties = check(out, oracle_for(spec, x, sample), spec, sample)
+    print(f"T={T}: delta max-err/RMS {rel:.2e}, near ties {ties}")
+
+
 def test_deterministic(B, decode_q4):
     ctx, spec = decode_q4
     x = I.hidden_np(0, 4, 2048, window=5)
