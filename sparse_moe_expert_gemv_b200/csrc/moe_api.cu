@@ -541,17 +541,18 @@ bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
 
 cudaError_t setup_prefill() {
   cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg<true>::SMEM);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg::SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(prefill_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PfCfg<false>::SMEM);
+                             PfCfg::SMEM);
   return e;
 }
 
 // Prefill through the grouped tcgen05 GEMM: Q4 experts, more tokens than a
-// decode window, f and d multiples of the 128-column GEMM slice.
+// decode window, f a multiple of the gate/up item (128 features) and d of
+// the down item (256 features).
 bool use_prefill_gemm(const moe_ctx *c, int N) {
-  return c->pf && c->fmt == MOE_Q4_SYM_G32_F16 && N > kDecMaxT && c->d % kPfBN == 0 &&
+  return c->pf && c->fmt == MOE_Q4_SYM_G32_F16 && N > kDecMaxT && c->d % (2 * kPfBN) == 0 &&
          c->f % kPfBN == 0 && c->E <= kPfMaxE;
 }
 
@@ -607,7 +608,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   CUDA_TRY(c, prof_mark(c, 1, s));
   PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
                   nullptr, c->status};
-  const int smem1 = PfCfg<true>::SMEM, smem2 = PfCfg<false>::SMEM;
+  const int smem1 = PfCfg::SMEM, smem2 = PfCfg::SMEM;
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(c->n_sm);

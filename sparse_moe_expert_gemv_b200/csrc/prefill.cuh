@@ -436,51 +436,57 @@ constexpr int kPfGemmThreads = 512;  // 16 warps
 constexpr int kPfDeqWarp0 = 8;       // warps 8..15 dequantise
 constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM lane quarters 0..3)
 
-template <bool GATED>
+// Both passes run two 128-column accumulators per item: gate and up of the
+// same 128 features (gate/up pass), or two adjacent 128-feature slices
+// (down pass, 256 features per item).
 struct PfCfg {
-  static constexpr int NM = GATED ? 2 : 1;
-  static constexpr int S = GATED ? 3 : 5;                   // pipeline stages
+  static constexpr int SA = 5;                              // A + code stages (TMA ring)
   static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB
-  static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per matrix
-  static constexpr uint32_t CODES = 8 * NM * 576;           // 8 row blocks of repacked tiles
-  static constexpr uint32_t STAGE = TILE_A + NM * TILE_B + CODES;
-  static constexpr uint32_t STAGE_AL = (STAGE + 1023) / 1024 * 1024;
-  static constexpr uint32_t SMEM = S * STAGE_AL + 1024;     // + alignment slack
-  static constexpr uint32_t ACC_COLS = NM * kPfBN;          // TMEM columns per accumulator buffer
-  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered (256 or 512)
+  static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per accumulator
+  static constexpr uint32_t CODES = 16 * 576;               // 16 repacked code tiles
+  static constexpr uint32_t STAGE_A = (TILE_A + CODES + 1023) / 1024 * 1024;
+  static constexpr uint32_t BBUF = 2 * TILE_B;              // one B buffer (two tiles)
+  static constexpr uint32_t SMEM = SA * STAGE_A + 2 * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t ACC_COLS = 2 * kPfBN;           // TMEM columns per accumulator buffer
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
 
 // Grouped GEMM over the tile list, warp-specialised.  Work item = (128-row
-// tile, 128-column slice); persistent CTAs walk items blockIdx.x, +gridDim.x.
+// tile, output slice of 128 (gate/up) or 256 (down) features); persistent
+// CTAs walk items blockIdx.x, +gridDim.x.
 //  warp 0 lane 0   producer: per 64-column reduction step, the A tile (2-D
-//                  TMA, 128-byte swizzle) and the 8 repacked code tiles of
-//                  the slice (1-D bulk copies) into a free stage
-//  warps 8..15     dequantise the stage's codes into the swizzled fp16 B
-//                  tile(s), then arrive on the stage's B barrier
-//  warp 1 lane 0   issues the MMAs (m128n128k16, A and B from shared memory,
-//                  fp32 accumulator in TMEM) and commits each stage's
-//                  release; accumulators alternate between two TMEM buffers
-//  warps 4..7      drain an accumulator buffer (TMEM lanes = tile rows) while
-//                  the next item accumulates into the other one
+//                  TMA, 128-byte swizzle) and the 16 repacked code tiles of
+//                  the step (1-D bulk copies) into a free stage of a 5-deep ring
+//  warps 8..15     dequantise a stage's codes into one of two swizzled fp16
+//                  B buffers, then arrive on the buffer's barrier
+//  warp 1 lane 0   issues the MMAs (m128n256k16: both accumulators at once,
+//                  operands in shared memory, fp32 in TMEM) and commits the
+//                  release of the stage and of the B buffer; accumulator
+//                  pairs alternate between two TMEM buffers
+//  warps 4..7      drain an accumulator buffer (TMEM lanes = tile rows)
+//                  while the next item accumulates into the other one
 // Every wait is bounded; a timeout raises kErrTimeout and every role stops.
 template <bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
-  using C = PfCfg<GATED>;
-  constexpr int S = C::S, NM = C::NM;
+  using C = PfCfg;
+  constexpr int SA = C::SA;
+  constexpr int COLS = GATED ? kPfBN : 2 * kPfBN;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
-  __shared__ __align__(8) unsigned long long s_full[S], s_deq[S], s_empty[S], s_accf[2], s_acce[2];
+  __shared__ __align__(8) unsigned long long s_full[SA], s_empty[SA], s_bfull[2], s_bempty[2],
+      s_accf[2], s_acce[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
   const uint32_t base = smem_addr(pf_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
   if (tid == 0) {
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < SA; ++i) {
       mbar_init(smem_addr(&s_full[i]), 1);
-      mbar_init(smem_addr(&s_deq[i]), 256);
       mbar_init(smem_addr(&s_empty[i]), 1);
     }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_addr(&s_bfull[b]), 256);
+      mbar_init(smem_addr(&s_bempty[b]), 1);
       mbar_init(smem_addr(&s_accf[b]), 1);
       mbar_init(smem_addr(&s_acce[b]), 128);
     }
@@ -499,11 +505,11 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   const uint32_t tmem = s_tmem;
   pdl_wait();
   const int ntiles = ldcg_i32(p.n_tiles);
-  const int nslices = p.N / kPfBN, nsteps = p.K / kPfBK;
+  const int nslices = p.N / COLS, nsteps = p.K / kPfBK;
   const int items = ntiles * nslices;
-  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_AL; };
-  auto stage_b = [&](uint32_t st) { return stage0 + st * C::STAGE_AL + C::TILE_A; };
-  auto stage_c = [&](uint32_t st) { return stage0 + st * C::STAGE_AL + C::TILE_A + NM * C::TILE_B; };
+  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_A; };
+  auto stage_c = [&](uint32_t st) { return stage0 + st * C::STAGE_A + C::TILE_A; };
+  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::STAGE_A + b * C::BBUF; };
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
   auto give_up = [&]() {
     *reinterpret_cast<volatile int *>(&s_abort) = 1;
@@ -516,10 +522,10 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       uint32_t it = 0;
       for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x) {
         const PfTile tile = p.tiles[item / nslices];
-        const int rb0 = (item % nslices) * (kPfBN / 16);
+        const int rb0 = (item % nslices) * (COLS / 16);
         const uint8_t *wbase = tile.w + p.region_off;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
-          const uint32_t st = it % S, use = it / S;
+          const uint32_t st = it % SA, use = it / SA;
           if (use > 0 && !mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1)) {
             give_up();
             break;
@@ -527,16 +533,26 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           const uint32_t bar = smem_addr(&s_full[st]);
           mbar_expect_tx(bar, C::TILE_A + C::CODES);
           tma_load_2d(stage_a(st), &amap, ks * kPfBK, tile.row0, bar);
-          for (int r = 0; r < 8; ++r)
-            bulk_g2s(stage_c(st) + r * NM * 576,
-                     wbase + ((long long)(rb0 + r) * p.ntile_k + ks) * NM * 576, NM * 576, bar);
+          // code tile q = 2 r + m: row block r of accumulator m
+          if constexpr (GATED) {  // gate and up tiles of a row block are adjacent
+            for (int r = 0; r < 8; ++r)
+              bulk_g2s(stage_c(st) + r * 2 * 576, wbase + ((long long)(rb0 + r) * p.ntile_k + ks) * 2 * 576,
+                       2 * 576, bar);
+          } else {
+            for (int q = 0; q < 16; ++q)
+              bulk_g2s(stage_c(st) + q * 576,
+                       wbase + ((long long)(rb0 + (q & 1) * 8 + (q >> 1)) * p.ntile_k + ks) * 576, 576, bar);
+          }
         }
       }
     }
   } else if (wid == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, kPfBN);
+      // the two B tiles of a buffer are one 256-row K-major tile (rows 0..127
+      // feed accumulator columns 0..127, rows 128..255 columns 128..255):
+      // one m128n256k16 MMA per 16-column step
+      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, 2 * kPfBN);
       uint32_t it = 0, ii = 0;
       for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x, ++ii) {
         const uint32_t buf = ii & 1, acc = tmem + buf * C::ACC_COLS;
@@ -547,22 +563,19 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
-          const uint32_t st = it % S, use = it / S;
-          if (!mbar_wait_bounded(smem_addr(&s_deq[st]), use & 1) ||
+          const uint32_t st = it % SA, use = it / SA, bb = it & 1, buse = it >> 1;
+          if (!mbar_wait_bounded(smem_addr(&s_bfull[bb]), buse & 1) ||
               !mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kPfBK / 16; ++kk) {
-            const uint64_t da = umma_desc_sw128(stage_a(st) + kk * 32);
-#pragma unroll
-            for (int m = 0; m < NM; ++m)
-              umma_f16(acc + m * kPfBN, da, umma_desc_sw128(stage_b(st) + m * C::TILE_B + kk * 32),
-                       IDESC, (ks | kk) != 0);
-          }
+          for (int kk = 0; kk < kPfBK / 16; ++kk)
+            umma_f16(acc, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(bbuf(bb) + kk * 32), IDESC,
+                     (ks | kk) != 0);
           umma_commit(smem_addr(&s_empty[st]));
+          umma_commit(smem_addr(&s_bempty[bb]));
         }
         if (!ok) {
           give_up();
@@ -571,7 +584,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         umma_commit(smem_addr(&s_accf[buf]));
       }
       // every committed MMA must be complete before TMEM is released
-      if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_empty[(it - 1) % S]), ((it - 1) / S) & 1);
+      if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_empty[(it - 1) % SA]), ((it - 1) / SA) & 1);
     }
   } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
@@ -586,15 +599,15 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       }
       tc_fence_after();
       const PfTile tile = p.tiles[item / nslices];
-      const int n0 = (item % nslices) * kPfBN;
+      const int n0 = (item % nslices) * COLS;
       const uint32_t lane_addr = tmem + buf * C::ACC_COLS + ((uint32_t)(quarter * 32) << 16);
       for (int c0 = 0; c0 < kPfBN; c0 += 32) {
         float g[32];
         tmem_ld32(lane_addr + c0, g);
-        if constexpr (GATED) {
-          float u[32];
-          tmem_ld32(lane_addr + kPfBN + c0, u);
-          if (r < tile.rows) {
+        float u[32];
+        tmem_ld32(lane_addr + kPfBN + c0, u);
+        if (r < tile.rows) {
+          if constexpr (GATED) {
             uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -608,12 +621,14 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
               }
               dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-          }
-        } else {
-          if (r < tile.rows) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
+          } else {
+            float4 *d0 = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
+            float4 *d1 = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + kPfBN + c0);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) dst[v] = make_float4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
+            for (int v = 0; v < 8; ++v) {
+              d0[v] = make_float4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
+              d1[v] = make_float4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+            }
           }
         }
       }
@@ -622,31 +637,31 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     }
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
-    // warp -> TPT (row block, matrix) code tiles, lane -> the tile's lane:
-    // contiguous 16-byte code reads, conflict-free stores (dequant_q4_lane)
-    const int dw = wid - kPfDeqWarp0;        // 0..7
-    constexpr int TPT = 8 * NM / 8;          // tiles per warp: 2 (gate/up) or 1 (down)
+    // warp -> two code tiles (q = 2 dw, 2 dw + 1: row block dw of both
+    // accumulators), lane -> the tile's lane: contiguous 16-byte code
+    // reads, conflict-free stores (dequant_q4_lane)
+    const int dw = wid - kPfDeqWarp0;  // 0..7 = row block
     const int g = lane >> 2, tig = lane & 3;
     uint32_t it = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
       for (int ks = 0; ks < nsteps; ++ks, ++it) {
-        const uint32_t st = it % S, use = it / S;
-        const bool got = mbar_wait_bounded(smem_addr(&s_full[st]), use & 1);
+        const uint32_t st = it % SA, use = it / SA, bb = it & 1, buse = it >> 1;
+        bool got = mbar_wait_bounded(smem_addr(&s_full[st]), use & 1);
+        if (got && buse > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb]), (buse - 1) & 1);
         if (__any_sync(0xffffffffu, !got) || aborted()) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
 #pragma unroll
-        for (int l = 0; l < TPT; ++l) {
-          const int q = dw * TPT + l, rbl = q / NM, m = q % NM;   // (row block, matrix) tile
-          const uint32_t tsm = stage_c(st) + q * 576;
+        for (int m = 0; m < 2; ++m) {
+          const uint32_t tsm = stage_c(st) + (dw * 2 + m) * 576;
           dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8),
-                          stage_b(st) + m * C::TILE_B, rbl * 16 + g, g, tig);
+                          bbuf(bb) + m * C::TILE_B, dw * 16 + g, g, tig);
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
-        mbar_arrive(smem_addr(&s_deq[st]));
+        mbar_arrive(smem_addr(&s_bfull[bb]));
       }
     }
   }
