@@ -148,6 +148,18 @@ MOE_DEV void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
+// expect_tx + 1-D bulk copy issued by the calling lane only when `issue`;
+// every lane may execute it (predicated, no branch).
+MOE_DEV void bulk_g2s_hint_pred(bool issue, uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %5, 0;\n\t"
+      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %2;\n\t"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n\t}" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy), "r"((uint32_t)issue)
+      : "memory");
+}
 // One arrival (this thread) on an mbarrier.
 MOE_DEV void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");

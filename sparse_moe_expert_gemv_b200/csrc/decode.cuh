@@ -64,15 +64,16 @@ MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global
 // complete), so its n-th barrier completes when the counter reaches
 // base + n * gridDim.x: the arrival needs no reply.  Returns false if the
 // wait gave up.
+// The arrival is a release and the poll an acquire at gpu scope; both are
+// cumulative over the CTA's accesses ordered by the CTA barriers around
+// them, so no separate fences are needed.
 MOE_DEV bool grid_sync(unsigned long long *count, unsigned long long target) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     red_release_add_u64(count, 1ull);
     bool ok = false;
     for (uint32_t i = 0; !ok && i < (1u << 22); ++i) ok = ld_acquire_u64(count) >= target;
-    __threadfence();
     s_ok = ok;
   }
   __syncthreads();
@@ -376,8 +377,7 @@ MOE_DEV bool sk_item(WarpRing &r, const Phase &ph, const SKCtx &sk, int ubase, i
         __threadfence_block();
         *reinterpret_cast<volatile unsigned long long *>(sk.s_flag + (sk.gw - cta_w0)) = sk.epoch;
       } else {
-        __threadfence();
-        st_release_u64(sk.flags + sk.gw, sk.epoch);
+        st_release_u64(sk.flags + sk.gw, sk.epoch);  // release covers the lanes' stores (syncwarp)
       }
     }
     return true;
@@ -774,10 +774,9 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   {
     const int u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1), i0 = u0 / ph1.UPI;
     ring_start(r, ph1, i0 / ph1.RB, i0 % ph1.RB, u0 - i0 * ph1.UPI, u1 - u0, 1);
-    if (lane == 0) {
-      fence_proxy_async_smem();  // a wide window occupied the rings until now
-      ring_prologue(r, ph1);
-    }
+    if (lane == 0) fence_proxy_async_smem();  // a wide window occupied the rings until now
+    __syncwarp();
+    ring_prologue(r, ph1, lane);
     if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg, s_rowmap,
                                 gsrc)) {
       if (lane == 0) atomicOr(p.status, kErrTimeout);
@@ -795,7 +794,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     const int i0 = v0 / ph2.UPI;
     ring_start(r, ph2, i0 / ph2.RB, i0 % ph2.RB, v0 - i0 * ph2.UPI, v1 - v0, 1);
   }
-  if (lane == 0) ring_prologue(r, ph2);  // weights stream in while the grid syncs
+  ring_prologue(r, ph2, lane);  // weights stream in while the grid syncs
   if (!grid_sync(p.bar, (ep0 + 2) * G)) {
     ring_drain(r);
     if (tid == 0) atomicOr(p.status, kErrTimeout);

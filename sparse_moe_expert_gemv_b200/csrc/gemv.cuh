@@ -139,7 +139,7 @@ struct WarpRing {
   uint32_t data_s, bar_s, slot_stride;
   int u;             // slot of the next unit to consume
   uint32_t phase;    // its mbarrier parity
-  int inflight;      // units issued and not yet consumed (lane 0)
+  int inflight;      // units issued and not yet consumed
   int istep;
   UnitCursor ld;      // next unit to load into the ring
   uint64_t policy;   // L2 policy of the ring loads (evict first)
@@ -164,23 +164,24 @@ MOE_DEV void ring_start(WarpRing &r, const Phase &ph, int job, int rb, int unit,
   cursor_start(r.ld, ph, job, rb, unit, n);
 }
 
-// lane 0: issue the producer's next unit into slot `slot`.  The slot's
-// previous unit was read with ld.shared by every lane, and those reads are
-// ordered before this copy by the __syncwarp that precedes the call (the
+// Every lane: the producer's next unit into slot `slot`, issued by lane 0
+// alone (predicated, no divergent branch); every lane keeps the cursor.  The
+// slot's previous unit was read with ld.shared by every lane, and those reads
+// are ordered before this copy by the __syncwarp that precedes the call (the
 // values were consumed by then), as in a TMA pipeline's consumer release.
-MOE_DEV void ring_issue(WarpRing &r, const Phase &ph, int slot) {
+MOE_DEV void ring_issue_warp(WarpRing &r, const Phase &ph, int slot, int lane) {
   if (r.ld.rem <= 0) return;
   const uint32_t bytes = (uint32_t)(ph.tps * ph.stride);
-  const uint32_t bar = r.bar_s + 8 * slot;
-  mbar_expect_tx(bar, bytes);
-  bulk_g2s_hint(r.data_s + slot * r.slot_stride, r.ld.addr, bytes, bar, r.policy);
+  bulk_g2s_hint_pred(lane == 0, r.data_s + slot * r.slot_stride, r.ld.addr, bytes, r.bar_s + 8 * slot,
+                     r.policy);
   ++r.inflight;
   cursor_advance(r.ld, ph, r.istep);
 }
 
-// lane 0: fill the kRingD slots that follow the consumer position
-MOE_DEV void ring_prologue(WarpRing &r, const Phase &ph) {
-  for (int i = 0; i < kRingD; ++i) ring_issue(r, ph, (r.u + i) % kRingD);
+// Every lane: fill the kRingD slots that follow the consumer position
+// (lane 0 issues).
+MOE_DEV void ring_prologue(WarpRing &r, const Phase &ph, int lane) {
+  for (int i = 0; i < kRingD; ++i) ring_issue_warp(r, ph, (r.u + i) % kRingD, lane);
 }
 
 // After a failed wait (all lanes of the warp): wait, bounded, for the units
@@ -390,10 +391,8 @@ struct ItemRun {
         tile(slot_s + tt * C::STRIDE, lane, b, hv, acc);
       }
       __syncwarp();
-      if (lane == 0) {
-        --r.inflight;
-        ring_issue(r, ph, r.u);
-      }
+      --r.inflight;
+      ring_issue_warp(r, ph, r.u, lane);
       if (++r.u == kRingD) {
         r.u = 0;
         r.phase ^= 1u;
@@ -480,7 +479,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, GATED, NTM>::WARPS * 32, 1)
   // the previous kernel, so the down projection starts streaming before its
   // wait)
   ring_start(r, ph, first / RB, first % RB, 0, my_items * ph.UPI, C::WARPS);
-  if (lane == 0) ring_prologue(r, ph);
+  ring_prologue(r, ph, lane);
   if (!GATED) {
     pdl_wait();
     MOE_TRACE(kTrDownWaited);
