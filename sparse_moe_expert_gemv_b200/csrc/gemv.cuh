@@ -384,11 +384,20 @@ struct ItemRun {
       const bool ok = mbar_wait_bounded(r.bar_s + 8 * r.u, r.phase);
       if (__any_sync(0xffffffffu, !ok)) return false;  // warp-uniform
       const uint32_t slot_s = r.data_s + r.u * r.slot_stride;
-      for (int tt = 0; tt < ph.tps; ++tt) {
+      if (ph.tps == 2) {
+        // both tiles of the unit in one block of straight-line code, so the
+        // scheduler can overlap one tile's unpack with the other's mma chains
+        uint4 b0[NTA][NB], b1[NTA][NB];
+        float2 hv0[NTA][2], hv1[NTA][2];
+        load_b(b0, hv0, br, 2 * u, tig);
+        load_b(b1, hv1, br, 2 * u + 1, tig);
+        tile(slot_s, lane, b0, hv0, acc);
+        tile(slot_s + C::STRIDE, lane, b1, hv1, acc);
+      } else {
         uint4 b[NTA][NB];
         float2 hv[NTA][2];
-        load_b(b, hv, br, u * ph.tps + tt, tig);
-        tile(slot_s + tt * C::STRIDE, lane, b, hv, acc);
+        load_b(b, hv, br, u, tig);
+        tile(slot_s, lane, b, hv, acc);
       }
       __syncwarp();
       --r.inflight;
