@@ -67,17 +67,25 @@ MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global
 // The arrival is a release and the poll an acquire at gpu scope; both are
 // cumulative over the CTA's accesses ordered by the CTA barriers around
 // them, so no separate fences are needed.
-MOE_DEV bool grid_sync(unsigned long long *count, unsigned long long target) {
-  __shared__ int s_ok;
+// Split form: grid_arrive, then work that only touches this CTA's shared
+// memory, then grid_wait.
+MOE_DEV void grid_arrive(unsigned long long *count) {
   __syncthreads();
+  if (threadIdx.x == 0) red_release_add_u64(count, 1ull);
+}
+MOE_DEV bool grid_wait(unsigned long long *count, unsigned long long target) {
+  __shared__ int s_ok;
   if (threadIdx.x == 0) {
-    red_release_add_u64(count, 1ull);
     bool ok = false;
     for (uint32_t i = 0; !ok && i < (1u << 22); ++i) ok = ld_acquire_u64(count) >= target;
     s_ok = ok;
   }
   __syncthreads();
   return s_ok != 0;
+}
+MOE_DEV bool grid_sync(unsigned long long *count, unsigned long long target) {
+  grid_arrive(count);
+  return grid_wait(count, target);
 }
 
 // Bounded wait for a partial-sum flag to carry this barrier epoch.
@@ -672,9 +680,6 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     }
     __syncthreads();
   }
-  // group sums of the window rows for the gate/up pass (read after the
-  // barriers below)
-  group_sums(win_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
   for (int task = wid, it = 0; task < ntask; task += WARPS, ++it) {
     const int rr = task / QP, q = task - rr * QP, e = blockIdx.x * RPC + rr;
     if (e >= E) continue;
@@ -707,7 +712,10 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   MOE_TRACE(kTrRouteLogits);
   const unsigned long long G = gridDim.x, ep0 = s_bar0 / G;
   const unsigned long long ep1 = ep0 + 1;
-  if (!grid_sync(p.bar, ep1 * G)) {
+  grid_arrive(p.bar);
+  // group sums of the window rows for the gate/up pass, while the grid syncs
+  group_sums(win_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
+  if (!grid_wait(p.bar, ep1 * G)) {
     if (tid == 0) atomicOr(p.status, kErrTimeout);
     return;
   }
