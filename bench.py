@@ -397,7 +397,7 @@ def run_native(args, world, rank, local):
         },
         "e2e": {"value": world * tok / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": K * (1 if single else (7 if prefill else 5)),
+        "gpu_launches": K * (1 if single else (8 if prefill else 6)),
         "clocks": clocks,
     }
     B.moe_destroy(ctx)
@@ -518,7 +518,7 @@ def run_stack(args, world, rank, local):
                                  f"{E * D * 4} B router W per layer"},
         "e2e": {"value": world * T * K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": K * NL * (1 if single else 5),
+        "gpu_launches": K * NL * (1 if single else 6),
         "clocks": clocks,
     }
     B.moe_destroy(ctx)

@@ -183,9 +183,10 @@ constexpr int kRouterWarps = 4;
 constexpr int kRouterSmem = 48 * 1024;  // bytes of h staged per pass
 
 // One warp per expert row: the row of W stays in registers (d/32 floats per
-// lane, d <= 4096) and is dotted with every token's h, which the CTA stages
-// in shared memory a chunk of tokens at a time; fp32 accumulate, four tokens
-// in flight per warp.
+// lane, d <= 4096) and is dotted with the h rows of the CTA's token chunks
+// (chunks blockIdx.y, + gridDim.y, ...), which the CTA stages in shared
+// memory one chunk at a time; fp32 accumulate, four tokens in flight per
+// warp.
 template <int VPL>  // float4 vectors per lane = d / 128
 __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(RouterParams p) {
   extern __shared__ __align__(16) unsigned char rsm[];
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(Router
   pdl_wait();
   pdl_launch_dependents();
   const int tc = kRouterSmem / (2 * d);  // tokens per pass
-  for (int t0 = 0; t0 < p.T; t0 += tc) {
+  for (int t0 = blockIdx.y * tc; t0 < p.T; t0 += gridDim.y * tc) {
     const int nt = min(tc, p.T - t0);
     __syncthreads();
     const int n16 = nt * d / 8;  // 16-byte vectors, 8 loads in flight per thread

@@ -383,9 +383,22 @@ cudaError_t launch_decode(moe_ctx *c, cudaStream_t s, const DecodeParams &dp) {
   return launch(k, dim3(c->n_sm), dim3(GemvCfg<1, true, 1>::WARPS * 32), kDecSmem, s, dp);
 }
 
+// Top-k of every token, one warp per token over ceil(T / 16) CTAs: idx, w and
+// the per-block token masks.
+cudaError_t launch_pf_topk(moe_ctx *c, cudaStream_t s, const PfRouteParams &tp) {
+  const dim3 tg((tp.T + kPfTok - 1) / kPfTok), tb(kPfTok * 32);
+  if (c->E <= 128) return launch(prefill_topk_kernel<4>, tg, tb, 0, s, tp);
+  if (c->E <= 512) return launch(prefill_topk_kernel<16>, tg, tb, 0, s, tp);
+  return launch(prefill_topk_kernel<32>, tg, tb, 0, s, tp);
+}
+
+// Router logits: CTA (x, y) takes expert rows [4x, 4x + 4) and every
+// gridDim.y-th chunk of tokens from chunk y.
 cudaError_t launch_router(moe_ctx *c, cudaStream_t s, const RouterParams &rp) {
-  const dim3 grid((c->E + kRouterWarps - 1) / kRouterWarps), block(kRouterWarps * 32);
-  const size_t sm = (size_t)std::min(rp.T, kRouterSmem / (2 * c->d)) * c->d * 2;
+  const int tc = kRouterSmem / (2 * c->d);
+  const dim3 grid((c->E + kRouterWarps - 1) / kRouterWarps, std::min((rp.T + tc - 1) / tc, 64)),
+      block(kRouterWarps * 32);
+  const size_t sm = (size_t)std::min(rp.T, tc) * c->d * 2;
   switch (c->d / 128) {
     case 1: return launch(router_logits_kernel<1>, grid, block, sm, s, rp);
     case 2: return launch(router_logits_kernel<2>, grid, block, sm, s, rp);
@@ -498,7 +511,18 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
                   c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
                   c->logits};
   CUDA_TRY(c, launch_router(c, s, rp));
-  CUDA_TRY(c, launch_finish(c, s, fp));
+  if (T > kDecMaxT && c->pf_bmask) {
+    // many tokens: the top-k runs one warp per token across the grid, and
+    // the single routing CTA only buckets the selections and builds the jobs
+    PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4]};
+    CUDA_TRY(c, launch_pf_topk(c, s, tp));
+    FinishParams fb = fp;
+    fb.logits = nullptr;
+    fb.idx_in = fp.idx;
+    CUDA_TRY(c, launch_finish(c, s, fb));
+  } else {
+    CUDA_TRY(c, launch_finish(c, s, fp));
+  }
   if (h_out) *h_out = h;
   return MOE_OK;
 }
@@ -575,10 +599,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
                      dim3(256), 0, s, rp));
   const int blocks = (N + kPfTok - 1) / kPfTok;
   PfRouteParams tp{c->logits, N, E, k, c->idx, c->w, c->pf_bmask, &c->stats[4]};
-  const dim3 tg(blocks), tb(kPfTok * 32);
-  if (E <= 128) CUDA_TRY(c, launch(prefill_topk_kernel<4>, tg, tb, 0, s, tp));
-  else if (E <= 512) CUDA_TRY(c, launch(prefill_topk_kernel<16>, tg, tb, 0, s, tp));
-  else CUDA_TRY(c, launch(prefill_topk_kernel<32>, tg, tb, 0, s, tp));
+  CUDA_TRY(c, launch_pf_topk(c, s, tp));
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;
   sp.blocks = blocks;
@@ -601,10 +622,11 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   sp.stats = c->stats;
   sp.last = c->last;
   sp.status = c->status;
+  CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32), dim3(kPfColWarps * 32), 0, s, sp));
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
   PfScatterParams cp{c->idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
                      c->pf_row_of, c->pf_hg};
-  CUDA_TRY(c, launch(prefill_scatter_kernel, tg, tb, 0, s, cp));
+  CUDA_TRY(c, launch(prefill_scatter_kernel, dim3(blocks), dim3(kPfTok * 32), 0, s, cp));
   CUDA_TRY(c, prof_mark(c, 1, s));
   PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
                   nullptr, c->status};

@@ -8,8 +8,10 @@
 //
 //   prefill_topk_kernel     one warp per token: top-k + softmax; per block of
 //                           16 tokens, each expert's token set (a bitmask)
-//   prefill_scan_kernel     per expert: tokens per block of 16 (column scan),
-//                           the expert's first row in grouped order, and the
+//   prefill_colscan_kernel  per expert: each block of 16 tokens' first row
+//                           relative to the expert's (a scan down the
+//                           expert's column of block masks) and its tokens
+//   prefill_scan_kernel     the experts' first rows in grouped order and the
 //                           list of 128-row tiles (expert, first row, rows)
 //   prefill_scatter_kernel  pair -> row in grouped order (stable: ascending t
 //                           within an expert) and the gather of every pair's
@@ -81,8 +83,8 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
 struct PfScanParams {
   const unsigned short *bmask;  // [blocks][E]
   int blocks, E, T, k;
-  int *boff;                    // [blocks][E] first row of (block, expert) in grouped order
-  int *eoff;                    // [E + 1]
+  int *boff;                    // [blocks][E] first row of (block, expert) relative to the expert's
+  int *eoff;                    // [E + 1] token counts (colscan), then first rows (scan)
   const int *slot_of;           // residency table [L*E]
   int n_slots, layer;
   const uint8_t *arena, *pool, *shared;
@@ -96,9 +98,41 @@ struct PfScanParams {
   int *status;
 };
 
-// One CTA of 1024 threads.  Thread e walks its expert's column of block
-// masks (block order = token order, so rows stay in ascending t), then one
-// block scan gives the experts' first rows and first tiles.
+// Down each expert's column of block masks (block order = token order, so
+// rows stay in ascending t): every block's first row relative to the
+// expert's first row (boff), and the expert's token count (eoff[e], turned
+// into the expert's first row by prefill_scan_kernel).  A CTA takes 32
+// experts (one per lane) and its 16 warps contiguous ranges of blocks.
+constexpr int kPfColWarps = 16;
+__global__ void __launch_bounds__(kPfColWarps * 32) prefill_colscan_kernel(PfScanParams p) {
+  __shared__ int s_part[kPfColWarps][33];
+  pdl_wait();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (p.blocks + kPfColWarps - 1) / kPfColWarps;
+  const int b0 = min(p.blocks, wid * per), b1 = min(p.blocks, b0 + per);
+  int run = 0;
+  if (e < p.E) {
+#pragma unroll 8
+    for (int b = b0; b < b1; ++b) run += __popc(p.bmask[(long long)b * p.E + e]);
+  }
+  s_part[wid][lane] = run;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < wid; ++w) base += s_part[w][lane];
+  if (e < p.E) {
+    for (int b = b0; b < b1; ++b) {
+      p.boff[(long long)b * p.E + e] = base;
+      base += __popc(p.bmask[(long long)b * p.E + e]);
+    }
+    if (wid == kPfColWarps - 1) p.eoff[e] = base;  // all blocks: the expert's tokens
+  }
+  pdl_launch_dependents();
+}
+
+// One CTA of 1024 threads: one block scan over the experts' token counts
+// gives their first rows, another their first tiles; then the tile list,
+// with the residency lookup.
 __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
   __shared__ int s_cnt[2 * kPfMaxE + 2];
   __shared__ int s_red[32];
@@ -108,11 +142,7 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
   int *cnt = s_cnt, *tl = s_cnt + kPfMaxE + 1;
   if (tid < 3) s_hm[tid] = 0;
   for (int e = tid; e < p.E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < p.blocks; ++b) {
-      p.boff[(long long)b * p.E + e] = run;  // relative to the expert's first row
-      run += __popc(p.bmask[(long long)b * p.E + e]);
-    }
+    const int run = p.eoff[e];  // token count from prefill_colscan_kernel
     cnt[e] = run;
     tl[e] = (run + kPfBM - 1) / kPfBM;
   }
