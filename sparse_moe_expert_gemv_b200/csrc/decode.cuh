@@ -124,6 +124,9 @@ struct DecSmem {
   int rpc, qp;       // router rows per CTA, parts per row
   int max_jobs;
   int npl;           // logits per lane of the top-k warp
+  int tk_parts;      // warps per token of the split top-k (1: one warp per token)
+  int tk_npl;        // logits per lane of a split top-k part
+  int cand;          // u64 [warps][k + 1] the parts' candidates
 };
 
 MOE_HOST_DEV_INLINE int dec_align(int x, int a) { return (x + a - 1) / a * a; }
@@ -163,6 +166,19 @@ inline DecSmem dec_layout(int ring, int warps, int chunk, int T, int d, int f, i
   L.hg = carve(T * L.ngd * 4, 16);
   L.hd_rows = kMaxStagedJobs * chunk;
   L.hd = carve(L.hd_rows * L.ngf * 4, 16);
+  // split top-k: parts (a power of two) warps per token, each keeping k + 1
+  // candidates of E / parts logits, while T * parts <= warps and the merge
+  // sees at most 64 candidates
+  L.tk_parts = 1;
+  while (L.tk_parts * 2 * T <= warps && L.tk_parts * 2 * (k + 1) <= 64 && E / (L.tk_parts * 2) >= k + 1)
+    L.tk_parts *= 2;
+  {
+    const int per = (E + L.tk_parts - 1) / L.tk_parts;
+    L.tk_npl = 1;
+    while (L.tk_npl * 32 < per) L.tk_npl *= 2;
+    if (L.tk_npl > 8) L.tk_parts = 1;
+  }
+  L.cand = carve(warps * (k + 1) * 8, 16);
   L.hand = carve(warps * 32 * kHandFloats * 4, 16);
   L.hflag = carve(warps * 8, 8);
   L.ring = carve(ring, 128);
@@ -247,6 +263,32 @@ __device__ __noinline__ void decode_topk(const float *logits, int T, int E, int 
   }
 }
 
+// Top-k of every token with `parts` warps per token (warp_topk_part, then
+// warp_topk_merge by warp t): the same selections and weights as
+// decode_topk in fewer dependent rounds per warp.  All threads.
+template <int NPL>
+__device__ __noinline__ void decode_topk_split(const float *logits, int T, int E, int k, int parts,
+                                               int *s_idx, float *s_w, unsigned *s_mask,
+                                               unsigned long long *s_cand,
+                                               unsigned long long *near_ties) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int kk = k < E ? k + 1 : k, per = (E + parts - 1) / parts;
+  const int t = wid / parts, q = wid - t * parts;
+  if (t < T)
+    warp_topk_part<NPL>(logits + (long long)t * E, E, per, q, kk, lane, s_cand + (t * parts + q) * kk);
+  __syncthreads();
+  if (wid < T) {
+    int e;
+    float w;
+    warp_topk_merge(s_cand + wid * parts * kk, parts * kk, E, k, lane, e, w, near_ties);
+    if (lane < k) {
+      s_idx[wid * k + lane] = e;
+      s_w[wid * k + lane] = w;
+      atomicOr(&s_mask[e], 1u << wid);
+    }
+  }
+}
+
 // All threads of the CTA: the bucketing of the pairs by expert and the job
 // list.  Experts come in ascending id, each split into jobs of <= chunk
 // tokens in ascending t; one exclusive scan over the experts' packed
@@ -293,8 +335,9 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
     for (int b = 0; m; ++b) {
       const int t = __ffs(m) - 1;
       m &= m - 1;
-      int j = 0;
-      while (j < k - 1 && s_idx[t * k + j] != e) ++j;
+      int j = k - 1;  // the token's selection slot of e (independent loads)
+#pragma unroll 4
+      for (int jj = k - 2; jj >= 0; --jj) j = s_idx[t * k + jj] == e ? jj : j;
       s_plist[px + b] = t * k + j;
     }
     for (int c0 = 0; c0 < n; c0 += CH, ++jx) {
@@ -723,9 +766,19 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
 
   // ---------------- phase 2: routing (every CTA, redundantly)
   unsigned long long *near = blockIdx.x == 0 ? &p.stats[4] : nullptr;
-  if (L.npl == 4) decode_topk<4>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
-  else if (L.npl == 16) decode_topk<16>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
-  else decode_topk<32>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  unsigned long long *s_cand = reinterpret_cast<unsigned long long *>(smem + L.cand);
+  if (L.tk_parts > 1) {
+    if (L.tk_npl == 1) decode_topk_split<1>(p.logits, T, E, k, L.tk_parts, s_idx, s_w, s_mask, s_cand, near);
+    else if (L.tk_npl == 2) decode_topk_split<2>(p.logits, T, E, k, L.tk_parts, s_idx, s_w, s_mask, s_cand, near);
+    else if (L.tk_npl == 4) decode_topk_split<4>(p.logits, T, E, k, L.tk_parts, s_idx, s_w, s_mask, s_cand, near);
+    else decode_topk_split<8>(p.logits, T, E, k, L.tk_parts, s_idx, s_w, s_mask, s_cand, near);
+  } else if (L.npl == 4) {
+    decode_topk<4>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  } else if (L.npl == 16) {
+    decode_topk<16>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  } else {
+    decode_topk<32>(p.logits, T, E, k, WARPS, s_idx, s_w, s_mask, near);
+  }
   __syncthreads();
   MOE_TRACE(kTrRouteTopk);
   {

@@ -167,6 +167,67 @@ MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int 
   sel_w = ex / den;
 }
 
+// The kk best of a warp's packed values (lane + 32 i holds pk[i]; 0 =
+// empty), in descending order: lane j < kk returns the j-th, 0 if fewer
+// exist.  Same round as warp_topk, with the winner cleared by value (the
+// packed values are distinct).
+template <int NPL>
+MOE_DEV unsigned long long warp_top_packed(unsigned long long (&pk)[NPL], int kk, int lane) {
+  unsigned long long mine = 0ull;
+  for (int j = 0; j < kk; ++j) {
+    const unsigned long long best = tournament_max<NPL>(pk);
+    const uint32_t hi = (uint32_t)(best >> 32);
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, hi == wmax ? (uint32_t)best : 0u);
+    const unsigned long long win = ((unsigned long long)wmax << 32) | wlo;
+    if (lane == j) mine = win;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) pk[i] = pk[i] == win ? 0ull : pk[i];
+  }
+  return mine;
+}
+
+// Top-k of one token split over `parts` warps (part 1): warp q of the token
+// keeps the kk = k + 1 best of experts [q per, (q+1) per) as packed values
+// in cand[q][kk].  The union of the parts' k + 1 best holds the token's
+// k + 1 best, so the merge (warp_topk_merge) selects exactly what warp_topk
+// selects over all E logits, in the same order.
+template <int NPL>
+MOE_DEV void warp_topk_part(const float *lr, int E, int per, int q, int kk, int lane,
+                            unsigned long long *cand) {
+  unsigned long long pk[NPL];
+  const int e0 = q * per, e1 = min(E, e0 + per);
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = e0 + lane + 32 * i;
+    pk[i] = e < e1 ? ((unsigned long long)order_key(__ldcg(lr + e)) << 32) | (uint32_t)~e : 0ull;
+  }
+  const unsigned long long v = warp_top_packed<NPL>(pk, kk, lane);
+  if (lane < kk) cand[lane] = v;
+}
+
+// Part 2: one warp merges the n <= 64 candidates of a token (cand[0..n))
+// and returns, like warp_topk, selection j and its weight in lane j < k,
+// counting a near tie of the k-th and (k+1)-th logits when near_ties is set.
+MOE_DEV void warp_topk_merge(const unsigned long long *cand, int n, int E, int k, int lane,
+                             int &sel_e, float &sel_w, unsigned long long *near_ties) {
+  unsigned long long pk[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) pk[i] = lane + 32 * i < n ? cand[lane + 32 * i] : 0ull;
+  const int kk = k < E ? k + 1 : k;
+  const unsigned long long v = warp_top_packed<2>(pk, kk, lane);
+  const uint32_t key = (uint32_t)(v >> 32);
+  const uint32_t k0 = __shfl_sync(0xffffffffu, key, 0);
+  const uint32_t kth = __shfl_sync(0xffffffffu, key, k - 1);
+  const uint32_t next = __shfl_sync(0xffffffffu, key, kk - 1);
+  if (k < E && near_ties && lane == 0 && key_to_float(kth) - key_to_float(next) < 1e-5f)
+    atomicAdd(near_ties, 1ULL);
+  const float ex = lane < k ? expf(key_to_float(key) - key_to_float(k0)) : 0.f;
+  const float den = warp_sum(ex);
+  sel_e = (int)~(uint32_t)v;
+  sel_w = ex / den;
+}
+
 // Shared-memory words the body needs (dynamic smem of the finish kernel;
 // the fused kernel reuses its staging area).
 MOE_HOST_DEV_INLINE int finish_smem_ints(int E, int P) {
