@@ -312,6 +312,7 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
   }
   block_exclusive_scan(s_cnt, s_cnt, E, s_red);
   const int routed_jobs = s_cnt[E] >> 16;
+  unsigned my_hits = 0, my_misses = 0, my_active = 0;  // CTA 0's statistics, warp-reduced below
   for (int e = tid; e < E; e += blockDim.x) {
     unsigned m = s_mask[e];
     const int n = __popc(m);
@@ -328,10 +329,8 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
       if (slot >= p.n_slots && cta0) atomicOr(p.status, kErrBadSlot);
       ptr = p.arena + ((long long)p.layer * E + e) * p.expert_bytes;
     }
-    if (cta0) {
-      atomicAdd(&s_hm[hit ? 0 : 1], (unsigned long long)n);
-      atomicAdd(&s_hm[2], 1ull);
-    }
+    (hit ? my_hits : my_misses) += (unsigned)n;
+    ++my_active;
     for (int b = 0; m; ++b) {
       const int t = __ffs(m) - 1;
       m &= m - 1;
@@ -354,6 +353,16 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
       s_jptr[routed_jobs + q] = (unsigned long long)p.shared;
       s_jbeg[routed_jobs + q] = P + q * CH;
       s_jn[routed_jobs + q] = min(CH, T - q * CH);
+    }
+  }
+  if (cta0) {
+    const unsigned h = __reduce_add_sync(0xffffffffu, my_hits);
+    const unsigned mi = __reduce_add_sync(0xffffffffu, my_misses);
+    const unsigned a = __reduce_add_sync(0xffffffffu, my_active);
+    if ((tid & 31) == 0) {
+      atomicAdd(&s_hm[0], (unsigned long long)h);
+      atomicAdd(&s_hm[1], (unsigned long long)mi);
+      atomicAdd(&s_hm[2], (unsigned long long)a);
     }
   }
   __syncthreads();
