@@ -146,6 +146,8 @@ class ClockSampler:
 
 
 def dist_setup(args):
+    """One process per GPU (torchrun env).  NCCL on GPUs; gloo where there is
+    no GPU (the host-side logic's CPU tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -153,9 +155,12 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=300)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -172,9 +177,16 @@ def max_over_ranks(world, v):
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank, ms_max):
+    """Units all ranks processed (replicas: the same per rank) over the
+    slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 # ------------------------------------------------------------ the workload
@@ -341,7 +353,7 @@ def run_native(args, world, rank, local):
     kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
     res = {
         "metric": "decode MoE tokens/s" if args.workload != "prefill" else "prefill MoE tokens/s",
-        "value": world * tok / (ms_max * 1e-3),
+        "value": whole_job_rate(world, tok, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -395,7 +407,7 @@ def run_native(args, world, rank, local):
                            else "fallback 6650 GB/s",
             "per_unit": per_unit,
         },
-        "e2e": {"value": world * tok / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(world, tok, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
         "gpu_launches": K * (1 if single else (8 if prefill else 6)),
         "clocks": clocks,
@@ -496,7 +508,7 @@ def run_stack(args, world, rank, local):
     gbs = kern_bytes / (ms_max * 1e-3) / 1e9
     single = T <= 32
     res = {
-        "metric": "stack MoE tokens/s", "value": world * T * K / (ms_max * 1e-3), "unit": "tokens/s",
+        "metric": "stack MoE tokens/s", "value": whole_job_rate(world, T * K, ms_max), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_max / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "q4-g32 weights, bf16 activations, fp32 accumulate",
@@ -516,7 +528,7 @@ def run_stack(args, world, rank, local):
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                      "per_unit": f"{Be} B per touched expert per layer (shared included) + "
                                  f"{E * D * 4} B router W per layer"},
-        "e2e": {"value": world * T * K / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(world, T * K, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
         "gpu_launches": K * NL * (1 if single else 6),
         "clocks": clocks,

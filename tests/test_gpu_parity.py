@@ -234,6 +234,37 @@ def test_equal_logits_go_to_lower_id(B):
         B.moe_destroy(ctx)
 
 
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_equal_logits_split_topk_outputs(B, T):
+    """The decode kernel's top-k splits a token over several warps at
+    T <= 8 (4 warps at T <= 4, 2 at T = 8) and merges their candidates.
+    Router rows are triplicated (experts e, e+8, e+16 have equal logits),
+    so the twins of one row fall into different warps' parts: only the
+    lower id may be taken.  A wrong twin changes the output (its weights
+    differ), and tokens whose distinct logits are well separated are
+    compared against the oracle, exact ties included."""
+    spec = LayerSpec(d=256, f=128, E=24, k=4, fmt=I.Q4, seed=15, shared=True)
+    spec.W[8:16] = spec.W[0:8]
+    spec.W[16:24] = spec.W[0:8]
+    ctx = make_ctx(B, spec, max_tokens=16)
+    try:
+        load_layer(B, ctx, spec)
+        x = I.hidden_np(15, T, 256, window=T)
+        delta = torch.empty((T, spec.d), dtype=torch.float32, device="cuda")
+        B.moe_forward_delta(ctx, 0, to_dev(x), T, delta)
+        B.moe_sync(ctx, 60000)
+        lg = O.router(x, spec.W, spec.bias)[:, :8]          # the 8 distinct logits
+        top = -np.sort(-lg, axis=1)
+        # k = 4 takes the three copies of the best row and the lowest copy of
+        # the second: fp32 can only disagree if these rows nearly tie
+        sep = np.minimum(top[:, 0] - top[:, 1], top[:, 1] - top[:, 2]) >= 1e-5
+        assert sep.any()
+        orc = spec.oracle(x)
+        assert_close_rms(delta.cpu().numpy()[sep], orc["delta"][sep], what="MoE delta")
+    finally:
+        B.moe_destroy(ctx)
+
+
 def test_one_hot_expert_many_jobs(B):
     """A large bias sends every token to expert 7: one expert with T tokens,
     split into several 16-token jobs."""
