@@ -289,55 +289,37 @@ __device__ __noinline__ void decode_topk_split(const float *logits, int T, int E
   }
 }
 
-// All threads of the CTA: the bucketing of the pairs by expert and the job
-// list.  Experts come in ascending id, each split into jobs of <= chunk
-// tokens in ascending t; one exclusive scan over the experts' packed
-// (jobs, tokens) counts gives every expert its first job and first pair.
-// Each selected expert is looked up in the residency table (slot pool, else
-// the backing arena; Strata engine analysis article "93 token/s on one 8 GB
-// card", section "Expert cache").  The shared expert's jobs come last.  CTA
-// 0 also writes the statistics.
-MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned *s_mask,
-                        const int *s_idx, int *s_cnt, int *s_plist, unsigned long long *s_jptr,
-                        int *s_jbeg, int *s_jn) {
+// All threads of the CTA: the job list.  Experts come in ascending id, each
+// split into jobs of <= chunk tokens in ascending t; one exclusive scan over
+// the experts' packed (jobs, tokens) counts gives every expert its first job
+// and first pair.  Each selected expert is looked up in the residency table
+// (slot pool, else the backing arena; Strata engine analysis article "93
+// token/s on one 8 GB card", section "Expert cache").  The shared expert's
+// jobs come last.  Ends with a CTA barrier: the weight streams can start
+// from here, before the pair list (decode_pairs) exists.
+MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned *s_mask, int *s_cnt,
+                        unsigned long long *s_jptr, int *s_jbeg, int *s_jn) {
   __shared__ int s_red[32];
-  __shared__ unsigned long long s_hm[3];  // hits, misses, active experts (CTA 0)
   const int tid = threadIdx.x;
-  const int E = p.E, k = p.k, T = p.T, P = T * k, CH = p.chunk;
-  const bool cta0 = blockIdx.x == 0;
-  if (tid < 3) s_hm[tid] = 0;
+  const int E = p.E, T = p.T, P = T * p.k, CH = p.chunk;
   for (int e = tid; e < E; e += blockDim.x) {
     const int n = __popc(s_mask[e]);
     s_cnt[e] = (((n + CH - 1) / CH) << 16) | n;
   }
   block_exclusive_scan(s_cnt, s_cnt, E, s_red);
   const int routed_jobs = s_cnt[E] >> 16;
-  unsigned my_hits = 0, my_misses = 0, my_active = 0;  // CTA 0's statistics, warp-reduced below
   for (int e = tid; e < E; e += blockDim.x) {
-    unsigned m = s_mask[e];
-    const int n = __popc(m);
-    if (cta0) p.cnt_out[e] = n;
+    const int n = __popc(s_mask[e]);
     if (!n) continue;
     int jx = s_cnt[e] >> 16;
     const int px = s_cnt[e] & 0xFFFF;
     const int slot = s_slot[e];
     const uint8_t *ptr;
-    const bool hit = slot >= 0 && slot < p.n_slots;
-    if (hit) {
+    if (slot >= 0 && slot < p.n_slots) {
       ptr = p.pool + (long long)slot * p.expert_bytes;
     } else {
-      if (slot >= p.n_slots && cta0) atomicOr(p.status, kErrBadSlot);
+      if (slot >= p.n_slots && blockIdx.x == 0) atomicOr(p.status, kErrBadSlot);
       ptr = p.arena + ((long long)p.layer * E + e) * p.expert_bytes;
-    }
-    (hit ? my_hits : my_misses) += (unsigned)n;
-    ++my_active;
-    for (int b = 0; m; ++b) {
-      const int t = __ffs(m) - 1;
-      m &= m - 1;
-      int j = k - 1;  // the token's selection slot of e (independent loads)
-#pragma unroll 4
-      for (int jj = k - 2; jj >= 0; --jj) j = s_idx[t * k + jj] == e ? jj : j;
-      s_plist[px + b] = t * k + j;
     }
     for (int c0 = 0; c0 < n; c0 += CH, ++jx) {
       s_jptr[jx] = (unsigned long long)ptr;
@@ -348,13 +330,49 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
   int shared_jobs = 0;
   if (p.shared) {
     shared_jobs = (T + CH - 1) / CH;
-    for (int t = tid; t < T; t += blockDim.x) s_plist[P + t] = P + t;
     for (int q = tid; q < shared_jobs; q += blockDim.x) {
       s_jptr[routed_jobs + q] = (unsigned long long)p.shared;
       s_jbeg[routed_jobs + q] = P + q * CH;
       s_jn[routed_jobs + q] = min(CH, T - q * CH);
     }
   }
+  __syncthreads();
+  return routed_jobs + shared_jobs;
+}
+
+// All threads of the CTA, after decode_jobs: the pair list (each expert's
+// tokens in ascending t, as pair ids t*k + j; the shared expert's pairs
+// P + t last) and, in CTA 0, the statistics (per-expert token counts,
+// residency hits and misses, warp-reduced).  Ends with a CTA barrier.
+MOE_DEV void decode_pairs(const DecodeParams &p, const int *s_slot, const unsigned *s_mask,
+                          const int *s_idx, const int *s_cnt, int *s_plist) {
+  __shared__ unsigned long long s_hm[3];  // hits, misses, active experts (CTA 0)
+  const int tid = threadIdx.x;
+  const int E = p.E, k = p.k, T = p.T, P = T * k;
+  const bool cta0 = blockIdx.x == 0;
+  if (tid < 3) s_hm[tid] = 0;
+  unsigned my_hits = 0, my_misses = 0, my_active = 0;
+  for (int e = tid; e < E; e += blockDim.x) {
+    unsigned m = s_mask[e];
+    const int n = __popc(m);
+    if (cta0) p.cnt_out[e] = n;
+    if (!n) continue;
+    const int px = s_cnt[e] & 0xFFFF;
+    const int slot = s_slot[e];
+    (slot >= 0 && slot < p.n_slots ? my_hits : my_misses) += (unsigned)n;
+    ++my_active;
+    for (int b = 0; m; ++b) {
+      const int t = __ffs(m) - 1;
+      m &= m - 1;
+      int j = k - 1;  // the token's selection slot of e (independent loads)
+#pragma unroll 4
+      for (int jj = k - 2; jj >= 0; --jj) j = s_idx[t * k + jj] == e ? jj : j;
+      s_plist[px + b] = t * k + j;
+    }
+  }
+  if (p.shared)
+    for (int t = tid; t < T; t += blockDim.x) s_plist[P + t] = P + t;
+  __syncthreads();  // s_hm cleared before any warp adds to it
   if (cta0) {
     const unsigned h = __reduce_add_sync(0xffffffffu, my_hits);
     const unsigned mi = __reduce_add_sync(0xffffffffu, my_misses);
@@ -375,7 +393,6 @@ MOE_DEV int decode_jobs(const DecodeParams &p, const int *s_slot, const unsigned
     p.last[1] = (int)s_hm[2];
     p.last[2] = p.layer;
   }
-  return routed_jobs + shared_jobs;
 }
 
 // ------------------------------------------------ phases 3 and 4: stream-K GEMV
@@ -791,7 +808,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   __syncthreads();
   MOE_TRACE(kTrRouteTopk);
   {
-    const int nj = decode_jobs(p, s_slot, s_mask, s_idx, s_cnt, s_plist, s_jptr, s_jbeg, s_jn);
+    const int nj = decode_jobs(p, s_slot, s_mask, s_cnt, s_jptr, s_jbeg, s_jn);
     if (tid == 0) s_njobs = nj;
   }
   __syncthreads();
@@ -802,6 +819,17 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   // ---------------- phase 3: gate/up
   const Phase ph1 = make_phase(s_jptr, f, d, CG::TK, CG::STRIDE, 0);
   const SKCtx sk1 = sk_make(n_jobs * ph1.RB * ph1.UPI, W, gw, ep1, p.ws, p.flags, s_hand, s_hflag, WARPS);
+  // The warp's first weight units go in flight as soon as the job list
+  // exists; the pair list and the token rows are built while they land.
+  const int u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1);
+  {
+    const int i0 = u0 / ph1.UPI;
+    ring_start(r, ph1, i0 / ph1.RB, i0 % ph1.RB, u0 - i0 * ph1.UPI, u1 - u0, 1);
+    if (lane == 0) fence_proxy_async_smem();  // a wide window occupied the rings until now
+    __syncwarp();
+    ring_prologue(r, ph1, lane);
+  }
+  decode_pairs(p, s_slot, s_mask, s_idx, s_cnt, s_plist);
   // Token rows for the gate/up B operand.  A window that fits the staging
   // area stays there (row t at staging row t).  A wide window was staged
   // over the rings and the staging area; now that the rings are needed, the
@@ -836,22 +864,16 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
                    rs_bar);
     }
     if (__syncthreads_or(!mbar_wait_bounded(rs_bar, 0))) {
+      ring_drain(r);  // the first weight units are in flight
       if (tid == 0) atomicOr(p.status, kErrTimeout);
       return;
     }
   }
   __syncthreads();
-  {
-    const int u0 = sk_start(sk1, gw), u1 = sk_start(sk1, gw + 1), i0 = u0 / ph1.UPI;
-    ring_start(r, ph1, i0 / ph1.RB, i0 % ph1.RB, u0 - i0 * ph1.UPI, u1 - u0, 1);
-    if (lane == 0) fence_proxy_async_smem();  // a wide window occupied the rings until now
-    __syncwarp();
-    ring_prologue(r, ph1, lane);
-    if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg, s_rowmap,
-                                gsrc)) {
-      if (lane == 0) atomicOr(p.status, kErrTimeout);
-      ring_drain(r);
-    }
+  if (!decode_gated<FMT, NTM>(r, ph1, sk1, u0, u1, p, s_plist, s_jbeg, s_jn, stage_g, s_hg, s_rowmap,
+                              gsrc)) {
+    if (lane == 0) atomicOr(p.status, kErrTimeout);
+    ring_drain(r);
   }
   if (lane == 0) trace_point(kTrGateEnd);
 
