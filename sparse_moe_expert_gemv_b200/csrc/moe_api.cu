@@ -643,13 +643,14 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<true>, c->pf_map_h, g1));
-    PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / 64, c->lay.p1_bytes, nullptr, c->ybuf,
-                    c->status};
+    PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / 64, c->lay.p1_bytes, nullptr,
+                    reinterpret_cast<__half *>(c->ybuf), c->status};
     cfg.dynamicSmemBytes = smem2;
     CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<false>, c->pf_map_a, g2));
   }
   CUDA_TRY(c, prof_mark(c, 2, s));
-  PfCombineParams mp{c->ybuf, c->w, c->pf_row_of, N, k, d, c->n_shared, x, delta};
+  PfCombineParams mp{reinterpret_cast<const __half *>(c->ybuf), c->w, c->pf_row_of, N, k, d, c->n_shared,
+                     x, delta};
   const long long n4 = (long long)N * d / 4;
   const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
   CUDA_TRY(c, launch(prefill_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));

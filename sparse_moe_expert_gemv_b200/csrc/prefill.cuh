@@ -247,8 +247,10 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
 // logits[t, e] = sum_i W[e, i] h[t, i] (+ b[e]) for a whole chunk, fp32 FMA
 // (routing decisions are compared bit-exactly, so no reduced-precision
 // tensor-core path).  CTA tile: 128 tokens x 128 experts, 256 threads, each
-// an 8 x 8 block of outputs; the reduction walks i in order, 16 at a time
-// through shared memory (h converted from bf16 on the way in).
+// an 8 x 8 block of outputs made of two 4-row and two 4-column halves 64
+// apart (so a warp's 16-byte shared-memory reads are contiguous: no bank
+// conflicts); the reduction walks i in order, 16 at a time through shared
+// memory (h converted from bf16 on the way in).
 struct RouterGemmParams {
   const uint16_t *h;   // bf16 [T, d]
   const float *W;      // fp32 [E, d]
@@ -306,10 +308,10 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
     if (kt + 1 < nk) load((kt + 1) * kRgBK, hv, w0, w1);
 #pragma unroll
     for (int k = 0; k < kRgBK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&Ws[buf][k][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&Ws[buf][k][tx * 8 + 4]);
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Ws[buf][k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Ws[buf][k][64 + tx * 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -323,11 +325,11 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
   pdl_launch_dependents();
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int t = t0 + ty * 8 + i;
+    const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
     if (t >= p.T) continue;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int e = e0 + tx * 8 + j;
+      const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
       if (e < p.E) p.logits[(long long)t * p.E + e] = acc[i][j] + (p.bias ? p.bias[e] : 0.f);
     }
   }
@@ -458,7 +460,7 @@ struct PfGemmParams {
   int ntile_k;           // repacked tiles along K: K / 64
   long long region_off;  // 0 (gate/up) or the down region's offset
   __half *out_a;         // gate/up: SiLU(G) * U, fp16 [rows][N]
-  float *out_y;          // down: fp32 [rows][N]
+  __half *out_y;         // down: y, fp16 (round to nearest, saturating) [rows][N]
   int *status;
 };
 
@@ -652,12 +654,19 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
               dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           } else {
-            float4 *d0 = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
-            float4 *d1 = reinterpret_cast<float4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + kPfBN + c0);
+            uint4 *d0 = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
+            uint4 *d1 = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + kPfBN + c0);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              d0[v] = make_float4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
-              d1[v] = make_float4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) {
+              uint32_t pg[4], pu[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int i = v * 8 + q * 2;
+                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pg[q]) : "f"(g[i + 1]), "f"(g[i]));
+                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pu[q]) : "f"(u[i + 1]), "f"(u[i]));
+              }
+              d0[v] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+              d1[v] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
             }
           }
         }
@@ -704,7 +713,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
 }
 
 struct PfCombineParams {
-  const float *y;     // [rows][d] grouped order
+  const __half *y;    // fp16 [rows][d] grouped order
   const float *w;     // [T][k]
   const int *row_of;  // [T*k + T]
   int T, k, d, has_shared;
@@ -721,16 +730,21 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p)
        i += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(i / per_t), o = (int)(i - (long long)t * per_t) * 4;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // four fp16 y values of a row: one 8-byte load
+    auto y4 = [&](long long row) {
+      const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(p.y + row * p.d + o));
+      return make_float4(half_lo(v.x), half_hi(v.x), half_lo(v.y), half_hi(v.y));
+    };
     for (int j = 0; j < p.k; ++j) {
       const float wj = __ldg(p.w + (long long)t * p.k + j);
-      const float4 v = ldcg_f4(p.y + (long long)__ldg(p.row_of + (long long)t * p.k + j) * p.d + o);
+      const float4 v = y4(__ldg(p.row_of + (long long)t * p.k + j));
       a0 = fmaf(wj, v.x, a0);
       a1 = fmaf(wj, v.y, a1);
       a2 = fmaf(wj, v.z, a2);
       a3 = fmaf(wj, v.w, a3);
     }
     if (p.has_shared) {
-      const float4 sh = ldcg_f4(p.y + (long long)(P + t) * p.d + o);
+      const float4 sh = y4(P + t);
       a0 += sh.x;
       a1 += sh.y;
       a2 += sh.z;
