@@ -46,6 +46,7 @@ struct moe_ctx {
   int *d_slot_of = nullptr;
   std::vector<int> h_slot_of;
   float *d_router = nullptr, *d_bias = nullptr, *d_gamma = nullptr;
+  __nv_bfloat16 *d_router3 = nullptr;  // [L][E][3d] exact bf16 parts of the router (prefill)
   std::vector<char> has_router, has_bias, has_norm, has_gamma, shared_loaded;
   std::vector<float> eps;
   std::vector<std::vector<char>> expert_loaded;
@@ -265,6 +266,8 @@ moe_status do_configure(moe_ctx *c) {
     c->pf_eoff = (int *)(c->pf + o_eo);
     c->pf_ntiles = (int *)(c->pf + o_nt);
     c->pf_tiles = (PfTile *)(c->pf + o_tl);
+    // the router rows as three exact bf16 parts, for the tensor-core router
+    CUDA_TRY(c, cudaMalloc(&c->d_router3, (size_t)c->L * E * 3 * d * sizeof(__nv_bfloat16)));
   }
   c->has_router.assign(c->L, 0);
   c->has_bias.assign(c->L, 0);
@@ -551,21 +554,32 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
+// 2-D map of a row-major matrix of 16-bit elements [rows][cols]: boxes of 64
+// columns (one 128-byte swizzle row) x box_rows rows, out-of-range rows read
+// as zeros.
+bool encode_map_16b(CUtensorMap *map, CUtensorMapDataType type, const void *base, int rows, int cols,
+                    int box_rows) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kPfBK, (cuuint32_t)kPfBM};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
+  static_assert(kPfBK == 64, "one swizzle row per box row");
+  return encode_map_16b(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rows, cols, kPfBM);
 }
 
 cudaError_t setup_prefill() {
   cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RtCfg::SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(prefill_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PfCfg::SMEM);
@@ -592,11 +606,29 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   cudaError_t e = cudaSuccess;
   const uint16_t *h = router_input(c, layer, x, N, s, &e);
   CUDA_TRY(c, e);
-  RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d,
-                      c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E,
-                      c->logits};
-  CUDA_TRY(c, launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN),
-                     dim3(256), 0, s, rp));
+  const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
+  CUtensorMap hm, wm;
+  if (c->d_router3 && E % kRtBN == 0 && N >= kRtBM && d % 64 == 0 &&
+      encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) &&
+      encode_map_16b(&wm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->d_router3 + (size_t)layer * E * 3 * d, E,
+                     3 * d, kRtBN)) {
+    RouterTcParams tp{bias, c->logits, N, E, d, c->status};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((N + kRtBM - 1) / kRtBM, E / kRtBN);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = RtCfg::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, tp));
+  } else {  // small expert counts or chunks: fp32 FMA
+    RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d, bias, N, d, E, c->logits};
+    CUDA_TRY(c, launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN),
+                       dim3(256), 0, s, rp));
+  }
   const int blocks = (N + kPfTok - 1) / kPfTok;
   PfRouteParams tp{c->logits, N, E, k, c->idx, c->w, c->pf_bmask, &c->stats[4]};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
@@ -902,6 +934,7 @@ moe_status moe_destroy(moe_ctx *c) {
   dfree(c->pool);
   dfree(c->d_slot_of);
   dfree(c->d_router);
+  dfree(c->d_router3);
   dfree(c->d_bias);
   dfree(c->d_gamma);
   dfree(c->scratch);
@@ -966,6 +999,13 @@ moe_status moe_set_router(moe_ctx *c, int layer, const float *W, const float *bi
   if (bias)
     CUDA_TRY(c, cudaMemcpyAsync(c->d_bias + (size_t)layer * c->E, bias, (size_t)c->E * sizeof(float),
                                 kind, c->io));
+  if (c->d_router3) {
+    const long long n = (long long)c->E * c->d;
+    router_split_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 4096), 256, 0, c->io>>>(
+        c->d_router + (size_t)layer * c->E * c->d, n, c->d,
+        c->d_router3 + (size_t)layer * c->E * 3 * c->d);
+    CUDA_TRY(c, cudaGetLastError());
+  }
   CUDA_TRY(c, cudaStreamSynchronize(c->io));
   c->has_router[layer] = 1;
   c->has_bias[layer] = bias != nullptr;

@@ -712,6 +712,164 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   pdl_launch_dependents();
 }
 
+// ------------------------------------------------ router on the tensor cores
+// logits[t, e] = sum_i W[e, i] h[t, i] (+ b[e]) for a whole chunk.  The fp32
+// router rows are split once, exactly, into three bf16 parts W = Wh + Wm + Wl
+// (8 significand bits each: router_split_kernel), and h is bf16, so the sum
+// runs as one bf16 GEMM with the reduction tripled: [h | h | h] x
+// [Wh | Wm | Wl]^T.  Every product is exact and the tensor core accumulates
+// in fp32, so the logits keep fp32 accuracy: this is not a reduced-precision
+// router.  One 128-token x 256-expert tile per CTA: warp 0 lane 0 loads the h
+// and W tiles of each 64-column step by TMA (128-byte swizzle) into a 4-deep
+// ring, warp 1 lane 0 issues the m128n256k16 MMAs (fp32 in TMEM), warps 4..7
+// read the accumulator back and add the bias.  Every wait is bounded.
+constexpr int kRtBM = 128, kRtBN = 256, kRtStages = 4;
+
+struct RtCfg {
+  static constexpr uint32_t TILE_A = kRtBM * 64 * 2;   // 16 KB
+  static constexpr uint32_t TILE_B = kRtBN * 64 * 2;   // 32 KB
+  static constexpr uint32_t STAGE = TILE_A + TILE_B;   // a multiple of 1024 B
+  static constexpr uint32_t SMEM = kRtStages * STAGE + 1024;  // + alignment slack
+};
+
+struct RouterTcParams {
+  const float *bias;  // [E] or null
+  float *logits;      // [T, E]
+  int T, E, d;
+  int *status;
+};
+
+// W3[e] = [Wh | Wm | Wl] (bf16, 3d per row) with W[e] = Wh + Wm + Wl exactly:
+// each part is the bf16 rounding of what the parts before it left, and each
+// difference is exact in fp32.
+__global__ void router_split_kernel(const float *W, long long n, int d, __nv_bfloat16 *W3) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long e = i / d, c = i - e * d;
+    const float w = W[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __nv_bfloat16 *row = W3 + e * 3 * d;
+    row[c] = hi;
+    row[d + c] = mid;
+    row[2 * d + c] = lo;
+  }
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (formats 1).
+constexpr uint32_t umma_idesc_bf16(int M, int N) { return umma_idesc_f16(M, N) | (1u << 7) | (1u << 10); }
+
+__global__ void __launch_bounds__(256, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap hmap, const __grid_constant__ CUtensorMap wmap,
+                     RouterTcParams p) {
+  using C = RtCfg;
+  constexpr int S = kRtStages;
+  extern __shared__ __align__(128) unsigned char rt_smem[];
+  __shared__ __align__(8) unsigned long long s_full[S], s_empty[S], s_accf;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+  const uint32_t base = smem_addr(rt_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_addr(&s_full[i]), 1);
+      mbar_init(smem_addr(&s_empty[i]), 1);
+    }
+    mbar_init(smem_addr(&s_accf), 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (wid == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&s_tmem)),
+                 "r"(kRtBN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  pdl_wait();
+  const int m0 = blockIdx.x * kRtBM, n0 = blockIdx.y * kRtBN;
+  const int nkh = p.d / 64, nk = 3 * nkh;
+  auto stage_a = [&](int st) { return stage0 + (uint32_t)st * C::STAGE; };
+  auto stage_b = [&](int st) { return stage0 + (uint32_t)st * C::STAGE + C::TILE_A; };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
+  auto give_up = [&]() {
+    *reinterpret_cast<volatile int *>(&s_abort) = 1;
+    atomicOr(p.status, kErrTimeout);
+  };
+  if (wid == 0) {
+    if (lane == 0) {  // producer
+      int issued = 0;
+      for (int ks = 0; ks < nk && !aborted(); ++ks) {
+        const int st = ks % S, use = ks / S;
+        if (use > 0 && !mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1)) {
+          give_up();
+          break;
+        }
+        const uint32_t bar = smem_addr(&s_full[st]);
+        mbar_expect_tx(bar, C::STAGE);
+        tma_load_2d(stage_a(st), &hmap, (ks % nkh) * 64, m0, bar);
+        tma_load_2d(stage_b(st), &wmap, ks * 64, n0, bar);
+        issued = ks + 1;
+      }
+      // no tile may land in shared memory after the CTA has moved on
+      for (int ks = max(0, issued - S); ks < issued; ++ks)
+        (void)mbar_wait_bounded(smem_addr(&s_full[ks % S]), (ks / S) & 1);
+    }
+  } else if (wid == 1) {
+    if (lane == 0) {  // MMA issuer
+      constexpr uint32_t IDESC = umma_idesc_bf16(kRtBM, kRtBN);
+      bool ok = true;
+      for (int ks = 0; ks < nk; ++ks) {
+        const int st = ks % S, use = ks / S;
+        if (!mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16(tmem, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(stage_b(st) + kk * 32), IDESC,
+                   (ks | kk) != 0);
+        umma_commit(smem_addr(&s_empty[st]));
+      }
+      if (!ok) give_up();
+      umma_commit(smem_addr(&s_accf));
+      // every issued MMA is complete before TMEM is released
+      (void)mbar_wait_bounded(smem_addr(&s_accf), 0);
+    }
+  } else if (wid >= 4) {  // epilogue: TMEM lane = tile row
+    const bool ok = mbar_wait_bounded(smem_addr(&s_accf), 0);
+    tc_fence_after();
+    if (__all_sync(0xffffffffu, ok && !aborted())) {  // warp-uniform: tcgen05.ld is collective
+      const int quarter = wid & 3, t = m0 + quarter * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+      for (int c0 = 0; c0 < kRtBN; c0 += 32) {
+        float v[32];
+        tmem_ld32(lane_addr + c0, v);
+        if (t < p.T) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = n0 + c0 + j;
+            if (e < p.E) p.logits[(long long)t * p.E + e] = v[j] + (p.bias ? p.bias[e] : 0.f);
+          }
+        }
+      }
+    } else if (lane == 0) {
+      give_up();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (wid == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kRtBN));
+  pdl_launch_dependents();
+}
+
 struct PfCombineParams {
   const __half *y;    // fp16 [rows][d] grouped order
   const float *w;     // [T][k]
