@@ -488,6 +488,8 @@ cudaError_t prof_mark(moe_ctx *c, int i, cudaStream_t s) {
 // The whole decode chain for one layer.  delta == nullptr: residual mode.
 // Routing for `layer` (norm + logits + top-k + buckets + jobs when
 // build_jobs); returns the router input h (x, or the normalised copy).
+bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, cudaError_t *err);
+
 moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const FinishParams &fp,
                       cudaStream_t s, const uint16_t **h_out) {
   if (use_fused_route(c, T)) {
@@ -513,7 +515,10 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
   RouterParams rp{h, c->d_router + (size_t)layer * c->E * c->d,
                   c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
                   c->logits};
-  CUDA_TRY(c, launch_router(c, s, rp));
+  if (launch_router_tc(c, s, h, T, layer, &e))  // large windows: tensor cores
+    CUDA_TRY(c, e);
+  else
+    CUDA_TRY(c, launch_router(c, s, rp));
   if (T > kDecMaxT && c->pf_bmask) {
     // many tokens: the top-k runs one warp per token across the grid, and
     // the single routing CTA only buckets the selections and builds the jobs
@@ -589,6 +594,37 @@ cudaError_t setup_prefill() {
 // Prefill through the grouped tcgen05 GEMM: Q4 experts, more tokens than a
 // decode window, f a multiple of the gate/up item (128 features) and d of
 // the down item (256 features).
+// Router logits of N tokens on the tensor cores (router_tc_kernel) when the
+// context holds the router's bf16 parts, the shapes fit its tiles and the
+// chunk has at least kRtMinTokens tokens (one tile per CTA runs its whole
+// reduction, about 75 us at d = 2048 whatever the grid: fewer tokens are
+// faster on the fp32 router's wider grid); returns false (nothing launched)
+// otherwise.
+constexpr int kRtMinTokens = 512;
+bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, cudaError_t *err) {
+  const int E = c->E, d = c->d;
+  CUtensorMap hm, wm;
+  if (!c->d_router3 || E % kRtBN != 0 || N < kRtMinTokens || d % 64 != 0 ||
+      !encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) ||
+      !encode_map_16b(&wm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->d_router3 + (size_t)layer * E * 3 * d, E,
+                      3 * d, kRtBN))
+    return false;
+  RouterTcParams tp{c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, c->logits, N, E, d,
+                    c->status};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((N + kRtBM - 1) / kRtBM, E / kRtBN);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = RtCfg::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  *err = cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, tp);
+  return true;
+}
+
 bool use_prefill_gemm(const moe_ctx *c, int N) {
   return c->pf && c->fmt == MOE_Q4_SYM_G32_F16 && N > kDecMaxT && c->d % (2 * kPfBN) == 0 &&
          c->f % kPfBN == 0 && c->E <= kPfMaxE;
@@ -607,23 +643,8 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   const uint16_t *h = router_input(c, layer, x, N, s, &e);
   CUDA_TRY(c, e);
   const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
-  CUtensorMap hm, wm;
-  if (c->d_router3 && E % kRtBN == 0 && N >= kRtBM && d % 64 == 0 &&
-      encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) &&
-      encode_map_16b(&wm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->d_router3 + (size_t)layer * E * 3 * d, E,
-                     3 * d, kRtBN)) {
-    RouterTcParams tp{bias, c->logits, N, E, d, c->status};
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((N + kRtBM - 1) / kRtBM, E / kRtBN);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = RtCfg::SMEM;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, tp));
+  if (launch_router_tc(c, s, h, N, layer, &e)) {
+    CUDA_TRY(c, e);
   } else {  // small expert counts or chunks: fp32 FMA
     RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d, bias, N, d, E, c->logits};
     CUDA_TRY(c, launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN),
