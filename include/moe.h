@@ -134,7 +134,10 @@ MOE_API moe_status moe_load_shared(moe_ctx *ctx, int layer, const void *codes,
                            int src_is_device);
 
 /* moe_set_router: router weight W fp32 [E, d] and optional bias fp32 [E]
- * (NULL = no bias) of `layer`.  Synchronous copy. */
+ * (NULL = no bias) of `layer`.  Synchronous copy.  In a context configured
+ * with max_tokens > 32 it also stores W as three bf16 parts whose sum is W
+ * exactly (L * E * 3d * 2 bytes for the context), from which chunks of 512
+ * or more tokens compute the logits on the tensor cores at fp32 accuracy. */
 MOE_API moe_status moe_set_router(moe_ctx *ctx, int layer, const float *W,
                           const float *bias, int src_is_device);
 
@@ -196,7 +199,10 @@ MOE_API moe_status moe_forward_stack(moe_ctx *ctx, void *x_dev, int T, void *str
  * cores (tcgen05): tokens sorted by expert, 128-token tiles, weights
  * dequantised to fp16 tile by tile in shared memory, fp32 accumulation in
  * tensor memory.  Activations enter as fp16 (exact for |h| < 65504; larger
- * values saturate).  Q2 experts and N <= 32 take the moe_forward path.
+ * values saturate), and the experts' outputs y are kept in fp16 until the
+ * combine.  Router logits: fp32 accuracy, on the tensor cores from N >= 512
+ * and E a multiple of 256 (see moe_set_router), else fp32 FMA.  Q2 experts
+ * and N <= 32 take the moe_forward path.
  * Requires a context configured with max_tokens >= N.  Errors: INVALID_ARG,
  * STATE; device faults through moe_sync. */
 MOE_API moe_status moe_prefill(moe_ctx *ctx, int layer, void *x_dev, int N,

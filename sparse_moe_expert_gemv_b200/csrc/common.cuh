@@ -148,8 +148,9 @@ MOE_DEV void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-// expect_tx + 1-D bulk copy issued by the calling lane only when `issue`;
-// every lane may execute it (predicated, no branch).
+// expect_tx + 1-D bulk copy with an L2 cache policy (l2_evict_first), issued
+// by the calling lane only when `issue`; every lane may execute it
+// (predicated, no branch).
 MOE_DEV void bulk_g2s_hint_pred(bool issue, uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
                                 uint64_t policy) {
   asm volatile(
@@ -173,26 +174,12 @@ MOE_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t ba
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
-// The same copy with an L2 cache policy (see l2_evict_first).
-MOE_DEV void bulk_g2s_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
-                           uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
-      "%2, [%3], %4;" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-      : "memory");
-}
 // Policy for data read once: its L2 lines are the first to be evicted, so a
 // stream of them does not push other data (or code) out of L2.
 MOE_DEV uint64_t l2_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
-}
-// Start moving [src, src + bytes) from HBM into L2 (16-byte aligned, bytes a
-// multiple of 16); no completion to wait for.
-MOE_DEV void prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 MOE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -249,20 +236,6 @@ MOE_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
-}
-
-// Q4: one 32-bit word holds the 8 nibbles of one mma step for one lane:
-// fragment register i takes its low element from bits [4i, 4i+4) and its
-// high element from bits [16+4i, 20+4i).  OR-ing a nibble c into the
-// mantissa of bf16 128.0 (0x4300) gives exactly 128 + c; one bf16x2 FMA
-// (x * 1 - 136) then gives the signed level c - 8 exactly.
-MOE_DEV void unpack_q4(uint32_t w, uint32_t (&a)[4]) {
-  const uint32_t M = 0x000F000Fu, C = 0x43004300u;
-  const uint32_t one = 0x3F803F80u, off = 0xC308C308u;  // 1.0, -136.0
-  a[0] = bf16x2_fma(lop3_and_or(w, M, C), one, off);
-  a[1] = bf16x2_fma(lop3_and_or(w >> 4, M, C), one, off);
-  a[2] = bf16x2_fma(lop3_and_or(w >> 8, M, C), one, off);
-  a[3] = bf16x2_fma(lop3_and_or(w >> 12, M, C), one, off);
 }
 
 // Q2: one word holds the 16 codes of two mma steps; fragment register r
