@@ -1,8 +1,9 @@
-"""The multi-GPU bench path is N independent replicas (no collective on the
-data path).  Its host-side logic runs here as world_size-2 gloo ranks on the
-CPU: process-group set-up from the torchrun environment, the barrier, the
-max-over-ranks timing, the whole-job rate, and the reference arm, where only
-rank 0 works and prints."""
+"""The bench's host-side logic on the CPU.  The multi-GPU path is N
+independent replicas (no collective on the data path): world_size-2 gloo
+ranks exercise the process-group set-up from the torchrun environment, the
+barrier, the max-over-ranks timing and the whole-job rate.  The reference
+arm (the oracle on the host cores) runs on rank 0 only and prints the
+contract's JSON line."""
 import json
 import os
 import socket
@@ -82,3 +83,27 @@ def test_reference_arm_rank_nonzero_exits_without_work():
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=240)
     assert p.returncode == 0, p.stderr[-2000:]
     assert p.stdout.strip() == ""
+
+
+def test_reference_arm_json_line():
+    """The reference arm times the oracle on the host cores and prints one
+    JSON line with the native arm's metric, unit and workload, its own
+    cpu_baseline and an end-to-end figure with no device copies."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("RANK", None)
+    env.pop("WORLD_SIZE", None)
+    p = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.strip().splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference"
+    assert j["metric"] == "decode MoE tokens/s" and j["unit"] == "tokens/s" and j["higher_is_better"]
+    assert j["steps"] == 1 and j["warmup"] == 3 and j["value"] > 0
+    assert "T=4" in j["config"]["workload"] and "d=2048" in j["config"]["workload"]
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
+    e = j["e2e"]
+    assert e["value"] == j["value"] and e["unit"] == j["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
