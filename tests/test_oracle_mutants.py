@@ -29,6 +29,10 @@ MUTANTS = {
     "bias_dropped": ("if (bias) acc += (double)bias[e];", "if (bias) acc += 0.0;"),
     "eps_outside_sqrt": ("double inv = 1.0 / sqrt(ss / (double)d + eps);",
                          "double inv = 1.0 / (sqrt(ss / (double)d) + eps);"),
+    "q4_round_half_away": ("double t = rint(w[i] / s);", "double t = round(w[i] / s);"),
+    "q2_round_half_away": ("double t = rint((w[i] - m) / s);", "double t = round((w[i] - m) / s);"),
+    "q4_clamp_low_7": ("q = t < -8.0 ? -8 : t > 7.0 ? 7 : (int)t;",
+                       "q = t < -7.0 ? -7 : t > 7.0 ? 7 : (int)t;"),
     "bucket_descending": ("for (int t = 0; t < T; ++t)\n    for (int j = 0; j < k; ++j) {\n      int e = idx[(long)t * k + j];\n      perm",
                           "for (int t = T - 1; t >= 0; --t)\n    for (int j = 0; j < k; ++j) {\n      int e = idx[(long)t * k + j];\n      perm"),
 }

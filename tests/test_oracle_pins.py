@@ -127,6 +127,62 @@ def test_q4_zero_group_encodes_to_level_zero():
     assert s[0] == 0 and np.all(c == 0x88)
 
 
+def _q4_levels(codes):
+    lo = (codes & 0xF).astype(np.int64) - 8
+    hi = (codes >> 4).astype(np.int64) - 8
+    return np.stack([lo, hi], 1).reshape(-1)
+
+
+def test_q4_rounding_ties_go_to_even_level():
+    # max|w| = 7 * 2^-4, so s = 2^-4 exactly and w / s is exact: the group
+    # holds w/s = +-0.5, +-1.5, +-2.5, +-3.5, +-4.5 (exact halves).  Round half
+    # to even gives 0, 2, 2, 4, 4 (and the negatives); half away from zero
+    # would give 1, 2, 3, 4, 5 and floor(x + 0.5) 1, 2, 3, 4, 5 / 0, -1, -2, -3, -4.
+    s = 2.0 ** -4
+    halves = np.array([0.5, 1.5, 2.5, 3.5, 4.5])
+    w = np.zeros(32)
+    w[0] = 7.0 * s
+    w[1:6] = halves * s
+    w[6:11] = -halves * s
+    w[11] = -7.0 * s
+    c, sc, _ = O.quantize(O.Q4, w[None, :])
+    assert O.f16_to_f64(int(sc[0])) == s
+    q = _q4_levels(c)
+    assert list(q[1:6]) == [0, 2, 2, 4, 4]
+    assert list(q[6:11]) == [0, -2, -2, -4, -4]
+    assert q[0] == 7 and q[11] == -7
+
+
+def test_q2_rounding_ties_go_to_even_code():
+    # m = 0, max = 3 * 2^-3: s = 2^-3 exactly; (w - m) / s = 0.5, 1.5, 2.5
+    # round half to even -> 0, 2, 2 (half away from zero: 1, 2, 3)
+    s = 2.0 ** -3
+    w = np.zeros(64)
+    w[1] = 3.0 * s
+    w[2:5] = np.array([0.5, 1.5, 2.5]) * s
+    c, sc, mn = O.quantize(O.Q2, w[None, :])
+    assert O.f16_to_f64(int(sc[0])) == s and O.f16_to_f64(int(mn[0])) == 0.0
+    q = np.array([(c[i // 4] >> (2 * (i % 4))) & 3 for i in range(64)])
+    assert list(q[2:5]) == [0, 2, 2]
+    assert q[1] == 3 and q[0] == 0
+
+
+def test_q4_clamp_reaches_level_minus_8_on_subnormal_scale():
+    # max|w| / 7 = 2.5 * 2^-24 lies halfway between the fp16 subnormals 2 and
+    # 3 * 2^-24 and rounds to 2 * 2^-24 (even): then w / s = -7 * 1.25 = -8.75
+    # for the largest-magnitude element, clamped to the lowest level -8, and
+    # +8.75 for its positive twin, clamped to +7.
+    amax = 7.0 * 2.5 * 2.0 ** -24
+    w = np.zeros(32)
+    w[0] = -amax
+    w[1] = amax
+    c, sc, _ = O.quantize(O.Q4, w[None, :])
+    assert int(sc[0]) == 2  # fp16 bits of 2 * 2^-24
+    q = _q4_levels(c)
+    assert q[0] == -8 and q[1] == 7
+    assert np.all(q[2:] == 0)
+
+
 def test_page_expert_byte_counts_match_shape():
     g = read_kv("page_expert_bytes.txt")
     d, f = 2048, 768
