@@ -1,17 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the sparse MoE expert layer on B200.
 
-Default workload (the headline): one Flash-Next-shaped MoE layer in decode,
-d=2048, f=768, E=512, top-10 renormalised softmax + 1 shared expert,
-4-bit symmetric group-32 experts, bf16 hidden N(0,1), verify window T=4,
-uniform routing.  A step = one moe_forward call (router, top-k, residency
-lookup, bucketing, dequant-SwiGLU experts, combine + residual) on a new
-4-token window.  Steps rotate over --rot-layers independent copies of the
-layer's weights (16 x 1.36 GB by default), so the weights a step reads were
-evicted from the 126 MB L2 long before (no flush needed).
+Headline workload: one Flash-Next-shaped MoE layer in decode, d=2048,
+f=768, E=512, top-10 renormalised softmax + 1 shared expert, 4-bit symmetric
+group-32 experts, bf16 hidden N(0,1), verify window T=4, uniform routing.  A
+step = one moe_forward call (router, top-k, residency lookup, bucketing,
+dequant-SwiGLU experts, combine + residual) on a new 4-token window.  Steps
+rotate over --rot-layers independent copies of the layer's weights (16 x
+1.36 GB by default), so the weights a step reads were evicted from the 126
+MB L2 long before (no flush needed).
 
-Other workloads: --workload q2 (2-bit asymmetric g64, Zipf(1.1) routing,
-64 sequences x T tokens per call), --workload prefill (8192-token chunk).
+At one GPU the same JSON line also carries the other workloads of the
+metric, each with its own roofline, end-to-end figure and clocks:
+  "prefill"  an 8192-token chunk through one layer (Q4, Zipf(1.1) routing):
+             prefill MoE tokens/s, tensor-pipe roofline of its grouped GEMMs;
+  "q2"       2-bit asymmetric g64 experts, Zipf(1.1) routing, 64 sequences x
+             T tokens per call, T = 1..5: tokens/s and expert GB/s per T;
+  "stack"    the 48-layer stack (RMSNorm -> router -> experts -> combine per
+             layer, 4096-slot residency table), 32 tokens per step.
+(--no-extras drops them; --workload q2|prefill|stack makes one of them the
+headline instead.)
 
 Contract: python bench.py --gpus N --steps K --warmup W [--impl reference];
 rank 0 prints one JSON line.  N > 1 runs N independent replicas (the layer
@@ -51,6 +59,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="headline only (no prefill / q2 / stack objects)")
+    ap.add_argument("--extra-steps", type=int, default=10)
     a = ap.parse_args()
     if a.steps is None:
         a.steps = {"prefill": 20, "stack": 10}.get(a.workload, 200)
@@ -58,13 +69,11 @@ def parse():
 
 
 # ----------------------------------------------------------------- helpers
-def kernel_traffic(kernel_bytes_per_launch):
-    """Per-launch DRAM traffic of decode_kernel from the committed ncu record,
-    scaled to this run's algorithmic bytes per launch (the record's launch
-    routed a different window).  None when the kernel sources changed since
-    the counters were taken."""
+def _traffic_record(name):
+    """A committed ncu traffic record (profiles/<name>), or None when it is
+    missing or the kernel sources changed since the counters were taken."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     with open(p) as fh:
@@ -75,7 +84,25 @@ def kernel_traffic(kernel_bytes_per_launch):
             h.update(fh.read())
     if h.hexdigest() != rec["sources_sha256"]:
         return None
-    return rec["traffic_over_algorithmic"] * kernel_bytes_per_launch
+    return rec
+
+
+def kernel_traffic(kernel_bytes_per_launch):
+    """Per-launch DRAM traffic of decode_kernel from the committed ncu record,
+    scaled to this run's algorithmic bytes per launch (the record's launch
+    routed a different window)."""
+    rec = _traffic_record("decode_kernel_traffic.json")
+    return None if rec is None else rec["traffic_over_algorithmic"] * kernel_bytes_per_launch
+
+
+def prefill_traffic(flops_per_call):
+    """DRAM bytes of the two grouped-GEMM launches of one 8192-token chunk,
+    from the committed ncu record (scaled by FLOPs when this chunk's work
+    differs from the record's)."""
+    rec = _traffic_record("prefill_gemm_traffic.json")
+    if rec is None:
+        return None
+    return rec["bytes_per_call"] * flops_per_call / rec["flops_per_call"]
 
 
 def peaks():
@@ -85,6 +112,24 @@ def peaks():
             j = json.load(fh)
         return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+def host_info():
+    """Logical cores and CPU model of this host (for the CPU baselines)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count() or 1
+    return {"nproc": os.cpu_count(), "usable_cores": usable, "cpu_model": model}
 
 
 class ClockSampler:
@@ -190,29 +235,33 @@ def whole_job_rate(world, units_per_rank, ms_max):
 
 
 # ------------------------------------------------------------ the workload
-def workload_spec(args):
+def workload_spec(name, T=4):
     from sparse_moe_expert_gemv_b200 import inputs as I
-    if args.workload == "decode":
-        return dict(name=f"one MoE layer decode, d=2048 f=768 E=512 top-10 + shared, Q4 g32, "
-                         f"T={args.T}, uniform routing", fmt=I.Q4, zipf=False, T=args.T, seqs=1)
-    if args.workload == "q2":
-        return dict(name=f"one MoE layer decode, Q2 g64 asym, Zipf(1.1) routing, 64 sequences x "
-                         f"T={args.T}", fmt=I.Q2, zipf=True, T=args.T * 64, seqs=64)
-    if args.workload == "stack":
-        return dict(name="48-layer MoE stack (RMSNorm -> router -> experts -> combine + residual), "
-                         "d=2048 f=768 E=512 top-10 + shared, Q4 g32, 4096-slot residency table by "
-                         "Zipf rank, Zipf(1.1) routing, T=4 x batch 8 = 32 tokens",
-                    fmt=I.Q4, zipf=True, T=32, seqs=8)
-    return dict(name="prefill chunk, 8192 tokens, one MoE layer, Q4 g32, Zipf(1.1) routing",
-                fmt=I.Q4, zipf=True, T=8192, seqs=1)
+    if name == "decode":
+        return dict(kind=name, name=f"one MoE layer decode, d=2048 f=768 E=512 top-10 + shared, "
+                                    f"Q4 g32, T={T}, uniform routing",
+                    fmt=I.Q4, zipf=False, T=T, seqs=1, prefill=False, metric="decode MoE tokens/s")
+    if name == "q2":
+        return dict(kind=name, name=f"one MoE layer decode, Q2 g64 asym, Zipf(1.1) routing, "
+                                    f"64 sequences x T={T}",
+                    fmt=I.Q2, zipf=True, T=T * 64, seqs=64, prefill=False, metric="decode MoE tokens/s")
+    if name == "stack":
+        return dict(kind=name, name="48-layer MoE stack (RMSNorm -> router -> experts -> combine + "
+                                    "residual), d=2048 f=768 E=512 top-10 + shared, Q4 g32, "
+                                    "4096-slot residency table by Zipf rank, Zipf(1.1) routing, "
+                                    "T=4 x batch 8 = 32 tokens",
+                    fmt=I.Q4, zipf=True, T=32, seqs=8, prefill=False, metric="stack MoE tokens/s")
+    return dict(kind="prefill", name="prefill chunk, 8192 tokens, one MoE layer, d=2048 f=768 E=512 "
+                                     "top-10 + shared, Q4 g32, Zipf(1.1) routing",
+                fmt=I.Q4, zipf=True, T=8192, seqs=1, prefill=True, metric="prefill MoE tokens/s")
 
 
-def build_native(args, spec, n_rot):
+def build_native(args, spec, n_rot, max_tokens=None):
     import torch
     from sparse_moe_expert_gemv_b200 import binding as B
     from sparse_moe_expert_gemv_b200 import inputs as I
     ctx = B.moe_create(D, F, E, K_TOP, spec["fmt"])
-    B.moe_configure(ctx, n_rot, 1, 0, spec["T"])
+    B.moe_configure(ctx, n_rot, 1, 0, max_tokens or spec["T"])
     for l in range(n_rot):
         W = I.router_np(args.seed, E, D, l)
         bias = I.zipf_bias_np(args.seed, E, l)[0] if spec["zipf"] else None
@@ -221,23 +270,31 @@ def build_native(args, spec, n_rot):
             c, s, m = I.experts_torch(args.seed, spec["fmt"], D, F, l, first, 64, "cuda")
             B.moe_load_experts(ctx, l, first, 64, c, s, m)
             del c, s, m
-        c, s, m = I.shared_np(args.seed, spec["fmt"], D, F, l)
+        c, s, m = I.experts_torch(args.seed, spec["fmt"], D, F, l, I.SHARED_INDEX, 1, "cuda")
         B.moe_load_shared(ctx, l, c, s, m)
+        del c, s, m
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return ctx
 
 
-def run_native(args, world, rank, local):
+def run_native(args, world, spec, n_rot, K, W):
+    """Build the layer copies, measure, free."""
+    from sparse_moe_expert_gemv_b200 import binding as B
+    ctx = build_native(args, spec, n_rot)
+    try:
+        return measure(args, world, ctx, spec, n_rot, K, W)
+    finally:
+        B.moe_destroy(ctx)
+
+
+def measure(args, world, ctx, spec, n_rot, K, W):
+    """K timed steps of one workload on a built context (n_rot layer copies)."""
     import torch
     from sparse_moe_expert_gemv_b200 import binding as B
     from sparse_moe_expert_gemv_b200 import inputs as I
 
-    spec = workload_spec(args)
     T = spec["T"]
-    n_rot = args.rot_layers
-    K, W = args.steps, args.warmup
-    ctx = build_native(args, spec, n_rot)
     Be = B.moe_expert_bytes(D, F, spec["fmt"])
 
     # one fresh window per step (timed and warm-up), pristine copies kept
@@ -262,7 +319,7 @@ def run_native(args, world, rank, local):
     total_bytes = expert_bytes + router_bytes + act_bytes
 
     stream = torch.cuda.current_stream()
-    prefill = args.workload == "prefill"
+    prefill = spec["prefill"]
     call = B.moe_prefill if prefill else B.moe_forward  # the public call a step makes
     # warm-up (eager), then capture the K timed steps as one CUDA graph
     for i in range(W):
@@ -371,7 +428,7 @@ def run_native(args, world, rank, local):
         per_unit = f"{Be} B per touched expert (codes+scales), shared expert included"
     kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
     res = {
-        "metric": "decode MoE tokens/s" if args.workload != "prefill" else "prefill MoE tokens/s",
+        "metric": spec["metric"],
         "value": whole_job_rate(world, tok, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -396,7 +453,8 @@ def run_native(args, world, rank, local):
         "distinct_experts_per_step": float(distinct.mean()),
         "segments_ms_per_step": {"route": route_ms / max(ncalls, 1),
                                  "experts": exp_ms / max(ncalls, 1),
-                                 "combine": comb_ms / max(ncalls, 1)},
+                                 "combine": comb_ms / max(ncalls, 1),
+                                 "timing": "a second, event-bracketed pass of the same steps"},
         "roofline": {
             "bound": "tensor",
             "kernel": "prefill_gemm_kernel (gate/up + down grouped GEMMs of one call, tcgen05 fp16)",
@@ -431,20 +489,23 @@ def run_native(args, world, rank, local):
         "gpu_launches": K * (1 if single else (8 if prefill else 6)),
         "clocks": clocks,
     }
-    B.moe_destroy(ctx)
-    return res, spec
+    if single:
+        # one launch per step: the profile pass only brackets that launch
+        del res["segments_ms_per_step"]
+    if prefill:
+        res["roofline"]["traffic"] = prefill_traffic(flops)
+    return res
 
 
-def run_stack(args, world, rank, local):
+def run_stack(args, world, K, W):
     """48-layer stack: each step is one moe_forward_stack call (one CUDA graph
     of the 48 layers) on a new 32-token window."""
     import torch
     from sparse_moe_expert_gemv_b200 import binding as B
     from sparse_moe_expert_gemv_b200 import inputs as I
 
-    spec = workload_spec(args)
+    spec = workload_spec("stack")
     T, NL, SLOTS = spec["T"], 48, 4096
-    K, W = args.steps, args.warmup
     ctx = B.moe_create(D, F, E, K_TOP, I.Q4)
     B.moe_configure(ctx, NL, 1, SLOTS, T)
     ranks = []
@@ -455,8 +516,9 @@ def run_stack(args, world, rank, local):
             c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, l, first, 64, "cuda")
             B.moe_load_experts(ctx, l, first, 64, c, s_, m)
             del c, s_, m
-        c, s_, m = I.shared_np(args.seed, I.Q4, D, F, l)
+        c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, l, I.SHARED_INDEX, 1, "cuda")
         B.moe_load_shared(ctx, l, c, s_, m)
+        del c, s_, m
         B.moe_set_norm(ctx, l, None, 1e-6)
         ranks.append(rank_of)
     B.moe_set_slots(ctx, I.slot_table_np(E, NL, SLOTS, np.stack(ranks)))
@@ -553,80 +615,149 @@ def run_stack(args, world, rank, local):
         "clocks": clocks,
     }
     B.moe_destroy(ctx)
-    return res, spec
+    return res
 
 
-def cpu_baseline(args, spec, seconds):
-    """The oracle, as it stands, on a bounded sample of the same workload."""
+# ------------------------------------------------ the oracle on host cores
+def oracle_rows_threaded(x_rows, spec, W, bias, experts, shared, threads, norm=False):
+    """The oracle's layer on token rows, the rows split over `threads`
+    host threads (tokens are independent; the C oracle runs without the
+    GIL).  `experts` maps id -> packed bytes for every id a row selects."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import oracle as O
+
+    chunks = [c for c in np.array_split(np.arange(x_rows.shape[0]), threads) if c.size]
+
+    def one(c):
+        x = np.ascontiguousarray(x_rows[c])
+        h = O.rmsnorm(x, None, 1e-6) if norm else x
+        idx, _, _ = O.topk(O.router(h, W, bias), K_TOP)
+        need = {e: experts[e] for e in set(idx.reshape(-1).tolist())}
+        O.moe_layer(x, fmt=spec["fmt"], d=D, f=F, E=E, k=K_TOP, router_w=W, router_bias=bias,
+                    experts=need, shared=shared, norm=norm)
+        return c.size
+
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        return sum(ex.map(one, chunks))
+
+
+def host_experts(args, fmt, layer, on_gpu):
+    """Packed bytes of every expert (and the shared one) of one layer, made
+    before any timing: on the GPU with the torch generator when there is one,
+    else with the numpy generator on host threads."""
+    from concurrent.futures import ThreadPoolExecutor
+
     from sparse_moe_expert_gemv_b200 import inputs as I
+    out = {}
+    if on_gpu:
+        for first in range(0, E, 64):
+            c, s, m = I.experts_torch(args.seed, fmt, D, F, layer, first, 64, "cuda")
+            c, s = c.cpu().numpy(), s.cpu().numpy().view(np.uint16)
+            m = None if m is None else m.cpu().numpy().view(np.uint16)
+            for i in range(64):
+                out[first + i] = (c[i], s[i], None if m is None else m[i])
+        c, s, m = I.experts_torch(args.seed, fmt, D, F, layer, I.SHARED_INDEX, 1, "cuda")
+        shared = (c[0].cpu().numpy(), s[0].cpu().numpy().view(np.uint16),
+                  None if m is None else m[0].cpu().numpy().view(np.uint16))
+        return out, shared
+    with ThreadPoolExecutor(host_info()["usable_cores"]) as ex:
+        vals = list(ex.map(lambda e: I.expert_np(args.seed, fmt, D, F, layer, e), range(E)))
+    return dict(enumerate(vals)), I.shared_np(args.seed, fmt, D, F, layer)
+
+
+def cpu_baseline(args, spec, seconds, on_gpu=True, norm=False, tokens=None, layers_per_token=1):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    token windows of the workload through the full layer, each window's
+    tokens split over the host's cores.  Runs for about `seconds`."""
+    from sparse_moe_expert_gemv_b200 import inputs as I
+    import oracle as O
     O.build()
-    T = spec["T"]
+    info = host_info()
+    threads = info["usable_cores"]
     W = I.router_np(args.seed, E, D, 0)
     bias = I.zipf_bias_np(args.seed, E, 0)[0] if spec["zipf"] else None
-    cache = {}
-    tok = 0
+    experts, shared = host_experts(args, spec["fmt"], 0, on_gpu)
+    per = tokens or min(spec["T"], max(threads, 4))
+    tok, win = 0, 0
     t0 = time.perf_counter()
-    win = 0
     while time.perf_counter() - t0 < seconds:
-        x = I.hidden_np(args.seed, min(T, 4), D, window=100000 + win)
+        x = I.hidden_np(args.seed, per, D, window=100000 + win)
+        tok += oracle_rows_threaded(x, spec, W, bias, experts, shared, threads, norm=norm)
         win += 1
-        lg = O.router(x, W, bias)
-        idx, _, _ = O.topk(lg, K_TOP)
-        experts = {}
-        for e in set(idx.reshape(-1).tolist()):
-            if e not in cache:
-                cache[e] = I.expert_np(args.seed, spec["fmt"], D, F, 0, e)
-            experts[e] = cache[e]
-        O.moe_layer(x, fmt=spec["fmt"], d=D, f=F, E=E, k=K_TOP, router_w=W, router_bias=bias,
-                    experts=experts, shared=I.shared_np(args.seed, spec["fmt"], D, F, 0))
-        tok += x.shape[0]
-        if len(cache) > 256:
-            cache.clear()
     dt = time.perf_counter() - t0
-    return {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{win} windows of {min(T, 4)} tokens through the full layer "
-                      f"(fp64 scalar C, single thread, {dt:.1f} s)"}
+    value = tok / dt / layers_per_token
+    what = (f"{win} windows of {per} tokens through one full layer"
+            + (f" (a token of the stack passes {layers_per_token} layers: tokens/s = "
+               f"layer-tokens/s / {layers_per_token})" if layers_per_token > 1 else ""))
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{what}; fp64 scalar C, each window's tokens split over {threads} "
+                      f"host threads; {dt:.1f} s", **info}
 
 
 def run_reference(args):
-    """Reference arm: the oracle (scalar fp64 C) on the host cores."""
-    spec = workload_spec(args)
+    """Reference arm: the oracle (scalar fp64 C) on the host cores, on the
+    headline's workload: each step is one window of the workload's tokens
+    through the full layer (capped at 8 tokens for the prefill and stack
+    workloads, whose steps the oracle cannot finish in minutes)."""
+    spec = workload_spec(args.workload, args.T)
     import oracle as O
     from sparse_moe_expert_gemv_b200 import inputs as I
     O.build()
+    info = host_info()
+    threads = info["usable_cores"]
     W = I.router_np(args.seed, E, D, 0)
     bias = I.zipf_bias_np(args.seed, E, 0)[0] if spec["zipf"] else None
-    shared = I.shared_np(args.seed, spec["fmt"], D, F, 0)
+    experts, shared = host_experts(args, spec["fmt"], 0, on_gpu=False)
+    per = spec["T"] if spec["kind"] in ("decode", "q2") and spec["T"] <= 8 else 8
+    norm = spec["kind"] == "stack"
 
     def step(i):
-        x = I.hidden_np(args.seed, 1, D, window=200000 + i)
-        lg = O.router(x, W, bias)
-        idx, _, _ = O.topk(lg, K_TOP)
-        experts = {e: I.expert_np(args.seed, spec["fmt"], D, F, 0, e)
-                   for e in set(idx.reshape(-1).tolist())}
-        O.moe_layer(x, fmt=spec["fmt"], d=D, f=F, E=E, k=K_TOP, router_w=W, router_bias=bias,
-                    experts=experts, shared=shared)
-        return 1
+        x = I.hidden_np(args.seed, per, D, window=i)
+        return oracle_rows_threaded(x, spec, W, bias, experts, shared, threads, norm=norm)
 
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
     tok = sum(step(args.warmup + i) for i in range(args.steps))
     dt = time.perf_counter() - t0
-    v = tok / dt
-    return {"impl": "reference", "metric": "decode MoE tokens/s" if args.workload != "prefill"
-            else "prefill MoE tokens/s", "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic",
-            "config": {"workload": spec["name"],
-                       "sample": "each step: 1 token through the full layer"},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "1 token per step through the full layer (router over "
-                                       "512 experts, its 10 experts + shared, fp64)"},
+    v = tok / dt / (48 if spec["kind"] == "stack" else 1)
+    same = per == spec["T"]
+    sample = (f"each step: {per} tokens (window {'= the workload' if same else 'sample'}) through "
+              f"the full layer{' (x 48 layers for the stack rate)' if norm else ''}, fp64 scalar C, "
+              f"tokens split over {threads} host threads")
+    return {"impl": "reference", "metric": spec["metric"], "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec["name"], "tokens_per_step": per, "same_window": same},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample, **info},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+def q2_sweep(args, world, K, W):
+    """Config Q2: one Q2 context (4 rotated layer copies), T = 1..5 tokens per
+    sequence x 64 sequences per call."""
+    from sparse_moe_expert_gemv_b200 import binding as B
+    spec0 = workload_spec("q2", 5)
+    n_rot = 4
+    ctx = build_native(args, spec0, n_rot, max_tokens=spec0["T"])
+    out = {}
+    try:
+        for T in range(1, 6):
+            r = measure(args, world, ctx, workload_spec("q2", T), n_rot, K, W)
+            out[f"T{T}"] = {key: r[key] for key in
+                            ("value", "unit", "ms_per_step", "steps", "warmup", "expert_weight_gbs",
+                             "distinct_experts_per_step", "roofline", "e2e", "gpu_launches",
+                             "segments_ms_per_step", "clocks")}
+            out[f"T{T}"]["tokens_per_step"] = 64 * T
+    finally:
+        B.moe_destroy(ctx)
+    return {"workload": "one MoE layer decode, d=2048 f=768 E=512 top-10 + shared, Q2 g64 asym "
+                        "(fp16 scale + min), Zipf(1.1) routing, 64 sequences x T tokens per call",
+            "metric": "decode MoE tokens/s", "by_T": out}
 
 
 def main():
@@ -639,10 +770,26 @@ def main():
     world, rank, local = dist_setup(args)
     from sparse_moe_expert_gemv_b200 import build as _b
     _b.build()
+    spec = workload_spec(args.workload, args.T)
     if args.workload == "stack":
-        res, spec = run_stack(args, world, rank, local)
+        res = run_stack(args, world, args.steps, args.warmup)
     else:
-        res, spec = run_native(args, world, rank, local)
+        n_rot = args.rot_layers if args.workload == "decode" else min(args.rot_layers, 4)
+        res = run_native(args, world, spec, n_rot, args.steps, args.warmup)
+    extras = world == 1 and not args.no_extras and args.workload == "decode"
+    if extras:
+        ks, ws = args.extra_steps, 3
+        pre = run_native(args, world, workload_spec("prefill"), 2, ks, ws)
+        if not args.no_cpu_baseline:
+            pre["cpu_baseline"] = cpu_baseline(args, workload_spec("prefill"), args.cpu_seconds,
+                                               tokens=16)
+        res["prefill"] = pre
+        res["q2"] = q2_sweep(args, world, 2 * ks, ws)
+        st = run_stack(args, world, max(ks // 2, 3), ws)
+        if not args.no_cpu_baseline:
+            st["cpu_baseline"] = cpu_baseline(args, workload_spec("stack"), args.cpu_seconds,
+                                              norm=True, tokens=8, layers_per_token=48)
+        res["stack"] = st
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(args, spec, args.cpu_seconds)

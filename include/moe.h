@@ -118,6 +118,9 @@ MOE_API moe_status moe_configure(moe_ctx *ctx, int n_layers, int n_shared, int n
 MOE_API moe_status moe_destroy(moe_ctx *ctx);
 
 /* moe_load_experts: copy n_experts packed experts (format above) into
+ * (the backing copy of every (layer, expert) that the residency table of the
+ * engine article "93 token/s on one 8 GB card", section "Expert cache",
+ * points at when an expert is not in a slot)
  * experts [first_expert, first_expert + n_experts) of `layer`, repacking them
  * into the library's device layout.  Also refreshes any slot-pool copies of
  * those experts.  Synchronous.  Errors: INVALID_ARG on a bad range or NULL
@@ -146,7 +149,9 @@ MOE_API moe_status moe_set_router(moe_ctx *ctx, int layer, const float *W,
  * Without this call a layer uses h = x (no norm). */
 MOE_API moe_status moe_set_norm(moe_ctx *ctx, int layer, const float *gamma, float eps);
 
-/* moe_set_slots: residency table, HOST int32 [n_layers * E]: slot id of
+/* moe_set_slots: the residency table of the engine article "93 token/s on
+ * one 8 GB card", section "Expert cache": (layer, expert) -> slot or -1.
+ * HOST int32 [n_layers * E]: slot id of
  * (layer, expert) in the slot pool, or -1 when it is served from the backing
  * arena (every expert always has a backing copy, so results do not depend on
  * the table).  Copies the experts into their slots (synchronous).
@@ -154,7 +159,12 @@ MOE_API moe_status moe_set_norm(moe_ctx *ctx, int layer, const float *gamma, flo
 MOE_API moe_status moe_set_slots(moe_ctx *ctx, const int32_t *slot_of);
 
 /* moe_route: router logits + top-k + softmax + bucketing for T tokens of
- * `layer`.  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
+ * `layer` (the engine article "93 token/s on one 8 GB card", section
+ * "Architecture overview": the router picks 10 of 512 experts per token;
+ * the "Doorbell handshake" section ends the "pre" half of a block with the
+ * router's ids and weights).  Windows of more than 32 tokens select the
+ * top-k one warp per token; from 512 tokens, with E a multiple of 256, the
+ * logits come from the tensor-core router (see moe_set_router).  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
  * w_dev fp32 [T, k] receive each token's experts and renormalised weights,
  * ordered by descending logit (equal logits: lower expert id first).
  * bucket_off_dev int32 [E+1] (exclusive prefix of tokens per expert) and
@@ -172,7 +182,10 @@ MOE_API moe_status moe_bucket(moe_ctx *ctx, const int32_t *idx_dev, int T,
                       int32_t *bucket_off_dev, int32_t *bucket_perm_dev,
                       void *stream);
 
-/* moe_forward: one decode window of T tokens through `layer`, in place:
+/* moe_forward: one decode window of T tokens through `layer`, in place
+ * (the engine article "93 token/s on one 8 GB card", section "Architecture
+ * overview": route, compute each selected expert from wherever it resides,
+ * combine into the residual):
  * x <- x + MoE(norm(x)).  x_dev: bf16 [T, d].  Runs router, top-k, residency
  * lookup, bucketing, the grouped dequant-SwiGLU experts (+ shared expert)
  * and the combine + residual kernel.  Errors: INVALID_ARG, STATE (router or
@@ -213,6 +226,23 @@ MOE_API moe_status moe_prefill(moe_ctx *ctx, int layer, void *x_dev, int N,
 MOE_API moe_status moe_prefill_delta(moe_ctx *ctx, int layer, const void *x_dev, int N,
                                      float *delta_dev, void *stream);
 
+/* moe_prefill_route: the routing half of moe_prefill alone, on router
+ * input h_dev bf16 [N, d] (no RMSNorm here, as in moe_route): the chunk's
+ * router logits (tensor cores from N >= 512 with E a multiple of 256, else
+ * fp32 FMA), top-k + softmax one warp per token, and the sort of the
+ * chunk's pairs by expert that feeds the grouped GEMM (the engine article
+ * "93 token/s on one 8 GB card", section "Architecture overview": prefill in
+ * chunks of up to 8192 tokens).  It launches exactly the kernels moe_prefill
+ * launches before its GEMMs.  Outputs as in moe_route: idx_dev int32
+ * [N, k], w_dev fp32 [N, k], bucket_off_dev int32 [E+1] (may be NULL),
+ * bucket_perm_dev int32 [N*k] (pair ids grouped by expert, ascending t
+ * inside an expert; may be NULL).  Errors: INVALID_ARG (N < 1, N >
+ * max_tokens, NULL idx/w, h not 16-byte aligned), STATE (router not set),
+ * NOT_SUPPORTED in a context configured with max_tokens <= 32. */
+MOE_API moe_status moe_prefill_route(moe_ctx *ctx, int layer, const void *h_dev, int N,
+                                     int32_t *idx_dev, float *w_dev, int32_t *bucket_off_dev,
+                                     int32_t *bucket_perm_dev, void *stream);
+
 /* moe_sync: wait (polling cudaEventQuery, at most timeout_ms; < 0 = no
  * limit) until the work queued by this context has finished, then read and
  * clear the device error status.  Returns TIMEOUT, BAD_SLOT, DEVICE, CUDA or
@@ -242,13 +272,25 @@ MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
  * kernels' shared-memory limit; make that first call before any stream
  * capture.  Each call clears the array's counters on `stream` before use;
  * calls whose execution overlaps on the GPU (other streams, other threads)
- * race on the array.  Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA;
- * an out-of-range routing id cannot occur (ids come from the top-k). */
+ * race on the array.  Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA at
+ * launch; an out-of-range routing id cannot occur (ids come from the
+ * top-k).  If a bounded wait inside the kernel gives up (the window's copy
+ * into shared memory never completed), the call routes nothing: idx, w and
+ * the buckets keep their previous contents, and moe_route_static_status
+ * reports it. */
 MOE_API moe_status moe_route_static(const void *h_dev, int T, int d, int E, int k,
                                     const float *W_dev, const float *bias_dev,
                                     int32_t *idx_dev, float *w_dev,
                                     int32_t *bucket_off_dev, int32_t *bucket_perm_dev,
                                     void *stream);
+
+/* moe_route_static_status: synchronises `stream`, then stores in
+ * *status_out the device status word of the most recent moe_route_static
+ * call on the current device (0, or the OR of its fault bits: 8 = a bounded
+ * wait gave up and nothing was routed).  Returns MOE_OK for 0, MOE_ERR_DEVICE
+ * for a non-zero word, MOE_ERR_CUDA or MOE_ERR_INVALID_ARG (NULL).  The
+ * word is cleared by the next moe_route_static call. */
+MOE_API moe_status moe_route_static_status(int *status_out, void *stream);
 
 /* Profiling: when enabled, every forward call records CUDA events on its
  * stream around its three segments -- routing (norm + router + top-k +
@@ -291,6 +333,13 @@ MOE_API const char *moe_status_string(int status);
  * the backing copy and sets the device status that moe_sync reports as
  * MOE_ERR_BAD_SLOT.  Not for production use. */
 MOE_API moe_status moe_debug_poke_slot(moe_ctx *ctx, int layer, int expert, int32_t slot);
+
+/* Debug hook: copies on `stream` the normalised router input h (bf16
+ * [T, d], h = RMSNorm(x) as the kernels computed it) of the most recent
+ * moe_forward / moe_forward_delta / moe_prefill call on a layer with
+ * RMSNorm into out_dev.  Lets tests compare the device's RMSNorm with a
+ * reference.  Errors: INVALID_ARG (NULL, T out of range). */
+MOE_API moe_status moe_debug_last_h(moe_ctx *ctx, void *out_dev, int T, void *stream);
 
 /* Bytes one packed expert occupies in the given format (codes + scales +
  * mins), or -1 for bad arguments. */

@@ -30,7 +30,8 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_forward_stack", "moe_prefill", "moe_sync", "moe_get_stats",
            "moe_last_error", "moe_status_string", "moe_expert_bytes",
            "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
-           "moe_set_trace", "moe_read_trace", "moe_route_static", "moe_prefill_delta")
+           "moe_set_trace", "moe_read_trace", "moe_route_static", "moe_prefill_delta",
+           "moe_prefill_route", "moe_route_static_status", "moe_debug_last_h")
 
 
 class MoeError(RuntimeError):
@@ -69,6 +70,9 @@ def _load():
         "moe_forward_stack": [P, P, I, P],
         "moe_prefill": [P, I, P, I, P],
         "moe_prefill_delta": [P, I, P, I, P, P],
+        "moe_prefill_route": [P, I, P, I, P, P, P, P, P],
+        "moe_route_static_status": [ctypes.POINTER(I), P],
+        "moe_debug_last_h": [P, P, I, P],
         "moe_sync": [P, I],
         "moe_get_stats": [P, ctypes.POINTER(MoeStats)],
         "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
@@ -205,6 +209,11 @@ def moe_prefill_delta(ctx, layer, x, N, delta, stream=None):
     _check(ctx, _lib.moe_prefill_delta(ctx, layer, _ptr(x), N, _ptr(delta), _stream(stream)))
 
 
+def moe_prefill_route(ctx, layer, h, N, idx, w, bucket_off=None, bucket_perm=None, stream=None):
+    _check(ctx, _lib.moe_prefill_route(ctx, layer, _ptr(h), N, _ptr(idx), _ptr(w),
+                                       _ptr(bucket_off), _ptr(bucket_perm), _stream(stream)))
+
+
 def moe_sync(ctx, timeout_ms=-1):
     _check(ctx, _lib.moe_sync(ctx, int(timeout_ms)))
 
@@ -232,6 +241,10 @@ def moe_expert_bytes(d, f, quant_fmt):
 
 def moe_debug_poke_slot(ctx, layer, expert, slot):
     _check(ctx, _lib.moe_debug_poke_slot(ctx, layer, expert, slot))
+
+
+def moe_debug_last_h(ctx, out, T, stream=None):
+    _check(ctx, _lib.moe_debug_last_h(ctx, _ptr(out), T, _stream(stream)))
 
 
 def moe_set_profiling(ctx, enable):
@@ -270,3 +283,15 @@ def moe_route_static(h, T, d, E, k, W, bias, idx, w, bucket_off, bucket_perm, st
     _check(None, _lib.moe_route_static(_ptr(h), T, d, E, k, _ptr(W), _ptr(bias), _ptr(idx),
                                        _ptr(w), _ptr(bucket_off), _ptr(bucket_perm),
                                        _stream(stream)))
+
+
+def moe_route_static_status(stream=None):
+    """Device status word of the last moe_route_static call on this device.
+    Returns the word (0 = fine); raises MoeError when it is non-zero."""
+    st = ctypes.c_int(0)
+    rc = _lib.moe_route_static_status(ctypes.byref(st), _stream(stream))
+    if rc not in (MOE_OK, 6):
+        _check(None, rc)
+    if rc == 6:
+        raise MoeError(rc, f"moe_route_static device status 0x{st.value:x}")
+    return st.value

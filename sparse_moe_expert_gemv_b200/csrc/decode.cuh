@@ -206,7 +206,7 @@ struct DecodeParams {
   const uint8_t *arena, *pool, *shared;
   long long expert_bytes, p1_bytes;
   float *logits;        // [T, E]
-  uint16_t *hbuf;       // bf16 [T, d]: the normalised window (wide windows with RMSNorm)
+  uint16_t *hbuf;       // bf16 [T, d]: the normalised window (written by CTA 0 with RMSNorm)
   uint16_t *abuf;       // bf16 [T*k + T, f]
   float *ybuf;          // fp32 [T*k + T, d]
   float *ws;            // stream-K partial sums [warps of the grid][32][16]
@@ -742,9 +742,10 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
         v.x = o[0] | ((uint32_t)o[1] << 16);
         v.y = o[2] | ((uint32_t)o[3] << 16);
         *reinterpret_cast<uint2 *>(hr + i) = v;
-        // wide windows re-stage rows after routing: CTA 0 publishes the
-        // normalised rows (visible to every CTA after the first barrier)
-        if (L.restage && blockIdx.x == 0) *reinterpret_cast<uint2 *>(p.hbuf + (long long)t * d + i) = v;
+        // CTA 0 publishes the normalised rows: wide windows re-stage them
+        // after routing (visible to every CTA after the first barrier), and
+        // moe_debug_last_h reads them back
+        if (blockIdx.x == 0) *reinterpret_cast<uint2 *>(p.hbuf + (long long)t * d + i) = v;
       }
     }
     __syncthreads();

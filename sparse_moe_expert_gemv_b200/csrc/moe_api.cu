@@ -60,7 +60,7 @@ struct moe_ctx {
   int *job_beg = nullptr, *job_n = nullptr, *n_jobs = nullptr;
   uint16_t *hbuf = nullptr, *abuf = nullptr;
   int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
-  unsigned int *ticket = nullptr;    // fused-routing CTA counter
+  unsigned int *ticket = nullptr;    // fused routing: [0] CTA counter, [1] abort flag
   // single-launch decode kernel: grid barrier counter, hand-over flags and
   // partial sums (one slot per warp of the grid)
   unsigned long long *dec_bar = nullptr, *dec_flags = nullptr;
@@ -202,7 +202,7 @@ moe_status do_configure(moe_ctx *c) {
     off += (bytes + 255) / 256 * 256;
     return at;
   };
-  const size_t o_status = carve(sizeof(int)), o_ticket = carve(sizeof(unsigned int));
+  const size_t o_status = carve(sizeof(int)), o_ticket = carve(2 * sizeof(unsigned int));
   const size_t dec_warps = (size_t)c->n_sm * 16;
   const size_t o_dbar = carve(sizeof(unsigned long long) * (1 + 2 * dec_warps));
   const size_t o_dws = carve(sizeof(float) * dec_warps * 32 * 16);
@@ -630,18 +630,15 @@ bool use_prefill_gemm(const moe_ctx *c, int N) {
          c->f % kPfBN == 0 && c->E <= kPfMaxE;
 }
 
-moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta, cudaStream_t s) {
-  const int E = c->E, k = c->k, d = c->d, f = c->f;
-  if (!c->pf_maps) {
-    if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
-        !encode_map_f16(&c->pf_map_a, c->abuf, c->pf_rows, f))
-      return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    c->pf_maps = true;
-  }
-  CUDA_TRY(c, prof_mark(c, 0, s));
+// The prefill chunk's routing on router input h: logits, top-k + softmax
+// (idx, w), the sort of the chunk's pairs by expert (each expert's rows in
+// ascending t), the 128-row tile list with the residency lookup, and the
+// gather of the grouped fp16 A rows.  perm (or null) receives the bucket
+// permutation; the bucket offsets are left in c->pf_eoff.
+moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int32_t *idx, float *w,
+                              int32_t *perm, cudaStream_t s) {
+  const int E = c->E, k = c->k, d = c->d;
   cudaError_t e = cudaSuccess;
-  const uint16_t *h = router_input(c, layer, x, N, s, &e);
-  CUDA_TRY(c, e);
   const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
   if (launch_router_tc(c, s, h, N, layer, &e)) {
     CUDA_TRY(c, e);
@@ -651,7 +648,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
                        dim3(256), 0, s, rp));
   }
   const int blocks = (N + kPfTok - 1) / kPfTok;
-  PfRouteParams tp{c->logits, N, E, k, c->idx, c->w, c->pf_bmask, &c->stats[4]};
+  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4]};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;
@@ -677,9 +674,26 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   sp.status = c->status;
   CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32), dim3(kPfColWarps * 32), 0, s, sp));
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
-  PfScatterParams cp{c->idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
-                     c->pf_row_of, c->pf_hg};
+  PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
+                     c->pf_row_of, c->pf_hg, perm};
   CUDA_TRY(c, launch(prefill_scatter_kernel, dim3(blocks), dim3(kPfTok * 32), 0, s, cp));
+  return MOE_OK;
+}
+
+moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta, cudaStream_t s) {
+  const int k = c->k, d = c->d, f = c->f;
+  if (!c->pf_maps) {
+    if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
+        !encode_map_f16(&c->pf_map_a, c->abuf, c->pf_rows, f))
+      return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    c->pf_maps = true;
+  }
+  CUDA_TRY(c, prof_mark(c, 0, s));
+  cudaError_t e = cudaSuccess;
+  const uint16_t *h = router_input(c, layer, x, N, s, &e);
+  CUDA_TRY(c, e);
+  moe_status st = prefill_route_impl(c, layer, h, N, c->idx, c->w, nullptr, s);
+  if (st) return st;
   CUDA_TRY(c, prof_mark(c, 1, s));
   PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
                   nullptr, c->status};
@@ -1202,6 +1216,27 @@ moe_status moe_prefill_delta(moe_ctx *c, int layer, const void *x, int N, float 
   return prefill_impl(c, layer, xp, N, delta, (cudaStream_t)stream);
 }
 
+moe_status moe_prefill_route(moe_ctx *c, int layer, const void *h, int N, int32_t *idx, float *w,
+                             int32_t *boff, int32_t *bperm, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !h || !idx || !w || N < 1 || N > c->max_tokens || !aligned16(h))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_prefill_route: bad arguments (N=%d max=%d)", N,
+                c->max_tokens);
+  if (!c->pf)
+    return fail(c, MOE_ERR_NOT_SUPPORTED,
+                "moe_prefill_route: context configured for decode windows only (max_tokens <= 32)");
+  if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  moe_status st = prefill_route_impl(c, layer, (const uint16_t *)h, N, idx, w, bperm, s);
+  if (st) return st;
+  if (boff)
+    CUDA_TRY(c, cudaMemcpyAsync(boff, c->pf_eoff, (size_t)(c->E + 1) * sizeof(int32_t),
+                                cudaMemcpyDeviceToDevice, s));
+  return MOE_OK;
+}
+
 moe_status moe_sync(moe_ctx *c, int timeout_ms) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (!c->configured) return MOE_OK;
@@ -1219,9 +1254,13 @@ moe_status moe_sync(moe_ctx *c, int timeout_ms) {
   int st = 0;
   CUDA_TRY(c, cudaMemcpyAsync(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost, c->io));
   CUDA_TRY(c, cudaMemsetAsync(c->status, 0, sizeof(int), c->io));
-  // a decode kernel that gave up a wait may have left its grid barrier
-  // counter mid-count: start it (and the hand-over flags) again from zero
-  if (st & kErrTimeout) CUDA_TRY(c, cudaMemsetAsync(c->dec_bar, 0, c->dec_sync_bytes, c->io));
+  // a kernel that gave up a wait may have left a counter mid-count: start
+  // the decode grid barrier, its hand-over flags and the fused-routing
+  // ticket again from zero
+  if (st & kErrTimeout) {
+    CUDA_TRY(c, cudaMemsetAsync(c->dec_bar, 0, c->dec_sync_bytes, c->io));
+    CUDA_TRY(c, cudaMemsetAsync(c->ticket, 0, 2 * sizeof(unsigned int), c->io));
+  }
   CUDA_TRY(c, cudaStreamSynchronize(c->io));
   if (st & kErrBadSlot) return fail(c, MOE_ERR_BAD_SLOT, "device status 0x%x: bad slot", st);
   if (st) return fail(c, MOE_ERR_DEVICE, "device status 0x%x", st);
@@ -1320,6 +1359,17 @@ moe_status moe_debug_poke_slot(moe_ctx *c, int layer, int expert, int32_t slot) 
   return MOE_OK;
 }
 
+// Debug hook: the normalised router input h (bf16 [T, d]) that the most
+// recent forward or prefill call of a layer with RMSNorm computed, copied on
+// `stream` into caller memory.
+moe_status moe_debug_last_h(moe_ctx *c, void *out, int T, void *stream) {
+  if (!c || !out || !c->configured || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_debug_last_h");
+  CUDA_TRY(c, cudaMemcpyAsync(out, c->hbuf, (size_t)T * c->d * 2, cudaMemcpyDeviceToDevice,
+                              (cudaStream_t)stream));
+  return MOE_OK;
+}
+
 }  // extern "C"
 
 // ======================================================================
@@ -1342,7 +1392,8 @@ namespace {
 constexpr int kStaticMaxT = kFusedMaxT;  // tokens per call
 constexpr int kStaticMaxE = 1024;        // experts
 constexpr int kStaticMaxD = kFusedMaxV * 128;
-constexpr size_t kStaticHeader = 256;    // ticket, status, statistics words
+constexpr size_t kStaticHeader = 256;    // ticket + abort flag, status, statistics words
+constexpr size_t kStaticStatusOff = 16;  // the status word, inside the header
 constexpr size_t kStaticScratchBytes =
     kStaticHeader + (size_t)kStaticMaxT * kStaticMaxE * sizeof(float);
 
@@ -1416,7 +1467,7 @@ moe_status moe_route_static(const void *h, int T, int d, int E, int k, const flo
   fp.off = boff;
   fp.perm = bperm;
   fp.build_jobs = 0;
-  fp.status = reinterpret_cast<int *>(base + 16);
+  fp.status = reinterpret_cast<int *>(base + kStaticStatusOff);
   fp.stats = reinterpret_cast<unsigned long long *>(base + 64);
   const int warps = T <= 8 ? 4 : kFusedWarps;
   const dim3 grid((E + warps - 1) / warps), block(warps * 32);
@@ -1434,6 +1485,30 @@ moe_status moe_route_static(const void *h, int T, int d, int E, int k, const flo
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+moe_status moe_route_static_status(int *status_out, void *stream) {
+  if (!status_out) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  unsigned char *base = nullptr;
+  if (static_scratch(dev, &base) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  int st = 0;
+  cudaError_t e = cudaMemcpyAsync(&st, base + kStaticStatusOff, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  *status_out = st;
+  return st ? MOE_ERR_DEVICE : MOE_OK;
 }
 
 }  // extern "C"

@@ -203,10 +203,13 @@ struct PfScatterParams {
   int T, E, k, d, has_shared;
   int *row_of;                  // [T*k + T]: grouped row of pair (shared pair P + t)
   __half *hg;                   // fp16 [rows][d] grouped A matrix
+  int *perm;                    // [T*k] or null: pair id of each routed grouped row
 };
 
 // One warp per token: its k pairs (and its shared-expert pair) get their
 // grouped rows, and the token's row is copied (fp16, saturating) to each.
+// With perm set, the routed rows' pair ids are also written in grouped
+// order: the bucket permutation (each expert's pairs in ascending t).
 __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterParams p) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   pdl_wait();
@@ -222,7 +225,11 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
     rows[j] = p.eoff[e] + p.boff[(long long)blockIdx.x * p.E + e] + rank;
   }
   if (p.has_shared) rows[p.k] = P + t;
-  if (lane < p.k) p.row_of[(long long)t * p.k + lane] = rows[lane];
+  if (lane < p.k) {
+    p.row_of[(long long)t * p.k + lane] = rows[lane];
+    // the bucket permutation: grouped row -> pair id (rows < P are routed)
+    if (p.perm) p.perm[rows[lane]] = t * p.k + lane;
+  }
   if (lane == 0 && p.has_shared) p.row_of[P + t] = P + t;
   // copy the token row to every destination, 8 elements per lane per step
   const uint4 *src = reinterpret_cast<const uint4 *>(p.h + (long long)t * p.d);

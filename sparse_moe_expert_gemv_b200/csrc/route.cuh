@@ -410,7 +410,8 @@ struct RouteFusedParams {
   const float *bias;       // fp32 [E] or null
   int d;
   float *logits;           // fp32 [T, E]
-  unsigned int *ticket;    // CTA completion counter, zero between calls
+  unsigned int *ticket;    // [0] CTA completion counter, [1] abort flag; both
+                           // zero between calls (the last CTA resets them)
   FinishParams f;
 };
 
@@ -424,7 +425,10 @@ constexpr int kFusedMaxV = 16;  // router row in registers: d <= 16 * 128
 // squares, IEEE sqrt and divide, bf16 round-to-nearest-even), and each warp
 // dots one router row (loaded into registers before the dependency wait)
 // with every token, four tokens at a time, fp32 accumulate.  The last CTA to finish (atomic ticket) runs the
-// routing body on the complete logits and resets the ticket.
+// routing body on the complete logits and resets the ticket.  A CTA whose
+// staging wait gives up reports kErrTimeout, raises the abort flag and still
+// takes its ticket, so the count completes: the last CTA then leaves the
+// outputs unwritten and resets both words, and the next call starts clean.
 template <int NPL>
 __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteFusedParams p) {
   extern __shared__ __align__(128) unsigned char fsm[];
@@ -457,11 +461,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteFuse
     mbar_expect_tx(smem_addr(&s_bar), bytes);
     bulk_g2s(smem_addr(fsm), p.x, bytes, smem_addr(&s_bar));
   }
-  if (!mbar_wait_bounded(smem_addr(&s_bar), 0)) {
-    if (threadIdx.x == 0) atomicOr(p.f.status, kErrTimeout);
-    return;
+  // the whole CTA agrees on the outcome of the wait (no thread leaves alone)
+  const bool staged = !__syncthreads_or(!mbar_wait_bounded(smem_addr(&s_bar), 0));
+  if (!staged && threadIdx.x == 0) {
+    atomicOr(p.f.status, kErrTimeout);
+    atomicOr(p.ticket + 1, 1u);
   }
-  if (p.use_norm) {
+  if (staged && p.use_norm) {
     for (int t = wid; t < T; t += nw) {
       uint16_t *hr = reinterpret_cast<uint16_t *>(fsm) + (long long)t * d;
       float ss = 0.f;
@@ -494,7 +500,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteFuse
   }
 
   // logits of this warp's expert for every token
-  if (e < E) {
+  if (staged && e < E) {
     const uint32_t hb0 = smem_addr(fsm);
     for (int t = 0; t < T; t += 4) {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -531,14 +537,21 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteFuse
   if (threadIdx.x == 0) {
     __threadfence();
     s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
-    if (s_last) __threadfence();
+    if (s_last) {
+      __threadfence();
+      // a CTA gave up: some logits are missing, route nothing
+      if (atomicAdd(p.ticket + 1, 0u) != 0u) s_last = 2;
+    }
   }
   __syncthreads();
   if (!s_last) return;
   MOE_TRACE(kTrRouteLastStart);
-  finish_body<NPL>(p.f, reinterpret_cast<int *>(fsm), slot_pref);
+  if (s_last == 1) finish_body<NPL>(p.f, reinterpret_cast<int *>(fsm), slot_pref);
   MOE_TRACE(kTrRouteEnd);
-  if (threadIdx.x == 0) *p.ticket = 0u;
+  if (threadIdx.x == 0) {
+    p.ticket[1] = 0u;
+    p.ticket[0] = 0u;
+  }
   // the expert kernels may launch now (not earlier: CTAs parked in their
   // dependency wait would compete with this CTA, the critical path)
   __syncthreads();

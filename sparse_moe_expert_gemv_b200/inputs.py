@@ -24,6 +24,11 @@ N(0, 0.02) weight matrix after quantisation in each format):
 * hidden states: bf16 N(0, 1) (float64 -> fp32 -> bf16, round to nearest even);
 * Zipf router bias: b[e] = ln p_rank(e), p_r proportional to r^-s, with a
   seeded per-layer permutation mapping rank to expert.
+
+Two more expert sources serve the parity tests: ``expert_weights_np`` draws
+an expert's unquantised matrices from N(0, 0.02) (float64), for a quantiser
+to encode; ``expert_uniform_codes_np`` draws every code value with equal
+probability (all 16 Q4 nibbles, level -8 included; all four Q2 codes).
 """
 from __future__ import annotations
 
@@ -38,6 +43,7 @@ _GOLD = 0x9E3779B9
 
 # stream kinds
 K_CODES, K_SCALES, K_MINS, K_ROUTER, K_ZIPF, K_HIDDEN, K_IDX, K_GAMMA = range(1, 9)
+K_WEIGHTS, K_UCODES = 9, 10
 SHARED_INDEX = 4095  # expert index used for the shared expert's streams
 
 Q4, Q2 = 1, 2
@@ -172,6 +178,15 @@ def shared_np(seed: int, fmt: int, d: int, f: int, layer: int):
     return expert_np(seed, fmt, d, f, layer, SHARED_INDEX)
 
 
+def expert_uniform_codes_np(seed: int, fmt: int, d: int, f: int, layer: int, e: int):
+    """One packed expert whose code bytes are uniform (every nibble / 2-bit
+    code equally likely); scales (and mins) as in ``expert_np``."""
+    nb, _ = expert_sizes(fmt, d, f)
+    u = u32_np(seed, stream_id(K_UCODES, layer, e), np.arange(nb, dtype=np.uint64))
+    _, scales, mins = expert_np(seed, fmt, d, f, layer, e)
+    return (u & 0xFF).astype(np.uint8), scales, mins
+
+
 def _normal_np(seed, stream, n):
     u = u32_np(seed, stream, np.arange(2 * n, dtype=np.uint64)).astype(np.float64)
     u1 = (u[0::2] + 0.5) / 4294967296.0
@@ -194,6 +209,14 @@ def hidden_np(seed: int, T: int, d: int, window: int = 0, layer: int = 0):
     """bf16 bits [T, d], N(0,1)."""
     z = _normal_np(seed, stream_id(K_HIDDEN, layer, window), T * d)
     return f32_to_bf16_bits(z.astype(np.float32)).reshape(T, d)
+
+
+def expert_weights_np(seed: int, d: int, f: int, layer: int, e: int, std: float = 0.02):
+    """Unquantised matrices of one expert, N(0, std) in float64:
+    (Wg [f, d], Wu [f, d], Wd [d, f])."""
+    z = _normal_np(seed, stream_id(K_WEIGHTS, layer, e), 3 * f * d) * std
+    return (z[:f * d].reshape(f, d), z[f * d:2 * f * d].reshape(f, d),
+            z[2 * f * d:].reshape(d, f))
 
 
 def router_np(seed: int, E: int, d: int, layer: int = 0, std: float = 0.02):

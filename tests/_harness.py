@@ -7,6 +7,9 @@ else.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 import oracle as O
@@ -19,20 +22,52 @@ TIE_MARGIN = 1e-5   # oracle k-th vs (k+1)-th fp64 logit gap below which a
                     # token is excluded from the bit-exact routing checks
 
 
-class LayerSpec:
-    """One MoE layer's synthetic weights (router, experts, shared expert)."""
+def quantised_expert(seed, fmt, d, f, layer, e):
+    """An expert whose N(0, 0.02) matrices are encoded by the oracle's
+    quantiser (the packed bytes both sides then consume)."""
+    mats = I.expert_weights_np(seed, d, f, layer, e)
+    parts = [O.quantize(fmt, W) for W in mats]
+    codes = np.concatenate([p[0] for p in parts])
+    scales = np.concatenate([p[1] for p in parts])
+    mins = None if fmt == O.Q4 else np.concatenate([p[2] for p in parts])
+    return codes, scales, mins
 
-    def __init__(self, *, d, f, E, k, fmt, seed=0, shared=True, zipf=False, layer=0):
+
+class LayerSpec:
+    """One MoE layer's synthetic weights (router, experts, shared expert).
+
+    weights: "codes" -- the generator's packed codes (``inputs.expert_np``);
+    "quantised" -- N(0, 0.02) matrices encoded by the oracle's quantiser,
+    for the experts in ``quantise`` (all when None; the others keep the
+    generator's codes); "uniform" -- uniform code bytes (every code value)."""
+
+    def __init__(self, *, d, f, E, k, fmt, seed=0, shared=True, zipf=False, layer=0,
+                 weights="codes", quantise=None):
         self.d, self.f, self.E, self.k, self.fmt = d, f, E, k, fmt
         self.seed, self.shared, self.zipf, self.layer = seed, shared, zipf, layer
+        self.weights, self.quantise = weights, quantise
         self.W = I.router_np(seed, E, d, layer)
         self.bias = I.zipf_bias_np(seed, E, layer)[0] if zipf else None
         self._host = {}
 
-    # ---- expert bytes (generator output), host side for the oracle
+    def special(self, e):
+        """Whether expert e (SHARED_INDEX for the shared one) differs from
+        the generator's codes."""
+        if self.weights == "codes":
+            return False
+        return self.quantise is None or e in self.quantise
+
+    def _make(self, e):
+        if self.special(e):
+            if self.weights == "quantised":
+                return quantised_expert(self.seed, self.fmt, self.d, self.f, self.layer, e)
+            return I.expert_uniform_codes_np(self.seed, self.fmt, self.d, self.f, self.layer, e)
+        return I.expert_np(self.seed, self.fmt, self.d, self.f, self.layer, e)
+
+    # ---- expert bytes, host side for the oracle
     def expert(self, e):
         if e not in self._host:
-            self._host[e] = I.expert_np(self.seed, self.fmt, self.d, self.f, self.layer, e)
+            self._host[e] = self._make(e)
         return self._host[e]
 
     def set_host_experts(self, codes, scales, mins):
@@ -42,7 +77,11 @@ class LayerSpec:
                              None if mins is None else mins[e].view(np.uint16))
 
     def shared_expert(self):
-        return I.shared_np(self.seed, self.fmt, self.d, self.f, self.layer) if self.shared else None
+        if not self.shared:
+            return None
+        if "shared" not in self._host:
+            self._host["shared"] = self._make(I.SHARED_INDEX)
+        return self._host["shared"]
 
     # ---- oracle
     def oracle(self, x_bits, norm=False, eps=1e-6, route_only_experts=None):
@@ -82,7 +121,86 @@ def load_layer(B, ctx, spec: LayerSpec, layer=0, device="cuda", chunk=64):
     scales = np.concatenate(hs)
     mins = None if hm[0] is None else np.concatenate(hm)
     spec.set_host_experts(codes, scales, mins)
+    # experts that are not the generator's codes: host bytes, one by one
+    for e in range(spec.E):
+        if spec.special(e):
+            spec._host.pop(e, None)
+            c, s, m = spec.expert(e)
+            B.moe_load_experts(ctx, layer, e, 1, c, s, m)
     return codes, scales, mins
+
+
+# ------------------------------------------------- oracle on many host cores
+def oracle_threads():
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def router_parallel(h_bits, W, bias=None, threads=None):
+    """O.router over row chunks on a thread pool (the C oracle runs without
+    the GIL); the result is the oracle's, row for row."""
+    h_bits = np.ascontiguousarray(h_bits, np.uint16)
+    n = threads or oracle_threads()
+    chunks = np.array_split(np.arange(h_bits.shape[0]), n)
+    with ThreadPoolExecutor(n) as ex:
+        parts = list(ex.map(lambda r: O.router(h_bits[r], W, bias), [c for c in chunks if c.size]))
+    return np.concatenate(parts)
+
+
+def oracle_rows(spec, x_bits, rows, threads=None, norm=False):
+    """The oracle's whole layer on the given rows (tokens are independent),
+    in chunks on a thread pool.  Returns (delta [n, d], x_out [n, d] bits,
+    margin [n]) in the order of ``rows``."""
+    rows = np.asarray(rows)
+    n = min(threads or oracle_threads(), max(1, rows.size))
+    chunks = [c for c in np.array_split(np.arange(rows.size), n) if c.size]
+
+    def one(c):
+        out = spec.oracle(x_bits[rows[c]], norm=norm)
+        return out["delta"], out["x_out"], out["margin"]
+
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        parts = list(ex.map(one, chunks))
+    return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts]),
+            np.concatenate([p[2] for p in parts]))
+
+
+def covering_sample(idx, E, tile=128, n_hot=3):
+    """Tokens (sorted) such that, in the expert-grouped order of the pairs
+    (each expert's tokens ascending), every expert's first and last
+    ``tile``-row tile holds a sampled token, every tile of the ``n_hot``
+    experts with most tokens does, and so do each expert's first and last
+    token (the edges of its first and last tiles).  Chosen greedily, so one
+    token covers the tiles of all its experts."""
+    T, k = idx.shape
+    lists = [[] for _ in range(E)]
+    for t in range(T):
+        for e in idx[t]:
+            lists[int(e)].append(t)
+    counts = np.array([len(l) for l in lists])
+    hot = set(np.argsort(-counts, kind="stable")[:n_hot].tolist())
+    need = {}   # (expert, tile) -> tokens of that tile
+    must = set()
+    for e in range(E):
+        L = lists[e]
+        if not L:
+            continue
+        nt = (len(L) + tile - 1) // tile
+        tiles = range(nt) if e in hot else sorted({0, nt - 1})
+        for m in tiles:
+            need[(e, m)] = set(L[m * tile:(m + 1) * tile])
+        must.add(L[0])
+        must.add(L[-1])
+    chosen = set(must)
+    open_ = {key for key, toks in need.items() if not (toks & chosen)}
+    while open_:
+        score = {}
+        for key in open_:
+            for t in need[key]:
+                score[t] = score.get(t, 0) + 1
+        best = min(score, key=lambda t: (-score[t], t))
+        chosen.add(best)
+        open_ = {key for key in open_ if best not in need[key]}
+    return np.array(sorted(chosen))
 
 
 def rms(a):

@@ -102,8 +102,10 @@ def test_reference_arm_json_line():
     assert j["metric"] == "decode MoE tokens/s" and j["unit"] == "tokens/s" and j["higher_is_better"]
     assert j["steps"] == 1 and j["warmup"] == 3 and j["value"] > 0
     assert "T=4" in j["config"]["workload"] and "d=2048" in j["config"]["workload"]
+    assert j["config"]["tokens_per_step"] == 4 and j["config"]["same_window"] is True
     cb = j["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
+    assert cb["nproc"] >= 1 and cb["usable_cores"] == cb["cores"] and "cpu_model" in cb
     e = j["e2e"]
     assert e["value"] == j["value"] and e["unit"] == j["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0

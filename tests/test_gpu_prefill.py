@@ -10,7 +10,8 @@ import torch
 
 import oracle as O
 from sparse_moe_expert_gemv_b200 import inputs as I
-from tests._harness import TIE_MARGIN, LayerSpec, assert_close_rms, load_layer
+from tests._harness import (TIE_MARGIN, LayerSpec, assert_close_rms, check_buckets, check_routing,
+                            covering_sample, load_layer, oracle_rows, router_parallel)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,6 +68,16 @@ def test_prefill_small_layer_all_tokens(B, N, zipf):
         delta, x_out = run_prefill(B, ctx, spec, x)
         rel, ties = check_rows(spec, x, delta, x_out, np.arange(N))
         print(f"N={N} zipf={zipf}: delta max-err/RMS {rel:.2e}, near ties {ties}")
+        # the same chunk's routing and buckets, bit for bit
+        out = _route_outputs(N, spec.k, spec.E)
+        B.moe_prefill_route(ctx, 0, to_dev(x), N, *out)
+        B.moe_sync(ctx, 60000)
+        idx, w, off, perm = [t.cpu().numpy() for t in out]
+        lg = O.router(x, spec.W, spec.bias)
+        oi, ow, om = O.topk(lg, spec.k)
+        orc = dict(idx=oi, w=ow, margin=om)
+        ok = check_routing(idx, w, orc, spec.k)
+        check_buckets(off, perm, oi, spec.E, spec.k, ok)
     finally:
         B.moe_destroy(ctx)
 
@@ -102,20 +113,94 @@ def test_prefill_q2_takes_the_gemv_path(B):
         B.moe_destroy(ctx)
 
 
-def test_prefill_chunk_8192_zipf_sampled(B):
+# ------------------------------------------------ the 8192-token chunk
+@pytest.fixture(scope="module")
+def chunk8192(B):
     """The prefill workload: d=2048, f=768, E=512, top-10 + shared, Q4 g32,
-    8192 tokens, Zipf(1.1)-biased routing; 16 sampled tokens against the
-    oracle."""
+    one chunk of 8192 tokens, Zipf(1.1)-biased routing; with the oracle's
+    fp64 routing of every token (computed on a thread pool)."""
     spec = LayerSpec(d=2048, f=768, E=512, k=10, fmt=I.Q4, seed=0, shared=True, zipf=True)
     ctx = make_ctx(B, spec, 8192)
+    load_layer(B, ctx, spec)
+    N = 8192
+    x = I.hidden_np(0, N, spec.d, window=4242)
+    lg = router_parallel(x, spec.W, spec.bias)
+    idx, w, margin = O.topk(lg, spec.k)
+    yield ctx, spec, x, dict(idx=idx, w=w, margin=margin)
+    B.moe_destroy(ctx)
+
+
+def _route_outputs(N, k, E):
+    return [torch.empty((N, k), dtype=torch.int32, device="cuda"),
+            torch.empty((N, k), dtype=torch.float32, device="cuda"),
+            torch.empty(E + 1, dtype=torch.int32, device="cuda"),
+            torch.empty(N * k, dtype=torch.int32, device="cuda")]
+
+
+def test_prefill_route_8192_bit_exact(B, chunk8192):
+    """The prefill path's own routing (tensor-core router, one warp per token
+    top-k, per-expert column scan, scan, scatter) against the oracle on all
+    8192 tokens: expert sets and bucket contents bit-exact, weights within
+    1e-5, near ties (oracle margin < 1e-5) excluded and counted."""
+    ctx, spec, x, orc = chunk8192
+    N = x.shape[0]
+    out = _route_outputs(N, spec.k, spec.E)
+    B.moe_prefill_route(ctx, 0, to_dev(x), N, *out)
+    B.moe_sync(ctx, 120000)
+    idx, w, off, perm = [t.cpu().numpy() for t in out]
+    ok = check_routing(idx, w, orc, spec.k)
+    check_buckets(off, perm, orc["idx"], spec.E, spec.k, ok)
+    ties = int((~ok).sum())
+    print(f"prefill routing, 8192 tokens: near ties {ties}")
+    assert ties <= 8
+
+
+@pytest.mark.parametrize("N", [512, 8192])
+def test_moe_route_large_windows_bit_exact(B, chunk8192, N):
+    """moe_route on 512 and 8192 tokens (E = 512): the tensor-core router
+    path of the multi-launch routing, against the oracle on every token."""
+    ctx, spec, x, orc = chunk8192
+    out = _route_outputs(N, spec.k, spec.E)
+    B.moe_route(ctx, 0, to_dev(x[:N]), N, *out)
+    B.moe_sync(ctx, 120000)
+    idx, w, off, perm = [t.cpu().numpy() for t in out]
+    sub = {key: v[:N] for key, v in orc.items()}
+    ok = check_routing(idx, w, sub, spec.k)
+    check_buckets(off, perm, sub["idx"], spec.E, spec.k, ok)
+    print(f"moe_route N={N}: near ties {int((~ok).sum())}")
+
+
+def test_prefill_chunk_8192_covering_sample(B, chunk8192):
+    """The whole prefill layer at 8192 tokens against the oracle on a
+    deterministic sample of tokens that covers every expert's first and last
+    128-row GEMM tile (and each expert's first and last row), every tile of
+    the three hottest experts, and the shared expert's first and last tiles."""
+    ctx, spec, x, orc = chunk8192
+    N = x.shape[0]
+    delta, x_out = run_prefill(B, ctx, spec, x)
+    assert np.isfinite(delta).all()
+    rows = np.union1d(covering_sample(orc["idx"], spec.E), [0, 127, 128, N - 129, N - 128, N - 1])
+    ok = orc["margin"][rows] >= TIE_MARGIN
+    od, ox, _ = oracle_rows(spec, x, rows)
+    rel = assert_close_rms(delta[rows][ok], od[ok], what="MoE delta")
+    assert_close_rms(I.bf16_bits_to_f32(x_out[rows][ok]), I.bf16_bits_to_f32(ox[ok]),
+                     what="residual x")
+    print(f"prefill 8192: {rows.size} sampled tokens, delta max-err/RMS {rel:.2e}, "
+          f"near ties {int((~ok).sum())}")
+
+
+def test_prefill_route_rejects_bad_calls(B):
+    spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=I.Q4, seed=5, shared=True)
+    ctx = make_ctx(B, spec, 16)  # decode-only context: no prefill buffers
     try:
         load_layer(B, ctx, spec)
-        N = 8192
-        x = I.hidden_np(0, N, spec.d, window=4242)
-        delta, x_out = run_prefill(B, ctx, spec, x)
-        rows = np.sort(np.random.default_rng(1).choice(N, size=16, replace=False))
-        rel, ties = check_rows(spec, x, delta, x_out, rows)
-        print(f"prefill 8192: delta max-err/RMS {rel:.2e}, near ties {ties}")
-        assert np.isfinite(delta).all()
+        x = to_dev(I.hidden_np(5, 8, spec.d))
+        out = _route_outputs(8, spec.k, spec.E)
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_prefill_route(ctx, 0, x, 8, *out)
+        assert ei.value.status == 8  # NOT_SUPPORTED
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_prefill_route(ctx, 0, x, 0, *out)
+        assert ei.value.status == 1
     finally:
         B.moe_destroy(ctx)

@@ -12,7 +12,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from sparse_moe_expert_gemv_b200 import inputs as I
+from tests._harness import check_buckets, check_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +50,40 @@ def test_route_static_matches_moe_route(B, zipf):
             assert torch.allclose(got[1], ref[1], rtol=0, atol=1e-5)
             assert torch.equal(got[2], ref[2])
             assert torch.equal(got[3], ref[3])
+            assert B.moe_route_static_status() == 0
     finally:
         B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("T,d,E,k,zipf", [
+    (1, 128, 16, 1, False),      # one token, smallest shapes
+    (9, 2048, 1024, 32, False),  # eight warps per CTA, 32 logits per lane, k at its limit
+    (32, 2048, 512, 10, True),   # the largest window, Zipf-biased
+    (32, 128, 1024, 1, True),
+    (9, 128, 16, 16, False),     # k = E
+])
+def test_route_static_matches_oracle(B, T, d, E, k, zipf):
+    """Across the shapes the entry point accepts, its expert sets and
+    bucket contents equal the oracle's bit for bit and its weights are
+    within 1e-5 (tokens whose oracle k-th and (k+1)-th logits differ by less
+    than 1e-5 are excluded and counted)."""
+    seed = 30 + T + E
+    W = I.router_np(seed, E, d)
+    bias = I.zipf_bias_np(seed, E)[0] if zipf else None
+    x = I.hidden_np(seed, T, d, window=E)
+    out = [torch.full((T, k), -7, dtype=torch.int32, device="cuda"),
+           torch.zeros((T, k), dtype=torch.float32, device="cuda"),
+           torch.zeros(E + 1, dtype=torch.int32, device="cuda"),
+           torch.zeros(T * k, dtype=torch.int32, device="cuda")]
+    B.moe_route_static(torch.from_numpy(x.view(np.int16)).cuda(), T, d, E, k,
+                       torch.from_numpy(W).cuda(),
+                       None if bias is None else torch.from_numpy(bias).cuda(), *out)
+    assert B.moe_route_static_status() == 0
+    idx, w, off, perm = [t.cpu().numpy() for t in out]
+    oi, ow, om = O.topk(O.router(x, W, bias), k)
+    ok = check_routing(idx, w, dict(idx=oi, w=ow, margin=om), k)
+    check_buckets(off, perm, oi, E, k, ok)
+    print(f"T={T} d={d} E={E} k={k}: near ties {int((~ok).sum())}")
 
 
 def test_route_static_rejects_sizes_beyond_its_scratch(B):
