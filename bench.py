@@ -424,7 +424,8 @@ def measure(args, world, ctx, spec, n_rot, K, W):
     else:
         kern_ms = exp_ms
         kern_bytes = expert_bytes
-        kern_name = "expert_gemv_kernel (gate/up + down launches of one call)"
+        kern_name = ("the experts of one call: prefill_gemm_kernel (gate/up + down, experts with "
+                     ">= 16 tokens) + expert_gemv_kernel (gate/up + down, the other experts)")
         per_unit = f"{Be} B per touched expert (codes+scales), shared expert included"
     kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
     res = {
@@ -457,7 +458,9 @@ def measure(args, world, ctx, spec, n_rot, K, W):
                                  "timing": "a second, event-bracketed pass of the same steps"},
         "roofline": {
             "bound": "tensor",
-            "kernel": "prefill_gemm_kernel (gate/up + down grouped GEMMs of one call, tcgen05 fp16)",
+            "kernel": ("the experts of one call: prefill_gemm_kernel (gate/up + down grouped GEMMs, "
+                       "tcgen05 fp16, experts with >= 16 tokens) + expert_gemv_kernel (the other "
+                       "experts)"),
             "achieved": gemm_tf,
             "peak": tflops,
             "unit": "TFLOP/s",
@@ -486,7 +489,8 @@ def measure(args, world, ctx, spec, n_rot, K, W):
         },
         "e2e": {"value": whole_job_rate(world, tok, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": K * (1 if single else (8 if prefill else 6)),
+        # chunks: router, top-k, column scan, scan, scatter, 2 GEMMs, 2 GEMVs, combine
+        "gpu_launches": K * (1 if single else 10),
         "clocks": clocks,
     }
     if single:

@@ -208,14 +208,14 @@ MOE_API moe_status moe_forward_stack(moe_ctx *ctx, void *x_dev, int T, void *str
  * `layer`, in place (x <- x + MoE(norm(x))).  The engine article "93 token/s
  * on one 8 GB card", section "Architecture overview", runs prefill in chunks
  * of up to 8192 tokens; per expert such a chunk is a dense contraction.  For
- * Q4 experts and N > 32 the experts run as a grouped GEMM on the tensor
- * cores (tcgen05): tokens sorted by expert, 128-token tiles, weights
- * dequantised to fp16 tile by tile in shared memory, fp32 accumulation in
- * tensor memory.  Activations enter as fp16 (exact for |h| < 65504; larger
- * values saturate), and the experts' outputs y are kept in fp16 until the
- * combine.  Router logits: fp32 accuracy, on the tensor cores from N >= 512
- * and E a multiple of 256 (see moe_set_router), else fp32 FMA.  Q2 experts
- * and N <= 32 take the moe_forward path.
+ * N > 32 the experts (Q4 or Q2) run as a grouped GEMM on the tensor cores
+ * (tcgen05): tokens sorted by expert, 128-token tiles, weights dequantised
+ * to fp16 tile by tile in shared memory (Q4: s (c - 8); Q2: s q + m, one
+ * fp16 rounding), fp32 accumulation in tensor memory.  Activations enter as
+ * fp16 (exact for |h| < 65504; larger values saturate), and the experts'
+ * outputs y are kept in fp16 until the combine.  Router logits: fp32
+ * accuracy, on the tensor cores from N >= 512 and E a multiple of 256 (see
+ * moe_set_router), else fp32 FMA.  N <= 32 takes the moe_forward path.
  * Requires a context configured with max_tokens >= N.  Errors: INVALID_ARG,
  * STATE; device faults through moe_sync. */
 MOE_API moe_status moe_prefill(moe_ctx *ctx, int layer, void *x_dev, int N,

@@ -174,6 +174,12 @@ MOE_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t ba
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// Bulk prefetch of [src, src + bytes) into L2 (no shared memory, no
+// completion); src 16-byte aligned, bytes a multiple of 16.
+MOE_DEV void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Policy for data read once: its L2 lines are the first to be evicted, so a
 // stream of them does not push other data (or code) out of L2.
 MOE_DEV uint64_t l2_evict_first() {

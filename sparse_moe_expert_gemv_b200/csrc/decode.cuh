@@ -216,6 +216,8 @@ struct DecodeParams {
   unsigned long long *stats;  // [0]=calls [1]=tokens [2]=hits [3]=misses [4]=near_ties
   int *last;
   int *status;
+  int prefetch;         // bit 0: L2-prefetch the warp's down units after routing;
+                        // bit 1: also its gate/up units beyond the ring's first ones
   DecSmem sm;
 };
 
@@ -829,6 +831,18 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     if (lane == 0) fence_proxy_async_smem();  // a wide window occupied the rings until now
     __syncwarp();
     ring_prologue(r, ph1, lane);
+  }
+  // The whole weight stream of the warp is known now: put it in flight to
+  // L2, so HBM streams every selected expert at full rate while the rings
+  // consume (gate/up units beyond the ring's first ones; the down units,
+  // which then wait in L2 for the second pass).
+  if (lane == 0 && p.prefetch) {
+    if (p.prefetch & 2) prefetch_units_l2(ph1, min(u0 + kRingD, u1), u1);
+    if (p.prefetch & 1) {
+      const Phase pd = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes);
+      const SKCtx sd = sk_make(n_jobs * pd.RB * pd.UPI, W, gw, 0, nullptr, nullptr, nullptr, nullptr, WARPS);
+      prefetch_units_l2(pd, sk_start(sd, gw), sk_start(sd, gw + 1));
+    }
   }
   decode_pairs(p, s_slot, s_mask, s_idx, s_cnt, s_plist);
   // Token rows for the gate/up B operand.  A window that fits the staging

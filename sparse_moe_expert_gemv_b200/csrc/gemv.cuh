@@ -101,6 +101,25 @@ MOE_DEV const unsigned char *item_base(const Phase &ph, int job, int rb) {
          (long long)rb * ph.NTILE * ph.stride;
 }
 
+// L2 prefetch of the pass's units [u0, u1) (job-major, then row block, then
+// unit).  A job's units are one contiguous byte range of its expert's
+// region, so the range is one prefetch run per job it touches, cut into
+// pieces of at most kPrefetchPiece bytes.  Issued by the calling lane.
+constexpr uint32_t kPrefetchPiece = 32768;
+MOE_DEV void prefetch_units_l2(const Phase &ph, int u0, int u1) {
+  if (u1 <= u0) return;
+  const int upj = ph.RB * ph.UPI;                 // units per job
+  const long long ubytes = (long long)ph.tps * ph.stride;
+  for (int job = u0 / upj; job * upj < u1; ++job) {
+    const int a = max(u0, job * upj), b = min(u1, (job + 1) * upj);
+    const unsigned char *p = reinterpret_cast<const unsigned char *>(ph.job_ptr[job]) + ph.region_off +
+                             (long long)(a - job * upj) * ubytes;
+    long long n = (long long)(b - a) * ubytes;
+    for (; n > 0; n -= kPrefetchPiece, p += kPrefetchPiece)
+      bulk_prefetch_l2(p, (uint32_t)(n < kPrefetchPiece ? n : kPrefetchPiece));
+  }
+}
+
 // A walk over consecutive weight units: n units from unit `unit` of item
 // (job, rb); the next item is istep row blocks further.  Only increments and
 // compares: no division per unit or item.

@@ -71,6 +71,10 @@ struct moe_ctx {
   __half *pf_hg = nullptr;              // grouped A rows, fp16 [rows][d]
   int *pf_row_of = nullptr, *pf_boff = nullptr, *pf_eoff = nullptr, *pf_ntiles = nullptr;
   unsigned short *pf_bmask = nullptr;
+  float *pf_part = nullptr;             // split router partial sums
+  __half *pf_a16 = nullptr, *pf_y16 = nullptr;  // GEMM a and y, fp16 [rows][f], [rows][d]
+  int *pf_perm = nullptr, *pf_hot = nullptr;     // bucket permutation [T*k], GEMM-expert flags [E]
+  long long pf_part_floats = 0;
   PfTile *pf_tiles = nullptr;
   int pf_max_tiles = 0, pf_rows = 0;
   CUtensorMap pf_map_h{}, pf_map_a{};   // TMA maps of the grouped A matrices
@@ -80,6 +84,7 @@ struct moe_ctx {
   std::vector<int32_t> host_counts;
 
   int gemv_blocks[2][2][2] = {};  // [fmt][gated][NTM-1]
+  int dec_prefetch = 3;           // decode_kernel L2 prefetch mode (DecodeParams::prefetch)
   // profiling: 4 events per call slot
   bool profiling = false;
   std::vector<cudaEvent_t> prof_ev;
@@ -257,6 +262,11 @@ moe_status do_configure(moe_ctx *c) {
     const size_t o_bm = pcarve((size_t)blocks * E * 2), o_bo = pcarve((size_t)blocks * E * 4);
     const size_t o_eo = pcarve((size_t)(E + 1) * 4), o_nt = pcarve(4);
     const size_t o_tl = pcarve((size_t)c->pf_max_tiles * sizeof(PfTile));
+    // a split reduction uses at most 2 n_sm 128 x 128 tiles of partial sums
+    c->pf_part_floats = 2LL * c->n_sm * kRgBM * kRgBN;
+    const size_t o_part = pcarve((size_t)c->pf_part_floats * sizeof(float));
+    const size_t o_a16 = pcarve((size_t)rows * f * 2), o_y16 = pcarve((size_t)rows * d * 2);
+    const size_t o_perm = pcarve((size_t)P * 4), o_hot = pcarve((size_t)E * 4);
     CUDA_TRY(c, cudaMalloc(&c->pf, po));
     CUDA_TRY(c, cudaMemset(c->pf, 0, po));
     c->pf_hg = (__half *)(c->pf + o_hg);
@@ -266,6 +276,11 @@ moe_status do_configure(moe_ctx *c) {
     c->pf_eoff = (int *)(c->pf + o_eo);
     c->pf_ntiles = (int *)(c->pf + o_nt);
     c->pf_tiles = (PfTile *)(c->pf + o_tl);
+    c->pf_part = (float *)(c->pf + o_part);
+    c->pf_a16 = (__half *)(c->pf + o_a16);
+    c->pf_y16 = (__half *)(c->pf + o_y16);
+    c->pf_perm = (int *)(c->pf + o_perm);
+    c->pf_hot = (int *)(c->pf + o_hot);
     // the router rows as three exact bf16 parts, for the tensor-core router
     CUDA_TRY(c, cudaMalloc(&c->d_router3, (size_t)c->L * E * 3 * d * sizeof(__nv_bfloat16)));
   }
@@ -490,6 +505,26 @@ cudaError_t prof_mark(moe_ctx *c, int i, cudaStream_t s) {
 // build_jobs); returns the router input h (x, or the normalised copy).
 bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, cudaError_t *err);
 
+// Router logits of a chunk of N > 32 tokens by fp32 FMA (router_gemm_kernel).
+// A chunk too small to give every SM a 128 x 128 tile splits the reduction
+// over blockIdx.z (a power of two dividing d / 128, partial sums bounded by
+// the pf_part buffer); *ksplit receives the split count: 1 = logits (with
+// bias) in c->logits, > 1 = partials in c->pf_part for the top-k to add.
+cudaError_t launch_router_fma(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, int *ksplit) {
+  const int E = c->E, d = c->d;
+  const int tiles = ((N + kRgBM - 1) / kRgBM) * ((E + kRgBN - 1) / kRgBN);
+  int ks = 1;
+  while (ks * tiles < c->n_sm && (d / 128) % (2 * ks) == 0 &&
+         (long long)2 * ks * N * E <= c->pf_part_floats)
+    ks *= 2;
+  *ksplit = ks;
+  RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d,
+                      c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E,
+                      ks > 1 ? c->pf_part : c->logits, d / ks};
+  return launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN, ks), dim3(256),
+                0, s, rp);
+}
+
 moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const FinishParams &fp,
                       cudaStream_t s, const uint16_t **h_out) {
   if (use_fused_route(c, T)) {
@@ -512,23 +547,26 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
   cudaError_t e = cudaSuccess;
   const uint16_t *h = router_input(c, layer, x, T, s, &e);
   CUDA_TRY(c, e);
-  RouterParams rp{h, c->d_router + (size_t)layer * c->E * c->d,
-                  c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr, T, c->d, c->E,
-                  c->logits};
-  if (launch_router_tc(c, s, h, T, layer, &e))  // large windows: tensor cores
-    CUDA_TRY(c, e);
-  else
-    CUDA_TRY(c, launch_router(c, s, rp));
+  const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * c->E : nullptr;
   if (T > kDecMaxT && c->pf_bmask) {
-    // many tokens: the top-k runs one warp per token across the grid, and
-    // the single routing CTA only buckets the selections and builds the jobs
-    PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4]};
+    // many tokens: logits on the tensor cores (large windows) or by a split
+    // fp32 GEMM, the top-k one warp per token across the grid, and the
+    // single routing CTA only buckets the selections and builds the jobs
+    int ks = 1;
+    if (launch_router_tc(c, s, h, T, layer, &e))
+      CUDA_TRY(c, e);
+    else
+      CUDA_TRY(c, launch_router_fma(c, s, h, T, layer, &ks));
+    PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4], c->pf_part, ks,
+                     bias};
     CUDA_TRY(c, launch_pf_topk(c, s, tp));
     FinishParams fb = fp;
     fb.logits = nullptr;
     fb.idx_in = fp.idx;
     CUDA_TRY(c, launch_finish(c, s, fb));
   } else {
+    RouterParams rp{h, c->d_router + (size_t)layer * c->E * c->d, bias, T, c->d, c->E, c->logits};
+    CUDA_TRY(c, launch_router(c, s, rp));
     CUDA_TRY(c, launch_finish(c, s, fp));
   }
   if (h_out) *h_out = h;
@@ -581,19 +619,47 @@ bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
 }
 
 cudaError_t setup_prefill() {
-  cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       RtCfg::SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RtCfg::SMEM);
+    e = cudaFuncSetAttribute(prefill_gemm_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfCfg<1>::SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PfCfg::SMEM);
+    e = cudaFuncSetAttribute(prefill_gemm_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfCfg<1>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_gemm_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfCfg<2>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_gemm_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PfCfg<2>::SMEM);
   return e;
 }
 
-// Prefill through the grouped tcgen05 GEMM: Q4 experts, more tokens than a
-// decode window, f a multiple of the gate/up item (128 features) and d of
-// the down item (256 features).
+// The two grouped GEMM launches of a prefill chunk (gate/up, then down).
+template <int FMT>
+cudaError_t launch_prefill_gemms(moe_ctx *c, cudaStream_t s) {
+  const int d = c->d, f = c->f, TK = c->lay.TK;
+  PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / TK, 0, c->pf_a16, nullptr, c->status};
+  PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / TK, c->lay.p1_bytes, nullptr, c->pf_y16, c->status};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c->n_sm);
+  cfg.blockDim = dim3(kPfGemmThreads);
+  cfg.dynamicSmemBytes = PfCfg<FMT>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, true>, c->pf_map_h, g1);
+  if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, false>, c->pf_map_a, g2);
+  return e;
+}
+
+// Prefill through the grouped tcgen05 GEMM: more tokens than a decode
+// window, f a multiple of the gate/up item (128 features) and d of the down
+// item (256 features); Q4 and Q2 experts.
 // Router logits of N tokens on the tensor cores (router_tc_kernel) when the
 // context holds the router's bf16 parts, the shapes fit its tiles and the
 // chunk has at least kRtMinTokens tokens (one tile per CTA runs its whole
@@ -625,9 +691,13 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
   return true;
 }
 
+// Experts with at least this many tokens in a chunk run on the grouped GEMM
+// (128-row tiles); fewer tokens would leave most of a tile empty, and the
+// GEMV streams such an expert once per job of <= 16 tokens instead.
+constexpr int kHotMinTokens = 16;
+
 bool use_prefill_gemm(const moe_ctx *c, int N) {
-  return c->pf && c->fmt == MOE_Q4_SYM_G32_F16 && N > kDecMaxT && c->d % (2 * kPfBN) == 0 &&
-         c->f % kPfBN == 0 && c->E <= kPfMaxE;
+  return c->pf && N > kDecMaxT && c->d % (2 * kPfBN) == 0 && c->f % kPfBN == 0 && c->E <= kPfMaxE;
 }
 
 // The prefill chunk's routing on router input h: logits, top-k + softmax
@@ -636,19 +706,17 @@ bool use_prefill_gemm(const moe_ctx *c, int N) {
 // gather of the grouped fp16 A rows.  perm (or null) receives the bucket
 // permutation; the bucket offsets are left in c->pf_eoff.
 moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int32_t *idx, float *w,
-                              int32_t *perm, cudaStream_t s) {
+                              int32_t *perm, cudaStream_t s, int hot_min) {
   const int E = c->E, k = c->k, d = c->d;
   cudaError_t e = cudaSuccess;
   const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
-  if (launch_router_tc(c, s, h, N, layer, &e)) {
+  int ks = 1;
+  if (launch_router_tc(c, s, h, N, layer, &e))
     CUDA_TRY(c, e);
-  } else {  // small expert counts or chunks: fp32 FMA
-    RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d, bias, N, d, E, c->logits};
-    CUDA_TRY(c, launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN),
-                       dim3(256), 0, s, rp));
-  }
+  else  // small expert counts or chunks: fp32 FMA
+    CUDA_TRY(c, launch_router_fma(c, s, h, N, layer, &ks));
   const int blocks = (N + kPfTok - 1) / kPfTok;
-  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4]};
+  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], c->pf_part, ks, bias};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;
@@ -668,6 +736,14 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   sp.tiles = c->pf_tiles;
   sp.n_tiles = c->pf_ntiles;
   sp.max_tiles = c->pf_max_tiles;
+  sp.hot_min = hot_min;
+  sp.chunk = job_chunk(N);
+  sp.hot = c->pf_hot;
+  sp.job_ptr = c->job_ptr;
+  sp.job_beg = c->job_beg;
+  sp.job_n = c->job_n;
+  sp.n_jobs = c->n_jobs;
+  sp.max_jobs = c->max_jobs;
   sp.cnt_out = c->cnt_out;
   sp.stats = c->stats;
   sp.last = c->last;
@@ -675,7 +751,7 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32), dim3(kPfColWarps * 32), 0, s, sp));
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
   PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
-                     c->pf_row_of, c->pf_hg, perm};
+                     c->pf_row_of, c->pf_hg, perm ? perm : c->pf_perm, c->pf_hot};
   CUDA_TRY(c, launch(prefill_scatter_kernel, dim3(blocks), dim3(kPfTok * 32), 0, s, cp));
   return MOE_OK;
 }
@@ -684,7 +760,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   const int k = c->k, d = c->d, f = c->f;
   if (!c->pf_maps) {
     if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
-        !encode_map_f16(&c->pf_map_a, c->abuf, c->pf_rows, f))
+        !encode_map_f16(&c->pf_map_a, c->pf_a16, c->pf_rows, f))
       return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     c->pf_maps = true;
   }
@@ -692,32 +768,44 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   cudaError_t e = cudaSuccess;
   const uint16_t *h = router_input(c, layer, x, N, s, &e);
   CUDA_TRY(c, e);
-  moe_status st = prefill_route_impl(c, layer, h, N, c->idx, c->w, nullptr, s);
+  moe_status st = prefill_route_impl(c, layer, h, N, c->idx, c->w, c->pf_perm, s, kHotMinTokens);
   if (st) return st;
   CUDA_TRY(c, prof_mark(c, 1, s));
-  PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / 64, 0, reinterpret_cast<__half *>(c->abuf),
-                  nullptr, c->status};
-  const int smem1 = PfCfg::SMEM, smem2 = PfCfg::SMEM;
-  {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(c->n_sm);
-    cfg.blockDim = dim3(kPfGemmThreads);
-    cfg.dynamicSmemBytes = smem1;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<true>, c->pf_map_h, g1));
-    PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / 64, c->lay.p1_bytes, nullptr,
-                    reinterpret_cast<__half *>(c->ybuf), c->status};
-    cfg.dynamicSmemBytes = smem2;
-    CUDA_TRY(c, cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<false>, c->pf_map_a, g2));
+  // experts with many tokens: grouped GEMM over 128-row tiles; the others:
+  // the GEMV over jobs of <= 16 tokens, rows read through the bucket
+  // permutation (grouped row -> pair id)
+  GemvParams g1{};
+  g1.job_ptr = c->job_ptr;
+  g1.job_beg = c->job_beg;
+  g1.job_n = c->job_n;
+  g1.n_jobs = c->n_jobs;
+  g1.plist = c->pf_perm;
+  g1.Tk = N * k;
+  g1.k = k;
+  g1.src = h;
+  g1.src_by_pair = 0;
+  g1.K = d;
+  g1.R = f;
+  g1.region_off = 0;
+  g1.out_a = c->abuf;
+  g1.status = c->status;
+  GemvParams g2 = g1;
+  g2.src = c->abuf;
+  g2.src_by_pair = 1;
+  g2.K = f;
+  g2.R = d;
+  g2.region_off = c->lay.p1_bytes;
+  g2.out_a = nullptr;
+  g2.out_y = c->ybuf;
+  if (c->fmt == MOE_Q4_SYM_G32_F16) {
+    CUDA_TRY(c, launch_prefill_gemms<1>(c, s));
+    CUDA_TRY(c, launch_experts<1>(c, s, N, g1, g2));
+  } else {
+    CUDA_TRY(c, launch_prefill_gemms<2>(c, s));
+    CUDA_TRY(c, launch_experts<2>(c, s, N, g1, g2));
   }
   CUDA_TRY(c, prof_mark(c, 2, s));
-  PfCombineParams mp{reinterpret_cast<const __half *>(c->ybuf), c->w, c->pf_row_of, N, k, d, c->n_shared,
-                     x, delta};
+  PfCombineParams mp{c->pf_y16, c->ybuf, c->w, c->pf_row_of, N, k, d, c->n_shared, x, delta};
   const long long n4 = (long long)N * d / 4;
   const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
   CUDA_TRY(c, launch(prefill_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));
@@ -769,6 +857,7 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.last = c->last;
     dp.status = c->status;
     dp.sm = decode_layout(c, T);
+    dp.prefetch = c->dec_prefetch;
     CUDA_TRY(c, launch_decode(c, s, dp));
     // one kernel: the profile's route / experts / combine marks coincide
     CUDA_TRY(c, prof_mark(c, 1, s));
@@ -780,6 +869,9 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     }
     return MOE_OK;
   }
+  // more tokens than a decode window: GEMM for the experts that many tokens
+  // share, GEMV for the rest (prefill_impl)
+  if (use_prefill_gemm(c, T)) return prefill_impl(c, layer, x, T, delta, s);
   FinishParams fp = finish_params(c, layer, T);
   fp.build_jobs = 1;
   const uint16_t *h = nullptr;
@@ -922,6 +1014,7 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   c->k = k;
   c->fmt = fmt;
   c->lay = make_layout(fmt, d, f);
+  if (const char *pf = getenv("MOE_DECODE_PREFETCH")) c->dec_prefetch = atoi(pf);  // TEMP A/B knob
   cudaError_t e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = setup_route_fused();
@@ -1229,7 +1322,7 @@ moe_status moe_prefill_route(moe_ctx *c, int layer, const void *h, int N, int32_
   if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
-  moe_status st = prefill_route_impl(c, layer, (const uint16_t *)h, N, idx, w, bperm, s);
+  moe_status st = prefill_route_impl(c, layer, (const uint16_t *)h, N, idx, w, bperm, s, kHotMinTokens);
   if (st) return st;
   if (boff)
     CUDA_TRY(c, cudaMemcpyAsync(boff, c->pf_eoff, (size_t)(c->E + 1) * sizeof(int32_t),

@@ -47,15 +47,20 @@ struct PfTile {                  // one 128-row tile of one expert
 };
 
 struct PfRouteParams {
-  const float *logits;  // [T, E]
+  float *logits;        // [T, E]: read; with ksplit > 1 first written here
   int T, E, k;
   int *idx;             // [T, k]
   float *w;             // [T, k]
   unsigned short *bmask;  // [blocks][E]: bit i = token 16 b + i selected the expert
   unsigned long long *near_ties;
+  const float *part;    // ksplit > 1: partial logits [ksplit][T][E] of a split reduction
+  int ksplit;
+  const float *bias;    // [E] or null, added to the summed partials
 };
 
-// One warp per token; then the block's per-expert token sets.
+// One warp per token; then the block's per-expert token sets.  When the
+// router's reduction was split (ksplit > 1), the warp first adds its token's
+// partial logits in split order (z = 0, 1, ...) and the bias.
 template <int NPL>
 __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams p) {
   __shared__ unsigned s_mask[kPfMaxE];
@@ -64,6 +69,17 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_mask[e] = 0u;
   __syncthreads();
   const int t = blockIdx.x * kPfTok + wid;
+  if (t < p.T && p.ksplit > 1) {
+    const long long plane = (long long)p.T * p.E;
+    for (int e = lane; e < p.E; e += 32) {
+      const long long at = (long long)t * p.E + e;
+      float s = __ldcg(p.part + at);
+      for (int z = 1; z < p.ksplit; ++z) s += __ldcg(p.part + z * plane + at);
+      p.logits[at] = s + (p.bias ? p.bias[e] : 0.f);
+    }
+    __threadfence();  // the lanes' sums before the warp's top-k reads them
+    __syncwarp();
+  }
   if (t < p.T) {
     int e;
     float w;
@@ -92,6 +108,13 @@ struct PfScanParams {
   PfTile *tiles;                // [max_tiles]
   int *n_tiles;
   int max_tiles;
+  // experts with fewer than hot_min tokens become GEMV jobs instead of GEMM
+  // tiles (hot_min <= 1: every expert is a GEMM expert)
+  int hot_min, chunk;           // chunk: tokens per GEMV job
+  int *hot;                     // [E] 1 = GEMM expert
+  unsigned long long *job_ptr;  // [max_jobs] expert base address per GEMV job
+  int *job_beg, *job_n, *n_jobs;  // first grouped row, rows; job count
+  int max_jobs;
   int *cnt_out;                 // [E] statistics
   unsigned long long *stats;
   int *last;
@@ -130,37 +153,46 @@ __global__ void __launch_bounds__(kPfColWarps * 32) prefill_colscan_kernel(PfSca
   pdl_launch_dependents();
 }
 
-// One CTA of 1024 threads: one block scan over the experts' token counts
-// gives their first rows, another their first tiles; then the tile list,
-// with the residency lookup.
+// One CTA of 1024 threads: block scans over the experts' token counts give
+// their first rows, their first GEMM tiles and their first GEMV jobs; then
+// the tile and job lists, with the residency lookup.  An expert with at
+// least hot_min tokens is a GEMM expert (128-row tiles); one with fewer is
+// cut into GEMV jobs of at most `chunk` tokens, which stream its weights
+// once per job instead of dequantising a mostly empty tile.
 __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
-  __shared__ int s_cnt[2 * kPfMaxE + 2];
+  __shared__ int s_cnt[3 * kPfMaxE + 3];
   __shared__ int s_red[32];
   __shared__ unsigned long long s_hm[3];
   pdl_wait();
   const int tid = threadIdx.x;
-  int *cnt = s_cnt, *tl = s_cnt + kPfMaxE + 1;
+  int *cnt = s_cnt, *tl = s_cnt + kPfMaxE + 1, *jl = s_cnt + 2 * kPfMaxE + 2;
   if (tid < 3) s_hm[tid] = 0;
   for (int e = tid; e < p.E; e += blockDim.x) {
     const int run = p.eoff[e];  // token count from prefill_colscan_kernel
+    const bool hot = run >= p.hot_min;
     cnt[e] = run;
-    tl[e] = (run + kPfBM - 1) / kPfBM;
+    tl[e] = hot ? (run + kPfBM - 1) / kPfBM : 0;
+    jl[e] = hot ? 0 : (run + p.chunk - 1) / p.chunk;
   }
   block_exclusive_scan(cnt, cnt, p.E, s_red);
   block_exclusive_scan(tl, tl, p.E, s_red);
-  const int routed_tiles = tl[p.E], P = cnt[p.E];
+  block_exclusive_scan(jl, jl, p.E, s_red);
+  const int routed_tiles = tl[p.E], P = cnt[p.E], n_jobs = jl[p.E];
   const int shared_tiles = p.shared ? (p.T + kPfBM - 1) / kPfBM : 0;
-  if (routed_tiles + shared_tiles > p.max_tiles) {
+  if (routed_tiles + shared_tiles > p.max_tiles || n_jobs > p.max_jobs) {
     if (tid == 0) {
       atomicOr(p.status, kErrJobOverflow);
       *p.n_tiles = 0;
+      *p.n_jobs = 0;
     }
     return;
   }
   for (int e = tid; e < p.E; e += blockDim.x) {
     p.eoff[e] = cnt[e];
     const int n = cnt[e + 1] - cnt[e];
+    const bool hot = n >= p.hot_min;
     p.cnt_out[e] = n;
+    p.hot[e] = hot;
     if (!n) continue;
     const int slot = p.slot_of ? p.slot_of[(long long)p.layer * p.E + e] : -1;
     const bool hit = slot >= 0 && slot < p.n_slots;
@@ -169,10 +201,18 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
                              : p.arena + ((long long)p.layer * p.E + e) * p.expert_bytes;
     atomicAdd(&s_hm[hit ? 0 : 1], (unsigned long long)n);
     atomicAdd(&s_hm[2], 1ull);
-    for (int m = 0, ti = tl[e]; m < n; m += kPfBM, ++ti) {
-      p.tiles[ti].w = ptr;
-      p.tiles[ti].row0 = cnt[e] + m;
-      p.tiles[ti].rows = min(kPfBM, n - m);
+    if (hot) {
+      for (int m = 0, ti = tl[e]; m < n; m += kPfBM, ++ti) {
+        p.tiles[ti].w = ptr;
+        p.tiles[ti].row0 = cnt[e] + m;
+        p.tiles[ti].rows = min(kPfBM, n - m);
+      }
+    } else {
+      for (int m = 0, j = jl[e]; m < n; m += p.chunk, ++j) {
+        p.job_ptr[j] = (unsigned long long)ptr;
+        p.job_beg[j] = cnt[e] + m;
+        p.job_n[j] = min(p.chunk, n - m);
+      }
     }
   }
   if (tid == 0) p.eoff[p.E] = P;
@@ -184,6 +224,7 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
   __syncthreads();
   if (tid == 0) {
     *p.n_tiles = routed_tiles + shared_tiles;
+    *p.n_jobs = n_jobs;
     atomicAdd(&p.stats[0], 1ULL);
     atomicAdd(&p.stats[1], (unsigned long long)p.T);
     atomicAdd(&p.stats[2], s_hm[0]);
@@ -201,9 +242,11 @@ struct PfScatterParams {
   const int *boff, *eoff;
   const uint16_t *h;            // bf16 [T, d]
   int T, E, k, d, has_shared;
-  int *row_of;                  // [T*k + T]: grouped row of pair (shared pair P + t)
-  __half *hg;                   // fp16 [rows][d] grouped A matrix
+  int *row_of;                  // [T*k + T]: grouped row of pair (shared pair P + t);
+                                // ~pair (negative) for a pair of a GEMV expert
+  __half *hg;                   // fp16 [rows][d] grouped A matrix (rows of GEMM experts)
   int *perm;                    // [T*k] or null: pair id of each routed grouped row
+  const int *hot;               // [E] or null (null: every expert is a GEMM expert)
 };
 
 // One warp per token: its k pairs (and its shared-expert pair) get their
@@ -217,18 +260,24 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
   if (t >= p.T) return;
   const int P = p.T * p.k;
   int rows[33];
+  unsigned long long copy = 0;  // bit j: row j feeds the GEMM (its A row is needed)
   const int nr = p.k + (p.has_shared ? 1 : 0);
   for (int j = 0; j < p.k; ++j) {
     const int e = __ldg(p.idx + (long long)t * p.k + j);
     const unsigned m = p.bmask[(long long)blockIdx.x * p.E + e];
     const int rank = __popc(m & ((1u << wid) - 1u));
     rows[j] = p.eoff[e] + p.boff[(long long)blockIdx.x * p.E + e] + rank;
+    if (!p.hot || p.hot[e]) copy |= 1ull << j;
   }
-  if (p.has_shared) rows[p.k] = P + t;
+  if (p.has_shared) {
+    rows[p.k] = P + t;
+    copy |= 1ull << p.k;
+  }
   if (lane < p.k) {
-    p.row_of[(long long)t * p.k + lane] = rows[lane];
+    const int q = t * p.k + lane;
+    p.row_of[q] = (copy >> lane) & 1 ? rows[lane] : ~q;
     // the bucket permutation: grouped row -> pair id (rows < P are routed)
-    if (p.perm) p.perm[rows[lane]] = t * p.k + lane;
+    if (p.perm) p.perm[rows[lane]] = q;
   }
   if (lane == 0 && p.has_shared) p.row_of[P + t] = P + t;
   // copy the token row to every destination, 8 elements per lane per step
@@ -245,7 +294,8 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
       out[q] = r;
     }
     const uint4 o = make_uint4(out[0], out[1], out[2], out[3]);
-    for (int j = 0; j < nr; ++j) reinterpret_cast<uint4 *>(p.hg + (long long)rows[j] * p.d)[i] = o;
+    for (int j = 0; j < nr; ++j)
+      if ((copy >> j) & 1) reinterpret_cast<uint4 *>(p.hg + (long long)rows[j] * p.d)[i] = o;
   }
   pdl_launch_dependents();
 }
@@ -253,7 +303,10 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
 // ------------------------------------------------------------ router GEMM
 // logits[t, e] = sum_i W[e, i] h[t, i] (+ b[e]) for a whole chunk, fp32 FMA
 // (routing decisions are compared bit-exactly, so no reduced-precision
-// tensor-core path).  CTA tile: 128 tokens x 128 experts, 256 threads, each
+// tensor-core path).  Small chunks split the reduction over blockIdx.z
+// (columns [z kchunk, (z+1) kchunk)) so the grid fills the GPU; each split
+// writes its partial sums, which prefill_topk_kernel adds in split order.
+// CTA tile: 128 tokens x 128 experts, 256 threads, each
 // an 8 x 8 block of outputs made of two 4-row and two 4-column halves 64
 // apart (so a warp's 16-byte shared-memory reads are contiguous: no bank
 // conflicts); the reduction walks i in order, 16 at a time through shared
@@ -263,7 +316,8 @@ struct RouterGemmParams {
   const float *W;      // fp32 [E, d]
   const float *bias;   // [E] or null
   int T, d, E;
-  float *logits;       // [T, E]
+  float *logits;       // [T, E]; with gridDim.z > 1 partial sums [gridDim.z][T][E], no bias
+  int kchunk;          // reduction columns of one CTA (blockIdx.z); d when unsplit
 };
 
 constexpr int kRgBM = 128, kRgBN = 128, kRgBK = 16;
@@ -306,13 +360,14 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
   };
   uint4 hv;
   float4 w0, w1;
-  load(0, hv, w0, w1);
+  const int kbase = blockIdx.z * p.kchunk;
+  load(kbase, hv, w0, w1);
   store(0, hv, w0, w1);
   __syncthreads();
-  const int nk = p.d / kRgBK;
+  const int nk = p.kchunk / kRgBK;
   for (int kt = 0; kt < nk; ++kt) {
     const int buf = kt & 1;
-    if (kt + 1 < nk) load((kt + 1) * kRgBK, hv, w0, w1);
+    if (kt + 1 < nk) load(kbase + (kt + 1) * kRgBK, hv, w0, w1);
 #pragma unroll
     for (int k = 0; k < kRgBK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
@@ -330,6 +385,8 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
     __syncthreads();
   }
   pdl_launch_dependents();
+  const bool split = gridDim.z > 1;
+  float *out = p.logits + (long long)blockIdx.z * p.T * p.E;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
@@ -337,7 +394,7 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(RouterGemmParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-      if (e < p.E) p.logits[(long long)t * p.E + e] = acc[i][j] + (p.bias ? p.bias[e] : 0.f);
+      if (e < p.E) out[(long long)t * p.E + e] = acc[i][j] + (!split && p.bias ? p.bias[e] : 0.f);
     }
   }
 }
@@ -414,6 +471,11 @@ MOE_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
+MOE_DEV uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
 
 // One code-word pair of a k-step pair: rows r0 (fp16 halves at nibble bits
 // 0/16 and 8/24) and r1 (bits 4/20 and 12/28), columns kb .. kb+7 from words
@@ -459,12 +521,61 @@ MOE_DEV void dequant_q4_lane(uint4 w, uint2 sc, uint32_t dst_s, int r0, int g, i
                "r"(s1.x), "r"(s1.y), "r"(s1.z), "r"(s1.w) : "memory");
 }
 
+// Q2 codes of one k-step half of a repacked tile into the swizzled fp16 B
+// tile.  A Q2 tile spans 128 reduction columns, two groups of 64; half h of
+// it is group h and sits in words 2h and 2h+1 of each lane (g, tig): word
+// 2h holds rows r0 = 16 rb + g and r0 + 8 at reduction columns
+// [8 tig, 8 tig + 8) of the half (16-byte chunk tig of both rows), word
+// 2h + 1 the same rows at chunk 4 + tig.  In a word, fragment register r
+// (r = 0..7) holds columns 2 (r >> 1) and 2 (r >> 1) + 1 -- row r0 for even
+// r, r0 + 8 for odd r -- at bits [2r, 2r + 2) and [16 + 2r, 18 + 2r).  A code
+// q placed at mantissa bit p of fp16 1024 gives 1024 + q 2^p; subtracting
+// 1024 is exact, and one fp16 FMA with s 2^-p (exact) and the min gives
+// s q + m, rounded once.  s and mn hold the group's (row r0, row r0 + 8)
+// fp16 scales and mins.  Stores as in dequant_q4_lane.
+MOE_DEV void dq_q2_word(uint32_t w, uint32_t sa, uint32_t sb, uint32_t ma, uint32_t mb, uint4 &row0,
+                        uint4 &row1) {
+  const uint32_t c1024 = 0x64006400u;
+  const uint32_t w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
+  // row r0: codes at p = 0 of w, w >> 4, w >> 8, w >> 12; row r1: p = 2
+  row0.x = hfma2(hsub2(lop3_and_or(w, 0x00030003u, c1024), c1024), sa, ma);
+  row0.y = hfma2(hsub2(lop3_and_or(w4, 0x00030003u, c1024), c1024), sa, ma);
+  row0.z = hfma2(hsub2(lop3_and_or(w8, 0x00030003u, c1024), c1024), sa, ma);
+  row0.w = hfma2(hsub2(lop3_and_or(w12, 0x00030003u, c1024), c1024), sa, ma);
+  row1.x = hfma2(hsub2(lop3_and_or(w, 0x000C000Cu, c1024), c1024), sb, mb);
+  row1.y = hfma2(hsub2(lop3_and_or(w4, 0x000C000Cu, c1024), c1024), sb, mb);
+  row1.z = hfma2(hsub2(lop3_and_or(w8, 0x000C000Cu, c1024), c1024), sb, mb);
+  row1.w = hfma2(hsub2(lop3_and_or(w12, 0x000C000Cu, c1024), c1024), sb, mb);
+}
+
+MOE_DEV void dequant_q2_lane(uint2 w, uint32_t s, uint32_t mn, uint32_t dst_s, int r0, int g, int tig) {
+  const int r1 = r0 + 8;
+  const uint32_t base0 = dst_s + (uint32_t)(r0 >> 3) * 1024 + (uint32_t)(r0 & 7) * 128;
+  const uint32_t base1 = dst_s + (uint32_t)(r1 >> 3) * 1024 + (uint32_t)(r1 & 7) * 128;
+  const uint32_t sa = h2_dup(s, false), sb = hmul2(h2_dup(s, true), 0x34003400u);  // s_r1 / 4
+  const uint32_t ma = h2_dup(mn, false), mb = h2_dup(mn, true);
+  uint4 a0, b0, a1, b1;
+  dq_q2_word(w.x, sa, sb, ma, mb, a0, b0);  // chunk tig
+  dq_q2_word(w.y, sa, sb, ma, mb, a1, b1);  // chunk 4 + tig
+  const bool odd = g & 1;
+  const uint32_t cf = (uint32_t)((odd ? 4 : 0) + tig), cs = (uint32_t)((odd ? 0 : 4) + tig);
+  const uint4 f0 = odd ? a1 : a0, s0 = odd ? a0 : a1, f1 = odd ? b1 : b0, s1 = odd ? b0 : b1;
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base0 + ((cf ^ (r0 & 7)) << 4)),
+               "r"(f0.x), "r"(f0.y), "r"(f0.z), "r"(f0.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base0 + ((cs ^ (r0 & 7)) << 4)),
+               "r"(s0.x), "r"(s0.y), "r"(s0.z), "r"(s0.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base1 + ((cf ^ (r1 & 7)) << 4)),
+               "r"(f1.x), "r"(f1.y), "r"(f1.z), "r"(f1.w) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(base1 + ((cs ^ (r1 & 7)) << 4)),
+               "r"(s1.x), "r"(s1.y), "r"(s1.z), "r"(s1.w) : "memory");
+}
+
 struct PfGemmParams {
   const PfTile *tiles;
   const int *n_tiles;
   int K;                 // reduction (d for gate/up, f for down)
   int N;                 // output features (f for gate/up, d for down)
-  int ntile_k;           // repacked tiles along K: K / 64
+  int ntile_k;           // repacked tiles along K: K / 64 (Q4) or K / 128 (Q2)
   long long region_off;  // 0 (gate/up) or the down region's offset
   __half *out_a;         // gate/up: SiLU(G) * U, fp16 [rows][N]
   __half *out_y;         // down: y, fp16 (round to nearest, saturating) [rows][N]
@@ -477,15 +588,23 @@ constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM 
 
 // Both passes run two 128-column accumulators per item: gate and up of the
 // same 128 features (gate/up pass), or two adjacent 128-feature slices
-// (down pass, 256 features per item).
+// (down pass, 256 features per item).  The A tiles (64 reduction columns of
+// 128 token rows) and the code tiles travel in two rings: an A stage is
+// released when its MMAs complete, a code stage when the dequantising warps
+// have read it.  A code stage holds the 16 repacked tiles of one tile
+// column: 64 reduction columns for Q4 (one k-step), 128 for Q2 (two k-steps,
+// one quantisation group each).
+template <int FMT>
 struct PfCfg {
-  static constexpr int SA = 5;                              // A + code stages (TMA ring)
+  static constexpr int TILE = FMT == 1 ? 576 : 640;         // repacked code tile (+ scales)
+  static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per code stage
+  static constexpr int SA = 6;                              // A ring
+  static constexpr int SC = 4;                              // code ring
   static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB
   static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per accumulator
-  static constexpr uint32_t CODES = 16 * 576;               // 16 repacked code tiles
-  static constexpr uint32_t STAGE_A = (TILE_A + CODES + 1023) / 1024 * 1024;
+  static constexpr uint32_t CODES = (16 * TILE + 1023) / 1024 * 1024;  // 16 repacked code tiles
   static constexpr uint32_t BBUF = 2 * TILE_B;              // one B buffer (two tiles)
-  static constexpr uint32_t SMEM = SA * STAGE_A + 2 * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + 2 * BBUF + 1024;  // + alignment slack
   static constexpr uint32_t ACC_COLS = 2 * kPfBN;           // TMEM columns per accumulator buffer
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
@@ -493,35 +612,41 @@ struct PfCfg {
 // Grouped GEMM over the tile list, warp-specialised.  Work item = (128-row
 // tile, output slice of 128 (gate/up) or 256 (down) features); persistent
 // CTAs walk items blockIdx.x, +gridDim.x.
-//  warp 0 lane 0   producer: per 64-column reduction step, the A tile (2-D
-//                  TMA, 128-byte swizzle) and the 16 repacked code tiles of
-//                  the step (1-D bulk copies) into a free stage of a 5-deep ring
-//  warps 8..15     dequantise a stage's codes into one of two swizzled fp16
-//                  B buffers, then arrive on the buffer's barrier
+//  warp 0 lane 0   producer: per 64-column reduction step the A tile (2-D
+//                  TMA, 128-byte swizzle) into a free stage of the A ring,
+//                  and at each new tile column the 16 repacked code tiles
+//                  (1-D bulk copies) into a free stage of the code ring
+//  warps 8..15     dequantise a k-step's codes into one of two swizzled fp16
+//                  B buffers, arrive on the buffer's barrier, and release
+//                  the code stage after its last k-step
 //  warp 1 lane 0   issues the MMAs (m128n256k16: both accumulators at once,
 //                  operands in shared memory, fp32 in TMEM) and commits the
-//                  release of the stage and of the B buffer; accumulator
+//                  release of the A stage and of the B buffer; accumulator
 //                  pairs alternate between two TMEM buffers
 //  warps 4..7      drain an accumulator buffer (TMEM lanes = tile rows)
 //                  while the next item accumulates into the other one
 // Every wait is bounded; a timeout raises kErrTimeout and every role stops.
-template <bool GATED>
+template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
-  using C = PfCfg;
-  constexpr int SA = C::SA;
+  using C = PfCfg<FMT>;
+  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, TILE = C::TILE;
   constexpr int COLS = GATED ? kPfBN : 2 * kPfBN;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
-  __shared__ __align__(8) unsigned long long s_full[SA], s_empty[SA], s_bfull[2], s_bempty[2],
-      s_accf[2], s_acce[2];
+  __shared__ __align__(8) unsigned long long s_afull[SA], s_aempty[SA], s_cfull[SC], s_cempty[SC],
+      s_bfull[2], s_bempty[2], s_accf[2], s_acce[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
   const uint32_t base = smem_addr(pf_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
   if (tid == 0) {
     for (int i = 0; i < SA; ++i) {
-      mbar_init(smem_addr(&s_full[i]), 1);
-      mbar_init(smem_addr(&s_empty[i]), 1);
+      mbar_init(smem_addr(&s_afull[i]), 1);
+      mbar_init(smem_addr(&s_aempty[i]), 1);
+    }
+    for (int i = 0; i < SC; ++i) {
+      mbar_init(smem_addr(&s_cfull[i]), 1);
+      mbar_init(smem_addr(&s_cempty[i]), 8);  // one arrival per dequantising warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_addr(&s_bfull[b]), 256);
@@ -546,9 +671,9 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   const int ntiles = ldcg_i32(p.n_tiles);
   const int nslices = p.N / COLS, nsteps = p.K / kPfBK;
   const int items = ntiles * nslices;
-  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_A; };
-  auto stage_c = [&](uint32_t st) { return stage0 + st * C::STAGE_A + C::TILE_A; };
-  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::STAGE_A + b * C::BBUF; };
+  auto stage_a = [&](uint32_t st) { return stage0 + st * C::TILE_A; };
+  auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::TILE_A + cs * C::CODES; };
+  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::TILE_A + SC * C::CODES + b * C::BBUF; };
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
   auto give_up = [&]() {
     *reinterpret_cast<volatile int *>(&s_abort) = 1;
@@ -558,32 +683,51 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   if (wid == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t it = 0;
-      for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x) {
+      uint32_t it = 0, ct = 0;  // k-steps and code stages issued
+      bool ok = true;
+      for (int item = blockIdx.x; item < items && ok && !aborted(); item += gridDim.x) {
         const PfTile tile = p.tiles[item / nslices];
         const int rb0 = (item % nslices) * (COLS / 16);
         const uint8_t *wbase = tile.w + p.region_off;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
+          if (ks % SPC == 0) {  // the next tile column's codes
+            const uint32_t cs = ct % SC, cuse = ct / SC, tk = ks / SPC;
+            if (cuse > 0 && !mbar_wait_bounded(smem_addr(&s_cempty[cs]), (cuse - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            const uint32_t cbar = smem_addr(&s_cfull[cs]);
+            mbar_expect_tx(cbar, 16 * TILE);
+            // code tile q = 2 r + m: row block r of accumulator m
+            if constexpr (GATED) {  // gate and up tiles of a row block are adjacent
+              for (int r = 0; r < 8; ++r)
+                bulk_g2s(stage_c(cs) + r * 2 * TILE,
+                         wbase + ((long long)(rb0 + r) * p.ntile_k + tk) * 2 * TILE, 2 * TILE, cbar);
+            } else {
+              for (int q = 0; q < 16; ++q)
+                bulk_g2s(stage_c(cs) + q * TILE,
+                         wbase + ((long long)(rb0 + (q & 1) * 8 + (q >> 1)) * p.ntile_k + tk) * TILE, TILE,
+                         cbar);
+            }
+            ++ct;
+          }
           const uint32_t st = it % SA, use = it / SA;
-          if (use > 0 && !mbar_wait_bounded(smem_addr(&s_empty[st]), (use - 1) & 1)) {
-            give_up();
+          if (use > 0 && !mbar_wait_bounded(smem_addr(&s_aempty[st]), (use - 1) & 1)) {
+            ok = false;
             break;
           }
-          const uint32_t bar = smem_addr(&s_full[st]);
-          mbar_expect_tx(bar, C::TILE_A + C::CODES);
+          const uint32_t bar = smem_addr(&s_afull[st]);
+          mbar_expect_tx(bar, C::TILE_A);
           tma_load_2d(stage_a(st), &amap, ks * kPfBK, tile.row0, bar);
-          // code tile q = 2 r + m: row block r of accumulator m
-          if constexpr (GATED) {  // gate and up tiles of a row block are adjacent
-            for (int r = 0; r < 8; ++r)
-              bulk_g2s(stage_c(st) + r * 2 * 576, wbase + ((long long)(rb0 + r) * p.ntile_k + ks) * 2 * 576,
-                       2 * 576, bar);
-          } else {
-            for (int q = 0; q < 16; ++q)
-              bulk_g2s(stage_c(st) + q * 576,
-                       wbase + ((long long)(rb0 + (q & 1) * 8 + (q >> 1)) * p.ntile_k + ks) * 576, 576, bar);
-          }
         }
       }
+      if (!ok) give_up();
+      // no copy may land in shared memory after the CTA has moved on (a give-up
+      // leaves stages in flight); consumed stages pass at once
+      for (uint32_t j = it > SA ? it - SA : 0; j < it; ++j)
+        (void)mbar_wait_bounded(smem_addr(&s_afull[j % SA]), (j / SA) & 1);
+      for (uint32_t j = ct > SC ? ct - SC : 0; j < ct; ++j)
+        (void)mbar_wait_bounded(smem_addr(&s_cfull[j % SC]), (j / SC) & 1);
     }
   } else if (wid == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -604,7 +748,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
           const uint32_t st = it % SA, use = it / SA, bb = it & 1, buse = it >> 1;
           if (!mbar_wait_bounded(smem_addr(&s_bfull[bb]), buse & 1) ||
-              !mbar_wait_bounded(smem_addr(&s_full[st]), use & 1)) {
+              !mbar_wait_bounded(smem_addr(&s_afull[st]), use & 1)) {
             ok = false;
             break;
           }
@@ -613,7 +757,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           for (int kk = 0; kk < kPfBK / 16; ++kk)
             umma_f16(acc, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(bbuf(bb) + kk * 32), IDESC,
                      (ks | kk) != 0);
-          umma_commit(smem_addr(&s_empty[st]));
+          umma_commit(smem_addr(&s_aempty[st]));
           umma_commit(smem_addr(&s_bempty[bb]));
         }
         if (!ok) {
@@ -623,7 +767,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         umma_commit(smem_addr(&s_accf[buf]));
       }
       // every committed MMA must be complete before TMEM is released
-      if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_empty[(it - 1) % SA]), ((it - 1) / SA) & 1);
+      if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_aempty[(it - 1) % SA]), ((it - 1) / SA) & 1);
     }
   } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
@@ -684,30 +828,42 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
     // warp -> two code tiles (q = 2 dw, 2 dw + 1: row block dw of both
-    // accumulators), lane -> the tile's lane: contiguous 16-byte code
-    // reads, conflict-free stores (dequant_q4_lane)
+    // accumulators), lane -> the tile's lane: contiguous code reads,
+    // conflict-free stores (dequant_q4_lane / dequant_q2_lane)
     const int dw = wid - kPfDeqWarp0;  // 0..7 = row block
     const int g = lane >> 2, tig = lane & 3;
-    uint32_t it = 0;
+    uint32_t it = 0, ct = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
       for (int ks = 0; ks < nsteps; ++ks, ++it) {
-        const uint32_t st = it % SA, use = it / SA, bb = it & 1, buse = it >> 1;
-        bool got = mbar_wait_bounded(smem_addr(&s_full[st]), use & 1);
+        const uint32_t cs = ct % SC, cuse = ct / SC, bb = it & 1, buse = it >> 1;
+        bool got = mbar_wait_bounded(smem_addr(&s_cfull[cs]), cuse & 1);
         if (got && buse > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb]), (buse - 1) & 1);
         if (__any_sync(0xffffffffu, !got) || aborted()) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
+        const int half = ks % SPC;
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-          const uint32_t tsm = stage_c(st) + (dw * 2 + m) * 576;
-          dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8),
-                          bbuf(bb) + m * C::TILE_B, dw * 16 + g, g, tig);
+          const uint32_t tsm = stage_c(cs) + (dw * 2 + m) * TILE;
+          if constexpr (FMT == 1) {
+            dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), bbuf(bb) + m * C::TILE_B,
+                            dw * 16 + g, g, tig);
+          } else {
+            const uint4 sc = lds_u4(tsm + 512 + g * 16);
+            dequant_q2_lane(lds_u2(tsm + lane * 16 + 8 * half), half ? sc.y : sc.x, half ? sc.w : sc.z,
+                            bbuf(bb) + m * C::TILE_B, dw * 16 + g, g, tig);
+          }
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
         mbar_arrive(smem_addr(&s_bfull[bb]));
+        if (half == SPC - 1) {  // the code stage's last k-step: release it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(&s_cempty[cs]));
+          ++ct;
+        }
       }
     }
   }
@@ -878,7 +1034,8 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 struct PfCombineParams {
-  const __half *y;    // fp16 [rows][d] grouped order
+  const __half *y;    // fp16 [rows][d] grouped order (GEMM experts)
+  const float *y32;   // fp32 [T*k][d] by pair id (GEMV experts: row_of < 0)
   const float *w;     // [T][k]
   const int *row_of;  // [T*k + T]
   int T, k, d, has_shared;
@@ -886,7 +1043,8 @@ struct PfCombineParams {
   float *delta;       // fp32 [T][d] (mode 1)
 };
 
-// x[t] <- bf16(x[t] + sum_j w[t,j] y[row(t,j)] + y[row(shared, t)]), j in order.
+// x[t] <- bf16(x[t] + sum_j w[t,j] y[row(t,j)] + y[row(shared, t)]), j in order;
+// a pair of a GEMV expert reads its fp32 y by pair id instead.
 __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p) {
   pdl_wait();
   const int per_t = p.d / 4, P = p.T * p.k;
@@ -902,7 +1060,8 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p)
     };
     for (int j = 0; j < p.k; ++j) {
       const float wj = __ldg(p.w + (long long)t * p.k + j);
-      const float4 v = y4(__ldg(p.row_of + (long long)t * p.k + j));
+      const int row = __ldg(p.row_of + (long long)t * p.k + j);
+      const float4 v = row >= 0 ? y4(row) : __ldcg(reinterpret_cast<const float4 *>(p.y32 + (long long)~row * p.d + o));
       a0 = fmaf(wj, v.x, a0);
       a1 = fmaf(wj, v.y, a1);
       a2 = fmaf(wj, v.z, a2);

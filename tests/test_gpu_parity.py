@@ -163,10 +163,11 @@ def test_every_code_value(B, fmt, T):
         B.moe_destroy(ctx)
 
 
-def test_every_code_value_prefill_gemm(B):
-    """The same uniform Q4 codes through the grouped tcgen05 GEMM (its own
-    fp16 dequantisation of every nibble)."""
-    spec = LayerSpec(d=256, f=256, E=16, k=4, fmt=I.Q4, seed=14, shared=True, weights="uniform")
+@pytest.mark.parametrize("fmt", [I.Q4, I.Q2])
+def test_every_code_value_prefill_gemm(B, fmt):
+    """The same uniform codes through the grouped tcgen05 GEMM (its own
+    fp16 dequantisation of every Q4 nibble and every Q2 code)."""
+    spec = LayerSpec(d=256, f=256, E=16, k=4, fmt=fmt, seed=14, shared=True, weights="uniform")
     ctx = make_ctx(B, spec, max_tokens=512)
     try:
         load_layer(B, ctx, spec)
@@ -194,6 +195,23 @@ def test_small_layer_ragged(B, fmt, shared, T):
     try:
         load_layer(B, ctx, spec)
         x = I.hidden_np(7, T, 256, window=T)
+        out = run(B, ctx, spec, x)
+        check(out, oracle_for(spec, x), spec)
+    finally:
+        B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("fmt", [I.Q4, I.Q2])
+@pytest.mark.parametrize("T", [12, 40])
+def test_multi_launch_path_d_not_multiple_of_256(B, fmt, T):
+    """d = 128 (not a multiple of 256): windows of more than 32 tokens take
+    the multi-launch routing and GEMV kernels, since the grouped GEMM's down
+    items are 256 features wide."""
+    spec = LayerSpec(d=128, f=256, E=24, k=3, fmt=fmt, seed=17, shared=True)
+    ctx = make_ctx(B, spec, max_tokens=64)
+    try:
+        load_layer(B, ctx, spec)
+        x = I.hidden_np(17, T, 128, window=T)
         out = run(B, ctx, spec, x)
         check(out, oracle_for(spec, x), spec)
     finally:

@@ -55,12 +55,14 @@ def check_rows(spec, x_bits, delta, x_out, rows):
     return rel, int((~ok).sum())
 
 
+@pytest.mark.parametrize("fmt", [I.Q4, I.Q2])
 @pytest.mark.parametrize("zipf", [False, True])
 @pytest.mark.parametrize("N", [33, 300, 1000])
-def test_prefill_small_layer_all_tokens(B, N, zipf):
+def test_prefill_small_layer_all_tokens(B, N, zipf, fmt):
     """d=256, f=128, E=16, k=2 + shared: partial and multiple 128-row tiles
-    per expert, several shared-expert tiles; every token checked."""
-    spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=I.Q4, seed=5, shared=True, zipf=zipf)
+    per expert, several shared-expert tiles; every token checked.  Q2 experts
+    are dequantised by the GEMM's own Q2 stage (a code tile per two k-steps)."""
+    spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=fmt, seed=5, shared=True, zipf=zipf)
     ctx = make_ctx(B, spec, 1024)
     try:
         load_layer(B, ctx, spec)
@@ -82,9 +84,9 @@ def test_prefill_small_layer_all_tokens(B, N, zipf):
         B.moe_destroy(ctx)
 
 
-def test_prefill_matches_decode_path(B):
-    """The grouped GEMM and the GEMV path compute the same layer: equal
-    within the output tolerance on every token."""
+def test_prefill_and_forward_agree(B):
+    """moe_prefill and moe_forward on a window of more than 32 tokens run
+    the same chunk path (GEMM experts + GEMV experts): equal outputs."""
     spec = LayerSpec(d=256, f=256, E=8, k=2, fmt=I.Q4, seed=9, shared=True)
     ctx = make_ctx(B, spec, 512)
     try:
@@ -96,12 +98,47 @@ def test_prefill_matches_decode_path(B):
         B.moe_prefill_delta(ctx, 0, x, N, d1)
         B.moe_forward_delta(ctx, 0, x, N, d2)
         B.moe_sync(ctx, 60000)
-        assert_close_rms(d1.cpu().numpy(), d2.cpu().numpy(), what="prefill vs decode path")
+        assert torch.equal(d1, d2)
     finally:
         B.moe_destroy(ctx)
 
 
-def test_prefill_q2_takes_the_gemv_path(B):
+def test_prefill_q2_gemm_and_gemv_experts(B):
+    """Q2 experts, 400 tokens over 8 experts: every routed expert is a GEMM
+    expert; the same layer with 24 experts and 40 tokens puts most of them
+    on the GEMV.  Both against the oracle on every token."""
+    for E, N in ((8, 400), (24, 40)):
+        spec = LayerSpec(d=256, f=256, E=E, k=2, fmt=I.Q2, seed=9 + E, shared=True)
+        ctx = make_ctx(B, spec, 512)
+        try:
+            load_layer(B, ctx, spec)
+            x = I.hidden_np(9, N, spec.d, window=E)
+            delta, x_out = run_prefill(B, ctx, spec, x)
+            check_rows(spec, x, delta, x_out, np.arange(N))
+        finally:
+            B.moe_destroy(ctx)
+
+
+def test_prefill_q2_matches_decode_path_small_windows(B):
+    """Q2 experts: a 32-token window (single-launch decode kernel) and the
+    same tokens inside a 64-token chunk (GEMM / GEMV experts) agree within
+    the output tolerance."""
+    spec = LayerSpec(d=256, f=256, E=8, k=2, fmt=I.Q2, seed=9, shared=True)
+    ctx = make_ctx(B, spec, 512)
+    try:
+        load_layer(B, ctx, spec)
+        x = to_dev(I.hidden_np(9, 64, spec.d, window=3))
+        d1 = torch.empty((64, spec.d), dtype=torch.float32, device="cuda")
+        d2 = torch.empty((32, spec.d), dtype=torch.float32, device="cuda")
+        B.moe_prefill_delta(ctx, 0, x, 64, d1)
+        B.moe_forward_delta(ctx, 0, x[:32], 32, d2)
+        B.moe_sync(ctx, 60000)
+        assert_close_rms(d1[:32].cpu().numpy(), d2.cpu().numpy(), what="chunk vs decode path")
+    finally:
+        B.moe_destroy(ctx)
+
+
+def test_prefill_q2_oracle(B):
     spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=I.Q2, seed=6, shared=True)
     ctx = make_ctx(B, spec, 256)
     try:
