@@ -218,6 +218,7 @@ struct DecodeParams {
   int *status;
   int prefetch;         // bit 0: L2-prefetch the warp's down units after routing;
                         // bit 1: also its gate/up units beyond the ring's first ones
+  int ring_lsu;         // ring slots filled by per-lane cp.async instead of bulk copies
   DecSmem sm;
 };
 
@@ -673,9 +674,10 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
 
   MOE_TRACE(kTrRouteStart);
   WarpRing r;
-  ring_init(r, smem_addr(smem + L.ring) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT);
+  ring_init(r, smem_addr(smem + L.ring) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT,
+            p.ring_lsu);
   if (lane == 0) {
-    for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, 1);
+    for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, p.ring_lsu ? 32 : 1);
     if (wid == 0) {
       mbar_init(h_bar, 1);
       mbar_init(st_bar, 1);

@@ -160,11 +160,13 @@ struct WarpRing {
   uint32_t phase;    // its mbarrier parity
   int inflight;      // units issued and not yet consumed
   int istep;
+  int lsu;           // 1: every lane fills the slot with 16-byte cp.async (slot
+                     // barriers count 32 arrivals); 0: lane 0 issues one bulk copy
   UnitCursor ld;      // next unit to load into the ring
   uint64_t policy;   // L2 policy of the ring loads (evict first)
 };
 
-MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t slot_stride) {
+MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t slot_stride, int lsu = 0) {
   r.data_s = data_s;
   r.bar_s = bar_s;
   r.slot_stride = slot_stride;
@@ -172,6 +174,7 @@ MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t sl
   r.phase = 0;
   r.inflight = 0;
   r.istep = 1;
+  r.lsu = lsu;
   r.ld.rem = 0;
   r.policy = l2_evict_first();
 }
@@ -191,8 +194,14 @@ MOE_DEV void ring_start(WarpRing &r, const Phase &ph, int job, int rb, int unit,
 MOE_DEV void ring_issue_warp(WarpRing &r, const Phase &ph, int slot, int lane) {
   if (r.ld.rem <= 0) return;
   const uint32_t bytes = (uint32_t)(ph.tps * ph.stride);
-  bulk_g2s_hint_pred(lane == 0, r.data_s + slot * r.slot_stride, r.ld.addr, bytes, r.bar_s + 8 * slot,
-                     r.policy);
+  if (r.lsu) {
+    const uint32_t dst = r.data_s + slot * r.slot_stride;
+    for (uint32_t c = 16u * lane; c < bytes; c += 512u) cp_async16_hint(dst + c, r.ld.addr + c, r.policy);
+    cp_async_mbar_arrive_noinc(r.bar_s + 8 * slot);
+  } else {
+    bulk_g2s_hint_pred(lane == 0, r.data_s + slot * r.slot_stride, r.ld.addr, bytes, r.bar_s + 8 * slot,
+                       r.policy);
+  }
   ++r.inflight;
   cursor_advance(r.ld, ph, r.istep);
 }

@@ -84,7 +84,8 @@ struct moe_ctx {
   std::vector<int32_t> host_counts;
 
   int gemv_blocks[2][2][2] = {};  // [fmt][gated][NTM-1]
-  int dec_prefetch = 3;           // decode_kernel L2 prefetch mode (DecodeParams::prefetch)
+  int dec_prefetch = 0;           // decode_kernel L2 prefetch mode (DecodeParams::prefetch)
+  int dec_ring_lsu = 0;           // decode_kernel ring fill (DecodeParams::ring_lsu)
   // profiling: 4 events per call slot
   bool profiling = false;
   std::vector<cudaEvent_t> prof_ev;
@@ -558,7 +559,7 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
     else
       CUDA_TRY(c, launch_router_fma(c, s, h, T, layer, &ks));
     PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4], c->pf_part, ks,
-                     bias};
+                     bias, h, c->d_router + (size_t)layer * c->E * c->d, c->d};
     CUDA_TRY(c, launch_pf_topk(c, s, tp));
     FinishParams fb = fp;
     fb.logits = nullptr;
@@ -716,7 +717,8 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   else  // small expert counts or chunks: fp32 FMA
     CUDA_TRY(c, launch_router_fma(c, s, h, N, layer, &ks));
   const int blocks = (N + kPfTok - 1) / kPfTok;
-  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], c->pf_part, ks, bias};
+  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], c->pf_part, ks, bias,
+                   h, c->d_router + (size_t)layer * E * d, d};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;
@@ -858,6 +860,7 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.status = c->status;
     dp.sm = decode_layout(c, T);
     dp.prefetch = c->dec_prefetch;
+    dp.ring_lsu = c->dec_ring_lsu;
     CUDA_TRY(c, launch_decode(c, s, dp));
     // one kernel: the profile's route / experts / combine marks coincide
     CUDA_TRY(c, prof_mark(c, 1, s));
@@ -1015,6 +1018,7 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   c->fmt = fmt;
   c->lay = make_layout(fmt, d, f);
   if (const char *pf = getenv("MOE_DECODE_PREFETCH")) c->dec_prefetch = atoi(pf);  // TEMP A/B knob
+  if (const char *pf = getenv("MOE_DECODE_LSU")) c->dec_ring_lsu = atoi(pf);        // TEMP A/B knob
   cudaError_t e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = setup_route_fused();

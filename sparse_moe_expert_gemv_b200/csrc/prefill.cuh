@@ -56,7 +56,28 @@ struct PfRouteParams {
   const float *part;    // ksplit > 1: partial logits [ksplit][T][E] of a split reduction
   int ksplit;
   const float *bias;    // [E] or null, added to the summed partials
+  const uint16_t *h;    // bf16 [T, d] router input and
+  const float *W;       // fp32 [E, d] router rows, for the boundary refinement
+  int d;
 };
+
+// Logits within this distance of a token's selection boundary (its k-th and
+// (k+1)-th logits) are recomputed exactly before the final selection.  The
+// chunk routers accumulate in fp32 in an order of their own (the tensor-core
+// router inside its MMAs); their error stays far below this band, so outside
+// it no two logits can change order.
+constexpr float kRefineBand = 2e-3f;
+
+// One warp: the exact logit of expert e for token row h (fp64 sum of the
+// exact fp32 x bf16 products, then the bias), rounded once to fp32.
+MOE_DEV float exact_logit(const float *W, const uint16_t *h, const float *bias, int d, int e, int lane) {
+  const float *wr = W + (long long)e * d;
+  double acc = 0.0;
+  for (int i = lane; i < d; i += 32) acc += (double)wr[i] * (double)__uint_as_float((uint32_t)h[i] << 16);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return (float)(acc + (bias ? (double)bias[e] : 0.0));
+}
 
 // One warp per token; then the block's per-expert token sets.  When the
 // router's reduction was split (ksplit > 1), the warp first adds its token's
@@ -82,8 +103,28 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
   }
   if (t < p.T) {
     int e;
-    float w;
-    warp_topk<NPL>(p.logits + (long long)t * p.E, p.E, p.k, lane, false, e, w, p.near_ties);
+    float w, lk, lk1;
+    float *lr = p.logits + (long long)t * p.E;
+    warp_topk<NPL>(lr, p.E, p.k, lane, false, e, w, nullptr, &lk, &lk1);
+    if (lk - lk1 < kRefineBand) {
+      // the boundary is close: recompute the logits in the band around it
+      // exactly, then select again (and count a near tie on exact values)
+      const uint16_t *hrow = p.h + (long long)t * p.d;
+      for (int i = 0; i < (p.E + 31) / 32; ++i) {
+        const int ei = lane + 32 * i;
+        const float v = ei < p.E ? __ldcg(lr + ei) : -INFINITY;
+        unsigned band = __ballot_sync(0xffffffffu, ei < p.E && v >= lk1 - kRefineBand && v <= lk + kRefineBand);
+        while (band) {
+          const int src = __ffs(band) - 1;
+          band &= band - 1;
+          const float x = exact_logit(p.W, hrow, p.bias, p.d, src + 32 * i, lane);
+          if (lane == src) lr[ei] = x;
+        }
+      }
+      __threadfence();
+      __syncwarp();
+      warp_topk<NPL>(lr, p.E, p.k, lane, false, e, w, p.near_ties);
+    }
     if (lane < p.k) {
       p.idx[(long long)t * p.k + lane] = e;
       p.w[(long long)t * p.k + lane] = w;

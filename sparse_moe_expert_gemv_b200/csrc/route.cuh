@@ -126,9 +126,12 @@ MOE_DEV unsigned long long tournament_max(const unsigned long long (&v)[N]) {
 // j < k returns the j-th selection (descending logit) and its weight
 // exp(l_j - l_0) / sum_j' exp(l_j' - l_0).  When near_ties is non-null, a
 // (k+1)-th logit within 1e-5 of the k-th counts one near tie.
+// When lk is non-null, *lk and *lk1 receive (in every lane) the k-th and the
+// (k+1)-th largest logits (-inf when k == E).
 template <int NPL>
 MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int &sel_e,
-                       float &sel_w, unsigned long long *near_ties) {
+                       float &sel_w, unsigned long long *near_ties, float *lk = nullptr,
+                       float *lk1 = nullptr) {
   unsigned long long pk[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -138,6 +141,7 @@ MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int 
   if (trace && lane == 0 && pk[0] != 1ull) trace_point(kTrRouteLoaded);
   uint32_t my_key = 0, k0 = 0, kk = 0;
   int my_i = 0;
+  if (lk1) *lk1 = -INFINITY;
   for (int j = 0; j <= k; ++j) {
     if (j == k && k == E) break;
     const unsigned long long best = tournament_max<NPL>(pk);
@@ -148,6 +152,7 @@ MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int 
     if (j == k) {  // the (k+1)-th logit: near-tie count only
       if (near_ties && lane == 0 && key_to_float(kk) - key_to_float(wmax) < 1e-5f)
         atomicAdd(near_ties, 1ULL);
+      if (lk1) *lk1 = key_to_float(wmax);
       break;
     }
     const bool mine = (wi & 31) == lane;
@@ -161,6 +166,7 @@ MOE_DEV void warp_topk(const float *lr, int E, int k, int lane, bool trace, int 
     kk = wmax;
   }
   if (trace && lane == 0) trace_point(kTrRouteSelected);
+  if (lk) *lk = key_to_float(kk);
   const float ex = lane < k ? expf(key_to_float(my_key) - key_to_float(k0)) : 0.f;
   const float den = warp_sum(ex);
   sel_e = my_i;

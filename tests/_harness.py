@@ -220,12 +220,37 @@ def assert_close_rms(got, want, tol=OUT_TOL, what="output"):
     return err / max(rms(want), 1e-300)
 
 
+def bf16_ulp(v):
+    """Spacing of bf16 values at magnitude |v| (normal range)."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def assert_close_residual(got_bits, want_bits, tol=OUT_TOL, what="residual x"):
+    """The layer's bf16 output x = bf16(x_in + delta).  Two sums that agree
+    within the tolerance can still round to neighbouring bf16 values, so the
+    bound is tol * RMS plus one bf16 ulp at the element's magnitude; the
+    strict check is the one on delta, before this rounding."""
+    got = I.bf16_bits_to_f32(got_bits).astype(np.float64)
+    want = I.bf16_bits_to_f32(want_bits).astype(np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    if want.size == 0:
+        return
+    bound = tol * rms(want) + bf16_ulp(np.maximum(np.abs(got), np.abs(want)))
+    bad = np.abs(got - want) > bound
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond tol*RMS + 1 ulp, "
+                           f"max|err| {np.abs(got - want).max():.3e}")
+
+
 def check_routing(gpu_idx, gpu_w, orc, k):
     """Expert sets bit-exact and weights within W_TOL, except near ties.
     Returns the boolean mask of tokens that were checked."""
     ok = orc["margin"] >= TIE_MARGIN
     for t in np.nonzero(ok)[0]:
-        assert set(gpu_idx[t].tolist()) == set(orc["idx"][t].tolist()), f"token {t}"
+        assert set(gpu_idx[t].tolist()) == set(orc["idx"][t].tolist()), (
+            f"token {t}: oracle margin {orc['margin'][t]:.3e}, gpu only "
+            f"{sorted(set(gpu_idx[t].tolist()) - set(orc['idx'][t].tolist()))}, oracle only "
+            f"{sorted(set(orc['idx'][t].tolist()) - set(gpu_idx[t].tolist()))}")
         # compare weights expert by expert
         wo = dict(zip(orc["idx"][t].tolist(), orc["w"][t].tolist()))
         for e, wv in zip(gpu_idx[t].tolist(), gpu_w[t].tolist()):

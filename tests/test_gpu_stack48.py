@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from sparse_moe_expert_gemv_b200 import inputs as I
-from tests._harness import TIE_MARGIN, LayerSpec, assert_close_rms
+from tests._harness import TIE_MARGIN, LayerSpec, assert_close_residual, assert_close_rms
 
 pytestmark = pytest.mark.gpu
 
@@ -103,5 +103,4 @@ def test_stack48_graph_layers_residency_and_oracle(B, stack):
         B.moe_forward_delta(ctx, l, to_dev(xs[l]), T, delta)
         B.moe_sync(ctx, 60000)
         assert_close_rms(delta.cpu().numpy()[rows][ok], orc["delta"][ok], what=f"layer {l} delta")
-        assert_close_rms(I.bf16_bits_to_f32(xs[l + 1][rows][ok]),
-                         I.bf16_bits_to_f32(orc["x_out"][ok]), what=f"layer {l} x")
+        assert_close_residual(xs[l + 1][rows][ok], orc["x_out"][ok], what=f"layer {l} x")
