@@ -498,7 +498,14 @@ cudaEvent_t prof_event(moe_ctx *c, int i) {
 
 cudaError_t prof_mark(moe_ctx *c, int i, cudaStream_t s) {
   cudaEvent_t ev = prof_event(c, i);
-  return ev ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal) : cudaSuccess;
+  if (!ev) return cudaSuccess;
+  // inside a stream capture the event becomes an external graph node (so a
+  // replay records it again); outside one it is an ordinary record
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                            : cudaEventRecord(ev, s);
 }
 
 // The whole decode chain for one layer.  delta == nullptr: residual mode.
@@ -509,21 +516,29 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
 // Router logits of a chunk of N > 32 tokens by fp32 FMA (router_gemm_kernel).
 // A chunk too small to give every SM a 128 x 128 tile splits the reduction
 // over blockIdx.z (a power of two dividing d / 128, partial sums bounded by
-// the pf_part buffer); *ksplit receives the split count: 1 = logits (with
-// bias) in c->logits, > 1 = partials in c->pf_part for the top-k to add.
+// the pf_part buffer); *ksplit receives the split count.  Either way the
+// logits (with bias) end in c->logits: a split writes partial sums to
+// c->pf_part and router_sum_kernel adds them in split order.
 cudaError_t launch_router_fma(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, int *ksplit) {
   const int E = c->E, d = c->d;
   const int tiles = ((N + kRgBM - 1) / kRgBM) * ((E + kRgBN - 1) / kRgBN);
   int ks = 1;
-  while (ks * tiles < c->n_sm && (d / 128) % (2 * ks) == 0 &&
-         (long long)2 * ks * N * E <= c->pf_part_floats)
+  while (ks * tiles < c->n_sm && 2 * ks <= kMaxRouterSplit && (d / 128) % (2 * ks) == 0 &&
+         (long long)2 * ks * N * E <= c->pf_part_floats && E % 4 == 0)
     ks *= 2;
   *ksplit = ks;
-  RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d,
-                      c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, N, d, E,
-                      ks > 1 ? c->pf_part : c->logits, d / ks};
-  return launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN, ks), dim3(256),
-                0, s, rp);
+  const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
+  RouterGemmParams rp{h, c->d_router + (size_t)layer * E * d, bias, N, d, E, ks > 1 ? c->pf_part : c->logits,
+                      d / ks};
+  cudaError_t e = launch(router_gemm_kernel, dim3((N + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN, ks),
+                         dim3(256), 0, s, rp);
+  if (e == cudaSuccess && ks > 1) {
+    const long long n4 = (long long)N * E / 4;
+    RouterSumParams sp{c->pf_part, ks, bias, N, E, c->logits};
+    e = launch(router_sum_kernel, dim3((unsigned)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm)),
+               dim3(256), 0, s, sp);
+  }
+  return e;
 }
 
 moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const FinishParams &fp,
@@ -558,8 +573,8 @@ moe_status route_impl(moe_ctx *c, int layer, const uint16_t *x, int T, const Fin
       CUDA_TRY(c, e);
     else
       CUDA_TRY(c, launch_router_fma(c, s, h, T, layer, &ks));
-    PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4], c->pf_part, ks,
-                     bias, h, c->d_router + (size_t)layer * c->E * c->d, c->d};
+    PfRouteParams tp{c->logits, T, c->E, c->k, fp.idx, fp.w, c->pf_bmask, &c->stats[4], bias, h,
+                     c->d_router + (size_t)layer * c->E * c->d, c->d};
     CUDA_TRY(c, launch_pf_topk(c, s, tp));
     FinishParams fb = fp;
     fb.logits = nullptr;
@@ -717,8 +732,8 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   else  // small expert counts or chunks: fp32 FMA
     CUDA_TRY(c, launch_router_fma(c, s, h, N, layer, &ks));
   const int blocks = (N + kPfTok - 1) / kPfTok;
-  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], c->pf_part, ks, bias,
-                   h, c->d_router + (size_t)layer * E * d, d};
+  PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], bias, h,
+                   c->d_router + (size_t)layer * E * d, d};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;

@@ -46,16 +46,59 @@ struct PfTile {                  // one 128-row tile of one expert
   int row0, rows;                // first row in grouped order, rows <= 128
 };
 
+// logits[t, e] = sum_z part[z][t, e] (z = 0, 1, ... in order) + bias[e]: the
+// partial sums of a router whose reduction was split over ksplit CTAs.  One
+// thread per four logits, every partial load in flight at once.
+constexpr int kMaxRouterSplit = 16;
+struct RouterSumParams {
+  const float *part;  // [ksplit][T][E]
+  int ksplit;
+  const float *bias;  // [E] or null
+  int T, E;           // E a multiple of 4
+  float *logits;      // [T][E]
+};
+
+__global__ void __launch_bounds__(256) router_sum_kernel(RouterSumParams p) {
+  const float *part = p.part, *bias = p.bias;
+  const int ksplit = p.ksplit, E = p.E;
+  float *logits = p.logits;
+  pdl_wait();
+  const long long n4 = (long long)p.T * E / 4, plane = (long long)p.T * E;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    float4 v[kMaxRouterSplit];
+#pragma unroll
+    for (int z = 0; z < kMaxRouterSplit; ++z)
+      if (z < ksplit) v[z] = __ldcg(reinterpret_cast<const float4 *>(part + z * plane) + i);
+    float4 s = v[0];
+#pragma unroll
+    for (int z = 1; z < kMaxRouterSplit; ++z)
+      if (z < ksplit) {
+        s.x += v[z].x;
+        s.y += v[z].y;
+        s.z += v[z].z;
+        s.w += v[z].w;
+      }
+    if (bias) {
+      const int e = (int)((i * 4) % E);
+      s.x += bias[e];
+      s.y += bias[e + 1];
+      s.z += bias[e + 2];
+      s.w += bias[e + 3];
+    }
+    reinterpret_cast<float4 *>(logits)[i] = s;
+  }
+  pdl_launch_dependents();
+}
+
 struct PfRouteParams {
-  float *logits;        // [T, E]: read; with ksplit > 1 first written here
+  float *logits;        // [T, E]
   int T, E, k;
   int *idx;             // [T, k]
   float *w;             // [T, k]
   unsigned short *bmask;  // [blocks][E]: bit i = token 16 b + i selected the expert
   unsigned long long *near_ties;
-  const float *part;    // ksplit > 1: partial logits [ksplit][T][E] of a split reduction
-  int ksplit;
-  const float *bias;    // [E] or null, added to the summed partials
+  const float *bias;    // [E] or null (for the boundary refinement)
   const uint16_t *h;    // bf16 [T, d] router input and
   const float *W;       // fp32 [E, d] router rows, for the boundary refinement
   int d;
@@ -79,9 +122,7 @@ MOE_DEV float exact_logit(const float *W, const uint16_t *h, const float *bias, 
   return (float)(acc + (bias ? (double)bias[e] : 0.0));
 }
 
-// One warp per token; then the block's per-expert token sets.  When the
-// router's reduction was split (ksplit > 1), the warp first adds its token's
-// partial logits in split order (z = 0, 1, ...) and the bias.
+// One warp per token; then the block's per-expert token sets.
 template <int NPL>
 __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams p) {
   __shared__ unsigned s_mask[kPfMaxE];
@@ -90,17 +131,6 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_mask[e] = 0u;
   __syncthreads();
   const int t = blockIdx.x * kPfTok + wid;
-  if (t < p.T && p.ksplit > 1) {
-    const long long plane = (long long)p.T * p.E;
-    for (int e = lane; e < p.E; e += 32) {
-      const long long at = (long long)t * p.E + e;
-      float s = __ldcg(p.part + at);
-      for (int z = 1; z < p.ksplit; ++z) s += __ldcg(p.part + z * plane + at);
-      p.logits[at] = s + (p.bias ? p.bias[e] : 0.f);
-    }
-    __threadfence();  // the lanes' sums before the warp's top-k reads them
-    __syncwarp();
-  }
   if (t < p.T) {
     int e;
     float w, lk, lk1;
@@ -346,7 +376,7 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
 // (routing decisions are compared bit-exactly, so no reduced-precision
 // tensor-core path).  Small chunks split the reduction over blockIdx.z
 // (columns [z kchunk, (z+1) kchunk)) so the grid fills the GPU; each split
-// writes its partial sums, which prefill_topk_kernel adds in split order.
+// writes its partial sums, which router_sum_kernel adds in split order.
 // CTA tile: 128 tokens x 128 experts, 256 threads, each
 // an 8 x 8 block of outputs made of two 4-row and two 4-column halves 64
 // apart (so a warp's 16-byte shared-memory reads are contiguous: no bank
@@ -641,11 +671,12 @@ struct PfCfg {
   static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per code stage
   static constexpr int SA = 6;                              // A ring
   static constexpr int SC = 4;                              // code ring
+  static constexpr int NBB = 2;                             // B buffers (dequantised weights)
   static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB
   static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per accumulator
   static constexpr uint32_t CODES = (16 * TILE + 1023) / 1024 * 1024;  // 16 repacked code tiles
   static constexpr uint32_t BBUF = 2 * TILE_B;              // one B buffer (two tiles)
-  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + 2 * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
   static constexpr uint32_t ACC_COLS = 2 * kPfBN;           // TMEM columns per accumulator buffer
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
@@ -671,11 +702,11 @@ template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
   using C = PfCfg<FMT>;
-  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, TILE = C::TILE;
+  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, TILE = C::TILE, NBB = C::NBB;
   constexpr int COLS = GATED ? kPfBN : 2 * kPfBN;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
   __shared__ __align__(8) unsigned long long s_afull[SA], s_aempty[SA], s_cfull[SC], s_cempty[SC],
-      s_bfull[2], s_bempty[2], s_accf[2], s_acce[2];
+      s_bfull[NBB], s_bempty[NBB], s_accf[2], s_acce[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
@@ -689,9 +720,11 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       mbar_init(smem_addr(&s_cfull[i]), 1);
       mbar_init(smem_addr(&s_cempty[i]), 8);  // one arrival per dequantising warp
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBB; ++b) {
       mbar_init(smem_addr(&s_bfull[b]), 256);
       mbar_init(smem_addr(&s_bempty[b]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(smem_addr(&s_accf[b]), 1);
       mbar_init(smem_addr(&s_acce[b]), 128);
     }
@@ -787,7 +820,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
-          const uint32_t st = it % SA, use = it / SA, bb = it & 1, buse = it >> 1;
+          const uint32_t st = it % SA, use = it / SA, bb = it % NBB, buse = it / NBB;
           if (!mbar_wait_bounded(smem_addr(&s_bfull[bb]), buse & 1) ||
               !mbar_wait_bounded(smem_addr(&s_afull[st]), use & 1)) {
             ok = false;
@@ -877,7 +910,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
       for (int ks = 0; ks < nsteps; ++ks, ++it) {
-        const uint32_t cs = ct % SC, cuse = ct / SC, bb = it & 1, buse = it >> 1;
+        const uint32_t cs = ct % SC, cuse = ct / SC, bb = it % NBB, buse = it / NBB;
         bool got = mbar_wait_bounded(smem_addr(&s_cfull[cs]), cuse & 1);
         if (got && buse > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb]), (buse - 1) & 1);
         if (__any_sync(0xffffffffu, !got) || aborted()) {
