@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true",
                     help="headline only (no prefill / q2 / stack objects)")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--experts", type=int, default=512,
+                    help="routed experts per layer (256: the pruned configuration)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = {"prefill": 20, "stack": 10}.get(a.workload, 200)
@@ -238,7 +240,7 @@ def whole_job_rate(world, units_per_rank, ms_max):
 def workload_spec(name, T=4):
     from sparse_moe_expert_gemv_b200 import inputs as I
     if name == "decode":
-        return dict(kind=name, name=f"one MoE layer decode, d=2048 f=768 E=512 top-10 + shared, "
+        return dict(kind=name, name=f"one MoE layer decode, d=2048 f=768 E={E} top-10 + shared, "
                                     f"Q4 g32, T={T}, uniform routing",
                     fmt=I.Q4, zipf=False, T=T, seqs=1, prefill=False, metric="decode MoE tokens/s")
     if name == "q2":
@@ -247,11 +249,11 @@ def workload_spec(name, T=4):
                     fmt=I.Q2, zipf=True, T=T * 64, seqs=64, prefill=False, metric="decode MoE tokens/s")
     if name == "stack":
         return dict(kind=name, name="48-layer MoE stack (RMSNorm -> router -> experts -> combine + "
-                                    "residual), d=2048 f=768 E=512 top-10 + shared, Q4 g32, "
+                                    f"residual), d=2048 f=768 E={E} top-10 + shared, Q4 g32, "
                                     "4096-slot residency table by Zipf rank, Zipf(1.1) routing, "
                                     "T=4 x batch 8 = 32 tokens",
                     fmt=I.Q4, zipf=True, T=32, seqs=8, prefill=False, metric="stack MoE tokens/s")
-    return dict(kind="prefill", name="prefill chunk, 8192 tokens, one MoE layer, d=2048 f=768 E=512 "
+    return dict(kind="prefill", name=f"prefill chunk, 8192 tokens, one MoE layer, d=2048 f=768 E={E} "
                                      "top-10 + shared, Q4 g32, Zipf(1.1) routing",
                 fmt=I.Q4, zipf=True, T=8192, seqs=1, prefill=True, metric="prefill MoE tokens/s")
 
@@ -765,7 +767,9 @@ def q2_sweep(args, world, K, W):
 
 
 def main():
+    global E
     args = parse()
+    E = args.experts
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return 0
@@ -780,7 +784,7 @@ def main():
     else:
         n_rot = args.rot_layers if args.workload == "decode" else min(args.rot_layers, 4)
         res = run_native(args, world, spec, n_rot, args.steps, args.warmup)
-    extras = world == 1 and not args.no_extras and args.workload == "decode"
+    extras = world == 1 and not args.no_extras and args.workload == "decode" and E == 512
     if extras:
         ks, ws = args.extra_steps, 3
         pre = run_native(args, world, workload_spec("prefill"), 2, ks, ws)

@@ -334,6 +334,16 @@ MOE_API const char *moe_status_string(int status);
  * MOE_ERR_BAD_SLOT.  Not for production use. */
 MOE_API moe_status moe_debug_poke_slot(moe_ctx *ctx, int layer, int expert, int32_t slot);
 
+/* Test hook for the device's bounded waits: the next single-launch decode
+ * (moe_forward or moe_forward_delta of a window of <= 32 tokens) runs with
+ * a first grid barrier that cannot complete and a poll limit of `polls`
+ * (about a microsecond each), so that wait runs out.  The kernel then sets
+ * the device status (a bounded wait gave up), skips the layer and leaves;
+ * moe_sync returns MOE_ERR_DEVICE and resets the barrier counters, and the
+ * next call runs normally.  No fault, trap or hang is involved.  Errors:
+ * INVALID_ARG (NULL ctx, polls < 1). */
+MOE_API moe_status moe_debug_stall_next_decode(moe_ctx *ctx, uint32_t polls);
+
 /* Debug hook: copies on `stream` the normalised router input h (bf16
  * [T, d], h = RMSNorm(x) as the kernels computed it) of the most recent
  * moe_forward / moe_forward_delta / moe_prefill call on a layer with

@@ -31,7 +31,8 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_last_error", "moe_status_string", "moe_expert_bytes",
            "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
            "moe_set_trace", "moe_read_trace", "moe_route_static", "moe_prefill_delta",
-           "moe_prefill_route", "moe_route_static_status", "moe_debug_last_h")
+           "moe_prefill_route", "moe_route_static_status", "moe_debug_last_h",
+           "moe_debug_stall_next_decode")
 
 
 class MoeError(RuntimeError):
@@ -73,6 +74,7 @@ def _load():
         "moe_prefill_route": [P, I, P, I, P, P, P, P, P],
         "moe_route_static_status": [ctypes.POINTER(I), P],
         "moe_debug_last_h": [P, P, I, P],
+        "moe_debug_stall_next_decode": [P, ctypes.c_uint32],
         "moe_sync": [P, I],
         "moe_get_stats": [P, ctypes.POINTER(MoeStats)],
         "moe_debug_poke_slot": [P, I, I, ctypes.c_int32],
@@ -241,6 +243,10 @@ def moe_expert_bytes(d, f, quant_fmt):
 
 def moe_debug_poke_slot(ctx, layer, expert, slot):
     _check(ctx, _lib.moe_debug_poke_slot(ctx, layer, expert, slot))
+
+
+def moe_debug_stall_next_decode(ctx, polls):
+    _check(ctx, _lib.moe_debug_stall_next_decode(ctx, int(polls)))
 
 
 def moe_debug_last_h(ctx, out, T, stream=None):

@@ -73,11 +73,11 @@ MOE_DEV void grid_arrive(unsigned long long *count) {
   __syncthreads();
   if (threadIdx.x == 0) red_release_add_u64(count, 1ull);
 }
-MOE_DEV bool grid_wait(unsigned long long *count, unsigned long long target) {
+MOE_DEV bool grid_wait(unsigned long long *count, unsigned long long target, uint32_t limit = 1u << 22) {
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
     bool ok = false;
-    for (uint32_t i = 0; !ok && i < (1u << 22); ++i) ok = ld_acquire_u64(count) >= target;
+    for (uint32_t i = 0; !ok && i < limit; ++i) ok = ld_acquire_u64(count) >= target;
     s_ok = ok;
   }
   __syncthreads();
@@ -219,6 +219,9 @@ struct DecodeParams {
   int prefetch;         // bit 0: L2-prefetch the warp's down units after routing;
                         // bit 1: also its gate/up units beyond the ring's first ones
   int ring_lsu;         // ring slots filled by per-lane cp.async instead of bulk copies
+  unsigned long long bar1_extra;  // added to the first grid barrier's target (0; a test
+                                  // sets it so that the bounded wait runs out)
+  uint32_t bar1_polls;  // poll limit of the first grid barrier
   DecSmem sm;
 };
 
@@ -789,7 +792,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   grid_arrive(p.bar);
   // group sums of the window rows for the gate/up pass, while the grid syncs
   group_sums(win_g, L.rsh, T, L.ngd, GQ, kSumScale, s_hg);
-  if (!grid_wait(p.bar, ep1 * G)) {
+  if (!grid_wait(p.bar, ep1 * G + p.bar1_extra, p.bar1_polls)) {
     if (tid == 0) atomicOr(p.status, kErrTimeout);
     return;
   }
@@ -841,7 +844,7 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   if (lane == 0 && p.prefetch) {
     if (p.prefetch & 2) prefetch_units_l2(ph1, min(u0 + kRingD, u1), u1);
     if (p.prefetch & 1) {
-      const Phase pd = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes);
+      const Phase pd = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes, CG::SLOT);
       const SKCtx sd = sk_make(n_jobs * pd.RB * pd.UPI, W, gw, 0, nullptr, nullptr, nullptr, nullptr, WARPS);
       prefetch_units_l2(pd, sk_start(sd, gw), sk_start(sd, gw + 1));
     }
@@ -895,7 +898,9 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
   if (lane == 0) trace_point(kTrGateEnd);
 
   // ---------------- phase 4: down projection
-  const Phase ph2 = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes);
+  // down units of up to four tiles: the ring slots hold a gate/up unit (two
+  // tiles of both matrices), so a down unit may fill the same bytes
+  const Phase ph2 = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes, CG::SLOT);
   const SKCtx sk2 = sk_make(n_jobs * ph2.RB * ph2.UPI, W, gw, ep0 + 2, p.ws, p.flags + W, s_hand,
                             s_hflag, WARPS);
   const int v0 = sk_start(sk2, gw), v1 = sk_start(sk2, gw + 1);

@@ -82,13 +82,16 @@ struct Phase {
   long long region_off;  // byte offset of the pass's region inside an expert
 };
 
+// Units are 4, 2 or 1 tiles: the most that divide the item's tiles and fit
+// one ring slot of slot_bytes (0: two tiles' worth).
 MOE_DEV Phase make_phase(const unsigned long long *job_ptr, int R, int K, int TK, int stride,
-                         long long region_off) {
+                         long long region_off, int slot_bytes = 0) {
   Phase ph;
   ph.job_ptr = job_ptr;
   ph.RB = R / 16;
   ph.NTILE = K / TK;
-  ph.tps = ph.NTILE % 2 == 0 ? 2 : 1;
+  if (slot_bytes <= 0) slot_bytes = 2 * stride;
+  ph.tps = ph.NTILE % 4 == 0 && 4 * stride <= slot_bytes ? 4 : ph.NTILE % 2 == 0 ? 2 : 1;
   ph.UPI = ph.NTILE / ph.tps;
   ph.stride = stride;
   ph.region_off = region_off;
@@ -412,7 +415,18 @@ struct ItemRun {
       const bool ok = mbar_wait_bounded(r.bar_s + 8 * r.u, r.phase);
       if (__any_sync(0xffffffffu, !ok)) return false;  // warp-uniform
       const uint32_t slot_s = r.data_s + r.u * r.slot_stride;
-      if (ph.tps == 2) {
+      if (ph.tps == 4) {
+        // two straight-line blocks of two tiles each
+#pragma unroll 1
+        for (int hp = 0; hp < 2; ++hp) {
+          uint4 b0[NTA][NB], b1[NTA][NB];
+          float2 hv0[NTA][2], hv1[NTA][2];
+          load_b(b0, hv0, br, 4 * u + 2 * hp, tig);
+          load_b(b1, hv1, br, 4 * u + 2 * hp + 1, tig);
+          tile(slot_s + 2 * hp * C::STRIDE, lane, b0, hv0, acc);
+          tile(slot_s + (2 * hp + 1) * C::STRIDE, lane, b1, hv1, acc);
+        }
+      } else if (ph.tps == 2) {
         // both tiles of the unit in one block of straight-line code, so the
         // scheduler can overlap one tile's unpack with the other's mma chains
         uint4 b0[NTA][NB], b1[NTA][NB];

@@ -85,6 +85,10 @@ struct moe_ctx {
 
   int gemv_blocks[2][2][2] = {};  // [fmt][gated][NTM-1]
   int dec_prefetch = 0;           // decode_kernel L2 prefetch mode (DecodeParams::prefetch)
+  bool dec_fits = true;           // one decode_kernel CTA fits on every SM (checked at create)
+  int dec_coop = -1;              // decode launches cooperative: -1 untried, 0 no, 1 yes
+  int dec_stall_next = 0;         // test hook: the next decode launch's first barrier cannot complete
+  uint32_t dec_stall_polls = 0;
   int dec_ring_lsu = 0;           // decode_kernel ring fill (DecodeParams::ring_lsu)
   // profiling: 4 events per call slot
   bool profiling = false;
@@ -390,16 +394,50 @@ DecSmem decode_layout(const moe_ctx *c, int T) {
 // Windows the single-launch decode kernel serves: token sets fit a 32-bit
 // mask, the pairs and the window fit its shared memory.
 bool use_decode_kernel(const moe_ctx *c, int T) {
-  if (T < 1 || T > kDecMaxT || T * c->k > kDecMaxPairs || c->E > kDecMaxE || c->k > kDecMaxK)
+  if (!c->dec_fits || T < 1 || T > kDecMaxT || T * c->k > kDecMaxPairs || c->E > kDecMaxE ||
+      c->k > kDecMaxK)
     return false;
   const DecSmem L = decode_layout(c, T);
   return L.stage_bytes >= L.rsh && (long long)T * L.rsh <= kDecSmem - L.win &&
          L.rsa <= L.stage_bytes;
 }
 
+// The decode kernel's CTAs wait on one another (grid barriers), so all of
+// them must be resident: one per SM.  Outside a stream capture the launch is
+// cooperative, so the driver refuses a grid that cannot be co-resident
+// instead of leaving the waits to run out; it is combined with programmatic
+// dependent launch when the driver accepts both (tried once per context,
+// else PDL alone).  Captured launches use PDL alone.
 cudaError_t launch_decode(moe_ctx *c, cudaStream_t s, const DecodeParams &dp) {
   void (*k)(DecodeParams) = c->fmt == MOE_Q4_SYM_G32_F16 ? decode_kernel<1, 1> : decode_kernel<2, 1>;
-  return launch(k, dim3(c->n_sm), dim3(GemvCfg<1, true, 1>::WARPS * 32), kDecSmem, s, dp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c->n_sm);
+  cfg.blockDim = dim3(GemvCfg<1, true, 1>::WARPS * 32);
+  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    cs = cudaStreamCaptureStatusActive;  // unknown: take the plain launch
+  }
+  if (c->dec_coop != 0 && cs == cudaStreamCaptureStatusNone) {
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k, dp);
+    if (e == cudaSuccess || c->dec_coop == 1) {
+      c->dec_coop = e == cudaSuccess ? 1 : c->dec_coop;
+      return e;
+    }
+    (void)cudaGetLastError();  // not accepted together: PDL alone from now on
+    c->dec_coop = 0;
+  }
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, dp);
 }
 
 // Top-k of every token, one warp per token over ceil(T / 16) CTAs: idx, w and
@@ -769,7 +807,9 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
   PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
                      c->pf_row_of, c->pf_hg, perm ? perm : c->pf_perm, c->pf_hot};
-  CUDA_TRY(c, launch(prefill_scatter_kernel, dim3(blocks), dim3(kPfTok * 32), 0, s, cp));
+  // small chunks split each token row's columns over more CTAs
+  const int ysplit = std::max(1, std::min(d / 256, (2 * c->n_sm + blocks - 1) / blocks));
+  CUDA_TRY(c, launch(prefill_scatter_kernel, dim3(blocks, ysplit), dim3(kPfTok * 32), 0, s, cp));
   return MOE_OK;
 }
 
@@ -876,6 +916,9 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.sm = decode_layout(c, T);
     dp.prefetch = c->dec_prefetch;
     dp.ring_lsu = c->dec_ring_lsu;
+    dp.bar1_extra = c->dec_stall_next ? (unsigned long long)c->n_sm : 0ull;
+    dp.bar1_polls = c->dec_stall_next ? c->dec_stall_polls : (1u << 22);
+    c->dec_stall_next = 0;
     CUDA_TRY(c, launch_decode(c, s, dp));
     // one kernel: the profile's route / experts / combine marks coincide
     CUDA_TRY(c, prof_mark(c, 1, s));
@@ -1048,6 +1091,15 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   if (e == cudaSuccess) e = setup_gemv<1, false, 2>(c->n_sm, &c->gemv_blocks[0][0][1]);
   if (e == cudaSuccess) e = setup_gemv<2, true, 2>(c->n_sm, &c->gemv_blocks[1][1][1]);
   if (e == cudaSuccess) e = setup_gemv<2, false, 2>(c->n_sm, &c->gemv_blocks[1][0][1]);
+  if (e == cudaSuccess) {
+    // the single-launch decode kernel needs one resident CTA per SM; where
+    // it does not fit (a smaller part, or shared-memory carve-outs), windows
+    // take the multi-launch path instead
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<1, 1>,
+                                                      GemvCfg<1, true, 1>::WARPS * 32, kDecSmem);
+    c->dec_fits = e == cudaSuccess && per_sm >= 1;
+  }
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     moe_destroy(c);
@@ -1468,6 +1520,17 @@ moe_status moe_debug_poke_slot(moe_ctx *c, int layer, int expert, int32_t slot) 
     return fail(c, MOE_ERR_INVALID_ARG, "moe_debug_poke_slot");
   CUDA_TRY(c, cudaMemcpy(c->d_slot_of + (size_t)layer * c->E + expert, &slot, sizeof slot,
                          cudaMemcpyHostToDevice));
+  return MOE_OK;
+}
+
+// Test hook: the next single-launch decode (moe_forward / moe_forward_delta
+// of a window of <= 32 tokens) gets a first grid barrier that cannot
+// complete, with a poll limit of `polls`; its bounded wait runs out, the
+// kernel reports kErrTimeout and leaves, and moe_sync reports it.
+moe_status moe_debug_stall_next_decode(moe_ctx *c, uint32_t polls) {
+  if (!c || polls < 1) return fail(c, MOE_ERR_INVALID_ARG, "moe_debug_stall_next_decode");
+  c->dec_stall_next = 1;
+  c->dec_stall_polls = polls;
   return MOE_OK;
 }
 

@@ -113,10 +113,29 @@ constexpr float kRefineBand = 2e-3f;
 
 // One warp: the exact logit of expert e for token row h (fp64 sum of the
 // exact fp32 x bf16 products, then the bias), rounded once to fp32.
+// d a multiple of 128; loads four columns per lane at a time, eight in flight.
 MOE_DEV float exact_logit(const float *W, const uint16_t *h, const float *bias, int d, int e, int lane) {
-  const float *wr = W + (long long)e * d;
+  const float4 *wr = reinterpret_cast<const float4 *>(W + (long long)e * d);
+  const uint2 *hr = reinterpret_cast<const uint2 *>(h);
+  const int n4 = d / 4;
   double acc = 0.0;
-  for (int i = lane; i < d; i += 32) acc += (double)wr[i] * (double)__uint_as_float((uint32_t)h[i] << 16);
+  for (int i0 = lane; i0 < n4; i0 += 32 * 8) {
+    float4 wv[8];
+    uint2 hv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = i0 + 32 * q;
+      wv[q] = i < n4 ? __ldg(wr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      hv[q] = i < n4 ? __ldg(hr + i) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      acc += (double)wv[q].x * (double)__uint_as_float(hv[q].x << 16);
+      acc += (double)wv[q].y * (double)__uint_as_float(hv[q].x & 0xFFFF0000u);
+      acc += (double)wv[q].z * (double)__uint_as_float(hv[q].y << 16);
+      acc += (double)wv[q].w * (double)__uint_as_float(hv[q].y & 0xFFFF0000u);
+    }
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return (float)(acc + (bias ? (double)bias[e] : 0.0));
@@ -322,6 +341,8 @@ struct PfScatterParams {
 
 // One warp per token: its k pairs (and its shared-expert pair) get their
 // grouped rows, and the token's row is copied (fp16, saturating) to each.
+// blockIdx.y splits the row's columns (small chunks: more CTAs); the CTAs
+// with blockIdx.y == 0 write the row map and the permutation.
 // With perm set, the routed rows' pair ids are also written in grouped
 // order: the bucket permutation (each expert's pairs in ascending t).
 __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterParams p) {
@@ -344,16 +365,19 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_scatter_kernel(PfScatterP
     rows[p.k] = P + t;
     copy |= 1ull << p.k;
   }
-  if (lane < p.k) {
+  if (lane < p.k && blockIdx.y == 0) {
     const int q = t * p.k + lane;
     p.row_of[q] = (copy >> lane) & 1 ? rows[lane] : ~q;
     // the bucket permutation: grouped row -> pair id (rows < P are routed)
     if (p.perm) p.perm[rows[lane]] = q;
   }
-  if (lane == 0 && p.has_shared) p.row_of[P + t] = P + t;
-  // copy the token row to every destination, 8 elements per lane per step
+  if (lane == 0 && p.has_shared && blockIdx.y == 0) p.row_of[P + t] = P + t;
+  // copy the token row's column slice to every destination, 8 elements per
+  // lane per step
   const uint4 *src = reinterpret_cast<const uint4 *>(p.h + (long long)t * p.d);
-  for (int i = lane; i < p.d / 8; i += 32) {
+  const int n8 = p.d / 8, per = (n8 + gridDim.y - 1) / gridDim.y;
+  const int i0 = blockIdx.y * per, i1 = min(n8, i0 + per);
+  for (int i = i0 + lane; i < i1; i += 32) {
     const uint4 v = __ldg(src + i);
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[4];

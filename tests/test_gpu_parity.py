@@ -520,6 +520,49 @@ def test_corrupt_slot_is_reported_not_trapped(B):
         B.moe_destroy(ctx)
 
 
+def test_decode_barrier_wait_runs_out_and_recovers(B):
+    """A bounded device wait made to run out: the test hook gives the next
+    single-launch decode a first grid barrier that cannot complete (poll
+    limit ~16 K).  The kernel reports the give-up and leaves; moe_sync
+    returns MOE_ERR_DEVICE with the timeout bit, resets the barrier counters,
+    and the next calls match the oracle.  No fault or hang is involved."""
+    spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=I.Q4, seed=18, shared=True)
+    ctx = make_ctx(B, spec, max_tokens=32)
+    try:
+        load_layer(B, ctx, spec)
+        x = I.hidden_np(18, 4, 256)
+        orc = oracle_for(spec, x)
+        check(run(B, ctx, spec, x), orc, spec)          # before
+        B.moe_debug_stall_next_decode(ctx, 1 << 14)
+        delta = torch.empty((4, 256), dtype=torch.float32, device="cuda")
+        B.moe_forward_delta(ctx, 0, to_dev(x), 4, delta)
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_sync(ctx, 60000)
+        assert ei.value.status == 6 and "0x8" in str(ei.value)
+        B.moe_sync(ctx, 60000)                          # status cleared
+        for _ in range(2):                              # after: counters reset
+            check(run(B, ctx, spec, x), orc, spec)
+    finally:
+        B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("T", [4, 40])
+def test_pruned_256_expert_layer(B, T):
+    """The pruned "Coder" configuration of the engine article's performance
+    validation (256 of the 512 experts kept, 10 active): d=2048, f=768,
+    E=256, top-10 + shared, Q4; a decode window and a 40-token window."""
+    spec = LayerSpec(d=2048, f=768, E=256, k=10, fmt=I.Q4, seed=0, shared=True)
+    ctx = make_ctx(B, spec, max_tokens=64)
+    try:
+        load_layer(B, ctx, spec)
+        x = I.hidden_np(0, T, 2048, window=256 + T)
+        sample = None if T <= 4 else np.array([0, 7, T // 2, T - 1])
+        rel, ties = check(run(B, ctx, spec, x), oracle_for(spec, x, sample), spec, sample)
+        print(f"E=256 T={T}: delta max-err/RMS {rel:.2e}, near ties {ties}")
+    finally:
+        B.moe_destroy(ctx)
+
+
 def test_sync_times_out_on_stalled_stream(B, decode_q4):
     ctx, spec = decode_q4
     x = to_dev(I.hidden_np(0, 4, 2048))

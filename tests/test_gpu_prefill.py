@@ -226,6 +226,36 @@ def test_prefill_chunk_8192_covering_sample(B, chunk8192):
           f"near ties {int((~ok).sum())}")
 
 
+def test_prefill_pruned_256_experts(B):
+    """A 1024-token chunk of the pruned 256-expert configuration (E a
+    multiple of 256: the tensor-core router), Zipf routing; routing and
+    buckets on every token, the layer on a covering sample."""
+    spec = LayerSpec(d=2048, f=768, E=256, k=10, fmt=I.Q4, seed=0, shared=True, zipf=True)
+    ctx = make_ctx(B, spec, 1024)
+    try:
+        load_layer(B, ctx, spec)
+        N = 1024
+        x = I.hidden_np(0, N, spec.d, window=2560)
+        lg = router_parallel(x, spec.W, spec.bias)
+        oi, ow, om = O.topk(lg, spec.k)
+        orc = dict(idx=oi, w=ow, margin=om)
+        out = _route_outputs(N, spec.k, spec.E)
+        B.moe_prefill_route(ctx, 0, to_dev(x), N, *out)
+        B.moe_sync(ctx, 60000)
+        idx, w, off, perm = [t.cpu().numpy() for t in out]
+        ok = check_routing(idx, w, orc, spec.k)
+        check_buckets(off, perm, oi, spec.E, spec.k, ok)
+        delta, x_out = run_prefill(B, ctx, spec, x)
+        rows = covering_sample(oi, spec.E)
+        keep = om[rows] >= TIE_MARGIN
+        od, ox, _ = oracle_rows(spec, x, rows)
+        rel = assert_close_rms(delta[rows][keep], od[keep], what="MoE delta")
+        assert_close_residual(x_out[rows][keep], ox[keep])
+        print(f"E=256 chunk: {rows.size} sampled, delta max-err/RMS {rel:.2e}, near ties {int((~ok).sum())}")
+    finally:
+        B.moe_destroy(ctx)
+
+
 def test_prefill_route_rejects_bad_calls(B):
     spec = LayerSpec(d=256, f=128, E=16, k=2, fmt=I.Q4, seed=5, shared=True)
     ctx = make_ctx(B, spec, 16)  # decode-only context: no prefill buffers
