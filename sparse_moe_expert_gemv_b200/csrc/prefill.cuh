@@ -36,12 +36,13 @@
 namespace moe {
 
 constexpr int kPfTok = 16;       // tokens per block of the top-k / scatter kernels (one warp each)
-constexpr int kPfBM = 128;       // GEMM tile rows (tokens of one expert)
+constexpr int kPfBM = 128;       // rows of one MMA (an M-half of a GEMM tile)
+constexpr int kPfTileRows = 2 * kPfBM;  // rows of one GEMM tile of an expert (two M-halves)
 constexpr int kPfBN = 128;       // GEMM tile columns (output features)
 constexpr int kPfBK = 64;        // reduction per stage (one 128-byte swizzle row of fp16)
 constexpr int kPfMaxE = 1024;
 
-struct PfTile {                  // one 128-row tile of one expert
+struct PfTile {                  // one tile of up to 256 rows of one expert
   const uint8_t *w;              // expert base (repacked layout)
   int row0, rows;                // first row in grouped order, rows <= 128
 };
@@ -261,14 +262,14 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
     const int run = p.eoff[e];  // token count from prefill_colscan_kernel
     const bool hot = run >= p.hot_min;
     cnt[e] = run;
-    tl[e] = hot ? (run + kPfBM - 1) / kPfBM : 0;
+    tl[e] = hot ? (run + kPfTileRows - 1) / kPfTileRows : 0;
     jl[e] = hot ? 0 : (run + p.chunk - 1) / p.chunk;
   }
   block_exclusive_scan(cnt, cnt, p.E, s_red);
   block_exclusive_scan(tl, tl, p.E, s_red);
   block_exclusive_scan(jl, jl, p.E, s_red);
   const int routed_tiles = tl[p.E], P = cnt[p.E], n_jobs = jl[p.E];
-  const int shared_tiles = p.shared ? (p.T + kPfBM - 1) / kPfBM : 0;
+  const int shared_tiles = p.shared ? (p.T + kPfTileRows - 1) / kPfTileRows : 0;
   if (routed_tiles + shared_tiles > p.max_tiles || n_jobs > p.max_jobs) {
     if (tid == 0) {
       atomicOr(p.status, kErrJobOverflow);
@@ -292,10 +293,10 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
     atomicAdd(&s_hm[hit ? 0 : 1], (unsigned long long)n);
     atomicAdd(&s_hm[2], 1ull);
     if (hot) {
-      for (int m = 0, ti = tl[e]; m < n; m += kPfBM, ++ti) {
+      for (int m = 0, ti = tl[e]; m < n; m += kPfTileRows, ++ti) {
         p.tiles[ti].w = ptr;
         p.tiles[ti].row0 = cnt[e] + m;
-        p.tiles[ti].rows = min(kPfBM, n - m);
+        p.tiles[ti].rows = min(kPfTileRows, n - m);
       }
     } else {
       for (int m = 0, j = jl[e]; m < n; m += p.chunk, ++j) {
@@ -308,8 +309,8 @@ __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
   if (tid == 0) p.eoff[p.E] = P;
   for (int q = tid; q < shared_tiles; q += blockDim.x) {
     p.tiles[routed_tiles + q].w = p.shared;
-    p.tiles[routed_tiles + q].row0 = P + q * kPfBM;
-    p.tiles[routed_tiles + q].rows = min(kPfBM, p.T - q * kPfBM);
+    p.tiles[routed_tiles + q].row0 = P + q * kPfTileRows;
+    p.tiles[routed_tiles + q].rows = min(kPfTileRows, p.T - q * kPfTileRows);
   }
   __syncthreads();
   if (tid == 0) {
@@ -681,53 +682,58 @@ constexpr int kPfGemmThreads = 512;  // 16 warps
 constexpr int kPfDeqWarp0 = 8;       // warps 8..15 dequantise
 constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM lane quarters 0..3)
 
-// Both passes run two 128-column accumulators per item: gate and up of the
-// same 128 features (gate/up pass), or two adjacent 128-feature slices
-// (down pass, 256 features per item).  The A tiles (64 reduction columns of
-// 128 token rows) and the code tiles travel in two rings: an A stage is
-// released when its MMAs complete, a code stage when the dequantising warps
-// have read it.  A code stage holds the 16 repacked tiles of one tile
-// column: 64 reduction columns for Q4 (one k-step), 128 for Q2 (two k-steps,
-// one quantisation group each).
+// A work item is one tile of up to 256 rows of one expert (two M-halves of
+// 128 rows) times one output slice: 64 features of the gate/up pass (gate
+// and up side by side: 128 weight rows) or 128 features of the down pass
+// (128 weight rows).  Each k-step dequantises the slice's 128 weight rows
+// once and feeds them to both halves' MMAs (m128n128k16 each), so the
+// dequantisation -- the pipeline's costliest stage -- is shared by 256 token
+// rows.  The A tiles (64 reduction columns of both halves' rows) and the
+// code tiles travel in two rings: an A stage is released when its MMAs
+// complete, a code stage when the dequantising warps have read it.  A code
+// stage holds the 8 repacked tiles of one tile column: 64 reduction columns
+// for Q4 (one k-step), 128 for Q2 (two k-steps, one quantisation group
+// each).
 template <int FMT>
 struct PfCfg {
   static constexpr int TILE = FMT == 1 ? 576 : 640;         // repacked code tile (+ scales)
   static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per code stage
-  static constexpr int SA = 6;                              // A ring
+  static constexpr int SA = 5;                              // A ring
   static constexpr int SC = 4;                              // code ring
   static constexpr int NBB = 2;                             // B buffers (dequantised weights)
-  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB
-  static constexpr uint32_t TILE_B = kPfBN * kPfBK * 2;     // 16 KB per accumulator
-  static constexpr uint32_t CODES = (16 * TILE + 1023) / 1024 * 1024;  // 16 repacked code tiles
-  static constexpr uint32_t BBUF = 2 * TILE_B;              // one B buffer (two tiles)
-  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
-  static constexpr uint32_t ACC_COLS = 2 * kPfBN;           // TMEM columns per accumulator buffer
+  static constexpr int NB_ROWS = 128;                       // weight rows per item (MMA N)
+  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB per M-half
+  static constexpr uint32_t STAGE_A = 2 * TILE_A;           // both halves
+  static constexpr uint32_t BBUF = NB_ROWS * kPfBK * 2;     // 16 KB
+  static constexpr uint32_t CODES = (8 * TILE + 1023) / 1024 * 1024;  // 8 repacked code tiles
+  static constexpr uint32_t SMEM = SA * STAGE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t ACC_COLS = 2 * NB_ROWS;         // TMEM columns per buffer (both halves)
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
 
-// Grouped GEMM over the tile list, warp-specialised.  Work item = (128-row
-// tile, output slice of 128 (gate/up) or 256 (down) features); persistent
-// CTAs walk items blockIdx.x, +gridDim.x.
-//  warp 0 lane 0   producer: per 64-column reduction step the A tile (2-D
-//                  TMA, 128-byte swizzle) into a free stage of the A ring,
-//                  and at each new tile column the 16 repacked code tiles
-//                  (1-D bulk copies) into a free stage of the code ring
-//  warps 8..15     dequantise a k-step's codes into one of two swizzled fp16
-//                  B buffers, arrive on the buffer's barrier, and release
-//                  the code stage after its last k-step
-//  warp 1 lane 0   issues the MMAs (m128n256k16: both accumulators at once,
-//                  operands in shared memory, fp32 in TMEM) and commits the
-//                  release of the A stage and of the B buffer; accumulator
-//                  pairs alternate between two TMEM buffers
-//  warps 4..7      drain an accumulator buffer (TMEM lanes = tile rows)
-//                  while the next item accumulates into the other one
+// Grouped GEMM over the tile list, warp-specialised; persistent CTAs walk
+// the items blockIdx.x, +gridDim.x.
+//  warp 0 lane 0   producer: per 64-column reduction step the A tiles of
+//                  both M-halves (2-D TMA, 128-byte swizzle; the second half
+//                  only when the tile has more than 128 rows) into a free
+//                  stage of the A ring, and at each new tile column the 8
+//                  repacked code tiles (1-D bulk copies) into the code ring
+//  warps 8..15     one code tile each: dequantise a k-step's codes into one
+//                  of two swizzled fp16 B buffers, arrive on the buffer's
+//                  barrier, and release the code stage after its last k-step
+//  warp 1 lane 0   issues the MMAs (per 16-column substep one m128n128k16
+//                  per M-half, operands in shared memory, fp32 in TMEM) and
+//                  commits the release of the A stage and of the B buffer;
+//                  accumulators alternate between two TMEM buffers
+//  warps 4..7      drain an accumulator buffer (TMEM lanes = rows of each
+//                  half) while the next item accumulates into the other one
 // Every wait is bounded; a timeout raises kErrTimeout and every role stops.
 template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
   using C = PfCfg<FMT>;
   constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, TILE = C::TILE, NBB = C::NBB;
-  constexpr int COLS = GATED ? kPfBN : 2 * kPfBN;  // output features per item
+  constexpr int COLS = GATED ? C::NB_ROWS / 2 : C::NB_ROWS;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
   __shared__ __align__(8) unsigned long long s_afull[SA], s_aempty[SA], s_cfull[SC], s_cempty[SC],
       s_bfull[NBB], s_bempty[NBB], s_accf[2], s_acce[2];
@@ -769,9 +775,9 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   const int ntiles = ldcg_i32(p.n_tiles);
   const int nslices = p.N / COLS, nsteps = p.K / kPfBK;
   const int items = ntiles * nslices;
-  auto stage_a = [&](uint32_t st) { return stage0 + st * C::TILE_A; };
-  auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::TILE_A + cs * C::CODES; };
-  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::TILE_A + SC * C::CODES + b * C::BBUF; };
+  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_A; };
+  auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::STAGE_A + cs * C::CODES; };
+  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::STAGE_A + SC * C::CODES + b * C::BBUF; };
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
   auto give_up = [&]() {
     *reinterpret_cast<volatile int *>(&s_abort) = 1;
@@ -785,7 +791,8 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < items && ok && !aborted(); item += gridDim.x) {
         const PfTile tile = p.tiles[item / nslices];
-        const int rb0 = (item % nslices) * (COLS / 16);
+        const bool two = tile.rows > kPfBM;  // the second M-half has rows
+        const int rb0 = (item % nslices) * (GATED ? COLS / 16 : COLS / 16);
         const uint8_t *wbase = tile.w + p.region_off;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
           if (ks % SPC == 0) {  // the next tile column's codes
@@ -795,17 +802,17 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
               break;
             }
             const uint32_t cbar = smem_addr(&s_cfull[cs]);
-            mbar_expect_tx(cbar, 16 * TILE);
-            // code tile q = 2 r + m: row block r of accumulator m
-            if constexpr (GATED) {  // gate and up tiles of a row block are adjacent
-              for (int r = 0; r < 8; ++r)
+            mbar_expect_tx(cbar, 8 * TILE);
+            if constexpr (GATED) {
+              // code tile q = 2 r + m: row block r of matrix m (gate, up);
+              // the two tiles of a row block are adjacent in memory
+              for (int r = 0; r < 4; ++r)
                 bulk_g2s(stage_c(cs) + r * 2 * TILE,
                          wbase + ((long long)(rb0 + r) * p.ntile_k + tk) * 2 * TILE, 2 * TILE, cbar);
             } else {
-              for (int q = 0; q < 16; ++q)
-                bulk_g2s(stage_c(cs) + q * TILE,
-                         wbase + ((long long)(rb0 + (q & 1) * 8 + (q >> 1)) * p.ntile_k + tk) * TILE, TILE,
-                         cbar);
+              for (int q = 0; q < 8; ++q)  // code tile q = row block q
+                bulk_g2s(stage_c(cs) + q * TILE, wbase + ((long long)(rb0 + q) * p.ntile_k + tk) * TILE,
+                         TILE, cbar);
             }
             ++ct;
           }
@@ -815,8 +822,9 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
             break;
           }
           const uint32_t bar = smem_addr(&s_afull[st]);
-          mbar_expect_tx(bar, C::TILE_A);
+          mbar_expect_tx(bar, two ? 2 * C::TILE_A : C::TILE_A);
           tma_load_2d(stage_a(st), &amap, ks * kPfBK, tile.row0, bar);
+          if (two) tma_load_2d(stage_a(st) + C::TILE_A, &amap, ks * kPfBK, tile.row0 + kPfBM, bar);
         }
       }
       if (!ok) give_up();
@@ -830,12 +838,10 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   } else if (wid == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // the two B tiles of a buffer are one 256-row K-major tile (rows 0..127
-      // feed accumulator columns 0..127, rows 128..255 columns 128..255):
-      // one m128n256k16 MMA per 16-column step
-      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, 2 * kPfBN);
+      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, C::NB_ROWS);
       uint32_t it = 0, ii = 0;
       for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x, ++ii) {
+        const bool two = p.tiles[item / nslices].rows > kPfBM;
         const uint32_t buf = ii & 1, acc = tmem + buf * C::ACC_COLS;
         if (ii >= 2 && !mbar_wait_bounded(smem_addr(&s_acce[buf]), ((ii >> 1) - 1) & 1)) {
           give_up();
@@ -852,9 +858,13 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kPfBK / 16; ++kk)
-            umma_f16(acc, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(bbuf(bb) + kk * 32), IDESC,
-                     (ks | kk) != 0);
+          for (int kk = 0; kk < kPfBK / 16; ++kk) {
+            const uint64_t db = umma_desc_sw128(bbuf(bb) + kk * 32);
+            umma_f16(acc, umma_desc_sw128(stage_a(st) + kk * 32), db, IDESC, (ks | kk) != 0);
+            if (two)
+              umma_f16(acc + C::NB_ROWS, umma_desc_sw128(stage_a(st) + C::TILE_A + kk * 32), db, IDESC,
+                       (ks | kk) != 0);
+          }
           umma_commit(smem_addr(&s_aempty[st]));
           umma_commit(smem_addr(&s_bempty[bb]));
         }
@@ -869,7 +879,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     }
   } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = wid & 3, r = quarter * 32 + lane;  // tile row = TMEM lane
+    const int quarter = wid & 3, lr = quarter * 32 + lane;  // TMEM lane = row of each half
     uint32_t ii = 0;
     for (int item = blockIdx.x; item < items; item += gridDim.x, ++ii) {
       const uint32_t buf = ii & 1;
@@ -881,41 +891,48 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       tc_fence_after();
       const PfTile tile = p.tiles[item / nslices];
       const int n0 = (item % nslices) * COLS;
-      const uint32_t lane_addr = tmem + buf * C::ACC_COLS + ((uint32_t)(quarter * 32) << 16);
-      for (int c0 = 0; c0 < kPfBN; c0 += 32) {
-        float g[32];
-        tmem_ld32(lane_addr + c0, g);
-        float u[32];
-        tmem_ld32(lane_addr + kPfBN + c0, u);
-        if (r < tile.rows) {
-          if constexpr (GATED) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
+      for (int half = 0; half < (tile.rows > kPfBM ? 2 : 1); ++half) {
+        const int r = half * kPfBM + lr;
+        const uint32_t lane_addr =
+            tmem + buf * C::ACC_COLS + half * C::NB_ROWS + ((uint32_t)(quarter * 32) << 16);
+        if constexpr (GATED) {
+          // accumulator columns [0, 64) = gate, [64, 128) = up of features n0 ..
+          for (int c0 = 0; c0 < COLS; c0 += 32) {
+            float g[32], u[32];
+            tmem_ld32(lane_addr + c0, g);
+            tmem_ld32(lane_addr + COLS + c0, u);
+            if (r < tile.rows) {
+              uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t pk[4];
+              for (int v = 0; v < 4; ++v) {
+                uint32_t pk[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int i = v * 8 + q * 2;
-                const float a0 = g[i] / (1.0f + __expf(-g[i])) * u[i];
-                const float a1 = g[i + 1] / (1.0f + __expf(-g[i + 1])) * u[i + 1];
-                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
+                for (int q = 0; q < 4; ++q) {
+                  const int i = v * 8 + q * 2;
+                  const float a0 = g[i] / (1.0f + __expf(-g[i])) * u[i];
+                  const float a1 = g[i + 1] / (1.0f + __expf(-g[i + 1])) * u[i + 1];
+                  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
+                }
+                dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
-              dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-          } else {
-            uint4 *d0 = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
-            uint4 *d1 = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + kPfBN + c0);
+          }
+        } else {
+          for (int c0 = 0; c0 < COLS; c0 += 32) {
+            float y[32];
+            tmem_ld32(lane_addr + c0, y);
+            if (r < tile.rows) {
+              uint4 *dst = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t pg[4], pu[4];
+              for (int v = 0; v < 4; ++v) {
+                uint32_t pk[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int i = v * 8 + q * 2;
-                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pg[q]) : "f"(g[i + 1]), "f"(g[i]));
-                asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pu[q]) : "f"(u[i + 1]), "f"(u[i]));
+                for (int q = 0; q < 4; ++q) {
+                  const int i = v * 8 + q * 2;
+                  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(y[i + 1]), "f"(y[i]));
+                }
+                dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
-              d0[v] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-              d1[v] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
             }
           }
         }
@@ -925,10 +942,11 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     }
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
-    // warp -> two code tiles (q = 2 dw, 2 dw + 1: row block dw of both
-    // accumulators), lane -> the tile's lane: contiguous code reads,
+    // warp -> one code tile q (gate/up: row block q >> 1 of matrix q & 1; down:
+    // row block q), lane -> the tile's lane: contiguous code reads,
     // conflict-free stores (dequant_q4_lane / dequant_q2_lane)
-    const int dw = wid - kPfDeqWarp0;  // 0..7 = row block
+    const int q = wid - kPfDeqWarp0;  // 0..7
+    const int brow0 = GATED ? (q & 1) * (C::NB_ROWS / 2) + (q >> 1) * 16 : q * 16;  // B row of its row 0
     const int g = lane >> 2, tig = lane & 3;
     uint32_t it = 0, ct = 0;
     bool ok = true;
@@ -943,17 +961,13 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           break;
         }
         const int half = ks % SPC;
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const uint32_t tsm = stage_c(cs) + (dw * 2 + m) * TILE;
-          if constexpr (FMT == 1) {
-            dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), bbuf(bb) + m * C::TILE_B,
-                            dw * 16 + g, g, tig);
-          } else {
-            const uint4 sc = lds_u4(tsm + 512 + g * 16);
-            dequant_q2_lane(lds_u2(tsm + lane * 16 + 8 * half), half ? sc.y : sc.x, half ? sc.w : sc.z,
-                            bbuf(bb) + m * C::TILE_B, dw * 16 + g, g, tig);
-          }
+        const uint32_t tsm = stage_c(cs) + q * TILE;
+        if constexpr (FMT == 1) {
+          dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), bbuf(bb), brow0 + g, g, tig);
+        } else {
+          const uint4 sc = lds_u4(tsm + 512 + g * 16);
+          dequant_q2_lane(lds_u2(tsm + lane * 16 + 8 * half), half ? sc.y : sc.x, half ? sc.w : sc.z, bbuf(bb),
+                          brow0 + g, g, tig);
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
         mbar_arrive(smem_addr(&s_bfull[bb]));
