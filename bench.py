@@ -108,12 +108,26 @@ def prefill_traffic(flops_per_call):
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, kind): the measured copy bandwidth and
+    cuBLAS bf16 rate in MEASURED_PEAKS.json when the file is present, else an
+    earlier measurement of the same part (kind "fallback")."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as fh:
             j = json.load(fh)
         return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+def peak_source(kind, what):
+    """What a roofline's peak is: `what` is "hbm" or "tensor"."""
+    if kind == "measured":
+        return ("measured hbm_gbs (MEASURED_PEAKS.json)" if what == "hbm" else
+                "measured bf16_tflops burst (MEASURED_PEAKS.json); fp16 dense rate = bf16 rate "
+                "(nominal ratio 1:1)")
+    return ("fallback 6650 GB/s (no MEASURED_PEAKS.json)" if what == "hbm" else
+            "fallback 1590 TFLOP/s bf16 burst (no MEASURED_PEAKS.json); fp16 dense rate = bf16 rate "
+            "(nominal ratio 1:1)")
 
 
 def host_info():
@@ -469,8 +483,7 @@ def measure(args, world, ctx, spec, n_rot, K, W):
             "frac": (gemm_tf / tflops) if gemm_tf else None,
             "launch_us": gemm_ms * 1e3,
             "traffic": None,
-            "peak_source": (f"{peak_kind} bf16_tflops (MEASURED_PEAKS.json); fp16 dense rate = bf16 "
-                            "rate (nominal ratio 1:1)"),
+            "peak_source": peak_source(peak_kind, "tensor"),
             "per_unit": f"6 d f = {6 * D * F} FLOP per (token, expert) row; "
                         f"{T * K_TOP + T} rows per call",
         } if prefill else {
@@ -485,8 +498,7 @@ def measure(args, world, ctx, spec, n_rot, K, W):
                 "launch_timing": "timed region / launches (one decode_kernel per step)"}
                if single else {}),
             "traffic": kernel_traffic(kern_bytes / K) if single else None,
-            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                           else "fallback 6650 GB/s",
+            "peak_source": peak_source(peak_kind, "hbm"),
             "per_unit": per_unit,
         },
         "e2e": {"value": whole_job_rate(world, tok, e2e_ms), "unit": "tokens/s",
@@ -612,7 +624,7 @@ def run_stack(args, world, K, W):
                                 "multi-launch layer path x 48"),
                      "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "traffic": None,
-                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                     "peak_source": peak_source(peak_kind, "hbm"),
                      "per_unit": f"{Be} B per touched expert per layer (shared included) + "
                                  f"{E * D * 4} B router W per layer"},
         "e2e": {"value": whole_job_rate(world, T * K, e2e_ms), "unit": "tokens/s",

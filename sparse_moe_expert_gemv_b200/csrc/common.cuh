@@ -174,24 +174,6 @@ MOE_DEV void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t ba
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
-// 16-byte asynchronous copy global -> shared through the load/store unit
-// (not the tensor memory accelerator), with an L2 cache policy.
-MOE_DEV void cp_async16_hint(uint32_t dst, const void *src, uint64_t policy) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "l"(policy)
-               : "memory");
-}
-// Arrive on an mbarrier once every cp.async this thread issued so far has
-// completed; the barrier's expected count includes this arrival (noinc).
-MOE_DEV void cp_async_mbar_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// Bulk prefetch of [src, src + bytes) into L2 (no shared memory, no
-// completion); src 16-byte aligned, bytes a multiple of 16.
-MOE_DEV void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // Policy for data read once: its L2 lines are the first to be evicted, so a
 // stream of them does not push other data (or code) out of L2.

@@ -216,9 +216,6 @@ struct DecodeParams {
   unsigned long long *stats;  // [0]=calls [1]=tokens [2]=hits [3]=misses [4]=near_ties
   int *last;
   int *status;
-  int prefetch;         // bit 0: L2-prefetch the warp's down units after routing;
-                        // bit 1: also its gate/up units beyond the ring's first ones
-  int ring_lsu;         // ring slots filled by per-lane cp.async instead of bulk copies
   unsigned long long bar1_extra;  // added to the first grid barrier's target (0; a test
                                   // sets it so that the bounded wait runs out)
   uint32_t bar1_polls;  // poll limit of the first grid barrier
@@ -677,10 +674,9 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
 
   MOE_TRACE(kTrRouteStart);
   WarpRing r;
-  ring_init(r, smem_addr(smem + L.ring) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT,
-            p.ring_lsu);
+  ring_init(r, smem_addr(smem + L.ring) + wid * kRingD * CG::SLOT, bars + wid * kRingD * 8, CG::SLOT);
   if (lane == 0) {
-    for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, p.ring_lsu ? 32 : 1);
+    for (int u = 0; u < kRingD; ++u) mbar_init(r.bar_s + 8 * u, 1);
     if (wid == 0) {
       mbar_init(h_bar, 1);
       mbar_init(st_bar, 1);
@@ -836,18 +832,6 @@ __global__ void __launch_bounds__(GemvCfg<FMT, true, NTM>::WARPS * 32, 1)
     if (lane == 0) fence_proxy_async_smem();  // a wide window occupied the rings until now
     __syncwarp();
     ring_prologue(r, ph1, lane);
-  }
-  // The whole weight stream of the warp is known now: put it in flight to
-  // L2, so HBM streams every selected expert at full rate while the rings
-  // consume (gate/up units beyond the ring's first ones; the down units,
-  // which then wait in L2 for the second pass).
-  if (lane == 0 && p.prefetch) {
-    if (p.prefetch & 2) prefetch_units_l2(ph1, min(u0 + kRingD, u1), u1);
-    if (p.prefetch & 1) {
-      const Phase pd = make_phase(s_jptr, d, f, CD::TK, CD::STRIDE, p.p1_bytes, CG::SLOT);
-      const SKCtx sd = sk_make(n_jobs * pd.RB * pd.UPI, W, gw, 0, nullptr, nullptr, nullptr, nullptr, WARPS);
-      prefetch_units_l2(pd, sk_start(sd, gw), sk_start(sd, gw + 1));
-    }
   }
   decode_pairs(p, s_slot, s_mask, s_idx, s_cnt, s_plist);
   // Token rows for the gate/up B operand.  A window that fits the staging

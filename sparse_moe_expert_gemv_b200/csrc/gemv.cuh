@@ -104,25 +104,6 @@ MOE_DEV const unsigned char *item_base(const Phase &ph, int job, int rb) {
          (long long)rb * ph.NTILE * ph.stride;
 }
 
-// L2 prefetch of the pass's units [u0, u1) (job-major, then row block, then
-// unit).  A job's units are one contiguous byte range of its expert's
-// region, so the range is one prefetch run per job it touches, cut into
-// pieces of at most kPrefetchPiece bytes.  Issued by the calling lane.
-constexpr uint32_t kPrefetchPiece = 32768;
-MOE_DEV void prefetch_units_l2(const Phase &ph, int u0, int u1) {
-  if (u1 <= u0) return;
-  const int upj = ph.RB * ph.UPI;                 // units per job
-  const long long ubytes = (long long)ph.tps * ph.stride;
-  for (int job = u0 / upj; job * upj < u1; ++job) {
-    const int a = max(u0, job * upj), b = min(u1, (job + 1) * upj);
-    const unsigned char *p = reinterpret_cast<const unsigned char *>(ph.job_ptr[job]) + ph.region_off +
-                             (long long)(a - job * upj) * ubytes;
-    long long n = (long long)(b - a) * ubytes;
-    for (; n > 0; n -= kPrefetchPiece, p += kPrefetchPiece)
-      bulk_prefetch_l2(p, (uint32_t)(n < kPrefetchPiece ? n : kPrefetchPiece));
-  }
-}
-
 // A walk over consecutive weight units: n units from unit `unit` of item
 // (job, rb); the next item is istep row blocks further.  Only increments and
 // compares: no division per unit or item.
@@ -163,13 +144,11 @@ struct WarpRing {
   uint32_t phase;    // its mbarrier parity
   int inflight;      // units issued and not yet consumed
   int istep;
-  int lsu;           // 1: every lane fills the slot with 16-byte cp.async (slot
-                     // barriers count 32 arrivals); 0: lane 0 issues one bulk copy
   UnitCursor ld;      // next unit to load into the ring
   uint64_t policy;   // L2 policy of the ring loads (evict first)
 };
 
-MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t slot_stride, int lsu = 0) {
+MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t slot_stride) {
   r.data_s = data_s;
   r.bar_s = bar_s;
   r.slot_stride = slot_stride;
@@ -177,7 +156,6 @@ MOE_DEV void ring_init(WarpRing &r, uint32_t data_s, uint32_t bar_s, uint32_t sl
   r.phase = 0;
   r.inflight = 0;
   r.istep = 1;
-  r.lsu = lsu;
   r.ld.rem = 0;
   r.policy = l2_evict_first();
 }
@@ -197,14 +175,8 @@ MOE_DEV void ring_start(WarpRing &r, const Phase &ph, int job, int rb, int unit,
 MOE_DEV void ring_issue_warp(WarpRing &r, const Phase &ph, int slot, int lane) {
   if (r.ld.rem <= 0) return;
   const uint32_t bytes = (uint32_t)(ph.tps * ph.stride);
-  if (r.lsu) {
-    const uint32_t dst = r.data_s + slot * r.slot_stride;
-    for (uint32_t c = 16u * lane; c < bytes; c += 512u) cp_async16_hint(dst + c, r.ld.addr + c, r.policy);
-    cp_async_mbar_arrive_noinc(r.bar_s + 8 * slot);
-  } else {
-    bulk_g2s_hint_pred(lane == 0, r.data_s + slot * r.slot_stride, r.ld.addr, bytes, r.bar_s + 8 * slot,
-                       r.policy);
-  }
+  bulk_g2s_hint_pred(lane == 0, r.data_s + slot * r.slot_stride, r.ld.addr, bytes, r.bar_s + 8 * slot,
+                     r.policy);
   ++r.inflight;
   cursor_advance(r.ld, ph, r.istep);
 }

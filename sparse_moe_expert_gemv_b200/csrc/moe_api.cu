@@ -79,17 +79,16 @@ struct moe_ctx {
   int pf_max_tiles = 0, pf_rows = 0;
   CUtensorMap pf_map_h{}, pf_map_a{};   // TMA maps of the grouped A matrices
   bool pf_maps = false;
+  int pf_pairs = 0;  // co-resident CTA pairs of the grouped GEMM (0: it cannot run)
   unsigned long long *trace = nullptr;  // moe_set_trace buffer
   unsigned long long *stats = nullptr;
   std::vector<int32_t> host_counts;
 
   int gemv_blocks[2][2][2] = {};  // [fmt][gated][NTM-1]
-  int dec_prefetch = 0;           // decode_kernel L2 prefetch mode (DecodeParams::prefetch)
   bool dec_fits = true;           // one decode_kernel CTA fits on every SM (checked at create)
   int dec_coop = -1;              // decode launches cooperative: -1 untried, 0 no, 1 yes
   int dec_stall_next = 0;         // test hook: the next decode launch's first barrier cannot complete
   uint32_t dec_stall_polls = 0;
-  int dec_ring_lsu = 0;           // decode_kernel ring fill (DecodeParams::ring_lsu)
   // profiling: 4 events per call slot
   bool profiling = false;
   std::vector<cudaEvent_t> prof_ev;
@@ -672,6 +671,27 @@ bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
   return encode_map_16b(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rows, cols, kPfBM);
 }
 
+// How many CTA pairs of the grouped GEMM fit on the device at once (the
+// persistent grid launches exactly that many, at most one CTA per SM).
+template <int FMT>
+cudaError_t prefill_pairs(int n_sm, int *pairs) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm / 2 * 2);
+  cfg.blockDim = dim3(kPfGemmThreads);
+  cfg.dynamicSmemBytes = PfCfg<FMT>::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, (const void *)prefill_gemm_kernel<FMT, true>, &cfg);
+  *pairs = e == cudaSuccess ? std::min(n, n_sm / 2) : 0;
+  return e;
+}
+
 cudaError_t setup_prefill() {
   cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        RtCfg::SMEM);
@@ -697,15 +717,19 @@ cudaError_t launch_prefill_gemms(moe_ctx *c, cudaStream_t s) {
   PfGemmParams g1{c->pf_tiles, c->pf_ntiles, d, f, d / TK, 0, c->pf_a16, nullptr, c->status};
   PfGemmParams g2{c->pf_tiles, c->pf_ntiles, f, d, f / TK, c->lay.p1_bytes, nullptr, c->pf_y16, c->status};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(c->n_sm);
+  cfg.gridDim = dim3(2 * c->pf_pairs);  // persistent CTA pairs, all co-resident
   cfg.blockDim = dim3(kPfGemmThreads);
   cfg.dynamicSmemBytes = PfCfg<FMT>::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, true>, c->pf_map_h, g1);
   if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, false>, c->pf_map_a, g2);
   return e;
@@ -746,17 +770,18 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
 }
 
 // Experts with at least this many tokens in a chunk run on the grouped GEMM
-// (128-row tiles); fewer tokens would leave most of a tile empty, and the
+// (256-row tiles); fewer tokens would leave most of a tile empty, and the
 // GEMV streams such an expert once per job of <= 16 tokens instead.
 constexpr int kHotMinTokens = 16;
 
 bool use_prefill_gemm(const moe_ctx *c, int N) {
-  return c->pf && N > kDecMaxT && c->d % (2 * kPfBN) == 0 && c->f % kPfBN == 0 && c->E <= kPfMaxE;
+  return c->pf && c->pf_pairs > 0 && N > kDecMaxT && c->d % (2 * kPfBN) == 0 && c->f % kPfBN == 0 &&
+         c->E <= kPfMaxE;
 }
 
 // The prefill chunk's routing on router input h: logits, top-k + softmax
 // (idx, w), the sort of the chunk's pairs by expert (each expert's rows in
-// ascending t), the 128-row tile list with the residency lookup, and the
+// ascending t), the 256-row tile list with the residency lookup, and the
 // gather of the grouped fp16 A rows.  perm (or null) receives the bucket
 // permutation; the bucket offsets are left in c->pf_eoff.
 moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int32_t *idx, float *w,
@@ -828,7 +853,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   moe_status st = prefill_route_impl(c, layer, h, N, c->idx, c->w, c->pf_perm, s, kHotMinTokens);
   if (st) return st;
   CUDA_TRY(c, prof_mark(c, 1, s));
-  // experts with many tokens: grouped GEMM over 128-row tiles; the others:
+  // experts with many tokens: grouped GEMM over 256-row tiles; the others:
   // the GEMV over jobs of <= 16 tokens, rows read through the bucket
   // permutation (grouped row -> pair id)
   GemvParams g1{};
@@ -914,8 +939,6 @@ moe_status forward_impl(moe_ctx *c, int layer, uint16_t *x, int T, float *delta,
     dp.last = c->last;
     dp.status = c->status;
     dp.sm = decode_layout(c, T);
-    dp.prefetch = c->dec_prefetch;
-    dp.ring_lsu = c->dec_ring_lsu;
     dp.bar1_extra = c->dec_stall_next ? (unsigned long long)c->n_sm : 0ull;
     dp.bar1_polls = c->dec_stall_next ? c->dec_stall_polls : (1u << 22);
     c->dec_stall_next = 0;
@@ -1075,8 +1098,6 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
   c->k = k;
   c->fmt = fmt;
   c->lay = make_layout(fmt, d, f);
-  if (const char *pf = getenv("MOE_DECODE_PREFETCH")) c->dec_prefetch = atoi(pf);  // TEMP A/B knob
-  if (const char *pf = getenv("MOE_DECODE_LSU")) c->dec_ring_lsu = atoi(pf);        // TEMP A/B knob
   cudaError_t e = cudaDeviceGetAttribute(&c->n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->io, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = setup_route_fused();
@@ -1100,6 +1121,8 @@ moe_status moe_create(int d, int f, int E, int k, int fmt, moe_ctx **out) {
                                                       GemvCfg<1, true, 1>::WARPS * 32, kDecSmem);
     c->dec_fits = e == cudaSuccess && per_sm >= 1;
   }
+  if (e == cudaSuccess)
+    e = fmt == MOE_Q4_SYM_G32_F16 ? prefill_pairs<1>(c->n_sm, &c->pf_pairs) : prefill_pairs<2>(c->n_sm, &c->pf_pairs);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     moe_destroy(c);

@@ -12,15 +12,16 @@
 //                           relative to the expert's (a scan down the
 //                           expert's column of block masks) and its tokens
 //   prefill_scan_kernel     the experts' first rows in grouped order and the
-//                           list of 128-row tiles (expert, first row, rows)
+//                           list of 256-row tiles (expert, first row, rows)
 //   prefill_scatter_kernel  pair -> row in grouped order (stable: ascending t
 //                           within an expert) and the gather of every pair's
 //                           token row into the grouped A matrix (fp16)
-//   prefill_gemm_kernel     A tile (TMA, 128B swizzle) x dequantised weight
-//                           tile (written by the CTA's warps straight into
-//                           the swizzled fp16 layout) -> tcgen05.mma, fp32
-//                           accumulators in TMEM; gate/up pass writes
-//                           SiLU(G) * U (fp16), down pass writes y (fp32)
+//   prefill_gemm_kernel     on CTA pairs: A tiles (TMA, 128B swizzle) x
+//                           dequantised weight tiles (written by each CTA's
+//                           warps straight into the swizzled fp16 layout) ->
+//                           tcgen05.mma.cta_group::2 m256n256k16, fp32
+//                           accumulators in both CTAs' TMEM; gate/up pass writes
+//                           SiLU(G) * U (fp16), down pass writes y (fp16)
 //   prefill_combine_kernel  x += sum_j w_j y[row(t, j)] + y_shared[t]
 //
 // Operands are fp16: a Q4 weight s*(c-8) with its fp16 scale is one
@@ -44,7 +45,7 @@ constexpr int kPfMaxE = 1024;
 
 struct PfTile {                  // one tile of up to 256 rows of one expert
   const uint8_t *w;              // expert base (repacked layout)
-  int row0, rows;                // first row in grouped order, rows <= 128
+  int row0, rows;                // first row in grouped order, rows <= 256
 };
 
 // logits[t, e] = sum_z part[z][t, e] (z = 0, 1, ... in order) + bias[e]: the
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(kPfColWarps * 32) prefill_colscan_kernel(PfSca
 // One CTA of 1024 threads: block scans over the experts' token counts give
 // their first rows, their first GEMM tiles and their first GEMV jobs; then
 // the tile and job lists, with the residency lookup.  An expert with at
-// least hot_min tokens is a GEMM expert (128-row tiles); one with fewer is
+// least hot_min tokens is a GEMM expert (256-row tiles); one with fewer is
 // cut into GEMV jobs of at most `chunk` tokens, which stream its weights
 // once per job instead of dequantising a mostly empty tile.
 __global__ void __launch_bounds__(1024) prefill_scan_kernel(PfScanParams p) {
@@ -666,6 +667,76 @@ MOE_DEV void dequant_q2_lane(uint2 w, uint32_t s, uint32_t mn, uint32_t dst_s, i
                "r"(s1.x), "r"(s1.y), "r"(s1.z), "r"(s1.w) : "memory");
 }
 
+// ------------------------------------------------------- CTA-pair helpers
+// The grouped GEMM runs on clusters of two CTAs (a CTA pair on two SMs) that
+// issue one tcgen05.mma.cta_group::2 per 16-column step: the pair's MMA is
+// m256n256k16, each CTA holding 128 of the A rows and 128 of the B rows in
+// its own shared memory (at the same offsets) and 128 accumulator rows in its
+// own TMEM.  Per SM that halves the shared-memory bytes per FLOP of the
+// one-CTA m128n128 form.
+MOE_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+MOE_DEV uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+MOE_DEV uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the variable at shared::cta address `a` in the
+// cluster's CTA `rank`
+MOE_DEV uint32_t mapa_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+// All threads of both CTAs; orders everything before it (release) against
+// everything after it (acquire) across the pair.
+MOE_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// One arrival on an mbarrier of either CTA of the pair (shared::cluster
+// address), with the instruction's default release semantics.  Waits on the
+// pair's barriers use the ordinary try_wait: the tensor-core and TMA
+// pipelines of the pair synchronise this way, and the release/acquire forms
+// at cluster scope made every step of this kernel a third slower.
+MOE_DEV void mbar_arrive_remote(uint32_t bar_cl) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cl) : "memory");
+}
+// 2-D TMA tile load into this CTA's shared memory whose completion is
+// counted on an mbarrier of either CTA of the pair (bar_cl: shared::cluster
+// address).  No multicast: the tile lands in this CTA only.
+MOE_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar_cl) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cl)
+      : "memory");
+}
+// The pair's MMA, issued by one thread of the even CTA: D (both CTAs' TMEM at
+// tmem_d) (+)= A (both CTAs' shared memory at da) x B (both at db)^T.
+MOE_DEV void umma_f16_pair(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+// One arrival on the mbarrier at shared::cta offset `bar` in both CTAs of the
+// pair once every tcgen05 operation this thread issued has completed.
+MOE_DEV void umma_commit_pair(uint32_t bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(both)
+      : "memory");
+}
+
 struct PfGemmParams {
   const PfTile *tiles;
   const int *n_tiles;
@@ -682,105 +753,122 @@ constexpr int kPfGemmThreads = 512;  // 16 warps
 constexpr int kPfDeqWarp0 = 8;       // warps 8..15 dequantise
 constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM lane quarters 0..3)
 
-// A work item is one tile of up to 256 rows of one expert (two M-halves of
-// 128 rows) times one output slice: 64 features of the gate/up pass (gate
-// and up side by side: 128 weight rows) or 128 features of the down pass
-// (128 weight rows).  Each k-step dequantises the slice's 128 weight rows
-// once and feeds them to both halves' MMAs (m128n128k16 each), so the
-// dequantisation -- the pipeline's costliest stage -- is shared by 256 token
-// rows.  The A tiles (64 reduction columns of both halves' rows) and the
-// code tiles travel in two rings: an A stage is released when its MMAs
-// complete, a code stage when the dequantising warps have read it.  A code
-// stage holds the 8 repacked tiles of one tile column: 64 reduction columns
-// for Q4 (one k-step), 128 for Q2 (two k-steps, one quantisation group
-// each).
+// A work item is one tile of up to 256 rows of one expert times one output
+// slice: 128 features of the gate/up pass or 256 features of the down pass.
+// Each CTA dequantises 128 weight rows of the slice -- gate/up: the gate and
+// up rows of 64 features (the even CTA features [0, 64) of the slice, the odd
+// CTA [64, 128)); down: 128 output features -- and holds 128 of the tile's
+// rows: the even CTA rows [0, 128), the odd CTA rows [128, 256).  The pair's
+// accumulator columns are then [gate | up] of the even CTA's 64 features and
+// [gate | up] of the odd CTA's (gate/up), or the slice's 256 features in
+// order (down).  Per 64-column reduction step each CTA loads its A tile (16
+// KB) and dequantises its 128 weight rows (16 KB of fp16) once for all 256
+// token rows.  The A tiles and the code tiles travel in two rings: an A stage
+// is released when the pair's MMAs complete, a code stage when the CTA's
+// dequantising warps have read it.  A code stage holds CT consecutive
+// repacked tiles of each of the CTA's row blocks (4 k-steps): the tiles of a
+// row block along the reduction are contiguous in memory (gate/up: gate and
+// up tile of each column side by side), so one bulk copy per row block fills
+// it -- issuing a copy costs the producer about 100 cycles, and one copy per
+// tile (8 per k-step) was the pipeline's bottleneck.
 template <int FMT>
 struct PfCfg {
   static constexpr int TILE = FMT == 1 ? 576 : 640;         // repacked code tile (+ scales)
-  static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per code stage
-  static constexpr int SA = 5;                              // A ring
-  static constexpr int SC = 4;                              // code ring
-  static constexpr int NBB = 2;                             // B buffers (dequantised weights)
-  static constexpr int NB_ROWS = 128;                       // weight rows per item (MMA N)
-  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB per M-half
-  static constexpr uint32_t STAGE_A = 2 * TILE_A;           // both halves
+  static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per tile (64 / 128 columns)
+  static constexpr int CT = FMT == 1 ? 4 : 2;               // tiles per row block per code stage
+  static constexpr int KSC = CT * SPC;                      // k-steps per code stage (4)
+  static constexpr int SA = FMT == 1 ? 7 : 8;               // A ring
+  static constexpr int SC = FMT == 1 ? 2 : 3;               // code ring
+  static constexpr int NBB = 3;                             // B buffers (dequantised weights)
+  static constexpr int NB_ROWS = 128;                       // weight rows per CTA per item
+  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB: this CTA's 128 rows
   static constexpr uint32_t BBUF = NB_ROWS * kPfBK * 2;     // 16 KB
-  static constexpr uint32_t CODES = (8 * TILE + 1023) / 1024 * 1024;  // 8 repacked code tiles
-  static constexpr uint32_t SMEM = SA * STAGE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
-  static constexpr uint32_t ACC_COLS = 2 * NB_ROWS;         // TMEM columns per buffer (both halves)
+  static constexpr uint32_t CODES = (8 * CT * TILE + 1023) / 1024 * 1024;  // 8 row blocks x CT tiles
+  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t ACC_COLS = 2 * NB_ROWS;         // TMEM columns per buffer (MMA N = 256)
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
 
-// Grouped GEMM over the tile list, warp-specialised; persistent CTAs walk
-// the items blockIdx.x, +gridDim.x.
-//  warp 0 lane 0   producer: per 64-column reduction step the A tiles of
-//                  both M-halves (2-D TMA, 128-byte swizzle; the second half
-//                  only when the tile has more than 128 rows) into a free
-//                  stage of the A ring, and at each new tile column the 8
-//                  repacked code tiles (1-D bulk copies) into the code ring
+// Grouped GEMM over the tile list, warp-specialised, on CTA pairs; the
+// persistent pairs walk the items clusterid.x, +nclusterid.x.  Both CTAs:
+//  warp 0 lane 0   producer: per 64-column reduction step this CTA's A tile
+//                  (2-D TMA, 128-byte swizzle; the odd CTA only when the tile
+//                  has more than 128 rows) into a free stage of the A ring,
+//                  counted on the even CTA's stage barrier, and every KSC
+//                  steps the next code stage (one 1-D bulk copy per row
+//                  block) into the code ring
 //  warps 8..15     one code tile each: dequantise a k-step's codes into one
-//                  of two swizzled fp16 B buffers, arrive on the buffer's
-//                  barrier, and release the code stage after its last k-step
-//  warp 1 lane 0   issues the MMAs (per 16-column substep one m128n128k16
-//                  per M-half, operands in shared memory, fp32 in TMEM) and
-//                  commits the release of the A stage and of the B buffer;
-//                  accumulators alternate between two TMEM buffers
-//  warps 4..7      drain an accumulator buffer (TMEM lanes = rows of each
-//                  half) while the next item accumulates into the other one
-// Every wait is bounded; a timeout raises kErrTimeout and every role stops.
+//                  of three swizzled fp16 B buffers, arrive on the even CTA's
+//                  buffer barrier, release the code stage after its last k-step
+//  warps 4..7      drain an accumulator buffer (TMEM lanes = the CTA's rows)
+//                  while the next item accumulates into the other one, then
+//                  arrive on the even CTA's buffer-empty barrier
+// Even CTA only:
+//  warp 1 lane 0   issues the pair's MMAs (m256n256k16 per 16-column step,
+//                  fp32 in TMEM) and commits the release of the A stage, the
+//                  B buffer and the accumulator to the barriers of both CTAs
+// Every wait is bounded; a timeout raises kErrTimeout and stops both CTAs.
 template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
   using C = PfCfg<FMT>;
-  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, TILE = C::TILE, NBB = C::NBB;
-  constexpr int COLS = GATED ? C::NB_ROWS / 2 : C::NB_ROWS;  // output features per item
+  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, CT = C::CT, KSC = C::KSC, TILE = C::TILE,
+                NBB = C::NBB;
+  constexpr int COLS = GATED ? C::NB_ROWS : 2 * C::NB_ROWS;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
   __shared__ __align__(8) unsigned long long s_afull[SA], s_aempty[SA], s_cfull[SC], s_cempty[SC],
       s_bfull[NBB], s_bempty[NBB], s_accf[2], s_acce[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the even CTA (issues the MMAs)
   const uint32_t base = smem_addr(pf_smem), stage0 = base + ((1024 - (base & 1023)) & 1023);
   if (tid == 0) {
     for (int i = 0; i < SA; ++i) {
-      mbar_init(smem_addr(&s_afull[i]), 1);
-      mbar_init(smem_addr(&s_aempty[i]), 1);
+      mbar_init(smem_addr(&s_afull[i]), 1);   // the even CTA's expect_tx; both CTAs' bytes
+      mbar_init(smem_addr(&s_aempty[i]), 1);  // the pair's MMA commit
     }
     for (int i = 0; i < SC; ++i) {
       mbar_init(smem_addr(&s_cfull[i]), 1);
       mbar_init(smem_addr(&s_cempty[i]), 8);  // one arrival per dequantising warp
     }
     for (int b = 0; b < NBB; ++b) {
-      mbar_init(smem_addr(&s_bfull[b]), 256);
+      mbar_init(smem_addr(&s_bfull[b]), 16);  // 8 dequantising warps of each CTA
       mbar_init(smem_addr(&s_bempty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_addr(&s_accf[b]), 1);
-      mbar_init(smem_addr(&s_acce[b]), 128);
+      mbar_init(smem_addr(&s_acce[b]), 8);  // 4 epilogue warps of each CTA
     }
     s_abort = 0;
     fence_mbar_init();
   }
   if (wid == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(&s_tmem)),
                  "r"(C::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either signals the other's
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   pdl_wait();
   const int ntiles = ldcg_i32(p.n_tiles);
   const int nslices = p.N / COLS, nsteps = p.K / kPfBK;
   const int items = ntiles * nslices;
-  auto stage_a = [&](uint32_t st) { return stage0 + st * C::STAGE_A; };
-  auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::STAGE_A + cs * C::CODES; };
-  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::STAGE_A + SC * C::CODES + b * C::BBUF; };
+  const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
+  auto stage_a = [&](uint32_t st) { return stage0 + st * C::TILE_A; };
+  auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::TILE_A + cs * C::CODES; };
+  auto bbuf = [&](uint32_t b) { return stage0 + SA * C::TILE_A + SC * C::CODES + b * C::BBUF; };
+  auto lead = [&](const void *v) { return mapa_shared(smem_addr(v), 0); };  // the even CTA's copy
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
-  auto give_up = [&]() {
+  auto give_up = [&]() {  // stop both CTAs' roles
     *reinterpret_cast<volatile int *>(&s_abort) = 1;
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(smem_addr(&s_abort), rank ^ 1u)),
+                 "r"(1)
+                 : "memory");
     atomicOr(p.status, kErrTimeout);
   };
 
@@ -789,30 +877,34 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, ct = 0;  // k-steps and code stages issued
       bool ok = true;
-      for (int item = blockIdx.x; item < items && ok && !aborted(); item += gridDim.x) {
+      for (int item = pair; item < items && ok && !aborted(); item += npairs) {
         const PfTile tile = p.tiles[item / nslices];
-        const bool two = tile.rows > kPfBM;  // the second M-half has rows
-        const int rb0 = (item % nslices) * (GATED ? COLS / 16 : COLS / 16);
+        const bool two = tile.rows > kPfBM;     // the odd CTA's rows exist
+        const bool mine = rank == 0 || two;     // this CTA loads A rows
+        const int slice = item % nslices;
         const uint8_t *wbase = tile.w + p.region_off;
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
-          if (ks % SPC == 0) {  // the next tile column's codes
-            const uint32_t cs = ct % SC, cuse = ct / SC, tk = ks / SPC;
+          if (ks % KSC == 0) {  // the next code stage: tiles tk0 .. tk0 + nt - 1
+            const uint32_t cs = ct % SC, cuse = ct / SC;
+            const int tk0 = ks / SPC, nt = min(CT, p.ntile_k - tk0);
             if (cuse > 0 && !mbar_wait_bounded(smem_addr(&s_cempty[cs]), (cuse - 1) & 1)) {
               ok = false;
               break;
             }
             const uint32_t cbar = smem_addr(&s_cfull[cs]);
-            mbar_expect_tx(cbar, 8 * TILE);
+            mbar_expect_tx(cbar, 8 * nt * TILE);
             if constexpr (GATED) {
-              // code tile q = 2 r + m: row block r of matrix m (gate, up);
-              // the two tiles of a row block are adjacent in memory
+              // row block r of the CTA's 64 features: its gate and up tiles
+              // of columns tk0 .. are one contiguous run
               for (int r = 0; r < 4; ++r)
-                bulk_g2s(stage_c(cs) + r * 2 * TILE,
-                         wbase + ((long long)(rb0 + r) * p.ntile_k + tk) * 2 * TILE, 2 * TILE, cbar);
+                bulk_g2s(stage_c(cs) + r * 2 * CT * TILE,
+                         wbase + ((long long)(slice * 8 + (int)rank * 4 + r) * p.ntile_k + tk0) * 2 * TILE,
+                         2 * nt * TILE, cbar);
             } else {
-              for (int q = 0; q < 8; ++q)  // code tile q = row block q
-                bulk_g2s(stage_c(cs) + q * TILE, wbase + ((long long)(rb0 + q) * p.ntile_k + tk) * TILE,
-                         TILE, cbar);
+              for (int q = 0; q < 8; ++q)  // row block q of the CTA's half of the slice
+                bulk_g2s(stage_c(cs) + q * CT * TILE,
+                         wbase + ((long long)(slice * 16 + (int)rank * 8 + q) * p.ntile_k + tk0) * TILE,
+                         nt * TILE, cbar);
             }
             ++ct;
           }
@@ -821,27 +913,27 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t bar = smem_addr(&s_afull[st]);
-          mbar_expect_tx(bar, two ? 2 * C::TILE_A : C::TILE_A);
-          tma_load_2d(stage_a(st), &amap, ks * kPfBK, tile.row0, bar);
-          if (two) tma_load_2d(stage_a(st) + C::TILE_A, &amap, ks * kPfBK, tile.row0 + kPfBM, bar);
+          if (rank == 0) mbar_expect_tx(smem_addr(&s_afull[st]), two ? 2 * C::TILE_A : C::TILE_A);
+          if (mine)
+            tma_load_2d_pair(stage_a(st), &amap, ks * kPfBK, tile.row0 + (int)rank * kPfBM, lead(&s_afull[st]));
         }
       }
       if (!ok) give_up();
-      // no copy may land in shared memory after the CTA has moved on (a give-up
-      // leaves stages in flight); consumed stages pass at once
-      for (uint32_t j = it > SA ? it - SA : 0; j < it; ++j)
-        (void)mbar_wait_bounded(smem_addr(&s_afull[j % SA]), (j / SA) & 1);
+      // no copy may land in shared memory after the pair has moved on (a
+      // give-up leaves stages in flight): the even CTA's stage barriers count
+      // both CTAs' A bytes; consumed stages pass at once
+      if (rank == 0)
+        for (uint32_t j = it > SA ? it - SA : 0; j < it; ++j)
+          (void)mbar_wait_bounded(smem_addr(&s_afull[j % SA]), (j / SA) & 1);
       for (uint32_t j = ct > SC ? ct - SC : 0; j < ct; ++j)
         (void)mbar_wait_bounded(smem_addr(&s_cfull[j % SC]), (j / SC) & 1);
     }
   } else if (wid == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = umma_idesc_f16(kPfBM, C::NB_ROWS);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = umma_idesc_f16(2 * kPfBM, C::ACC_COLS);
       uint32_t it = 0, ii = 0;
-      for (int item = blockIdx.x; item < items && !aborted(); item += gridDim.x, ++ii) {
-        const bool two = p.tiles[item / nslices].rows > kPfBM;
+      for (int item = pair; item < items && !aborted(); item += npairs, ++ii) {
         const uint32_t buf = ii & 1, acc = tmem + buf * C::ACC_COLS;
         if (ii >= 2 && !mbar_wait_bounded(smem_addr(&s_acce[buf]), ((ii >> 1) - 1) & 1)) {
           give_up();
@@ -858,30 +950,26 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kPfBK / 16; ++kk) {
-            const uint64_t db = umma_desc_sw128(bbuf(bb) + kk * 32);
-            umma_f16(acc, umma_desc_sw128(stage_a(st) + kk * 32), db, IDESC, (ks | kk) != 0);
-            if (two)
-              umma_f16(acc + C::NB_ROWS, umma_desc_sw128(stage_a(st) + C::TILE_A + kk * 32), db, IDESC,
-                       (ks | kk) != 0);
-          }
-          umma_commit(smem_addr(&s_aempty[st]));
-          umma_commit(smem_addr(&s_bempty[bb]));
+          for (int kk = 0; kk < kPfBK / 16; ++kk)
+            umma_f16_pair(acc, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(bbuf(bb) + kk * 32),
+                          IDESC, (ks | kk) != 0);
+          umma_commit_pair(smem_addr(&s_aempty[st]));
+          umma_commit_pair(smem_addr(&s_bempty[bb]));
         }
         if (!ok) {
           give_up();
           break;
         }
-        umma_commit(smem_addr(&s_accf[buf]));
+        umma_commit_pair(smem_addr(&s_accf[buf]));
       }
-      // every committed MMA must be complete before TMEM is released
+      // every committed MMA must be complete before either CTA releases TMEM
       if (it > 0) (void)mbar_wait_bounded(smem_addr(&s_aempty[(it - 1) % SA]), ((it - 1) / SA) & 1);
     }
   } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = wid & 3, lr = quarter * 32 + lane;  // TMEM lane = row of each half
+    const int quarter = wid & 3;  // TMEM lanes [32 quarter, +32) = the warp's rows of this CTA
     uint32_t ii = 0;
-    for (int item = blockIdx.x; item < items; item += gridDim.x, ++ii) {
+    for (int item = pair; item < items; item += npairs, ++ii) {
       const uint32_t buf = ii & 1;
       const bool ok = mbar_wait_bounded(smem_addr(&s_accf[buf]), (ii >> 1) & 1);
       if (__any_sync(0xffffffffu, !ok) || aborted()) {
@@ -891,18 +979,20 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       tc_fence_after();
       const PfTile tile = p.tiles[item / nslices];
       const int n0 = (item % nslices) * COLS;
-      for (int half = 0; half < (tile.rows > kPfBM ? 2 : 1); ++half) {
-        const int r = half * kPfBM + lr;
-        const uint32_t lane_addr =
-            tmem + buf * C::ACC_COLS + half * C::NB_ROWS + ((uint32_t)(quarter * 32) << 16);
+      const int r0 = (int)rank * kPfBM + quarter * 32;  // the warp's first row in the tile
+      const int r = r0 + lane;
+      const uint32_t lane_addr = tmem + buf * C::ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+      if (r0 < tile.rows) {  // warp-uniform: the warp has rows in this tile
         if constexpr (GATED) {
-          // accumulator columns [0, 64) = gate, [64, 128) = up of features n0 ..
-          for (int c0 = 0; c0 < COLS; c0 += 32) {
+          // accumulator columns [128 h, 128 h + 64) = gate, [128 h + 64,
+          // 128 h + 128) = up of features n0 + 64 h ..
+          for (int c = 0; c < COLS; c += 32) {
+            const int h = c >> 6, c0 = c & 63;
             float g[32], u[32];
-            tmem_ld32(lane_addr + c0, g);
-            tmem_ld32(lane_addr + COLS + c0, u);
+            tmem_ld32(lane_addr + h * 128 + c0, g);
+            tmem_ld32(lane_addr + h * 128 + 64 + c0, u);
             if (r < tile.rows) {
-              uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c0);
+              uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c);
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 uint32_t pk[4];
@@ -938,19 +1028,24 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_addr(&s_acce[buf]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(&s_acce[buf]));
     }
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
-    // warp -> one code tile q (gate/up: row block q >> 1 of matrix q & 1; down:
-    // row block q), lane -> the tile's lane: contiguous code reads,
+    // warp -> one row block of the CTA's 128 weight rows (gate/up: row
+    // block q >> 1 of matrix q & 1, i.e. B rows (q & 1) 64 + (q >> 1) 16 ..;
+    // down: row block q), lane -> the tile's lane: contiguous code reads,
     // conflict-free stores (dequant_q4_lane / dequant_q2_lane)
     const int q = wid - kPfDeqWarp0;  // 0..7
-    const int brow0 = GATED ? (q & 1) * (C::NB_ROWS / 2) + (q >> 1) * 16 : q * 16;  // B row of its row 0
+    const int brow0 = GATED ? (q & 1) * 64 + (q >> 1) * 16 : q * 16;  // B row of its row 0
+    // its tiles in a code stage: tile j at tbase + j * tstep
+    const uint32_t tbase = GATED ? (uint32_t)(((q >> 1) * 2 * CT + (q & 1)) * TILE) : (uint32_t)(q * CT * TILE);
+    constexpr uint32_t tstep = GATED ? 2 * TILE : TILE;
     const int g = lane >> 2, tig = lane & 3;
     uint32_t it = 0, ct = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    for (int item = pair; item < items && ok; item += npairs) {
       for (int ks = 0; ks < nsteps; ++ks, ++it) {
         const uint32_t cs = ct % SC, cuse = ct / SC, bb = it % NBB, buse = it / NBB;
         bool got = mbar_wait_bounded(smem_addr(&s_cfull[cs]), cuse & 1);
@@ -960,8 +1055,8 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           ok = false;
           break;
         }
-        const int half = ks % SPC;
-        const uint32_t tsm = stage_c(cs) + q * TILE;
+        const int half = ks % SPC, j = (ks % KSC) / SPC;
+        const uint32_t tsm = stage_c(cs) + tbase + j * tstep;
         if constexpr (FMT == 1) {
           dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), bbuf(bb), brow0 + g, g, tig);
         } else {
@@ -970,9 +1065,9 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
                           brow0 + g, g, tig);
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
-        mbar_arrive(smem_addr(&s_bfull[bb]));
-        if (half == SPC - 1) {  // the code stage's last k-step: release it
-          __syncwarp();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead(&s_bfull[bb]));
+        if (ks % KSC == KSC - 1 || ks == nsteps - 1) {  // the code stage's last k-step: release it
           if (lane == 0) mbar_arrive(smem_addr(&s_cempty[cs]));
           ++ct;
         }
@@ -981,9 +1076,10 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the pair's MMAs, remote arrivals and copies are done
   tc_fence_after();
   if (wid == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
   pdl_launch_dependents();
 }
 
