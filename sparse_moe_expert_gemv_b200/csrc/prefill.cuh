@@ -777,9 +777,9 @@ struct PfCfg {
   static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per tile (64 / 128 columns)
   static constexpr int CT = FMT == 1 ? 4 : 2;               // tiles per row block per code stage
   static constexpr int KSC = CT * SPC;                      // k-steps per code stage (4)
-  static constexpr int SA = FMT == 1 ? 7 : 8;               // A ring
+  static constexpr int SA = 7;                              // A ring
   static constexpr int SC = FMT == 1 ? 2 : 3;               // code ring
-  static constexpr int NBB = 3;                             // B buffers (dequantised weights)
+  static constexpr int NBB = 4;                             // B buffers (dequantised weights)
   static constexpr int NB_ROWS = 128;                       // weight rows per CTA per item
   static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB: this CTA's 128 rows
   static constexpr uint32_t BBUF = NB_ROWS * kPfBK * 2;     // 16 KB
@@ -791,15 +791,16 @@ struct PfCfg {
 
 // Grouped GEMM over the tile list, warp-specialised, on CTA pairs; the
 // persistent pairs walk the items clusterid.x, +nclusterid.x.  Both CTAs:
-//  warp 0 lane 0   producer: per 64-column reduction step this CTA's A tile
-//                  (2-D TMA, 128-byte swizzle; the odd CTA only when the tile
-//                  has more than 128 rows) into a free stage of the A ring,
-//                  counted on the even CTA's stage barrier, and every KSC
-//                  steps the next code stage (one 1-D bulk copy per row
-//                  block) into the code ring
-//  warps 8..15     one code tile each: dequantise a k-step's codes into one
-//                  of three swizzled fp16 B buffers, arrive on the even CTA's
-//                  buffer barrier, release the code stage after its last k-step
+//  warp 0 lane 0   A producer: per 64-column reduction step this CTA's A
+//                  tile (2-D TMA, 128-byte swizzle; the odd CTA only when the
+//                  tile has more than 128 rows) into a free stage of the A
+//                  ring, counted on the even CTA's stage barrier
+//  warp 2 lane 0   code producer: every KSC steps the next code stage (one
+//                  1-D bulk copy per row block) into the code ring; apart
+//                  from the A producer so that neither ring waits on the other
+//  warps 8..15     one row block each: dequantise two k-steps' codes into two
+//                  of four swizzled fp16 B buffers, arrive on the even CTA's
+//                  buffer barriers, release the code stage after its last k-step
 //  warps 4..7      drain an accumulator buffer (TMEM lanes = the CTA's rows)
 //                  while the next item accumulates into the other one, then
 //                  arrive on the even CTA's buffer-empty barrier
@@ -873,41 +874,15 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   };
 
   if (wid == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ A producer
     if (lane == 0) {
-      uint32_t it = 0, ct = 0;  // k-steps and code stages issued
+      uint32_t it = 0;  // k-steps issued
       bool ok = true;
       for (int item = pair; item < items && ok && !aborted(); item += npairs) {
         const PfTile tile = p.tiles[item / nslices];
-        const bool two = tile.rows > kPfBM;     // the odd CTA's rows exist
-        const bool mine = rank == 0 || two;     // this CTA loads A rows
-        const int slice = item % nslices;
-        const uint8_t *wbase = tile.w + p.region_off;
+        const bool two = tile.rows > kPfBM;  // the odd CTA's rows exist
+        const bool mine = rank == 0 || two;  // this CTA loads A rows
         for (int ks = 0; ks < nsteps; ++ks, ++it) {
-          if (ks % KSC == 0) {  // the next code stage: tiles tk0 .. tk0 + nt - 1
-            const uint32_t cs = ct % SC, cuse = ct / SC;
-            const int tk0 = ks / SPC, nt = min(CT, p.ntile_k - tk0);
-            if (cuse > 0 && !mbar_wait_bounded(smem_addr(&s_cempty[cs]), (cuse - 1) & 1)) {
-              ok = false;
-              break;
-            }
-            const uint32_t cbar = smem_addr(&s_cfull[cs]);
-            mbar_expect_tx(cbar, 8 * nt * TILE);
-            if constexpr (GATED) {
-              // row block r of the CTA's 64 features: its gate and up tiles
-              // of columns tk0 .. are one contiguous run
-              for (int r = 0; r < 4; ++r)
-                bulk_g2s(stage_c(cs) + r * 2 * CT * TILE,
-                         wbase + ((long long)(slice * 8 + (int)rank * 4 + r) * p.ntile_k + tk0) * 2 * TILE,
-                         2 * nt * TILE, cbar);
-            } else {
-              for (int q = 0; q < 8; ++q)  // row block q of the CTA's half of the slice
-                bulk_g2s(stage_c(cs) + q * CT * TILE,
-                         wbase + ((long long)(slice * 16 + (int)rank * 8 + q) * p.ntile_k + tk0) * TILE,
-                         nt * TILE, cbar);
-            }
-            ++ct;
-          }
           const uint32_t st = it % SA, use = it / SA;
           if (use > 0 && !mbar_wait_bounded(smem_addr(&s_aempty[st]), (use - 1) & 1)) {
             ok = false;
@@ -925,6 +900,42 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       if (rank == 0)
         for (uint32_t j = it > SA ? it - SA : 0; j < it; ++j)
           (void)mbar_wait_bounded(smem_addr(&s_afull[j % SA]), (j / SA) & 1);
+    }
+  } else if (wid == 2) {
+    // ------------------------------------------------------------ code producer
+    if (lane == 0) {
+      uint32_t ct = 0;  // code stages issued
+      bool ok = true;
+      for (int item = pair; item < items && ok && !aborted(); item += npairs) {
+        const PfTile tile = p.tiles[item / nslices];
+        const int slice = item % nslices;
+        const uint8_t *wbase = tile.w + p.region_off;
+        for (int ks = 0; ks < nsteps; ks += KSC) {  // code stage: tiles tk0 .. tk0 + nt - 1
+          const uint32_t cs = ct % SC, cuse = ct / SC;
+          const int tk0 = ks / SPC, nt = min(CT, p.ntile_k - tk0);
+          if (cuse > 0 && !mbar_wait_bounded(smem_addr(&s_cempty[cs]), (cuse - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t cbar = smem_addr(&s_cfull[cs]);
+          mbar_expect_tx(cbar, 8 * nt * TILE);
+          if constexpr (GATED) {
+            // row block r of the CTA's 64 features: its gate and up tiles of
+            // columns tk0 .. are one contiguous run
+            for (int r = 0; r < 4; ++r)
+              bulk_g2s(stage_c(cs) + r * 2 * CT * TILE,
+                       wbase + ((long long)(slice * 8 + (int)rank * 4 + r) * p.ntile_k + tk0) * 2 * TILE,
+                       2 * nt * TILE, cbar);
+          } else {
+            for (int q = 0; q < 8; ++q)  // row block q of the CTA's half of the slice
+              bulk_g2s(stage_c(cs) + q * CT * TILE,
+                       wbase + ((long long)(slice * 16 + (int)rank * 8 + q) * p.ntile_k + tk0) * TILE,
+                       nt * TILE, cbar);
+          }
+          ++ct;
+        }
+      }
+      if (!ok) give_up();
       for (uint32_t j = ct > SC ? ct - SC : 0; j < ct; ++j)
         (void)mbar_wait_bounded(smem_addr(&s_cfull[j % SC]), (j / SC) & 1);
     }
@@ -1043,31 +1054,42 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     const uint32_t tbase = GATED ? (uint32_t)(((q >> 1) * 2 * CT + (q & 1)) * TILE) : (uint32_t)(q * CT * TILE);
     constexpr uint32_t tstep = GATED ? 2 * TILE : TILE;
     const int g = lane >> 2, tig = lane & 3;
+    // Two k-steps per round (nsteps is even: K is a multiple of 128), into
+    // two B buffers: twice the independent work between waits, which hides
+    // the latency of the code loads and of the proxy fence.
     uint32_t it = 0, ct = 0;
     bool ok = true;
     for (int item = pair; item < items && ok; item += npairs) {
-      for (int ks = 0; ks < nsteps; ++ks, ++it) {
-        const uint32_t cs = ct % SC, cuse = ct / SC, bb = it % NBB, buse = it / NBB;
+      for (int ks = 0; ks < nsteps; ks += 2, it += 2) {
+        const uint32_t cs = ct % SC, cuse = ct / SC;
+        const uint32_t bb0 = it % NBB, bb1 = (it + 1) % NBB, bu0 = it / NBB, bu1 = (it + 1) / NBB;
         bool got = mbar_wait_bounded(smem_addr(&s_cfull[cs]), cuse & 1);
-        if (got && buse > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb]), (buse - 1) & 1);
+        if (got && bu0 > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb0]), (bu0 - 1) & 1);
+        if (got && bu1 > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb1]), (bu1 - 1) & 1);
         if (__any_sync(0xffffffffu, !got) || aborted()) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
-        const int half = ks % SPC, j = (ks % KSC) / SPC;
-        const uint32_t tsm = stage_c(cs) + tbase + j * tstep;
-        if constexpr (FMT == 1) {
-          dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), bbuf(bb), brow0 + g, g, tig);
-        } else {
-          const uint4 sc = lds_u4(tsm + 512 + g * 16);
-          dequant_q2_lane(lds_u2(tsm + lane * 16 + 8 * half), half ? sc.y : sc.x, half ? sc.w : sc.z, bbuf(bb),
-                          brow0 + g, g, tig);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k1 = ks + u, half = k1 % SPC, j = (k1 % KSC) / SPC;
+          const uint32_t tsm = stage_c(cs) + tbase + j * tstep, dst = bbuf(u ? bb1 : bb0);
+          if constexpr (FMT == 1) {
+            dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), dst, brow0 + g, g, tig);
+          } else {
+            const uint4 sc = lds_u4(tsm + 512 + g * 16);
+            dequant_q2_lane(lds_u2(tsm + lane * 16 + 8 * half), half ? sc.y : sc.x, half ? sc.w : sc.z, dst,
+                            brow0 + g, g, tig);
+          }
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead(&s_bfull[bb]));
-        if (ks % KSC == KSC - 1 || ks == nsteps - 1) {  // the code stage's last k-step: release it
+        if (lane == 0) {
+          mbar_arrive_remote(lead(&s_bfull[bb0]));
+          mbar_arrive_remote(lead(&s_bfull[bb1]));
+        }
+        if ((ks + 1) % KSC == KSC - 1 || ks + 1 == nsteps - 1) {  // the code stage's last k-step: release it
           if (lane == 0) mbar_arrive(smem_addr(&s_cempty[cs]));
           ++ct;
         }
