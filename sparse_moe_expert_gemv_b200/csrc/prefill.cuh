@@ -761,28 +761,30 @@ constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM 
 // rows: the even CTA rows [0, 128), the odd CTA rows [128, 256).  The pair's
 // accumulator columns are then [gate | up] of the even CTA's 64 features and
 // [gate | up] of the odd CTA's (gate/up), or the slice's 256 features in
-// order (down).  Per 64-column reduction step each CTA loads its A tile (16
-// KB) and dequantises its 128 weight rows (16 KB of fp16) once for all 256
-// token rows.  The A tiles and the code tiles travel in two rings: an A stage
-// is released when the pair's MMAs complete, a code stage when the CTA's
-// dequantising warps have read it.  A code stage holds CT consecutive
-// repacked tiles of each of the CTA's row blocks (4 k-steps): the tiles of a
+// order (down).  Per step of 128 reduction columns each CTA loads its A tile
+// (32 KB) and dequantises its 128 weight rows (32 KB of fp16) once for all
+// 256 token rows.  The A tiles and the code tiles travel in two rings: an A
+// stage is released when the pair's MMAs complete, a code stage when the
+// CTA's dequantising warps have read it.  A code stage holds CT consecutive
+// repacked tiles of each of the CTA's row blocks (two steps): the tiles of a
 // row block along the reduction are contiguous in memory (gate/up: gate and
 // up tile of each column side by side), so one bulk copy per row block fills
 // it -- issuing a copy costs the producer about 100 cycles, and one copy per
-// tile (8 per k-step) was the pipeline's bottleneck.
+// tile (8 per 64 columns) was the pipeline's bottleneck.
 template <int FMT>
 struct PfCfg {
   static constexpr int TILE = FMT == 1 ? 576 : 640;         // repacked code tile (+ scales)
-  static constexpr int SPC = FMT == 1 ? 1 : 2;              // k-steps per tile (64 / 128 columns)
+  static constexpr int APT = FMT == 1 ? 1 : 2;              // 64-column atoms per tile (64 / 128 columns)
   static constexpr int CT = FMT == 1 ? 4 : 2;               // tiles per row block per code stage
-  static constexpr int KSC = CT * SPC;                      // k-steps per code stage (4)
-  static constexpr int SA = 7;                              // A ring
+  static constexpr int APC = CT * APT;                      // atoms per code stage (4: two steps)
+  static constexpr int SA = 3;                              // A ring (stages of one step)
   static constexpr int SC = FMT == 1 ? 2 : 3;               // code ring
-  static constexpr int NBB = 4;                             // B buffers (dequantised weights)
+  static constexpr int NBB = 2;                             // B buffers (dequantised weights of one step)
   static constexpr int NB_ROWS = 128;                       // weight rows per CTA per item
-  static constexpr uint32_t TILE_A = kPfBM * kPfBK * 2;     // 16 KB: this CTA's 128 rows
-  static constexpr uint32_t BBUF = NB_ROWS * kPfBK * 2;     // 16 KB
+  static constexpr uint32_t ATOM_A = kPfBM * kPfBK * 2;     // 16 KB: this CTA's 128 rows x 64 columns
+  static constexpr uint32_t TILE_A = 2 * ATOM_A;            // one step: 128 columns
+  static constexpr uint32_t ATOM_B = NB_ROWS * kPfBK * 2;   // 16 KB
+  static constexpr uint32_t BBUF = 2 * ATOM_B;              // one step
   static constexpr uint32_t CODES = (8 * CT * TILE + 1023) / 1024 * 1024;  // 8 row blocks x CT tiles
   static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
   static constexpr uint32_t ACC_COLS = 2 * NB_ROWS;         // TMEM columns per buffer (MMA N = 256)
@@ -791,30 +793,35 @@ struct PfCfg {
 
 // Grouped GEMM over the tile list, warp-specialised, on CTA pairs; the
 // persistent pairs walk the items clusterid.x, +nclusterid.x.  Both CTAs:
-//  warp 0 lane 0   A producer: per 64-column reduction step this CTA's A
-//                  tile (2-D TMA, 128-byte swizzle; the odd CTA only when the
-//                  tile has more than 128 rows) into a free stage of the A
-//                  ring, counted on the even CTA's stage barrier
-//  warp 2 lane 0   code producer: every KSC steps the next code stage (one
+//  warp 0 lane 0   A producer: per step (128 reduction columns, two 64-column
+//                  atoms) this CTA's A tile (two 2-D TMA boxes, 128-byte
+//                  swizzle; the odd CTA only when the tile has more than 128
+//                  rows) into a free stage of the A ring, counted on the even
+//                  CTA's stage barrier
+//  warp 2 lane 0   code producer: every two steps the next code stage (one
 //                  1-D bulk copy per row block) into the code ring; apart
 //                  from the A producer so that neither ring waits on the other
-//  warps 8..15     one row block each: dequantise two k-steps' codes into two
-//                  of four swizzled fp16 B buffers, arrive on the even CTA's
-//                  buffer barriers, release the code stage after its last k-step
+//  warps 8..15     one row block each: dequantise a step's codes into one of
+//                  two swizzled fp16 B buffers, arrive on the even CTA's
+//                  buffer barrier, release the code stage after its last step
 //  warps 4..7      drain an accumulator buffer (TMEM lanes = the CTA's rows)
 //                  while the next item accumulates into the other one, then
 //                  arrive on the even CTA's buffer-empty barrier
 // Even CTA only:
-//  warp 1 lane 0   issues the pair's MMAs (m256n256k16 per 16-column step,
-//                  fp32 in TMEM) and commits the release of the A stage, the
-//                  B buffer and the accumulator to the barriers of both CTAs
+//  warp 1 lane 0   issues the pair's MMAs (8 x m256n256k16 per step, fp32 in
+//                  TMEM) and commits the release of the A stage, the B buffer
+//                  and the accumulator to the barriers of both CTAs
+// A step of 128 columns (rather than one 64-column atom) halves the barrier
+// waits and commits per MMA: the issuing thread's per-wait overhead left the
+// tensor pipe idle between atoms.
 // Every wait is bounded; a timeout raises kErrTimeout and stops both CTAs.
 template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
   using C = PfCfg<FMT>;
-  constexpr int SA = C::SA, SC = C::SC, SPC = C::SPC, CT = C::CT, KSC = C::KSC, TILE = C::TILE,
+  constexpr int SA = C::SA, SC = C::SC, APT = C::APT, CT = C::CT, APC = C::APC, TILE = C::TILE,
                 NBB = C::NBB;
+  constexpr int SPS = APC / 2;  // steps per code stage
   constexpr int COLS = GATED ? C::NB_ROWS : 2 * C::NB_ROWS;  // output features per item
   extern __shared__ __align__(128) unsigned char pf_smem[];  // stages start at the next 1024 B
   __shared__ __align__(8) unsigned long long s_afull[SA], s_aempty[SA], s_cfull[SC], s_cempty[SC],
@@ -857,7 +864,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   const uint32_t tmem = s_tmem;
   pdl_wait();
   const int ntiles = ldcg_i32(p.n_tiles);
-  const int nslices = p.N / COLS, nsteps = p.K / kPfBK;
+  const int nslices = p.N / COLS, nsteps = p.K / (2 * kPfBK);  // K is a multiple of 128
   const int items = ntiles * nslices;
   const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
   auto stage_a = [&](uint32_t st) { return stage0 + st * C::TILE_A; };
@@ -876,7 +883,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   if (wid == 0) {
     // ------------------------------------------------------------ A producer
     if (lane == 0) {
-      uint32_t it = 0;  // k-steps issued
+      uint32_t it = 0;  // steps issued
       bool ok = true;
       for (int item = pair; item < items && ok && !aborted(); item += npairs) {
         const PfTile tile = p.tiles[item / nslices];
@@ -890,7 +897,10 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           }
           if (rank == 0) mbar_expect_tx(smem_addr(&s_afull[st]), two ? 2 * C::TILE_A : C::TILE_A);
           if (mine)
-            tma_load_2d_pair(stage_a(st), &amap, ks * kPfBK, tile.row0 + (int)rank * kPfBM, lead(&s_afull[st]));
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+              tma_load_2d_pair(stage_a(st) + s * C::ATOM_A, &amap, (2 * ks + s) * kPfBK,
+                               tile.row0 + (int)rank * kPfBM, lead(&s_afull[st]));
         }
       }
       if (!ok) give_up();
@@ -910,9 +920,9 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         const PfTile tile = p.tiles[item / nslices];
         const int slice = item % nslices;
         const uint8_t *wbase = tile.w + p.region_off;
-        for (int ks = 0; ks < nsteps; ks += KSC) {  // code stage: tiles tk0 .. tk0 + nt - 1
+        for (int ks = 0; ks < nsteps; ks += SPS) {  // code stage: tiles tk0 .. tk0 + nt - 1
           const uint32_t cs = ct % SC, cuse = ct / SC;
-          const int tk0 = ks / SPC, nt = min(CT, p.ntile_k - tk0);
+          const int tk0 = 2 * ks / APT, nt = min(CT, p.ntile_k - tk0);
           if (cuse > 0 && !mbar_wait_bounded(smem_addr(&s_cempty[cs]), (cuse - 1) & 1)) {
             ok = false;
             break;
@@ -961,9 +971,11 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kPfBK / 16; ++kk)
-            umma_f16_pair(acc, umma_desc_sw128(stage_a(st) + kk * 32), umma_desc_sw128(bbuf(bb) + kk * 32),
-                          IDESC, (ks | kk) != 0);
+          for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int kk = 0; kk < kPfBK / 16; ++kk)
+              umma_f16_pair(acc, umma_desc_sw128(stage_a(st) + s * C::ATOM_A + kk * 32),
+                            umma_desc_sw128(bbuf(bb) + s * C::ATOM_B + kk * 32), IDESC, (ks | s | kk) != 0);
           umma_commit_pair(smem_addr(&s_aempty[st]));
           umma_commit_pair(smem_addr(&s_bempty[bb]));
         }
@@ -1054,27 +1066,22 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     const uint32_t tbase = GATED ? (uint32_t)(((q >> 1) * 2 * CT + (q & 1)) * TILE) : (uint32_t)(q * CT * TILE);
     constexpr uint32_t tstep = GATED ? 2 * TILE : TILE;
     const int g = lane >> 2, tig = lane & 3;
-    // Two k-steps per round (nsteps is even: K is a multiple of 128), into
-    // two B buffers: twice the independent work between waits, which hides
-    // the latency of the code loads and of the proxy fence.
     uint32_t it = 0, ct = 0;
     bool ok = true;
     for (int item = pair; item < items && ok; item += npairs) {
-      for (int ks = 0; ks < nsteps; ks += 2, it += 2) {
-        const uint32_t cs = ct % SC, cuse = ct / SC;
-        const uint32_t bb0 = it % NBB, bb1 = (it + 1) % NBB, bu0 = it / NBB, bu1 = (it + 1) / NBB;
+      for (int ks = 0; ks < nsteps; ++ks, ++it) {
+        const uint32_t cs = ct % SC, cuse = ct / SC, bb = it % NBB, buse = it / NBB;
         bool got = mbar_wait_bounded(smem_addr(&s_cfull[cs]), cuse & 1);
-        if (got && bu0 > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb0]), (bu0 - 1) & 1);
-        if (got && bu1 > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb1]), (bu1 - 1) & 1);
+        if (got && buse > 0) got = mbar_wait_bounded(smem_addr(&s_bempty[bb]), (buse - 1) & 1);
         if (__any_sync(0xffffffffu, !got) || aborted()) {
           if (lane == 0) give_up();
           ok = false;
           break;
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int k1 = ks + u, half = k1 % SPC, j = (k1 % KSC) / SPC;
-          const uint32_t tsm = stage_c(cs) + tbase + j * tstep, dst = bbuf(u ? bb1 : bb0);
+        for (int s = 0; s < 2; ++s) {  // the step's two 64-column atoms
+          const int at = (2 * ks + s) % APC, half = at % APT, j = at / APT;
+          const uint32_t tsm = stage_c(cs) + tbase + j * tstep, dst = bbuf(bb) + s * C::ATOM_B;
           if constexpr (FMT == 1) {
             dequant_q4_lane(lds_u4(tsm + lane * 16), lds_u2(tsm + 512 + g * 8), dst, brow0 + g, g, tig);
           } else {
@@ -1085,17 +1092,15 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
         }
         fence_proxy_async_smem();  // the tensor core reads B through the async proxy
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_remote(lead(&s_bfull[bb0]));
-          mbar_arrive_remote(lead(&s_bfull[bb1]));
-        }
-        if ((ks + 1) % KSC == KSC - 1 || ks + 1 == nsteps - 1) {  // the code stage's last k-step: release it
+        if (lane == 0) mbar_arrive_remote(lead(&s_bfull[bb]));
+        if (ks % SPS == SPS - 1 || ks == nsteps - 1) {  // the code stage's last step: release it
           if (lane == 0) mbar_arrive(smem_addr(&s_cempty[cs]));
           ++ct;
         }
       }
     }
   }
+
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // the pair's MMAs, remote arrivals and copies are done
