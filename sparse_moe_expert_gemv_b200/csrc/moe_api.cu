@@ -78,6 +78,7 @@ struct moe_ctx {
   PfTile *pf_tiles = nullptr;
   int pf_max_tiles = 0, pf_rows = 0;
   CUtensorMap pf_map_h{}, pf_map_a{};   // TMA maps of the grouped A matrices
+  CUtensorMap pf_omap_a{}, pf_omap_y{};  // TMA maps of the GEMMs' outputs (a, y)
   bool pf_maps = false;
   int pf_pairs = 0;  // co-resident CTA pairs of the grouped GEMM (0: it cannot run)
   unsigned long long *trace = nullptr;  // moe_set_trace buffer
@@ -666,6 +667,20 @@ bool encode_map_16b(CUtensorMap *map, CUtensorMapDataType type, const void *base
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map of the grouped GEMM's epilogue: fp16 [rows][cols], boxes of
+// 32 rows x 32 columns (64 B) with the 64-byte swizzle of the staging tiles.
+bool encode_out_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kPfOutCols, (cuuint32_t)kPfOutRows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
   static_assert(kPfBK == 64, "one swizzle row per box row");
   return encode_map_16b(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rows, cols, kPfBM);
@@ -730,8 +745,9 @@ cudaError_t launch_prefill_gemms(moe_ctx *c, cudaStream_t s) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, true>, c->pf_map_h, g1);
-  if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, false>, c->pf_map_a, g2);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, true>, c->pf_map_h, c->pf_omap_a, g1);
+  if (e == cudaSuccess)
+    e = cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<FMT, false>, c->pf_map_a, c->pf_omap_y, g2);
   return e;
 }
 
@@ -842,7 +858,9 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   const int k = c->k, d = c->d, f = c->f;
   if (!c->pf_maps) {
     if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
-        !encode_map_f16(&c->pf_map_a, c->pf_a16, c->pf_rows, f))
+        !encode_map_f16(&c->pf_map_a, c->pf_a16, c->pf_rows, f) ||
+        !encode_out_map_f16(&c->pf_omap_a, c->pf_a16, c->pf_rows, f) ||
+        !encode_out_map_f16(&c->pf_omap_y, c->pf_y16, c->pf_rows, d))
       return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     c->pf_maps = true;
   }

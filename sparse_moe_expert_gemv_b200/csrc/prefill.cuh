@@ -719,6 +719,22 @@ MOE_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cl)
       : "memory");
 }
+// 2-D TMA tile store from this CTA's shared memory (bulk-group completion).
+MOE_DEV void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+MOE_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all of this thread's bulk groups are complete.
+MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // The pair's MMA, issued by one thread of the even CTA: D (both CTAs' TMEM at
 // tmem_d) (+)= A (both CTAs' shared memory at da) x B (both at db)^T.
 MOE_DEV void umma_f16_pair(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate) {
@@ -750,6 +766,8 @@ struct PfGemmParams {
 };
 
 constexpr int kPfGemmThreads = 512;  // 16 warps
+constexpr int kPfOutRows = 32, kPfOutCols = 32;  // epilogue TMA store box (one warp's rows x 64 B)
+constexpr uint32_t kPfOutStage = kPfOutRows * kPfOutCols * 2;  // 2 KB
 constexpr int kPfDeqWarp0 = 8;       // warps 8..15 dequantise
 constexpr int kPfEpiWarp0 = 4;       // warps 4..7 drain the accumulators (TMEM lane quarters 0..3)
 
@@ -786,7 +804,8 @@ struct PfCfg {
   static constexpr uint32_t ATOM_B = NB_ROWS * kPfBK * 2;   // 16 KB
   static constexpr uint32_t BBUF = 2 * ATOM_B;              // one step
   static constexpr uint32_t CODES = (8 * CT * TILE + 1023) / 1024 * 1024;  // 8 row blocks x CT tiles
-  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + 1024;  // + alignment slack
+  static constexpr uint32_t OUT = 4 * 2 * kPfOutStage;       // epilogue staging: 2 per epilogue warp
+  static constexpr uint32_t SMEM = SA * TILE_A + SC * CODES + NBB * BBUF + OUT + 1024;  // + alignment slack
   static constexpr uint32_t ACC_COLS = 2 * NB_ROWS;         // TMEM columns per buffer (MMA N = 256)
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;       // double buffered: all 512
 };
@@ -817,7 +836,8 @@ struct PfCfg {
 // Every wait is bounded; a timeout raises kErrTimeout and stops both CTAs.
 template <int FMT, bool GATED>
 __global__ void __launch_bounds__(kPfGemmThreads, 1)
-    prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, PfGemmParams p) {
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap omap,
+                        PfGemmParams p) {
   using C = PfCfg<FMT>;
   constexpr int SA = C::SA, SC = C::SC, APT = C::APT, CT = C::CT, APC = C::APC, TILE = C::TILE,
                 NBB = C::NBB;
@@ -870,6 +890,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
   auto stage_a = [&](uint32_t st) { return stage0 + st * C::TILE_A; };
   auto stage_c = [&](uint32_t cs) { return stage0 + SA * C::TILE_A + cs * C::CODES; };
   auto bbuf = [&](uint32_t b) { return stage0 + SA * C::TILE_A + SC * C::CODES + b * C::BBUF; };
+  const uint32_t out0 = stage0 + SA * C::TILE_A + SC * C::CODES + NBB * C::BBUF;  // 1024-aligned
   auto lead = [&](const void *v) { return mapa_shared(smem_addr(v), 0); };  // the even CTA's copy
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
   auto give_up = [&]() {  // stop both CTAs' roles
@@ -990,8 +1011,13 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
     }
   } else if (wid >= kPfEpiWarp0 && wid < kPfEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
+    // A warp whose 32 rows all belong to the tile stages each 32-column
+    // chunk (fp16, 64-byte swizzle: conflict-free lane stores) and writes it
+    // with one TMA store, two stages in flight; rows at a tile's ragged end
+    // are stored lane by lane, so no store reaches another expert's rows.
     const int quarter = wid & 3;  // TMEM lanes [32 quarter, +32) = the warp's rows of this CTA
-    uint32_t ii = 0;
+    const uint32_t stg = out0 + (uint32_t)quarter * 2 * kPfOutStage;
+    uint32_t ii = 0, ob = 0;  // items, staged stores
     for (int item = pair; item < items; item += npairs, ++ii) {
       const uint32_t buf = ii & 1;
       const bool ok = mbar_wait_bounded(smem_addr(&s_accf[buf]), (ii >> 1) & 1);
@@ -1004,7 +1030,30 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       const int n0 = (item % nslices) * COLS;
       const int r0 = (int)rank * kPfBM + quarter * 32;  // the warp's first row in the tile
       const int r = r0 + lane;
+      const bool full = r0 + 32 <= tile.rows;  // warp-uniform
       const uint32_t lane_addr = tmem + buf * C::ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+      __half *const out = GATED ? p.out_a : p.out_y;
+      auto emit = [&](const uint32_t (&pk)[16], int col) {
+        if (full) {
+          const uint32_t sb = stg + (ob & 1) * kPfOutStage;
+          if (lane == 0 && ob >= 2) bulk_wait_read<1>();  // the store of two chunks ago has read its stage
+          __syncwarp();
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sb + lane * 64 +
+                                                                      ((v ^ ((lane >> 1) & 3)) << 4)),
+                         "r"(pk[4 * v]), "r"(pk[4 * v + 1]), "r"(pk[4 * v + 2]), "r"(pk[4 * v + 3])
+                         : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tma_store_2d(&omap, sb, col, tile.row0 + r0);
+          ++ob;
+        } else if (r < tile.rows) {
+          uint4 *dst = reinterpret_cast<uint4 *>(out + (long long)(tile.row0 + r) * p.N + col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      };
       if (r0 < tile.rows) {  // warp-uniform: the warp has rows in this tile
         if constexpr (GATED) {
           // accumulator columns [128 h, 128 h + 64) = gate, [128 h + 64,
@@ -1014,39 +1063,24 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
             float g[32], u[32];
             tmem_ld32(lane_addr + h * 128 + c0, g);
             tmem_ld32(lane_addr + h * 128 + 64 + c0, u);
-            if (r < tile.rows) {
-              uint4 *dst = reinterpret_cast<uint4 *>(p.out_a + (long long)(tile.row0 + r) * p.N + n0 + c);
+            uint32_t pk[16];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const int i = v * 8 + q * 2;
-                  const float a0 = g[i] / (1.0f + __expf(-g[i])) * u[i];
-                  const float a1 = g[i + 1] / (1.0f + __expf(-g[i + 1])) * u[i + 1];
-                  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
-                }
-                dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
+            for (int q = 0; q < 16; ++q) {
+              const float a0 = g[2 * q] / (1.0f + __expf(-g[2 * q])) * u[2 * q];
+              const float a1 = g[2 * q + 1] / (1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
+              asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
             }
+            emit(pk, n0 + c);
           }
         } else {
           for (int c0 = 0; c0 < COLS; c0 += 32) {
             float y[32];
             tmem_ld32(lane_addr + c0, y);
-            if (r < tile.rows) {
-              uint4 *dst = reinterpret_cast<uint4 *>(p.out_y + (long long)(tile.row0 + r) * p.N + n0 + c0);
+            uint32_t pk[16];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const int i = v * 8 + q * 2;
-                  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(y[i + 1]), "f"(y[i]));
-                }
-                dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
-            }
+            for (int q = 0; q < 16; ++q)
+              asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(y[2 * q + 1]), "f"(y[2 * q]));
+            emit(pk, n0 + c0);
           }
         }
       }
@@ -1054,6 +1088,7 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(lead(&s_acce[buf]));
     }
+    if (lane == 0) bulk_wait_all();  // every staged store has landed before the CTA exits
   } else if (wid >= kPfDeqWarp0) {
     // ------------------------------------------------------------ dequantise
     // warp -> one row block of the CTA's 128 weight rows (gate/up: row
