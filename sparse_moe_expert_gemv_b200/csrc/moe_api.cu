@@ -787,8 +787,14 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
 
 // Experts with at least this many tokens in a chunk run on the grouped GEMM
 // (256-row tiles); fewer tokens would leave most of a tile empty, and the
-// GEMV streams such an expert once per job of <= 16 tokens instead.
+// GEMV streams such an expert once per job of <= 8 tokens instead.
 constexpr int kHotMinTokens = 16;
+// The chunk path's GEMV experts (fewer than kHotMinTokens tokens: most have
+// one to three) run as jobs of <= 8 tokens through the one-column-tile GEMV;
+// jobs of 16 doubled its tensor work per weight byte, and the pass is
+// weight-bound (a chunk of 8192 tokens touched about 106 such experts with
+// 401 tokens between them: 281 MB of weights).
+constexpr int kColdChunk = 8;
 
 bool use_prefill_gemm(const moe_ctx *c, int N) {
   return c->pf && c->pf_pairs > 0 && N > kDecMaxT && c->d % (2 * kPfBN) == 0 && c->f % kPfBN == 0 &&
@@ -833,7 +839,7 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   sp.n_tiles = c->pf_ntiles;
   sp.max_tiles = c->pf_max_tiles;
   sp.hot_min = hot_min;
-  sp.chunk = job_chunk(N);
+  sp.chunk = kColdChunk;
   sp.hot = c->pf_hot;
   sp.job_ptr = c->job_ptr;
   sp.job_beg = c->job_beg;
@@ -872,7 +878,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   if (st) return st;
   CUDA_TRY(c, prof_mark(c, 1, s));
   // experts with many tokens: grouped GEMM over 256-row tiles; the others:
-  // the GEMV over jobs of <= 16 tokens, rows read through the bucket
+  // the GEMV over jobs of <= 8 tokens, rows read through the bucket
   // permutation (grouped row -> pair id)
   GemvParams g1{};
   g1.job_ptr = c->job_ptr;
@@ -899,10 +905,10 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
   g2.out_y = c->ybuf;
   if (c->fmt == MOE_Q4_SYM_G32_F16) {
     CUDA_TRY(c, launch_prefill_gemms<1>(c, s));
-    CUDA_TRY(c, launch_experts<1>(c, s, N, g1, g2));
+    CUDA_TRY(c, launch_experts<1>(c, s, kColdChunk, g1, g2));
   } else {
     CUDA_TRY(c, launch_prefill_gemms<2>(c, s));
-    CUDA_TRY(c, launch_experts<2>(c, s, N, g1, g2));
+    CUDA_TRY(c, launch_experts<2>(c, s, kColdChunk, g1, g2));
   }
   CUDA_TRY(c, prof_mark(c, 2, s));
   PfCombineParams mp{c->pf_y16, c->ybuf, c->w, c->pf_row_of, N, k, d, c->n_shared, x, delta};
