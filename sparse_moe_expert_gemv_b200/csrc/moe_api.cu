@@ -667,6 +667,20 @@ bool encode_map_16b(CUtensorMap *map, CUtensorMapDataType type, const void *base
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 logits [rows][cols] in boxes of 32 x 32 with the 128-byte swizzle of
+// the router's staging tiles.
+bool encode_logit_map(CUtensorMap *map, const void *base, int rows, int cols) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  const cuuint32_t box[2] = {32u, 32u};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output map of the grouped GEMM's epilogue: fp16 [rows][cols], boxes of
 // 32 rows x 32 columns (64 B) with the 64-byte swizzle of the staging tiles.
 bool encode_out_map_f16(CUtensorMap *map, const void *base, int rows, int cols) {
@@ -763,11 +777,12 @@ cudaError_t launch_prefill_gemms(moe_ctx *c, cudaStream_t s) {
 constexpr int kRtMinTokens = 512;
 bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, cudaError_t *err) {
   const int E = c->E, d = c->d;
-  CUtensorMap hm, wm;
+  CUtensorMap hm, wm, lm;
   if (!c->d_router3 || E % kRtBN != 0 || N < kRtMinTokens || d % 64 != 0 ||
       !encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) ||
       !encode_map_16b(&wm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->d_router3 + (size_t)layer * E * 3 * d, E,
-                      3 * d, kRtBN))
+                      3 * d, kRtBN) ||
+      !encode_logit_map(&lm, c->logits, N, E))
     return false;
   RouterTcParams tp{c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, c->logits, N, E, d,
                     c->status};
@@ -781,7 +796,7 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  *err = cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, tp);
+  *err = cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, lm, tp);
   return true;
 }
 

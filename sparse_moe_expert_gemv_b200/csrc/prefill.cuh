@@ -1196,7 +1196,7 @@ constexpr uint32_t umma_idesc_bf16(int M, int N) { return umma_idesc_f16(M, N) |
 
 __global__ void __launch_bounds__(256, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap hmap, const __grid_constant__ CUtensorMap wmap,
-                     RouterTcParams p) {
+                     const __grid_constant__ CUtensorMap lmap, RouterTcParams p) {
   using C = RtCfg;
   constexpr int S = kRtStages;
   extern __shared__ __align__(128) unsigned char rt_smem[];
@@ -1279,19 +1279,33 @@ __global__ void __launch_bounds__(256, 1)
     const bool ok = mbar_wait_bounded(smem_addr(&s_accf), 0);
     tc_fence_after();
     if (__all_sync(0xffffffffu, ok && !aborted())) {  // warp-uniform: tcgen05.ld is collective
-      const int quarter = wid & 3, t = m0 + quarter * 32 + lane;
+      // Every MMA is complete, so the ring is free: each warp stages its 32
+      // rows x 32 logits (128-byte swizzle: conflict-free lane stores) in
+      // two 4 KB buffers there and writes each block with one TMA store
+      // (rows past T are clipped by the tensor map).
+      const int quarter = wid & 3, r0 = m0 + quarter * 32;
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-      for (int c0 = 0; c0 < kRtBN; c0 += 32) {
+      const uint32_t stg = stage0 + (uint32_t)quarter * 2 * 4096;
+      for (int c0 = 0, ob = 0; c0 < kRtBN; c0 += 32, ++ob) {
         float v[32];
         tmem_ld32(lane_addr + c0, v);
-        if (t < p.T) {
+        if (p.bias) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = n0 + c0 + j;
-            if (e < p.E) p.logits[(long long)t * p.E + e] = v[j] + (p.bias ? p.bias[e] : 0.f);
-          }
+          for (int j = 0; j < 32; ++j) v[j] += __ldg(p.bias + n0 + c0 + j);
         }
+        const uint32_t sb = stg + (uint32_t)(ob & 1) * 4096;
+        if (lane == 0 && ob >= 2) bulk_wait_read<1>();  // the store of two blocks ago has read its buffer
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(sb + lane * 128 + ((q ^ (lane & 7)) << 4)),
+                       "f"(v[4 * q]), "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
+                       : "memory");
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && r0 < p.T) tma_store_2d(&lmap, sb, n0 + c0, r0);
       }
+      if (lane == 0) bulk_wait_all();
     } else if (lane == 0) {
       give_up();
     }
