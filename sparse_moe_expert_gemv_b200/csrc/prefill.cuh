@@ -6,7 +6,8 @@
 // in chunks of up to 8192 tokens), so the experts run as a grouped GEMM on
 // the 5th-generation tensor cores:
 //
-//   prefill_topk_kernel     one warp per token: top-k + softmax; per block of
+//   prefill_topk_kernel     one warp per token: top-k + softmax (candidate
+//                           filter, warp_topk_fast); per block of
 //                           16 tokens, each expert's token set (a bitmask)
 //   prefill_colscan_kernel  per expert: each block of 16 tokens' first row
 //                           relative to the expert's (a scan down the
@@ -147,6 +148,7 @@ MOE_DEV float exact_logit(const float *W, const uint16_t *h, const float *bias, 
 template <int NPL>
 __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams p) {
   __shared__ unsigned s_mask[kPfMaxE];
+  __shared__ unsigned long long s_cand[kPfTok][64];  // each warp's top-k candidates
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   pdl_wait();
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_mask[e] = 0u;
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
     int e;
     float w, lk, lk1;
     float *lr = p.logits + (long long)t * p.E;
-    warp_topk<NPL>(lr, p.E, p.k, lane, false, e, w, nullptr, &lk, &lk1);
+    if (!warp_topk_fast<NPL>(lr, p.E, p.k, lane, s_cand[wid], e, w, nullptr, &lk, &lk1))
+      warp_topk<NPL>(lr, p.E, p.k, lane, false, e, w, nullptr, &lk, &lk1);
     if (lk - lk1 < kRefineBand) {
       // the boundary is close: recompute the logits in the band around it
       // exactly, then select again (and count a near tie on exact values)

@@ -234,6 +234,70 @@ MOE_DEV void warp_topk_merge(const unsigned long long *cand, int n, int E, int k
   sel_w = ex / den;
 }
 
+// Top-k of one token by one warp through a candidate filter; same result
+// as warp_topk (selections, weights, *lk, *lk1).  The (k+1)-th largest of
+// the lanes' maxima is a threshold that at least k + 1 logits reach, so the
+// k + 1 best are among the values at or above it: those (usually a few
+// dozen) are compacted into cand[0..64) (this warp's shared memory) and the
+// k + 1 best of them are selected two per lane.  A full selection round over
+// all NPL values per lane runs only once (the lane maxima) instead of k + 1
+// times.  Returns false, with nothing written, when k + 1 > 32, k >= E or
+// more than 64 values pass; the caller then runs warp_topk.  Near ties are
+// counted as warp_topk counts them.
+template <int NPL>
+MOE_DEV bool warp_topk_fast(const float *lr, int E, int k, int lane, unsigned long long *cand, int &sel_e,
+                            float &sel_w, unsigned long long *near_ties, float *lk, float *lk1) {
+  if (k + 1 > 32 || k >= E) return false;
+  unsigned long long pk[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    pk[i] = e < E ? ((unsigned long long)order_key(__ldcg(lr + e)) << 32) | (uint32_t)~e : 0ull;
+  }
+  // the (k+1)-th largest lane maximum: min(E, 32) >= k + 1 lanes hold one
+  unsigned long long m = tournament_max<NPL>(pk), thr = 0ull;
+  for (int j = 0; j <= k; ++j) {
+    const uint32_t hi = (uint32_t)(m >> 32);
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, hi == wmax ? (uint32_t)m : 0u);
+    thr = ((unsigned long long)wmax << 32) | wlo;
+    m = m == thr ? 0ull : m;
+  }
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) c += (pk[i] != 0ull && pk[i] >= thr) ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total > 64) return false;
+  int pos = incl - c;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i)
+    if (pk[i] != 0ull && pk[i] >= thr) cand[pos++] = pk[i];
+  __syncwarp();
+  unsigned long long pc[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) pc[i] = lane + 32 * i < total ? cand[lane + 32 * i] : 0ull;
+  __syncwarp();  // cand[] may be rewritten by this warp's next token
+  const unsigned long long v = warp_top_packed<2>(pc, k + 1, lane);  // lane j <= k: the j-th best
+  const uint32_t key = (uint32_t)(v >> 32);
+  const uint32_t k0 = __shfl_sync(0xffffffffu, key, 0);
+  const uint32_t kth = __shfl_sync(0xffffffffu, key, k - 1);
+  const uint32_t next = __shfl_sync(0xffffffffu, key, k);
+  if (near_ties && lane == 0 && key_to_float(kth) - key_to_float(next) < 1e-5f) atomicAdd(near_ties, 1ULL);
+  if (lk) *lk = key_to_float(kth);
+  if (lk1) *lk1 = key_to_float(next);
+  const float ex = lane < k ? expf(key_to_float(key) - key_to_float(k0)) : 0.f;
+  const float den = warp_sum(ex);
+  sel_e = lane < k ? (int)~(uint32_t)v : 0;
+  sel_w = ex / den;
+  return true;
+}
+
 // Shared-memory words the body needs (dynamic smem of the finish kernel;
 // the fused kernel reuses its staging area).
 MOE_HOST_DEV_INLINE int finish_smem_ints(int E, int P) {
