@@ -163,8 +163,9 @@ MOE_API moe_status moe_set_slots(moe_ctx *ctx, const int32_t *slot_of);
  * "Architecture overview": the router picks 10 of 512 experts per token;
  * the "Doorbell handshake" section ends the "pre" half of a block with the
  * router's ids and weights).  Windows of more than 32 tokens select the
- * top-k one warp per token; from 512 tokens, with E a multiple of 256, the
- * logits come from the tensor-core router (see moe_set_router).  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
+ * top-k one warp per token; with E a multiple of 256 and a context
+ * configured for chunks (max_tokens > 32), the logits come from the
+ * tensor-core router (see moe_set_router).  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
  * w_dev fp32 [T, k] receive each token's experts and renormalised weights,
  * ordered by descending logit (equal logits: lower expert id first).
  * bucket_off_dev int32 [E+1] (exclusive prefix of tokens per expert) and
@@ -209,12 +210,12 @@ MOE_API moe_status moe_forward_stack(moe_ctx *ctx, void *x_dev, int T, void *str
  * on one 8 GB card", section "Architecture overview", runs prefill in chunks
  * of up to 8192 tokens; per expert such a chunk is a dense contraction.  For
  * N > 32 the experts (Q4 or Q2) run as a grouped GEMM on the tensor cores
- * (tcgen05): tokens sorted by expert, 128-token tiles, weights dequantised
+ * (tcgen05): tokens sorted by expert, 256-token tiles, weights dequantised
  * to fp16 tile by tile in shared memory (Q4: s (c - 8); Q2: s q + m, one
  * fp16 rounding), fp32 accumulation in tensor memory.  Activations enter as
  * fp16 (exact for |h| < 65504; larger values saturate), and the experts'
  * outputs y are kept in fp16 until the combine.  Router logits: fp32
- * accuracy, on the tensor cores from N >= 512 and E a multiple of 256 (see
+ * accuracy, on the tensor cores when E is a multiple of 256 (see
  * moe_set_router), else fp32 FMA.  N <= 32 takes the moe_forward path.
  * Requires a context configured with max_tokens >= N.  Errors: INVALID_ARG,
  * STATE; device faults through moe_sync. */
@@ -228,8 +229,8 @@ MOE_API moe_status moe_prefill_delta(moe_ctx *ctx, int layer, const void *x_dev,
 
 /* moe_prefill_route: the routing half of moe_prefill alone, on router
  * input h_dev bf16 [N, d] (no RMSNorm here, as in moe_route): the chunk's
- * router logits (tensor cores from N >= 512 with E a multiple of 256, else
- * fp32 FMA), top-k + softmax one warp per token, and the sort of the
+ * router logits (tensor cores when E is a multiple of 256, else fp32
+ * FMA), top-k + softmax one warp per token, and the sort of the
  * chunk's pairs by expert that feeds the grouped GEMM (the engine article
  * "93 token/s on one 8 GB card", section "Architecture overview": prefill in
  * chunks of up to 8192 tokens).  It launches exactly the kernels moe_prefill

@@ -213,7 +213,7 @@ moe_status do_configure(moe_ctx *c) {
     return at;
   };
   const size_t o_status = carve(sizeof(int)), o_ticket = carve(2 * sizeof(unsigned int));
-  const size_t dec_warps = (size_t)c->n_sm * 16;
+  const size_t dec_warps = (size_t)c->n_sm * GemvCfg<1, true, 1>::WARPS;  // decode_kernel warps
   const size_t o_dbar = carve(sizeof(unsigned long long) * (1 + 2 * dec_warps));
   const size_t o_dws = carve(sizeof(float) * dec_warps * 32 * 16);
   const size_t o_njobs = carve(sizeof(int)), o_last = carve(4 * sizeof(int));
@@ -667,16 +667,17 @@ bool encode_map_16b(CUtensorMap *map, CUtensorMapDataType type, const void *base
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 logits [rows][cols] in boxes of 32 x 32 with the 128-byte swizzle of
-// the router's staging tiles.
-bool encode_logit_map(CUtensorMap *map, const void *base, int rows, int cols) {
+// fp32 logits [planes][rows][cols] (planes = the splits of a split
+// reduction, else 1) in boxes of 32 x 32 x 1 with the 128-byte swizzle of
+// the router's staging tiles; a plane clips its own rows.
+bool encode_logit_map(CUtensorMap *map, const void *base, int planes, int rows, int cols) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-  const cuuint32_t box[2] = {32u, 32u};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+  const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)rows * cols * 4};
+  const cuuint32_t box[3] = {32u, 32u, 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -769,25 +770,29 @@ cudaError_t launch_prefill_gemms(moe_ctx *c, cudaStream_t s) {
 // window, f a multiple of the gate/up item (128 features) and d of the down
 // item (256 features); Q4 and Q2 experts.
 // Router logits of N tokens on the tensor cores (router_tc_kernel) when the
-// context holds the router's bf16 parts, the shapes fit its tiles and the
-// chunk has at least kRtMinTokens tokens (one tile per CTA runs its whole
-// reduction, about 75 us at d = 2048 whatever the grid: fewer tokens are
-// faster on the fp32 router's wider grid); returns false (nothing launched)
-// otherwise.
-constexpr int kRtMinTokens = 512;
+// context holds the router's bf16 parts and E and d fit its tiles; returns
+// false (nothing launched) otherwise.  A chunk with fewer 128 x 256 tiles
+// than SMs splits the reduction over blockIdx.z (each split at least four
+// 64-column steps) and router_sum_kernel adds the partial sums, in split
+// order, with the bias.
 bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int layer, cudaError_t *err) {
   const int E = c->E, d = c->d;
+  if (!c->d_router3 || E % kRtBN != 0 || d % 64 != 0) return false;
+  const int tiles = ((N + kRtBM - 1) / kRtBM) * (E / kRtBN), nk = 3 * d / 64;
+  int splits = 1;
+  while (2 * splits * tiles <= c->n_sm && 2 * splits <= kMaxRouterSplit && nk % (2 * splits) == 0 &&
+         nk / (2 * splits) >= 4 && (long long)2 * splits * N * E <= c->pf_part_floats)
+    splits *= 2;
+  const float *bias = c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr;
   CUtensorMap hm, wm, lm;
-  if (!c->d_router3 || E % kRtBN != 0 || N < kRtMinTokens || d % 64 != 0 ||
-      !encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) ||
+  if (!encode_map_16b(&hm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h, N, d, kRtBM) ||
       !encode_map_16b(&wm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->d_router3 + (size_t)layer * E * 3 * d, E,
                       3 * d, kRtBN) ||
-      !encode_logit_map(&lm, c->logits, N, E))
+      !encode_logit_map(&lm, splits > 1 ? c->pf_part : c->logits, splits, N, E))
     return false;
-  RouterTcParams tp{c->has_bias[layer] ? c->d_bias + (size_t)layer * E : nullptr, c->logits, N, E, d,
-                    c->status};
+  RouterTcParams tp{splits > 1 ? nullptr : bias, c->logits, N, E, d, nk / splits, c->status};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((N + kRtBM - 1) / kRtBM, E / kRtBN);
+  cfg.gridDim = dim3((N + kRtBM - 1) / kRtBM, E / kRtBN, splits);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = RtCfg::SMEM;
   cfg.stream = s;
@@ -797,6 +802,12 @@ bool launch_router_tc(moe_ctx *c, cudaStream_t s, const uint16_t *h, int N, int 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   *err = cudaLaunchKernelEx(&cfg, router_tc_kernel, hm, wm, lm, tp);
+  if (*err == cudaSuccess && splits > 1) {
+    const long long n4 = (long long)N * E / 4;
+    RouterSumParams sp{c->pf_part, splits, bias, N, E, c->logits};
+    *err = launch(router_sum_kernel, dim3((unsigned)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm)),
+                  dim3(256), 0, s, sp);
+  }
   return true;
 }
 

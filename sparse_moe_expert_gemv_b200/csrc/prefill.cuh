@@ -8,8 +8,8 @@
 //
 //   prefill_topk_kernel     one warp per token: top-k + softmax (candidate
 //                           filter, warp_topk_fast); per block of
-//                           16 tokens, each expert's token set (a bitmask)
-//   prefill_colscan_kernel  per expert: each block of 16 tokens' first row
+//                           kPfTok tokens, each expert's token set (a bitmask)
+//   prefill_colscan_kernel  per expert: each block of tokens' first row
 //                           relative to the expert's (a scan down the
 //                           expert's column of block masks) and its tokens
 //   prefill_scan_kernel     the experts' first rows in grouped order and the
@@ -37,7 +37,11 @@
 
 namespace moe {
 
-constexpr int kPfTok = 16;       // tokens per block of the top-k / scatter kernels (one warp each)
+// Tokens per block of the top-k / scatter kernels (one warp each; a block's
+// per-expert token set is a 16-bit mask).  Eight rather than 16: a top-k
+// CTA waits for its slowest token (the few with an exact refinement), and
+// 8-warp CTAs fit three to an SM instead of one.
+constexpr int kPfTok = 8;
 constexpr int kPfBM = 128;       // rows of one MMA (an M-half of a GEMM tile)
 constexpr int kPfTileRows = 2 * kPfBM;  // rows of one GEMM tile of an expert (two M-halves)
 constexpr int kPfBN = 128;       // GEMM tile columns (output features)
@@ -730,6 +734,14 @@ MOE_DEV void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+// 3-D TMA tile store from this CTA's shared memory (bulk-group completion).
+MOE_DEV void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
 // Wait until at most N of this thread's bulk groups still read shared memory.
 template <int N>
 MOE_DEV void bulk_wait_read() {
@@ -1169,9 +1181,10 @@ struct RtCfg {
 };
 
 struct RouterTcParams {
-  const float *bias;  // [E] or null
-  float *logits;      // [T, E]
+  const float *bias;  // [E] or null (null with a split reduction: router_sum_kernel adds it)
+  float *logits;      // [T, E] (written through the output map)
   int T, E, d;
+  int ksteps;         // 64-column reduction steps per split (blockIdx.z): 3 d / 64 / splits
   int *status;
 };
 
@@ -1229,7 +1242,8 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = s_tmem;
   pdl_wait();
   const int m0 = blockIdx.x * kRtBM, n0 = blockIdx.y * kRtBN;
-  const int nkh = p.d / 64, nk = 3 * nkh;
+  // this CTA's reduction steps [k0, k0 + nk) of the tripled reduction
+  const int nkh = p.d / 64, nk = p.ksteps, k0 = blockIdx.z * p.ksteps;
   auto stage_a = [&](int st) { return stage0 + (uint32_t)st * C::STAGE; };
   auto stage_b = [&](int st) { return stage0 + (uint32_t)st * C::STAGE + C::TILE_A; };
   auto aborted = [&]() { return *reinterpret_cast<volatile int *>(&s_abort) != 0; };
@@ -1248,8 +1262,8 @@ __global__ void __launch_bounds__(256, 1)
         }
         const uint32_t bar = smem_addr(&s_full[st]);
         mbar_expect_tx(bar, C::STAGE);
-        tma_load_2d(stage_a(st), &hmap, (ks % nkh) * 64, m0, bar);
-        tma_load_2d(stage_b(st), &wmap, ks * 64, n0, bar);
+        tma_load_2d(stage_a(st), &hmap, ((k0 + ks) % nkh) * 64, m0, bar);
+        tma_load_2d(stage_b(st), &wmap, (k0 + ks) * 64, n0, bar);
         issued = ks + 1;
       }
       // no tile may land in shared memory after the CTA has moved on
@@ -1306,7 +1320,7 @@ __global__ void __launch_bounds__(256, 1)
                        : "memory");
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && r0 < p.T) tma_store_2d(&lmap, sb, n0 + c0, r0);
+        if (lane == 0 && r0 < p.T) tma_store_3d(&lmap, sb, n0 + c0, r0, blockIdx.z);
       }
       if (lane == 0) bulk_wait_all();
     } else if (lane == 0) {
