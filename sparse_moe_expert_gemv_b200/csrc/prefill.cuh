@@ -552,6 +552,30 @@ MOE_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// The same 32 columns, issued without waiting: the registers hold the data
+// only after tmem_ld32_wait on them (which names them as operands, so no
+// use can move above the wait).
+#define MOE_R32(r)                                                                                         \
+  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),        \
+      "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), \
+      "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),          \
+      "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),          \
+      "+r"(r[30]), "+r"(r[31])
+MOE_DEV void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+MOE_DEV void tmem_ld32_wait(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : MOE_R32(r)::"memory");
+}
+
 // 2-D TMA tile load (x = element offset along the contiguous dimension, y = row)
 MOE_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -1079,23 +1103,40 @@ __global__ void __launch_bounds__(kPfGemmThreads, 1)
             tmem_ld32(lane_addr + h * 128 + c0, g);
             tmem_ld32(lane_addr + h * 128 + 64 + c0, u);
             uint32_t pk[16];
+            // SiLU(g) u with the fast divide: a is rounded to fp16 next, so
+            // its few-ulp fp32 error is invisible, and the IEEE divide made
+            // this epilogue as slow as the item's MMAs (for g below about
+            // -88 the denominator is inf and the quotient the correct 0)
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-              const float a0 = g[2 * q] / (1.0f + __expf(-g[2 * q])) * u[2 * q];
-              const float a1 = g[2 * q + 1] / (1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
+              const float a0 = __fdividef(g[2 * q], 1.0f + __expf(-g[2 * q])) * u[2 * q];
+              const float a1 = __fdividef(g[2 * q + 1], 1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
               asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(a1), "f"(a0));
             }
             emit(pk, n0 + c);
           }
         } else {
-          for (int c0 = 0; c0 < COLS; c0 += 32) {
-            float y[32];
-            tmem_ld32(lane_addr + c0, y);
+          // the next chunk's TMEM load is in flight while this one is
+          // converted and stored
+          uint32_t ra[32], rb[32];
+          auto put = [&](const uint32_t (&r)[32], int col) {
             uint32_t pk[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q)
-              asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(pk[q]) : "f"(y[2 * q + 1]), "f"(y[2 * q]));
-            emit(pk, n0 + c0);
+              asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
+                  : "=r"(pk[q])
+                  : "f"(__uint_as_float(r[2 * q + 1])), "f"(__uint_as_float(r[2 * q])));
+            emit(pk, col);
+          };
+          tmem_ld32_issue(lane_addr, ra);
+          tmem_ld32_wait(ra);
+          for (int c0 = 0; c0 < COLS; c0 += 64) {  // COLS is a multiple of 64
+            tmem_ld32_issue(lane_addr + c0 + 32, rb);
+            put(ra, n0 + c0);
+            tmem_ld32_wait(rb);
+            if (c0 + 64 < COLS) tmem_ld32_issue(lane_addr + c0 + 64, ra);
+            put(rb, n0 + c0 + 32);
+            if (c0 + 64 < COLS) tmem_ld32_wait(ra);
           }
         }
       }
