@@ -19,7 +19,10 @@ metric, each with its own roofline, end-to-end figure and clocks:
   "stack"    the 48-layer stack (RMSNorm -> router -> experts -> combine per
              layer, 4096-slot residency table), 32 tokens per step.
 (--no-extras drops them; --workload q2|prefill|stack makes one of them the
-headline instead.)
+headline instead.)  --workload tier runs the host tier: 4 layers whose
+experts are backed in pinned host memory, a 512-slot HBM cache, Zipf-routed
+16-token windows through moe_forward_tiered, both replacement policies and
+the all-HBM forward of the same windows (use it with --no-cpu-baseline).
 
 Contract: python bench.py --gpus N --steps K --warmup W [--impl reference];
 rank 0 prints one JSON line.  N > 1 runs N independent replicas (the layer
@@ -53,7 +56,7 @@ def parse():
                     help="timed steps (default 200 decode windows, 20 prefill chunks)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "q2", "prefill", "stack"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "q2", "prefill", "stack", "tier"])
     ap.add_argument("--T", type=int, default=4, help="window (decode) / per-sequence window (q2)")
     ap.add_argument("--rot-layers", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -66,7 +69,7 @@ def parse():
                     help="routed experts per layer (256: the pruned configuration)")
     a = ap.parse_args()
     if a.steps is None:
-        a.steps = {"prefill": 20, "stack": 10}.get(a.workload, 200)
+        a.steps = {"prefill": 20, "stack": 10, "tier": 100}.get(a.workload, 200)
     return a
 
 
@@ -713,6 +716,80 @@ def cpu_baseline(args, spec, seconds, on_gpu=True, norm=False, tokens=None, laye
                       f"host threads; {dt:.1f} s", **info}
 
 
+def run_tier(args, world, K, W):
+    """Host tier: the experts' backing copies in pinned host memory, a slot
+    pool of a quarter of the (layer, expert) pairs in HBM, Zipf-routed
+    windows through moe_forward_tiered (route, bring the misses in, forward);
+    both replacement policies, and the all-HBM forward of the same windows for
+    comparison.  Timed with CUDA events around the K windows (the miss path
+    synchronises the stream once per window to read the routing back)."""
+    import torch
+    from sparse_moe_expert_gemv_b200 import binding as B
+    from sparse_moe_expert_gemv_b200 import inputs as I
+    NL, T, slots = 4, 16, 512
+    xs = torch.from_numpy(np.stack([I.hidden_np(args.seed, T, D, window=i) for i in range(W + K)])
+                          .view(np.int16)).cuda()
+
+    def build(tier, policy):
+        ctx = B.moe_create(D, F, E, K_TOP, I.Q4)
+        if tier:
+            B.moe_set_host_tier(ctx, 1, policy, 64.0)
+        B.moe_configure(ctx, NL, 1, slots if tier else 0, T)
+        for l in range(NL):
+            B.moe_set_router(ctx, l, I.router_np(args.seed, E, D, l), I.zipf_bias_np(args.seed, E, l)[0])
+            for first in range(0, E, 64):
+                c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, l, first, 64, "cuda")
+                B.moe_load_experts(ctx, l, first, 64, c, s_, m)
+                del c, s_, m
+            c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, l, I.SHARED_INDEX, 1, "cuda")
+            B.moe_load_shared(ctx, l, c, s_, m)
+        torch.cuda.synchronize()
+        return ctx
+
+    def run(ctx, fwd):
+        work = xs.clone()
+        for i in range(W):
+            fwd(ctx, i % NL, work[i], T)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        st0 = B.moe_tier_stats(ctx) if fwd is B.moe_forward_tiered else None
+        e0.record()
+        for i in range(W, W + K):
+            fwd(ctx, i % NL, work[i], T)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        st1 = B.moe_tier_stats(ctx) if st0 else None
+        B.moe_sync(ctx, 60000)
+        return ms, (None if st0 is None else {k: st1[k] - st0[k] for k in st1})
+
+    out = {}
+    ctx = build(False, 0)
+    ms_hbm, _ = run(ctx, B.moe_forward)
+    B.moe_destroy(ctx)
+    for name, pol in (("lru", B.TIER_LRU), ("adaptive", B.TIER_ADAPTIVE)):
+        ctx = build(True, pol)
+        ms, d = run(ctx, B.moe_forward_tiered)
+        B.moe_destroy(ctx)
+        torch.cuda.empty_cache()
+        req = d["hits"] + d["misses"]
+        out[name] = {"value": K * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_window": ms / K,
+                     "hit_rate": d["hits"] / max(req, 1), "misses_per_window": d["misses"] / K,
+                     "h2d_gbs": d["bytes"] / (ms * 1e-3) / 1e9}
+    return {"metric": "tier MoE tokens/s", "value": out["adaptive"]["value"], "unit": "tokens/s",
+            "n_gpus": 1, "steps": K, "warmup": W, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "q4-g32 weights, bf16 activations, fp32 accumulate",
+            "data": "synthetic (seeded generator; random-init weights of the layer's shape)",
+            "config": {"workload": f"{NL} MoE layers, d=2048 f=768 E={E} top-10 + shared, Q4 g32, Zipf(1.1) "
+                                   f"routing, windows of T={T}; experts backed in pinned host memory, "
+                                   f"{slots} HBM slots ({slots / (NL * E):.0%} of the pairs)",
+                       "tokens_per_step": T, "parallelism": "1 GPU",
+                       "timing": "CUDA events around K moe_forward_tiered calls (each reads its routing back)"},
+            "policies": out,
+            "all_hbm": {"value": K * T / (ms_hbm * 1e-3), "unit": "tokens/s", "ms_per_window": ms_hbm / K},
+            "gpu_launches": None}
+
+
 def run_reference(args):
     """Reference arm: the oracle (scalar fp64 C) on the host cores, on the
     headline's workload: each step is one window of the workload's tokens
@@ -793,6 +870,8 @@ def main():
     spec = workload_spec(args.workload, args.T)
     if args.workload == "stack":
         res = run_stack(args, world, args.steps, args.warmup)
+    elif args.workload == "tier":
+        res = run_tier(args, world, args.steps, args.warmup)
     else:
         n_rot = args.rot_layers if args.workload == "decode" else min(args.rot_layers, 4)
         res = run_native(args, world, spec, n_rot, args.steps, args.warmup)

@@ -293,6 +293,72 @@ MOE_API moe_status moe_route_static(const void *h_dev, int T, int d, int E, int 
  * word is cleared by the next moe_route_static call. */
 MOE_API moe_status moe_route_static_status(int *status_out, void *stream);
 
+/* Host tier (the engine article "93 token/s on one 8 GB card", section
+ * "Expert cache": a model larger than the GPU keeps its hot experts in a
+ * fixed set of device slots, (layer, expert) -> slot or -1, and brings
+ * misses in while other work runs; the user report "EPYC 7B13 + 2x RTX 3090"
+ * makes that cache adaptive).  With the host tier, every expert's backing
+ * copy lives in pinned, mapped host memory, and the n_slots slots of
+ * moe_configure form an HBM cache over it.  The shared experts, routers and
+ * scratch stay in HBM.  Results are those of the all-HBM context bit for bit:
+ * residency only moves where an expert is read from.
+ *
+ * moe_set_host_tier: before moe_configure.  enable 0/1; policy 0 = least
+ * recently used, 1 = adaptive (an exponentially decayed use count with the
+ * given half-life in requests, ties by recency).  Errors: INVALID_ARG,
+ * STATE (already configured). */
+MOE_API moe_status moe_set_host_tier(moe_ctx *ctx, int enable, int policy, double half_life);
+
+/* moe_tier_prepare: make the experts a window selects resident.  idx_dev is
+ * the window's routing, int32 [T, k] on the device (e.g. from moe_route),
+ * written by work already queued on `stream`: the call waits for the stream,
+ * reads the ids back, gives each selected expert without a slot a slot (by
+ * the policy; never one the window itself uses), copies the missed experts
+ * host -> HBM on the context's copy stream with the changed slot-table rows
+ * after them, and makes `stream` wait for those copies.  A later forward of
+ * this window on `stream` then reads only HBM.  Errors: INVALID_ARG (bad
+ * arguments, or more distinct experts than slots), STATE (no host tier),
+ * DEVICE (an id outside [0, E)), CUDA. */
+MOE_API moe_status moe_tier_prepare(moe_ctx *ctx, int layer, const int32_t *idx_dev, int T,
+                                    void *stream);
+
+/* moe_tier_prefetch: as moe_tier_prepare, but the copies stay in flight
+ * (no stream waits for them; the next prepare or prefetch is ordered after
+ * them), so they overlap whatever runs meanwhile -- the pages stream the
+ * next layer's misses during the current layer's work.  The previous
+ * request's slots are not evicted either, since its window may still be
+ * running; other work in flight must only use experts of that request. */
+MOE_API moe_status moe_tier_prefetch(moe_ctx *ctx, int layer, const int32_t *idx_dev, int T,
+                                     void *stream);
+
+/* moe_forward_tiered: moe_forward with the miss path in front: the window's
+ * routing (with the layer's RMSNorm, as the forward computes it),
+ * moe_tier_prepare on it, then the forward.  Same arguments, results and
+ * errors as moe_forward, plus those of moe_tier_prepare. */
+MOE_API moe_status moe_forward_tiered(moe_ctx *ctx, int layer, void *x_dev, int T, void *stream);
+
+/* moe_tier_stats: out[0] hits, out[1] misses, out[2] evictions (distinct
+ * experts per request), out[3] bytes copied host -> HBM, out[4] requests,
+ * out[5] slots in use.  Errors: INVALID_ARG, STATE (no host tier). */
+MOE_API moe_status moe_tier_stats(moe_ctx *ctx, long long *out);
+
+/* moe_tier_dump_trace: write the routing trace of every request so far to a
+ * text file, one line per request: "request layer n expert...".  Errors:
+ * INVALID_ARG (cannot open or write), STATE (no host tier). */
+MOE_API moe_status moe_tier_dump_trace(moe_ctx *ctx, const char *path);
+
+/* Host-only model of the tier's replacement policy (no device involved), for
+ * policy studies and tests: a cache of n_slots slots over keys [0, n_keys).
+ * moe_tier_sim_request takes one request of n distinct keys, writes each
+ * key's slot into slots_out[n] (may be NULL) and returns the request's misses,
+ * -1 for bad arguments, -2 when the misses outnumber the slots that may be
+ * taken.  moe_tier_sim_counts writes hits, misses, evictions. */
+MOE_API void *moe_tier_sim_create(int n_slots, int policy, double half_life, long long n_keys);
+MOE_API int moe_tier_sim_request(void *sim, const long long *keys, int n, int protect_prev,
+                                 int *slots_out);
+MOE_API void moe_tier_sim_counts(void *sim, long long *out);
+MOE_API void moe_tier_sim_destroy(void *sim);
+
 /* Profiling: when enabled, every forward call records CUDA events on its
  * stream around its three segments -- routing (norm + router + top-k +
  * bucketing), experts (the two grouped dequant-GEMV kernels) and combine --

@@ -32,7 +32,10 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_debug_poke_slot", "moe_set_profiling", "moe_read_profile",
            "moe_set_trace", "moe_read_trace", "moe_route_static", "moe_prefill_delta",
            "moe_prefill_route", "moe_route_static_status", "moe_debug_last_h",
-           "moe_debug_stall_next_decode")
+           "moe_debug_stall_next_decode", "moe_set_host_tier", "moe_tier_prepare",
+           "moe_tier_prefetch", "moe_forward_tiered", "moe_tier_stats", "moe_tier_dump_trace",
+           "moe_tier_sim_create", "moe_tier_sim_request", "moe_tier_sim_counts",
+           "moe_tier_sim_destroy")
 
 
 class MoeError(RuntimeError):
@@ -83,6 +86,13 @@ def _load():
         "moe_route_static": [P, I, I, I, I, P, P, P, P, P, P, P],
         "moe_read_trace": [P, ctypes.POINTER(ctypes.c_int64), I],
         "moe_read_profile": [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
+        "moe_set_host_tier": [P, I, I, ctypes.c_double],
+        "moe_tier_prepare": [P, I, P, I, P],
+        "moe_tier_prefetch": [P, I, P, I, P],
+        "moe_forward_tiered": [P, I, P, I, P],
+        "moe_tier_stats": [P, ctypes.POINTER(ctypes.c_int64)],
+        "moe_tier_dump_trace": [P, ctypes.c_char_p],
+        "moe_tier_sim_request": [P, ctypes.POINTER(ctypes.c_int64), I, I, ctypes.POINTER(I)],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -94,6 +104,12 @@ def _load():
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_expert_bytes.argtypes = [I, I, I]
     L.moe_expert_bytes.restype = ctypes.c_int64
+    L.moe_tier_sim_create.argtypes = [I, I, ctypes.c_double, ctypes.c_int64]
+    L.moe_tier_sim_create.restype = P
+    L.moe_tier_sim_counts.argtypes = [P, ctypes.POINTER(ctypes.c_int64)]
+    L.moe_tier_sim_counts.restype = None
+    L.moe_tier_sim_destroy.argtypes = [P]
+    L.moe_tier_sim_destroy.restype = None
     return L
 
 
@@ -301,3 +317,70 @@ def moe_route_static_status(stream=None):
     if rc == 6:
         raise MoeError(rc, f"moe_route_static device status 0x{st.value:x}")
     return st.value
+
+
+# ------------------------------------------------------------- host tier
+TIER_LRU, TIER_ADAPTIVE = 0, 1
+
+
+def moe_set_host_tier(ctx, enable=1, policy=TIER_ADAPTIVE, half_life=64.0):
+    """Backing copies in pinned host memory, the slot pool as an HBM cache
+    (before moe_configure; see include/moe.h)."""
+    _check(ctx, _lib.moe_set_host_tier(ctx, int(enable), int(policy), float(half_life)))
+
+
+def moe_tier_prepare(ctx, layer, idx, T, stream=None):
+    _check(ctx, _lib.moe_tier_prepare(ctx, layer, _ptr(idx), T, _stream(stream)))
+
+
+def moe_tier_prefetch(ctx, layer, idx, T, stream=None):
+    _check(ctx, _lib.moe_tier_prefetch(ctx, layer, _ptr(idx), T, _stream(stream)))
+
+
+def moe_forward_tiered(ctx, layer, x, T, stream=None):
+    _check(ctx, _lib.moe_forward_tiered(ctx, layer, _ptr(x), T, _stream(stream)))
+
+
+def moe_tier_stats(ctx):
+    """{"hits", "misses", "evictions", "bytes", "requests", "slots_used"}"""
+    out = (ctypes.c_int64 * 6)()
+    _check(ctx, _lib.moe_tier_stats(ctx, out))
+    return dict(zip(("hits", "misses", "evictions", "bytes", "requests", "slots_used"), out))
+
+
+def moe_tier_dump_trace(ctx, path):
+    _check(ctx, _lib.moe_tier_dump_trace(ctx, os.fsencode(path)))
+
+
+class TierSim:
+    """Host-only model of the tier's replacement policy (moe_tier_sim_*)."""
+
+    def __init__(self, n_slots, policy, half_life, n_keys):
+        self.h = _lib.moe_tier_sim_create(n_slots, policy, float(half_life), n_keys)
+        if not self.h:
+            raise ValueError("moe_tier_sim_create: bad arguments")
+
+    def request(self, keys, protect_prev=False):
+        """(misses, slots) for one request of distinct keys; raises on -1 / -2."""
+        n = len(keys)
+        karr = (ctypes.c_int64 * max(n, 1))(*keys)
+        sarr = (ctypes.c_int * max(n, 1))()
+        r = _lib.moe_tier_sim_request(self.h, karr, n, int(protect_prev), sarr)
+        if r == -1:
+            raise ValueError("moe_tier_sim_request: bad arguments")
+        if r == -2:
+            raise MoeError(1, "the request needs more slots than may be taken")
+        return r, list(sarr[:n])
+
+    def counts(self):
+        out = (ctypes.c_int64 * 3)()
+        _lib.moe_tier_sim_counts(self.h, out)
+        return dict(zip(("hits", "misses", "evictions"), out))
+
+    def close(self):
+        if self.h:
+            _lib.moe_tier_sim_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        self.close()

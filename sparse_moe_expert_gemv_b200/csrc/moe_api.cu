@@ -12,6 +12,7 @@
 //   scratch sized for max_tokens tokens per call.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <chrono>
 #include <cstdarg>
 #include <cstdio>
@@ -27,6 +28,7 @@
 #include "decode.cuh"
 #include "kernels.cuh"
 #include "prefill.cuh"
+#include "tier.h"
 
 using namespace moe;
 
@@ -45,6 +47,19 @@ struct moe_ctx {
   uint8_t *arena = nullptr, *shared = nullptr, *pool = nullptr;
   int *d_slot_of = nullptr;
   std::vector<int> h_slot_of;
+  // host tier: the backing arena in pinned, mapped host memory and the slot
+  // pool as a cache over it (moe_set_host_tier)
+  int host_tier = 0, tier_policy = 0;
+  double tier_half_life = 64.0;
+  uint8_t *h_arena = nullptr;            // host address of the arena (host tier)
+  moe::TierCache tier;
+  cudaStream_t tier_stream = nullptr;    // host -> HBM expert copies
+  cudaEvent_t tier_done = nullptr;       // the latest copies and slot-table update
+  int32_t *tier_idx = nullptr;           // device [max_tokens * k] routing of the tiered forward
+  float *tier_w = nullptr;
+  int32_t *h_tier_idx = nullptr;         // pinned host copy of a window's routing
+  long long tier_bytes = 0, tier_calls = 0;
+  std::vector<int> tier_trace;           // per request: call, layer, n, then n expert ids
   float *d_router = nullptr, *d_bias = nullptr, *d_gamma = nullptr;
   __nv_bfloat16 *d_router3 = nullptr;  // [L][E][3d] exact bf16 parts of the router (prefill)
   std::vector<char> has_router, has_bias, has_norm, has_gamma, shared_loaded;
@@ -192,7 +207,21 @@ moe_status do_configure(moe_ctx *c) {
   const Layout &L = c->lay;
   const long long Be = L.expert_bytes;
   const int T = c->max_tokens, E = c->E, k = c->k, d = c->d, f = c->f;
-  CUDA_TRY(c, cudaMalloc(&c->arena, (size_t)c->L * E * Be));
+  if (c->host_tier) {
+    // every expert's backing copy in pinned host memory, mapped so that the
+    // kernels can still address it; the HBM slot pool caches it
+    CUDA_TRY(c, cudaHostAlloc((void **)&c->h_arena, (size_t)c->L * E * Be,
+                              cudaHostAllocMapped | cudaHostAllocPortable));
+    CUDA_TRY(c, cudaHostGetDevicePointer((void **)&c->arena, c->h_arena, 0));
+    CUDA_TRY(c, cudaStreamCreateWithFlags(&c->tier_stream, cudaStreamNonBlocking));
+    CUDA_TRY(c, cudaEventCreateWithFlags(&c->tier_done, cudaEventDisableTiming));
+    CUDA_TRY(c, cudaMalloc(&c->tier_idx, (size_t)T * k * sizeof(int32_t)));
+    CUDA_TRY(c, cudaMalloc(&c->tier_w, (size_t)T * k * sizeof(float)));
+    CUDA_TRY(c, cudaHostAlloc((void **)&c->h_tier_idx, (size_t)T * k * sizeof(int32_t), cudaHostAllocDefault));
+    c->tier.init(c->n_slots, c->tier_policy, c->tier_half_life, (long long)c->L * E);
+  } else {
+    CUDA_TRY(c, cudaMalloc(&c->arena, (size_t)c->L * E * Be));
+  }
   if (c->n_shared) CUDA_TRY(c, cudaMalloc(&c->shared, (size_t)c->L * Be));
   if (c->n_slots) CUDA_TRY(c, cudaMalloc(&c->pool, (size_t)c->n_slots * Be));
   CUDA_TRY(c, cudaMalloc(&c->d_slot_of, (size_t)c->L * E * sizeof(int)));
@@ -1095,9 +1124,61 @@ moe_status refresh_slots(moe_ctx *c, int layer, int first, int n) {
     if (slot >= 0)
       CUDA_TRY(c, cudaMemcpyAsync(c->pool + (size_t)slot * Be,
                                   c->arena + ((size_t)layer * c->E + e) * Be, (size_t)Be,
-                                  cudaMemcpyDeviceToDevice, c->io));
+                                  cudaMemcpyDefault, c->io));
   }
   CUDA_TRY(c, cudaStreamSynchronize(c->io));
+  return MOE_OK;
+}
+
+// One request of the host tier.  The window's routing (idx_dev [T, k], on
+// stream s) is read back once the stream's work is done; its distinct
+// experts are the request.  Each miss takes a slot by the cache's policy, its
+// expert is copied from the host arena into the slot on the tier stream, and
+// the slot-table rows that changed follow on the same stream.  With wait,
+// stream s waits for those copies; otherwise (a prefetch) they stay in
+// flight and the next request's wait covers them, and the previous
+// request's slots are protected from eviction (its window may still run).
+moe_status tier_request(moe_ctx *c, int layer, const int32_t *idx_dev, int T, cudaStream_t s, bool wait) {
+  const int E = c->E, k = c->k;
+  const long long Be = c->lay.expert_bytes;
+  CUDA_TRY(c, cudaMemcpyAsync(c->h_tier_idx, idx_dev, (size_t)T * k * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(c, cudaStreamSynchronize(s));
+  std::vector<char> seen(E, 0);
+  std::vector<long long> keys;
+  for (int i = 0; i < T * k; ++i) {
+    const int e = c->h_tier_idx[i];
+    if (e < 0 || e >= E) return fail(c, MOE_ERR_DEVICE, "routing id %d out of range", e);
+    if (!seen[e]) {
+      seen[e] = 1;
+      keys.push_back((long long)layer * E + e);
+    }
+  }
+  std::sort(keys.begin(), keys.end());
+  std::vector<long long> fill_key, fill_ev;
+  std::vector<int> fill_slot;
+  if (!c->tier.request(keys, c->h_slot_of, !wait, fill_key, fill_slot, fill_ev))
+    return fail(c, MOE_ERR_INVALID_ARG, "the window needs %zu experts resident; the pool has %d slots",
+                keys.size(), c->n_slots);
+  ++c->tier_calls;
+  c->tier_trace.push_back((int)c->tier_calls);
+  c->tier_trace.push_back(layer);
+  c->tier_trace.push_back((int)keys.size());
+  for (long long key : keys) c->tier_trace.push_back((int)(key - (long long)layer * E));
+  std::vector<char> dirty(c->L, 0);
+  for (size_t i = 0; i < fill_key.size(); ++i) {
+    CUDA_TRY(c, cudaMemcpyAsync(c->pool + (size_t)fill_slot[i] * Be, c->h_arena + (size_t)fill_key[i] * Be,
+                                (size_t)Be, cudaMemcpyHostToDevice, c->tier_stream));
+    c->tier_bytes += Be;
+    dirty[fill_key[i] / E] = 1;
+    if (fill_ev[i] >= 0) dirty[fill_ev[i] / E] = 1;
+  }
+  // pageable source: the call returns once the row has been staged
+  for (int l = 0; l < c->L; ++l)
+    if (dirty[l])
+      CUDA_TRY(c, cudaMemcpyAsync(c->d_slot_of + (size_t)l * E, c->h_slot_of.data() + (size_t)l * E,
+                                  (size_t)E * sizeof(int), cudaMemcpyHostToDevice, c->tier_stream));
+  CUDA_TRY(c, cudaEventRecord(c->tier_done, c->tier_stream));
+  if (wait) CUDA_TRY(c, cudaStreamWaitEvent(s, c->tier_done, 0));
   return MOE_OK;
 }
 
@@ -1201,7 +1282,17 @@ moe_status moe_destroy(moe_ctx *c) {
   for (auto &kv : c->stack_graphs) cudaGraphExecDestroy(kv.second);
   for (cudaEvent_t ev : c->prof_ev) cudaEventDestroy(ev);
   dfree(c->pf);
+  if (c->h_arena) {
+    cudaFreeHost(c->h_arena);
+    c->h_arena = nullptr;
+    c->arena = nullptr;
+  }
   dfree(c->arena);
+  dfree(c->tier_idx);
+  dfree(c->tier_w);
+  if (c->h_tier_idx) cudaFreeHost(c->h_tier_idx);
+  if (c->tier_done) cudaEventDestroy(c->tier_done);
+  if (c->tier_stream) cudaStreamDestroy(c->tier_stream);
   dfree(c->shared);
   dfree(c->pool);
   dfree(c->d_slot_of);
@@ -1313,6 +1404,7 @@ moe_status moe_set_slots(moe_ctx *c, const int32_t *slot_of) {
     }
   }
   c->h_slot_of.assign(slot_of, slot_of + n);
+  if (c->host_tier) c->tier.adopt(c->h_slot_of);
   CUDA_TRY(c, cudaMemcpy(c->d_slot_of, slot_of, n * sizeof(int), cudaMemcpyHostToDevice));
   for (int l = 0; l < c->L; ++l) {
     st = refresh_slots(c, l, 0, c->E);
@@ -1343,6 +1435,128 @@ moe_status moe_route(moe_ctx *c, int layer, const void *h, int T, int32_t *idx, 
   c->has_norm[layer] = saved;
   return st;
 }
+
+moe_status moe_set_host_tier(moe_ctx *c, int enable, int policy, double half_life) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->configured) return fail(c, MOE_ERR_STATE, "moe_set_host_tier after configuration/loads");
+  if ((enable != 0 && enable != 1) || (policy != moe::kLru && policy != moe::kAdaptive) || !(half_life > 0))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_set_host_tier: bad arguments");
+  c->host_tier = enable;
+  c->tier_policy = policy;
+  c->tier_half_life = half_life;
+  return MOE_OK;
+}
+
+moe_status moe_tier_prepare(moe_ctx *c, int layer, const int32_t *idx_dev, int T, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured || !c->host_tier) return fail(c, MOE_ERR_STATE, "moe_tier_prepare: no host tier");
+  if (!valid_layer(c, layer) || !idx_dev || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_tier_prepare: bad arguments");
+  return tier_request(c, layer, idx_dev, T, (cudaStream_t)stream, true);
+}
+
+moe_status moe_tier_prefetch(moe_ctx *c, int layer, const int32_t *idx_dev, int T, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured || !c->host_tier) return fail(c, MOE_ERR_STATE, "moe_tier_prefetch: no host tier");
+  if (!valid_layer(c, layer) || !idx_dev || T < 1 || T > c->max_tokens)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_tier_prefetch: bad arguments");
+  return tier_request(c, layer, idx_dev, T, (cudaStream_t)stream, false);
+}
+
+moe_status moe_forward_tiered(moe_ctx *c, int layer, void *x, int T, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured || !c->host_tier) return fail(c, MOE_ERR_STATE, "moe_forward_tiered: no host tier");
+  if (!valid_layer(c, layer) || !x || T < 1 || T > c->max_tokens || !aligned16(x))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_forward_tiered: bad arguments");
+  moe_status st = check_ready(c, layer);
+  if (st) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  // the window's routing (with the layer's RMSNorm, as the forward computes it)
+  FinishParams fp = finish_params(c, layer, T);
+  fp.idx = c->tier_idx;
+  fp.w = c->tier_w;
+  fp.off = c->off;
+  fp.perm = c->perm;
+  fp.build_jobs = 0;
+  st = route_impl(c, layer, (const uint16_t *)x, T, fp, s, nullptr);
+  if (st) return st;
+  st = tier_request(c, layer, c->tier_idx, T, s, true);
+  if (st) return st;
+  return forward_impl(c, layer, (uint16_t *)x, T, nullptr, s);
+}
+
+moe_status moe_tier_stats(moe_ctx *c, long long *out) {
+  if (!c || !out) return MOE_ERR_INVALID_ARG;
+  if (!c->host_tier) return fail(c, MOE_ERR_STATE, "moe_tier_stats: no host tier");
+  int used = 0;
+  for (long long o : c->tier.owner) used += o >= 0 ? 1 : 0;
+  out[0] = c->tier.hits;
+  out[1] = c->tier.misses;
+  out[2] = c->tier.evictions;
+  out[3] = c->tier_bytes;
+  out[4] = c->tier_calls;
+  out[5] = used;
+  return MOE_OK;
+}
+
+moe_status moe_tier_dump_trace(moe_ctx *c, const char *path) {
+  if (!c || !path) return MOE_ERR_INVALID_ARG;
+  if (!c->host_tier) return fail(c, MOE_ERR_STATE, "moe_tier_dump_trace: no host tier");
+  FILE *fh = fopen(path, "w");
+  if (!fh) return fail(c, MOE_ERR_INVALID_ARG, "cannot open %s", path);
+  fprintf(fh, "# request layer n_experts experts...\n");
+  const std::vector<int> &tr = c->tier_trace;
+  for (size_t i = 0; i + 3 <= tr.size();) {
+    const int n = tr[i + 2];
+    fprintf(fh, "%d %d %d", tr[i], tr[i + 1], n);
+    for (int j = 0; j < n; ++j) fprintf(fh, " %d", tr[i + 3 + j]);
+    fprintf(fh, "\n");
+    i += 3 + (size_t)n;
+  }
+  const bool ok = fclose(fh) == 0;
+  return ok ? MOE_OK : fail(c, MOE_ERR_INVALID_ARG, "cannot write %s", path);
+}
+
+// Host-only model of the tier's replacement policy (no device needed).
+typedef std::pair<moe::TierCache, std::vector<int>> TierSim;
+
+void *moe_tier_sim_create(int n_slots, int policy, double half_life, long long n_keys) {
+  if (n_slots < 1 || n_keys < 1 || (policy != moe::kLru && policy != moe::kAdaptive) || !(half_life > 0))
+    return nullptr;
+  TierSim *sim = new TierSim();
+  sim->first.init(n_slots, policy, half_life, n_keys);
+  sim->second.assign((size_t)n_keys, -1);
+  return sim;
+}
+
+int moe_tier_sim_request(void *h, const long long *keys, int n, int protect_prev, int *slots_out) {
+  TierSim *sim = static_cast<TierSim *>(h);
+  if (!sim || (!keys && n > 0) || n < 0) return -1;
+  std::vector<long long> ks;
+  std::vector<char> seen(sim->second.size(), 0);
+  for (int i = 0; i < n; ++i) {
+    if (keys[i] < 0 || keys[i] >= (long long)sim->second.size() || seen[(size_t)keys[i]]) return -1;
+    seen[(size_t)keys[i]] = 1;
+    ks.push_back(keys[i]);
+  }
+  std::vector<long long> fk, fe;
+  std::vector<int> fs;
+  if (!sim->first.request(ks, sim->second, protect_prev != 0, fk, fs, fe)) return -2;
+  if (slots_out)
+    for (int i = 0; i < n; ++i) slots_out[i] = sim->second[(size_t)keys[i]];
+  return (int)fk.size();  // misses of this request
+}
+
+void moe_tier_sim_counts(void *h, long long *out) {
+  TierSim *sim = static_cast<TierSim *>(h);
+  if (!sim || !out) return;
+  out[0] = sim->first.hits;
+  out[1] = sim->first.misses;
+  out[2] = sim->first.evictions;
+}
+
+void moe_tier_sim_destroy(void *h) { delete static_cast<TierSim *>(h); }
 
 moe_status moe_bucket(moe_ctx *c, const int32_t *idx, int T, int32_t *boff, int32_t *bperm,
                       void *stream) {
