@@ -244,6 +244,72 @@ MOE_API moe_status moe_prefill_route(moe_ctx *ctx, int layer, const void *h_dev,
                                      int32_t *idx_dev, float *w_dev, int32_t *bucket_off_dev,
                                      int32_t *bucket_perm_dev, void *stream);
 
+/* moe_rmsnorm: the router input of `layer` for T tokens, h = RMSNorm(x)
+ * as moe_forward and moe_prefill compute it (h = bf16(x (mean(x^2) +
+ * eps)^-1/2 gamma), fp32 inside), or a copy of x when the layer has no
+ * norm.  x_dev, h_dev: bf16 [T, d], 16-byte aligned, caller-owned; T >= 1
+ * (no scratch is used).  Errors: INVALID_ARG, STATE (not configured). */
+MOE_API moe_status moe_rmsnorm(moe_ctx *ctx, int layer, const void *x_dev, int T, void *h_dev,
+                               void *stream);
+
+/* moe_experts_given: the experts of `layer` on caller-given routing, with
+ * the chunk path's kernels (bucketing by expert, grouped tcgen05 GEMM for
+ * experts with at least 16 rows, GEMV for the others, combine): the
+ * "experts by residency, then combine" half of the engine article's
+ * per-layer flow ("93 token/s on one 8 GB card", section "Architecture
+ * overview") without its router.  It is what an expert-parallel owner runs
+ * on the rows it receives.
+ *   h_dev    bf16 [N, d] router input rows (already normalised; no RMSNorm here)
+ *   idx_dev  int32 [N, kk] expert ids, distinct within a row, each expert loaded
+ *   w_dev    fp32 [N, kk] weights
+ *   kk       0..k experts per row (0: shared expert only)
+ *   with_shared  1: add the shared expert's output (the context must have one)
+ *   delta_dev fp32 [N, d] receives sum_j w[t,j] y_j(h_t) (+ y_shared(h_t)),
+ *            j in order, with the arithmetic of moe_prefill_delta.
+ * Every buffer is caller-owned device memory, 16-byte aligned where it
+ * holds rows.  N <= max_tokens.  The ids are copied to the host and checked
+ * before any launch (the call synchronizes `stream` once).  Errors:
+ * INVALID_ARG (bad sizes or pointers, an id outside [0, E), a repeated id
+ * in a row), STATE (an expert or the shared expert not loaded),
+ * NOT_SUPPORTED (context configured with max_tokens <= 32, or shapes the
+ * grouped GEMM does not take: d a multiple of 256, f of 128, E <= 1024). */
+MOE_API moe_status moe_experts_given(moe_ctx *ctx, int layer, const void *h_dev, int N, int kk,
+                                     const int32_t *idx_dev, const float *w_dev, int with_shared,
+                                     float *delta_dev, void *stream);
+
+/* Expert parallelism over n_ranks ranks: expert e belongs to rank
+ * e / (E / n_ranks) (E a multiple of n_ranks, n_ranks <= 64).
+ *
+ * moe_ep_dispatch: the send side of the exchange for N tokens routed by
+ * idx_dev int32 [N, k] (this context's k and E): every pair q = t k + j is
+ * sent to its expert's owner.  Writes, in device memory the caller owns:
+ *   send_h_dev  bf16 [N k, d]: the router-input row h_dev[t] of each sent
+ *               pair, grouped by destination rank (rank 0 first), ascending
+ *               pair id inside a rank's segment;
+ *   send_e_dev  int32 [N k]: the pair's expert id at the same position;
+ *   row_of_dev  int32 [N k]: the send position of pair q (-1: id outside
+ *               [0, E), not sent; the device status is set and moe_sync
+ *               reports DEVICE);
+ * and counts_host int32 [n_ranks] (host memory): rows for each rank, the
+ * all-to-all's send split.  h_dev bf16 [N, d].  Synchronizes `stream`
+ * (the counts are read back).  Errors: INVALID_ARG, STATE. */
+MOE_API moe_status moe_ep_dispatch(moe_ctx *ctx, const int32_t *idx_dev, int N, int n_ranks,
+                                   const void *h_dev, void *send_h_dev, int32_t *send_e_dev,
+                                   int32_t *row_of_dev, int32_t *counts_host, void *stream);
+
+/* moe_ep_combine: the receive side.  y_dev fp32 [rows, d]: the expert
+ * outputs returned by the owners, in send order (row_of_dev from
+ * moe_ep_dispatch maps pair q to its row); w_dev fp32 [N, k];
+ * y_shared_dev fp32 [N, d] (the shared expert's output, e.g. from
+ * moe_experts_given with kk = 0) or NULL.  Exactly one of x_dev (bf16
+ * [N, d], updated in place: x <- bf16(x + acc)) and delta_dev (fp32 [N, d]
+ * <- acc) is non-NULL; acc = sum_j w[t,j] y[row_of(t,j)] + y_shared[t],
+ * j in order, the one-GPU combine's arithmetic, so an expert-parallel layer
+ * matches moe_prefill bit for bit.  Errors: INVALID_ARG. */
+MOE_API moe_status moe_ep_combine(moe_ctx *ctx, int N, const float *w_dev, const float *y_dev,
+                                  const int32_t *row_of_dev, const float *y_shared_dev, void *x_dev,
+                                  float *delta_dev, void *stream);
+
 /* moe_sync: wait (polling cudaEventQuery, at most timeout_ms; < 0 = no
  * limit) until the work queued by this context has finished, then read and
  * clear the device error status.  Returns TIMEOUT, BAD_SLOT, DEVICE, CUDA or

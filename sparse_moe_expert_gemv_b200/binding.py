@@ -20,6 +20,8 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_OOM", 3: "MOE_ERR_CUDA",
                 4: "MOE_ERR_STATE", 5: "MOE_ERR_BAD_SLOT", 6: "MOE_ERR_DEVICE",
                 7: "MOE_ERR_TIMEOUT", 8: "MOE_ERR_NOT_SUPPORTED"}
+(MOE_ERR_INVALID_ARG, MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_STATE, MOE_ERR_BAD_SLOT,
+ MOE_ERR_DEVICE, MOE_ERR_TIMEOUT, MOE_ERR_NOT_SUPPORTED) = range(1, 9)
 MOE_Q4_SYM_G32_F16 = 1
 MOE_Q2_ASYM_G64_F16 = 2
 
@@ -35,7 +37,8 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_debug_stall_next_decode", "moe_set_host_tier", "moe_tier_prepare",
            "moe_tier_prefetch", "moe_forward_tiered", "moe_tier_stats", "moe_tier_dump_trace",
            "moe_tier_sim_create", "moe_tier_sim_request", "moe_tier_sim_counts",
-           "moe_tier_sim_destroy")
+           "moe_tier_sim_destroy", "moe_rmsnorm", "moe_experts_given", "moe_ep_dispatch",
+           "moe_ep_combine")
 
 
 class MoeError(RuntimeError):
@@ -93,6 +96,10 @@ def _load():
         "moe_tier_stats": [P, ctypes.POINTER(ctypes.c_int64)],
         "moe_tier_dump_trace": [P, ctypes.c_char_p],
         "moe_tier_sim_request": [P, ctypes.POINTER(ctypes.c_int64), I, I, ctypes.POINTER(I)],
+        "moe_rmsnorm": [P, I, P, I, P, P],
+        "moe_experts_given": [P, I, P, I, I, P, P, I, P, P],
+        "moe_ep_dispatch": [P, P, I, I, P, P, P, P, ctypes.POINTER(ctypes.c_int32), P],
+        "moe_ep_combine": [P, I, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -230,6 +237,28 @@ def moe_prefill_delta(ctx, layer, x, N, delta, stream=None):
 def moe_prefill_route(ctx, layer, h, N, idx, w, bucket_off=None, bucket_perm=None, stream=None):
     _check(ctx, _lib.moe_prefill_route(ctx, layer, _ptr(h), N, _ptr(idx), _ptr(w),
                                        _ptr(bucket_off), _ptr(bucket_perm), _stream(stream)))
+
+
+def moe_rmsnorm(ctx, layer, x, T, h, stream=None):
+    _check(ctx, _lib.moe_rmsnorm(ctx, layer, _ptr(x), T, _ptr(h), _stream(stream)))
+
+
+def moe_experts_given(ctx, layer, h, N, kk, idx, w, with_shared, delta, stream=None):
+    _check(ctx, _lib.moe_experts_given(ctx, layer, _ptr(h), N, kk, _ptr(idx), _ptr(w),
+                                       int(bool(with_shared)), _ptr(delta), _stream(stream)))
+
+
+def moe_ep_dispatch(ctx, idx, N, n_ranks, h, send_h, send_e, row_of, stream=None):
+    """Returns the rows sent to each rank (a list of n_ranks ints)."""
+    counts = (ctypes.c_int32 * n_ranks)()
+    _check(ctx, _lib.moe_ep_dispatch(ctx, _ptr(idx), N, n_ranks, _ptr(h), _ptr(send_h),
+                                     _ptr(send_e), _ptr(row_of), counts, _stream(stream)))
+    return list(counts)
+
+
+def moe_ep_combine(ctx, N, w, y, row_of, y_shared=None, x=None, delta=None, stream=None):
+    _check(ctx, _lib.moe_ep_combine(ctx, N, _ptr(w), _ptr(y), _ptr(row_of), _ptr(y_shared),
+                                    _ptr(x), _ptr(delta), _stream(stream)))
 
 
 def moe_sync(ctx, timeout_ms=-1):

@@ -28,6 +28,7 @@
 #include "decode.cuh"
 #include "kernels.cuh"
 #include "prefill.cuh"
+#include "ep.cuh"
 #include "tier.h"
 
 using namespace moe;
@@ -75,6 +76,7 @@ struct moe_ctx {
   int *job_beg = nullptr, *job_n = nullptr, *n_jobs = nullptr;
   uint16_t *hbuf = nullptr, *abuf = nullptr;
   int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
+  int *ep_counts = nullptr;  // [kEpMaxRanks] rows per rank of the last expert-parallel dispatch
   unsigned int *ticket = nullptr;    // fused routing: [0] CTA counter, [1] abort flag
   // single-launch decode kernel: grid barrier counter, hand-over flags and
   // partial sums (one slot per warp of the grid)
@@ -861,6 +863,9 @@ bool use_prefill_gemm(const moe_ctx *c, int N) {
 // ascending t), the 256-row tile list with the residency lookup, and the
 // gather of the grouped fp16 A rows.  perm (or null) receives the bucket
 // permutation; the bucket offsets are left in c->pf_eoff.
+moe_status pf_bucket_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int kk, const int32_t *idx,
+                          bool with_shared, int32_t *perm, cudaStream_t s, int hot_min);
+
 moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int32_t *idx, float *w,
                               int32_t *perm, cudaStream_t s, int hot_min) {
   const int E = c->E, k = c->k, d = c->d;
@@ -871,16 +876,27 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
     CUDA_TRY(c, e);
   else  // small expert counts or chunks: fp32 FMA
     CUDA_TRY(c, launch_router_fma(c, s, h, N, layer, &ks));
-  const int blocks = (N + kPfTok - 1) / kPfTok;
   PfRouteParams tp{c->logits, N, E, k, idx, w, c->pf_bmask, &c->stats[4], bias, h,
                    c->d_router + (size_t)layer * E * d, d};
   CUDA_TRY(c, launch_pf_topk(c, s, tp));
+  return pf_bucket_impl(c, layer, h, N, k, idx, c->n_shared != 0, perm, s, hot_min);
+}
+
+// The chunk's pairs sorted by expert from the block masks in c->pf_bmask
+// (the top-k's, or prefill_mask_kernel's for given routing): bucket
+// offsets, the GEMM tile and GEMV job lists with the residency lookup, and
+// the grouped fp16 A rows.  kk: experts per token; with_shared adds the
+// shared expert's T rows after the routed ones.
+moe_status pf_bucket_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int kk, const int32_t *idx,
+                          bool with_shared, int32_t *perm, cudaStream_t s, int hot_min) {
+  const int E = c->E, d = c->d;
+  const int blocks = (N + kPfTok - 1) / kPfTok;
   PfScanParams sp{};
   sp.bmask = c->pf_bmask;
   sp.blocks = blocks;
   sp.E = E;
   sp.T = N;
-  sp.k = k;
+  sp.k = kk;
   sp.boff = c->pf_boff;
   sp.eoff = c->pf_eoff;
   sp.slot_of = c->d_slot_of;
@@ -888,7 +904,7 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   sp.layer = layer;
   sp.arena = c->arena;
   sp.pool = c->pool;
-  sp.shared = c->n_shared ? c->shared + (size_t)layer * c->lay.expert_bytes : nullptr;
+  sp.shared = with_shared ? c->shared + (size_t)layer * c->lay.expert_bytes : nullptr;
   sp.expert_bytes = c->lay.expert_bytes;
   sp.tiles = c->pf_tiles;
   sp.n_tiles = c->pf_ntiles;
@@ -907,7 +923,7 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   sp.status = c->status;
   CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32), dim3(kPfColWarps * 32), 0, s, sp));
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
-  PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, k, d, c->n_shared,
+  PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, kk, d, with_shared ? 1 : 0,
                      c->pf_row_of, c->pf_hg, perm ? perm : c->pf_perm, c->pf_hot};
   // small chunks split each token row's columns over more CTAs
   const int ysplit = std::max(1, std::min(d / 256, (2 * c->n_sm + blocks - 1) / blocks));
@@ -915,46 +931,44 @@ moe_status prefill_route_impl(moe_ctx *c, int layer, const uint16_t *h, int N, i
   return MOE_OK;
 }
 
-moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta, cudaStream_t s) {
-  const int k = c->k, d = c->d, f = c->f;
-  if (!c->pf_maps) {
-    if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
-        !encode_map_f16(&c->pf_map_a, c->pf_a16, c->pf_rows, f) ||
-        !encode_out_map_f16(&c->pf_omap_a, c->pf_a16, c->pf_rows, f) ||
-        !encode_out_map_f16(&c->pf_omap_y, c->pf_y16, c->pf_rows, d))
-      return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    c->pf_maps = true;
-  }
-  CUDA_TRY(c, prof_mark(c, 0, s));
-  cudaError_t e = cudaSuccess;
-  const uint16_t *h = router_input(c, layer, x, N, s, &e);
-  CUDA_TRY(c, e);
-  moe_status st = prefill_route_impl(c, layer, h, N, c->idx, c->w, c->pf_perm, s, kHotMinTokens);
-  if (st) return st;
-  CUDA_TRY(c, prof_mark(c, 1, s));
-  // experts with many tokens: grouped GEMM over 256-row tiles; the others:
-  // the GEMV over jobs of <= 8 tokens, rows read through the bucket
-  // permutation (grouped row -> pair id)
+// Tensor maps of the grouped GEMM's operands (encoded once per context).
+moe_status pf_maps(moe_ctx *c) {
+  if (c->pf_maps) return MOE_OK;
+  const int d = c->d, f = c->f;
+  if (!encode_map_f16(&c->pf_map_h, c->pf_hg, c->pf_rows, d) ||
+      !encode_map_f16(&c->pf_map_a, c->pf_a16, c->pf_rows, f) ||
+      !encode_out_map_f16(&c->pf_omap_a, c->pf_a16, c->pf_rows, f) ||
+      !encode_out_map_f16(&c->pf_omap_y, c->pf_y16, c->pf_rows, d))
+    return fail(c, MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  c->pf_maps = true;
+  return MOE_OK;
+}
+
+// The experts of a bucketed chunk: experts with many tokens run as the
+// grouped GEMM over 256-row tiles, the others as the GEMV over jobs of <= 8
+// tokens, rows read through the bucket permutation (grouped row -> pair
+// id).  h: the router input the pairs' rows come from; kk: experts per token.
+moe_status pf_experts_impl(moe_ctx *c, const uint16_t *h, int N, int kk, cudaStream_t s) {
   GemvParams g1{};
   g1.job_ptr = c->job_ptr;
   g1.job_beg = c->job_beg;
   g1.job_n = c->job_n;
   g1.n_jobs = c->n_jobs;
   g1.plist = c->pf_perm;
-  g1.Tk = N * k;
-  g1.k = k;
+  g1.Tk = N * kk;
+  g1.k = kk > 0 ? kk : 1;  // kk == 0: no routed pairs, so no GEMV jobs
   g1.src = h;
   g1.src_by_pair = 0;
-  g1.K = d;
-  g1.R = f;
+  g1.K = c->d;
+  g1.R = c->f;
   g1.region_off = 0;
   g1.out_a = c->abuf;
   g1.status = c->status;
   GemvParams g2 = g1;
   g2.src = c->abuf;
   g2.src_by_pair = 1;
-  g2.K = f;
-  g2.R = d;
+  g2.K = c->f;
+  g2.R = c->d;
   g2.region_off = c->lay.p1_bytes;
   g2.out_a = nullptr;
   g2.out_y = c->ybuf;
@@ -965,17 +979,61 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
     CUDA_TRY(c, launch_prefill_gemms<2>(c, s));
     CUDA_TRY(c, launch_experts<2>(c, s, kColdChunk, g1, g2));
   }
-  CUDA_TRY(c, prof_mark(c, 2, s));
-  PfCombineParams mp{c->pf_y16, c->ybuf, c->w, c->pf_row_of, N, k, d, c->n_shared, x, delta};
+  return MOE_OK;
+}
+
+// x[t] <- bf16(x[t] + sum_j w[t,j] y(t,j) + y_shared[t]) (delta == null) or
+// delta[t] <- the same sum, from the chunk's grouped outputs.
+moe_status pf_combine_impl(moe_ctx *c, int N, int kk, const float *w, bool with_shared, uint16_t *x,
+                           float *delta, cudaStream_t s) {
+  const int d = c->d;
+  PfCombineParams mp{c->pf_y16, c->ybuf, w, c->pf_row_of, N, kk, d, with_shared ? 1 : 0, x, delta};
   const long long n4 = (long long)N * d / 4;
   const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
   CUDA_TRY(c, launch(prefill_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));
+  return MOE_OK;
+}
+
+moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta, cudaStream_t s) {
+  const int k = c->k;
+  moe_status st = pf_maps(c);
+  if (st) return st;
+  CUDA_TRY(c, prof_mark(c, 0, s));
+  cudaError_t e = cudaSuccess;
+  const uint16_t *h = router_input(c, layer, x, N, s, &e);
+  CUDA_TRY(c, e);
+  st = prefill_route_impl(c, layer, h, N, c->idx, c->w, c->pf_perm, s, kHotMinTokens);
+  if (st) return st;
+  CUDA_TRY(c, prof_mark(c, 1, s));
+  st = pf_experts_impl(c, h, N, k, s);
+  if (st) return st;
+  CUDA_TRY(c, prof_mark(c, 2, s));
+  st = pf_combine_impl(c, N, k, c->w, c->n_shared != 0, x, delta, s);
+  if (st) return st;
   CUDA_TRY(c, prof_mark(c, 3, s));
   if (c->profiling) {
     c->prof_next = (c->prof_next + 1) % kProfSlots;
     c->prof_pending = std::min(c->prof_pending + 1, kProfSlots);
   }
   return MOE_OK;
+}
+
+// The experts of a chunk on caller-given routing (the rows an
+// expert-parallel owner received, or any precomputed routing): block masks
+// from idx, then the chunk path's bucketing, experts and combine into
+// delta.  idx was checked on the host (ids in [0, E), distinct per token).
+moe_status given_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int kk, const int32_t *idx,
+                      const float *w, bool with_shared, float *delta, cudaStream_t s) {
+  moe_status st = pf_maps(c);
+  if (st) return st;
+  const int blocks = (N + kPfTok - 1) / kPfTok;
+  PfMaskParams mp{idx, N, c->E, kk, c->pf_bmask};
+  CUDA_TRY(c, launch(prefill_mask_kernel, dim3(blocks), dim3(kPfTok * 32), 0, s, mp));
+  st = pf_bucket_impl(c, layer, h, N, kk, idx, with_shared, c->pf_perm, s, kHotMinTokens);
+  if (st) return st;
+  st = pf_experts_impl(c, h, N, kk, s);
+  if (st) return st;
+  return pf_combine_impl(c, N, kk, w, with_shared, nullptr, delta, s);
 }
 
 // The whole decode chain for one layer.  delta == nullptr: residual mode.
@@ -1282,6 +1340,7 @@ moe_status moe_destroy(moe_ctx *c) {
   for (auto &kv : c->stack_graphs) cudaGraphExecDestroy(kv.second);
   for (cudaEvent_t ev : c->prof_ev) cudaEventDestroy(ev);
   dfree(c->pf);
+  dfree(c->ep_counts);
   if (c->h_arena) {
     cudaFreeHost(c->h_arena);
     c->h_arena = nullptr;
@@ -1685,6 +1744,102 @@ moe_status moe_prefill_route(moe_ctx *c, int layer, const void *h, int N, int32_
   if (boff)
     CUDA_TRY(c, cudaMemcpyAsync(boff, c->pf_eoff, (size_t)(c->E + 1) * sizeof(int32_t),
                                 cudaMemcpyDeviceToDevice, s));
+  return MOE_OK;
+}
+
+moe_status moe_rmsnorm(moe_ctx *c, int layer, const void *x, int T, void *h, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !x || !h || T < 1 || !aligned16(x) || !aligned16(h))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_rmsnorm: bad arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  if (!c->has_norm[layer]) {
+    CUDA_TRY(c, cudaMemcpyAsync(h, x, (size_t)T * c->d * 2, cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+  }
+  NormParams np{(const uint16_t *)x, c->has_gamma[layer] ? c->d_gamma + (size_t)layer * c->d : nullptr,
+                c->eps[layer], T, c->d, (uint16_t *)h};
+  CUDA_TRY(c, launch(rmsnorm_kernel, dim3(T), dim3(256), 0, s, np));
+  return MOE_OK;
+}
+
+moe_status moe_experts_given(moe_ctx *c, int layer, const void *h, int N, int kk, const int32_t *idx,
+                             const float *w, int with_shared, float *delta, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  if (!valid_layer(c, layer) || !h || !delta || N < 1 || N > c->max_tokens || kk < 0 || kk > c->k ||
+      (kk > 0 && (!idx || !w)) || (kk == 0 && !with_shared) || !aligned16(h) || !aligned16(delta))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: bad arguments (N=%d max=%d kk=%d k=%d)", N,
+                c->max_tokens, kk, c->k);
+  if (with_shared && !c->n_shared)
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: no shared expert configured");
+  if (!c->pf || c->pf_pairs <= 0 || c->d % (2 * kPfBN) != 0 || c->f % kPfBN != 0 || c->E > kPfMaxE)
+    return fail(c, MOE_ERR_NOT_SUPPORTED,
+                "moe_experts_given: needs a chunk-configured context (max_tokens > 32) and the "
+                "grouped GEMM's shapes");
+  if (with_shared && !c->shared_loaded[layer])
+    return fail(c, MOE_ERR_STATE, "shared expert of layer %d not loaded", layer);
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  if (kk > 0) {
+    // the ids index the kernels' tables: check them before any launch
+    std::vector<int32_t> ids((size_t)N * kk);
+    CUDA_TRY(c, cudaMemcpyAsync(ids.data(), idx, ids.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(c, cudaStreamSynchronize(s));
+    const auto &loaded = c->expert_loaded[layer];
+    for (int t = 0; t < N; ++t)
+      for (int j = 0; j < kk; ++j) {
+        const int e = ids[(size_t)t * kk + j];
+        if (e < 0 || e >= c->E)
+          return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: id %d of token %d outside [0, %d)", e, t,
+                      c->E);
+        if (!loaded[e])
+          return fail(c, MOE_ERR_STATE, "moe_experts_given: expert %d of layer %d not loaded", e, layer);
+        for (int i = 0; i < j; ++i)
+          if (ids[(size_t)t * kk + i] == e)
+            return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: token %d selects expert %d twice", t, e);
+      }
+  }
+  return given_impl(c, layer, (const uint16_t *)h, N, kk, idx, w, with_shared != 0, delta, s);
+}
+
+moe_status moe_ep_dispatch(moe_ctx *c, const int32_t *idx, int N, int n_ranks, const void *h,
+                           void *send_h, int32_t *send_e, int32_t *row_of, int32_t *counts_host,
+                           void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (!idx || !h || !send_h || !send_e || !row_of || !counts_host || N < 1 || n_ranks < 1 ||
+      n_ranks > kEpMaxRanks || c->E % n_ranks != 0 || !aligned16(h) || !aligned16(send_h) ||
+      (long long)N * c->k > (1LL << 30))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_ep_dispatch: bad arguments (N=%d ranks=%d E=%d)", N, n_ranks,
+                c->E);
+  if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  if (!c->ep_counts) CUDA_TRY(c, cudaMalloc(&c->ep_counts, kEpMaxRanks * sizeof(int)));
+  EpPlanParams pp{idx, N, c->k, c->E, n_ranks, row_of, send_e, c->ep_counts, c->status};
+  CUDA_TRY(c, launch(ep_plan_kernel, dim3(1), dim3(1024), 0, s, pp));
+  const long long P = (long long)N * c->k;
+  EpGatherParams gp{(const uint16_t *)h, row_of, N, c->k, c->d, (uint16_t *)send_h};
+  const int gblocks = (int)std::min<long long>((P + 7) / 8, 8LL * c->n_sm);
+  CUDA_TRY(c, launch(ep_gather_kernel, dim3(gblocks), dim3(256), 0, s, gp));
+  CUDA_TRY(c, cudaMemcpyAsync(counts_host, c->ep_counts, n_ranks * sizeof(int), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(c, cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(moe_ctx *c, int N, const float *w, const float *y, const int32_t *row_of,
+                          const float *y_shared, void *x, float *delta, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (N < 1 || !w || !y || !row_of || (!x == !delta) || !aligned16(y) ||
+      (y_shared && !aligned16(y_shared)) || (x && !aligned16(x)) || (delta && !aligned16(delta)))
+    return fail(c, MOE_ERR_INVALID_ARG, "moe_ep_combine: bad arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  EpCombineParams mp{y, row_of, w, y_shared, N, c->k, c->d, (uint16_t *)x, delta};
+  const long long n4 = (long long)N * c->d / 4;
+  const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
+  CUDA_TRY(c, launch(ep_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));
   return MOE_OK;
 }
 

@@ -195,6 +195,29 @@ __global__ void __launch_bounds__(kPfTok * 32) prefill_topk_kernel(PfRouteParams
   pdl_launch_dependents();
 }
 
+// Caller-given routing (idx [T, k], distinct ids in [0, E) per token,
+// checked on the host): the block masks prefill_topk_kernel would have
+// written for it, so the chunk path's bucketing can run without the router.
+struct PfMaskParams {
+  const int *idx;         // [T, k]
+  int T, E, k;
+  unsigned short *bmask;  // [blocks][E]
+};
+
+__global__ void __launch_bounds__(kPfTok * 32) prefill_mask_kernel(PfMaskParams p) {
+  __shared__ unsigned s_mask[kPfMaxE];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  pdl_wait();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_mask[e] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kPfTok + wid;
+  if (t < p.T && lane < p.k) atomicOr(&s_mask[__ldg(p.idx + (long long)t * p.k + lane)], 1u << wid);
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+    p.bmask[(long long)blockIdx.x * p.E + e] = (unsigned short)s_mask[e];
+  pdl_launch_dependents();
+}
+
 struct PfScanParams {
   const unsigned short *bmask;  // [blocks][E]
   int blocks, E, T, k;
