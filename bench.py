@@ -56,7 +56,7 @@ def parse():
                     help="timed steps (default 200 decode windows, 20 prefill chunks)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "q2", "prefill", "stack", "tier"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "q2", "prefill", "stack", "tier", "ep"])
     ap.add_argument("--T", type=int, default=4, help="window (decode) / per-sequence window (q2)")
     ap.add_argument("--rot-layers", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -69,7 +69,7 @@ def parse():
                     help="routed experts per layer (256: the pruned configuration)")
     a = ap.parse_args()
     if a.steps is None:
-        a.steps = {"prefill": 20, "stack": 10, "tier": 100}.get(a.workload, 200)
+        a.steps = {"prefill": 20, "stack": 10, "tier": 100, "ep": 10}.get(a.workload, 200)
     return a
 
 
@@ -790,6 +790,167 @@ def run_tier(args, world, K, W):
             "gpu_launches": None}
 
 
+def ep_launches_per_step(N, rows, max_rows):
+    """Library kernels one ExpertParallelMoE.forward launches for N tokens of
+    its own and `rows` received rows (8192-token chunks: the tensor-core
+    router needs no split).  A chunk step on n rows adds a column-count pass
+    when its column scan is split (n / 8 mask blocks over ranges of 64)."""
+    def colcount(n):
+        return 1 if min(32, (n + 7) // 8 // 64) > 1 else 0
+    route = 5 + colcount(N)                       # router, top-k, [count], column scan, scan, scatter
+    dispatch = 3                                  # count, offsets, place + copy
+    given = 0
+    for a in range(0, rows, max_rows):            # mask, [count], column scan, scan, scatter,
+        given += 9 + colcount(min(max_rows, rows - a))   # two GEMM, two GEMV, combine
+    shared = 9 + colcount(N)
+    return route + dispatch + given + shared + 1  # + the combine
+
+
+def run_ep(args, world, rank, K, W):
+    """Expert parallelism (ep.py): each rank holds E / world experts of the
+    layer (router and shared expert replicated) and 8192 tokens of its own;
+    one step is ExpertParallelMoE.forward on them (route, dispatch by owner,
+    NCCL all-to-all, owners' experts, all-to-all back, shared expert,
+    combine).  With one GPU the process group has one rank and the
+    exchange is a local copy; the one-GPU layer (moe_prefill) on the same
+    tokens is timed beside it.  Phases are timed in one extra untimed step."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    from sparse_moe_expert_gemv_b200 import binding as B
+    from sparse_moe_expert_gemv_b200 import inputs as I
+    from sparse_moe_expert_gemv_b200.ep import DeviceOps, Exchange, ExpertParallelMoE
+
+    own_group = not dist.is_initialized()
+    if own_group:
+        with socket.socket() as s_:
+            s_.bind(("127.0.0.1", 0))
+            port = s_.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                device_id=torch.device("cuda", 0))
+    N = 8192
+    per = E // world
+    ctx = B.moe_create(D, F, E, K_TOP, I.Q4)
+    try:
+        B.moe_configure(ctx, 1, 1, 0, N * K_TOP)
+        B.moe_set_router(ctx, 0, I.router_np(args.seed, E, D, 0), I.zipf_bias_np(args.seed, E, 0)[0])
+        for first in range(rank * per, (rank + 1) * per, 64):
+            n = min(64, (rank + 1) * per - first)
+            c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, 0, first, n, "cuda")
+            B.moe_load_experts(ctx, 0, first, n, c, s_, m)
+            del c, s_, m
+        c, s_, m = I.experts_torch(args.seed, I.Q4, D, F, 0, I.SHARED_INDEX, 1, "cuda")
+        B.moe_load_shared(ctx, 0, c, s_, m)
+        del c, s_, m
+        torch.cuda.synchronize()
+        ops = DeviceOps(B, ctx, d=D, k=K_TOP, E=E, max_tokens=N * K_TOP, has_shared=True)
+        marks = []
+        moe = ExpertParallelMoE(ops, Exchange(), on_phase=None)
+        x0 = torch.from_numpy(I.hidden_np(args.seed, N, D, window=1000 + rank).view(np.int16)).cuda()
+        x = x0.clone()
+        for _ in range(W):
+            x.copy_(x0)
+            moe.forward(0, x, N)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as cs:
+            e0.record()
+            for _ in range(K):
+                x.copy_(x0)
+                moe.forward(0, x, N)
+            e1.record()
+            torch.cuda.synchronize()
+        barrier(world)
+        ms_max = max_over_ranks(world, e0.elapsed_time(e1))
+        clocks = cs.summary()
+        # phases of one more step
+        ev0 = torch.cuda.Event(enable_timing=True)
+
+        def on_phase(name):
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            marks.append((name, ev))
+
+        moe.on_phase = on_phase
+        x.copy_(x0)
+        ev0.record()
+        moe.forward(0, x, N)
+        torch.cuda.synchronize()
+        moe.on_phase = None
+        seg, prev = {}, ev0
+        for name, ev in marks:
+            seg[name] = prev.elapsed_time(ev)
+            prev = ev
+        # end to end: the input copied in from pinned host memory and the
+        # result read back, every step, through the same public call
+        x_host = x0.cpu().pin_memory()
+        out_host = torch.empty_like(x_host).pin_memory()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K):
+            x.copy_(x_host, non_blocking=True)
+            moe.forward(0, x, N)
+            out_host.copy_(x, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
+        one_gpu = None
+        if world == 1:   # the one-GPU layer on the same tokens, for comparison
+            for _ in range(W):
+                x.copy_(x0)
+                B.moe_prefill(ctx, 0, x, N)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(K):
+                x.copy_(x0)
+                B.moe_prefill(ctx, 0, x, N)
+            e1.record()
+            torch.cuda.synchronize()
+            one_gpu = {"ms_per_step": e0.elapsed_time(e1) / K,
+                       "value": K * N / (e0.elapsed_time(e1) * 1e-3), "unit": "tokens/s"}
+        B.moe_sync(ctx, 120000)
+    finally:
+        B.moe_destroy(ctx)
+    _, tflops_peak, peak_kind = peaks()
+    flops = 6.0 * D * F * (N * K_TOP + N)
+    t_exp = (seg["experts"] + seg["shared"]) * 1e-3
+    P = N * K_TOP
+    gather_bytes = N * D * 2 + P * D * 2
+    combine_bytes = P * D * 4 + N * D * 4 + 2 * N * D * 2 + P * 8
+    res = {
+        "metric": "expert-parallel MoE tokens/s", "value": whole_job_rate(world, N * K, ms_max),
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "q4-g32 weights, bf16 activations, fp16 tensor-core operands, fp32 accumulate",
+        "data": "synthetic (seeded generator; random-init weights of the layer's shape)",
+        "config": {"workload": f"expert-parallel MoE layer, d=2048 f=768 E={E} top-10 + shared, Q4 g32, "
+                               f"Zipf(1.1) routing, {N} tokens per rank, {per} experts per rank",
+                   "tokens_per_step": N * world, "parallelism": f"ep{world}",
+                   "l2": "no flush: a step moves ~1 GB of rows and outputs (>> 126 MB L2)",
+                   "timing": "K ExpertParallelMoE.forward calls, CUDA events, max over ranks"},
+        "segments_ms_one_step": seg,
+        "roofline": {"bound": "tensor", "kernel": "owners' experts + shared expert (moe_experts_given)",
+                     "achieved": flops / t_exp / 1e12, "peak": tflops_peak, "unit": "TFLOP/s",
+                     "frac": flops / t_exp / 1e12 / tflops_peak, "traffic": None,
+                     "peak_source": peak_source(peak_kind, "bf16"),
+                     "per_unit": "6 d f FLOP per (token, expert) row; the rank's 8192 x (10 + 1) rows"},
+        "dispatch_gbs": gather_bytes / (seg["dispatch"] * 1e-3) / 1e9,
+        "combine_gbs": combine_bytes / (seg["combine"] * 1e-3) / 1e9,
+        "e2e": {"value": whole_job_rate(world, N * K, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": N * D * 2, "d2h_bytes_per_step": N * D * 2},
+        "gpu_launches": K * ep_launches_per_step(N, ops.last_rows, N * K_TOP),
+        "clocks": clocks,
+    }
+    if one_gpu:
+        res["one_gpu_layer"] = one_gpu
+    if own_group:
+        dist.destroy_process_group()
+    return res
+
+
 def run_reference(args):
     """Reference arm: the oracle (scalar fp64 C) on the host cores, on the
     headline's workload: each step is one window of the workload's tokens
@@ -872,6 +1033,8 @@ def main():
         res = run_stack(args, world, args.steps, args.warmup)
     elif args.workload == "tier":
         res = run_tier(args, world, args.steps, args.warmup)
+    elif args.workload == "ep":
+        res = run_ep(args, world, rank, args.steps, args.warmup)
     else:
         n_rot = args.rot_layers if args.workload == "decode" else min(args.rot_layers, 4)
         res = run_native(args, world, spec, n_rot, args.steps, args.warmup)

@@ -17,84 +17,111 @@ namespace moe {
 
 constexpr int kEpMaxRanks = 64;
 
+// Pairs are placed in blocks of kEpBlockPairs consecutive pair ids, one
+// per lane of the block's warps.
+constexpr int kEpWarps = 8, kEpBlockPairs = kEpWarps * 32;
+
 struct EpPlanParams {
-  const int *idx;  // [N, k] expert ids
-  int N, k, E, R;
-  int *row_of;     // [N*k] send position of pair q = t k + j (-1: invalid id, not sent)
-  int *send_e;     // [N*k] expert id of the row at each send position
-  int *counts;     // [R] rows for each rank
+  const int *idx;       // [N, k] expert ids
+  const uint16_t *h;    // bf16 [N, d] router input
+  int N, k, d, E, R;
+  int blocks;           // blocks of kEpBlockPairs pairs
+  int *blk_cnt;         // [blocks][R] pairs of each block for each rank
+  int *blk_off;         // [blocks][R] first send position of the block's pairs for each rank
+  int *counts;          // [R] rows for each rank
+  int *row_of;          // [N*k] send position of pair q = t k + j (-1: invalid id, not sent)
+  int *send_e;          // [N*k] expert id of the row at each send position
+  uint16_t *send_h;     // bf16 [rows sent, d]
   int *status;
 };
 
-// One CTA of 1024 threads.  Each thread takes a run of consecutive pairs;
-// for each rank in turn a block scan over the runs' counts gives every
-// run's first position inside that rank's segment, so each segment lists
-// its pairs in ascending pair id (t, then j).  An id outside [0, E) sets
-// the device status and its pair is left out (row_of = -1).
-__global__ void __launch_bounds__(1024) ep_plan_kernel(EpPlanParams p) {
+// Owner rank of pair q's expert, or -1 for an id outside [0, E).
+MOE_DEV int ep_owner(const EpPlanParams &p, long long q, int *e_out) {
+  const int e = __ldg(p.idx + q);
+  *e_out = e;
+  return (e >= 0 && e < p.E) ? e / (p.E / p.R) : -1;
+}
+
+// Pass 1: each block's pair count for every rank (order does not matter).
+__global__ void __launch_bounds__(kEpBlockPairs) ep_count_kernel(EpPlanParams p) {
+  __shared__ int s_cnt[kEpMaxRanks];
+  pdl_wait();
+  for (int r = threadIdx.x; r < p.R; r += blockDim.x) s_cnt[r] = 0;
+  __syncthreads();
+  const long long P = (long long)p.N * p.k;
+  const long long q = (long long)blockIdx.x * kEpBlockPairs + threadIdx.x;
+  if (q < P) {
+    int e;
+    const int r = ep_owner(p, q, &e);
+    if (r >= 0)
+      atomicAdd(&s_cnt[r], 1);
+    else
+      atomicOr(p.status, kErrBadExpert);
+  }
+  __syncthreads();
+  for (int r = threadIdx.x; r < p.R; r += blockDim.x) p.blk_cnt[(long long)blockIdx.x * p.R + r] = s_cnt[r];
+  pdl_launch_dependents();
+}
+
+// Pass 2, one CTA: per rank, an exclusive scan of the blocks' counts in
+// block order (the rank segments one after another) and the rank totals.
+__global__ void __launch_bounds__(1024) ep_offsets_kernel(EpPlanParams p) {
+  const int blocks = p.blocks;
   __shared__ int s_cnt[1025];
   __shared__ int s_red[32];
   pdl_wait();
-  const int tid = threadIdx.x;
-  const int P = p.N * p.k, per = p.E / p.R;
-  const int ept = (P + blockDim.x - 1) / blockDim.x;
-  const int q0 = min(P, tid * ept), q1 = min(P, q0 + ept);
-  bool bad = false;
-  for (int q = q0; q < q1; ++q) {
-    const int e = __ldg(p.idx + q);
-    if (e < 0 || e >= p.E) {
-      p.row_of[q] = -1;
-      bad = true;
-    }
-  }
-  if (bad) atomicOr(p.status, kErrBadExpert);
   int base = 0;
   for (int r = 0; r < p.R; ++r) {
-    int n = 0;
-    for (int q = q0; q < q1; ++q) {
-      const int e = __ldg(p.idx + q);
-      n += (e >= 0 && e < p.E && e / per == r);
+    const int start = base;
+    for (int b0 = 0; b0 < blocks; b0 += 1024) {
+      const int nb = min(1024, blocks - b0);
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) s_cnt[i] = p.blk_cnt[(long long)(b0 + i) * p.R + r];
+      block_exclusive_scan(s_cnt, s_cnt, nb, s_red);
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) p.blk_off[(long long)(b0 + i) * p.R + r] = base + s_cnt[i];
+      base += s_cnt[nb];
+      __syncthreads();  // s_cnt is rewritten by the next range
     }
-    s_cnt[tid] = n;
-    block_exclusive_scan(s_cnt, s_cnt, blockDim.x, s_red);
-    int pos = base + s_cnt[tid];
-    for (int q = q0; q < q1; ++q) {
-      const int e = __ldg(p.idx + q);
-      if (e >= 0 && e < p.E && e / per == r) {
-        p.row_of[q] = pos;
-        p.send_e[pos] = e;
-        ++pos;
-      }
-    }
-    const int total = s_cnt[blockDim.x];
-    if (tid == 0) p.counts[r] = total;
-    base += total;
-    __syncthreads();  // s_cnt is rewritten by the next rank's counts
+    if (threadIdx.x == 0) p.counts[r] = base - start;
   }
   pdl_launch_dependents();
 }
 
-struct EpGatherParams {
-  const uint16_t *h;   // bf16 [N, d] router input
-  const int *row_of;   // [N*k]
-  int N, k, d;
-  uint16_t *send_h;    // bf16 [rows sent, d]
-};
-
-// One warp per pair: the token's row to the pair's send position, 16 bytes
-// per lane per step.
-__global__ void __launch_bounds__(256) ep_gather_kernel(EpGatherParams p) {
+// Pass 3: each pair's send position, stable in pair id inside a rank's
+// segment (the block's offset, the earlier warps' counts, the earlier lanes
+// with the same owner), then the warp copies the pairs' token rows to their
+// positions, 16 bytes per lane per step.
+__global__ void __launch_bounds__(kEpBlockPairs) ep_place_kernel(EpPlanParams p) {
+  __shared__ int s_wcnt[kEpWarps][kEpMaxRanks];
+  __shared__ int s_pos[kEpWarps][32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   pdl_wait();
-  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kEpWarps * kEpMaxRanks; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
+  __syncthreads();
   const long long P = (long long)p.N * p.k;
+  const long long q = (long long)blockIdx.x * kEpBlockPairs + threadIdx.x;
+  int e = -1, r = -1;
+  if (q < P) r = ep_owner(p, q, &e);
+  const unsigned same = __match_any_sync(0xffffffffu, r);
+  const int before = __popc(same & ((1u << lane) - 1u));
+  if (r >= 0 && before == 0) s_wcnt[wid][r] = __popc(same);
+  __syncthreads();
+  int pos = -1;
+  if (r >= 0) {
+    pos = p.blk_off[(long long)blockIdx.x * p.R + r] + before;
+    for (int w = 0; w < wid; ++w) pos += s_wcnt[w][r];
+    p.send_e[pos] = e;
+  }
+  if (q < P) p.row_of[q] = pos;
+  s_pos[wid][lane] = pos;
+  __syncwarp();
   const int n8 = p.d / 8;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long q = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < P; q += nw) {
-    const int pos = __ldg(p.row_of + q);
-    if (pos < 0) continue;
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.h + (q / p.k) * p.d);
-    uint4 *dst = reinterpret_cast<uint4 *>(p.send_h + (long long)pos * p.d);
-    for (int i = lane; i < n8; i += 32) dst[i] = __ldg(src + i);
+  const long long q0 = (long long)blockIdx.x * kEpBlockPairs + wid * 32;
+  for (int i = 0; i < 32 && q0 + i < P; ++i) {
+    const int at = s_pos[wid][i];
+    if (at < 0) continue;
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.h + ((q0 + i) / p.k) * p.d);
+    uint4 *dst = reinterpret_cast<uint4 *>(p.send_h + (long long)at * p.d);
+    for (int c = lane; c < n8; c += 32) dst[c] = __ldg(src + c);
   }
   pdl_launch_dependents();
 }

@@ -76,7 +76,9 @@ struct moe_ctx {
   int *job_beg = nullptr, *job_n = nullptr, *n_jobs = nullptr;
   uint16_t *hbuf = nullptr, *abuf = nullptr;
   int *status = nullptr, *cnt_out = nullptr, *last = nullptr;
-  int *ep_counts = nullptr;  // [kEpMaxRanks] rows per rank of the last expert-parallel dispatch
+  int *ep_counts = nullptr;  // expert-parallel dispatch: [kEpMaxRanks] rows per rank, then the
+                             // blocks' per-rank counts and offsets
+  long long ep_scratch_n = 0;
   unsigned int *ticket = nullptr;    // fused routing: [0] CTA counter, [1] abort flag
   // single-launch decode kernel: grid barrier counter, hand-over flags and
   // partial sums (one slot per warp of the grid)
@@ -91,6 +93,7 @@ struct moe_ctx {
   float *pf_part = nullptr;             // split router partial sums
   __half *pf_a16 = nullptr, *pf_y16 = nullptr;  // GEMM a and y, fp16 [rows][f], [rows][d]
   int *pf_perm = nullptr, *pf_hot = nullptr;     // bucket permutation [T*k], GEMM-expert flags [E]
+  int *pf_colpart = nullptr;                     // [kPfColSplitMax][E] split column-scan counts
   long long pf_part_floats = 0;
   PfTile *pf_tiles = nullptr;
   int pf_max_tiles = 0, pf_rows = 0;
@@ -303,6 +306,7 @@ moe_status do_configure(moe_ctx *c) {
     const size_t o_part = pcarve((size_t)c->pf_part_floats * sizeof(float));
     const size_t o_a16 = pcarve((size_t)rows * f * 2), o_y16 = pcarve((size_t)rows * d * 2);
     const size_t o_perm = pcarve((size_t)P * 4), o_hot = pcarve((size_t)E * 4);
+    const size_t o_colp = pcarve((size_t)kPfColSplitMax * E * 4);
     CUDA_TRY(c, cudaMalloc(&c->pf, po));
     CUDA_TRY(c, cudaMemset(c->pf, 0, po));
     c->pf_hg = (__half *)(c->pf + o_hg);
@@ -317,6 +321,7 @@ moe_status do_configure(moe_ctx *c) {
     c->pf_y16 = (__half *)(c->pf + o_y16);
     c->pf_perm = (int *)(c->pf + o_perm);
     c->pf_hot = (int *)(c->pf + o_hot);
+    c->pf_colpart = (int *)(c->pf + o_colp);
     // the router rows as three exact bf16 parts, for the tensor-core router
     CUDA_TRY(c, cudaMalloc(&c->d_router3, (size_t)c->L * E * 3 * d * sizeof(__nv_bfloat16)));
   }
@@ -921,7 +926,12 @@ moe_status pf_bucket_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int k
   sp.stats = c->stats;
   sp.last = c->last;
   sp.status = c->status;
-  CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32), dim3(kPfColWarps * 32), 0, s, sp));
+  // long chunks: the column scan split over ranges of about 64 blocks
+  const int splits = std::max(1, std::min(kPfColSplitMax, blocks / 64));
+  sp.col_part = c->pf_colpart;
+  if (splits > 1)
+    CUDA_TRY(c, launch(prefill_colcount_kernel, dim3((E + 31) / 32, splits), dim3(kPfColWarps * 32), 0, s, sp));
+  CUDA_TRY(c, launch(prefill_colscan_kernel, dim3((E + 31) / 32, splits), dim3(kPfColWarps * 32), 0, s, sp));
   CUDA_TRY(c, launch(prefill_scan_kernel, dim3(1), dim3(1024), 0, s, sp));
   PfScatterParams cp{idx, c->pf_bmask, c->pf_boff, c->pf_eoff, h, N, E, kk, d, with_shared ? 1 : 0,
                      c->pf_row_of, c->pf_hg, perm ? perm : c->pf_perm, c->pf_hot};
@@ -1816,13 +1826,21 @@ moe_status moe_ep_dispatch(moe_ctx *c, const int32_t *idx, int N, int n_ranks, c
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
-  if (!c->ep_counts) CUDA_TRY(c, cudaMalloc(&c->ep_counts, kEpMaxRanks * sizeof(int)));
-  EpPlanParams pp{idx, N, c->k, c->E, n_ranks, row_of, send_e, c->ep_counts, c->status};
-  CUDA_TRY(c, launch(ep_plan_kernel, dim3(1), dim3(1024), 0, s, pp));
   const long long P = (long long)N * c->k;
-  EpGatherParams gp{(const uint16_t *)h, row_of, N, c->k, c->d, (uint16_t *)send_h};
-  const int gblocks = (int)std::min<long long>((P + 7) / 8, 8LL * c->n_sm);
-  CUDA_TRY(c, launch(ep_gather_kernel, dim3(gblocks), dim3(256), 0, s, gp));
+  const int blocks = (int)((P + kEpBlockPairs - 1) / kEpBlockPairs);
+  const long long need = kEpMaxRanks + 2LL * blocks * n_ranks;
+  if (need > c->ep_scratch_n) {  // grows to the largest dispatch seen
+    CUDA_TRY(c, cudaStreamSynchronize(s));
+    dfree(c->ep_counts);
+    CUDA_TRY(c, cudaMalloc(&c->ep_counts, (size_t)need * sizeof(int)));
+    c->ep_scratch_n = need;
+  }
+  EpPlanParams pp{idx, (const uint16_t *)h, N, c->k, c->d, c->E, n_ranks, blocks,
+                  c->ep_counts + kEpMaxRanks, c->ep_counts + kEpMaxRanks + (long long)blocks * n_ranks,
+                  c->ep_counts, row_of, send_e, (uint16_t *)send_h, c->status};
+  CUDA_TRY(c, launch(ep_count_kernel, dim3(blocks), dim3(kEpBlockPairs), 0, s, pp));
+  CUDA_TRY(c, launch(ep_offsets_kernel, dim3(1), dim3(1024), 0, s, pp));
+  CUDA_TRY(c, launch(ep_place_kernel, dim3(blocks), dim3(kEpBlockPairs), 0, s, pp));
   CUDA_TRY(c, cudaMemcpyAsync(counts_host, c->ep_counts, n_ranks * sizeof(int), cudaMemcpyDeviceToHost, s));
   CUDA_TRY(c, cudaStreamSynchronize(s));
   return MOE_OK;

@@ -222,6 +222,7 @@ struct PfScanParams {
   const unsigned short *bmask;  // [blocks][E]
   int blocks, E, T, k;
   int *boff;                    // [blocks][E] first row of (block, expert) relative to the expert's
+  int *col_part;                // [kPfColSplitMax][E] per-range token counts (split column scan)
   int *eoff;                    // [E + 1] token counts (colscan), then first rows (scan)
   const int *slot_of;           // residency table [L*E]
   int n_slots, layer;
@@ -247,15 +248,51 @@ struct PfScanParams {
 // rows stay in ascending t): every block's first row relative to the
 // expert's first row (boff), and the expert's token count (eoff[e], turned
 // into the expert's first row by prefill_scan_kernel).  A CTA takes 32
-// experts (one per lane) and its 16 warps contiguous ranges of blocks.
-constexpr int kPfColWarps = 16;
+// experts (one per lane) and one of gridDim.y contiguous ranges of blocks,
+// its 16 warps contiguous sub-ranges.  With more than one range,
+// prefill_colcount_kernel has left each range's counts in col_part, and a
+// range starts from the sum of the earlier ranges' counts.
+constexpr int kPfColWarps = 16, kPfColSplitMax = 32;
+
+MOE_DEV void colscan_range(const PfScanParams &p, int *b0_out, int *b1_out) {
+  const int per_s = (p.blocks + gridDim.y - 1) / gridDim.y;
+  *b0_out = min(p.blocks, (int)blockIdx.y * per_s);
+  *b1_out = min(p.blocks, *b0_out + per_s);
+}
+
+__global__ void __launch_bounds__(kPfColWarps * 32) prefill_colcount_kernel(PfScanParams p) {
+  __shared__ int s_part[kPfColWarps][33];
+  pdl_wait();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  int sb0, sb1;
+  colscan_range(p, &sb0, &sb1);
+  const int per = (sb1 - sb0 + kPfColWarps - 1) / kPfColWarps;
+  const int b0 = min(sb1, sb0 + wid * per), b1 = min(sb1, b0 + per);
+  int run = 0;
+  if (e < p.E) {
+#pragma unroll 8
+    for (int b = b0; b < b1; ++b) run += __popc(p.bmask[(long long)b * p.E + e]);
+  }
+  s_part[wid][lane] = run;
+  __syncthreads();
+  if (wid == 0 && e < p.E) {
+    int tot = 0;
+    for (int w = 0; w < kPfColWarps; ++w) tot += s_part[w][lane];
+    p.col_part[(long long)blockIdx.y * p.E + e] = tot;
+  }
+  pdl_launch_dependents();
+}
+
 __global__ void __launch_bounds__(kPfColWarps * 32) prefill_colscan_kernel(PfScanParams p) {
   __shared__ int s_part[kPfColWarps][33];
   pdl_wait();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
-  const int per = (p.blocks + kPfColWarps - 1) / kPfColWarps;
-  const int b0 = min(p.blocks, wid * per), b1 = min(p.blocks, b0 + per);
+  int sb0, sb1;
+  colscan_range(p, &sb0, &sb1);
+  const int per = (sb1 - sb0 + kPfColWarps - 1) / kPfColWarps;
+  const int b0 = min(sb1, sb0 + wid * per), b1 = min(sb1, b0 + per);
   int run = 0;
   if (e < p.E) {
 #pragma unroll 8
@@ -264,13 +301,16 @@ __global__ void __launch_bounds__(kPfColWarps * 32) prefill_colscan_kernel(PfSca
   s_part[wid][lane] = run;
   __syncthreads();
   int base = 0;
+  if (e < p.E)
+    for (int s = 0; s < (int)blockIdx.y; ++s) base += p.col_part[(long long)s * p.E + e];
   for (int w = 0; w < wid; ++w) base += s_part[w][lane];
   if (e < p.E) {
     for (int b = b0; b < b1; ++b) {
       p.boff[(long long)b * p.E + e] = base;
       base += __popc(p.bmask[(long long)b * p.E + e]);
     }
-    if (wid == kPfColWarps - 1) p.eoff[e] = base;  // all blocks: the expert's tokens
+    // the last range's last warp: all blocks, the expert's tokens
+    if (wid == kPfColWarps - 1 && blockIdx.y == gridDim.y - 1) p.eoff[e] = base;
   }
   pdl_launch_dependents();
 }

@@ -39,6 +39,7 @@ class DeviceOps:
         self.B, self.ctx = B, ctx
         self.d, self.k, self.E = d, k, E
         self.max_tokens, self.has_shared, self.device = max_tokens, has_shared, device
+        self.last_rows = 0    # rows of the last experts() call
 
     def norm(self, layer, x, N):
         h = torch.empty_like(x)
@@ -65,6 +66,7 @@ class DeviceOps:
     def experts(self, layer, rows_h, M, rows_e):
         """y [M, d] fp32: row i's output of expert rows_e[i].  More rows than
         the context holds run in slices of max_tokens rows."""
+        self.last_rows = M
         y = torch.empty((M, self.d), dtype=torch.float32, device=self.device)
         ones = torch.ones(min(M, self.max_tokens), dtype=torch.float32, device=self.device)
         for a in range(0, M, self.max_tokens):
@@ -123,25 +125,38 @@ class ExpertParallelMoE:
     """One rank's view of expert-parallel MoE layers (``ops`` on this rank's
     context, ``exchange`` over the process group)."""
 
-    def __init__(self, ops, exchange):
+    def __init__(self, ops, exchange, on_phase=None):
         self.ops, self.ex = ops, exchange
+        self.on_phase = on_phase   # optional callable(name), called after each phase
+
+    def _mark(self, name):
+        if self.on_phase is not None:
+            self.on_phase(name)
 
     def forward(self, layer, x, N):
         """x [N, d] bf16, in place: x <- x + MoE(norm(x)) for this rank's tokens."""
         h = self.ops.norm(layer, x, N)
         idx, w = self.ops.route(layer, h, N)
+        self._mark("route")
         self.forward_routed(layer, x, h, N, idx, w)
 
     def forward_routed(self, layer, x, h, N, idx, w):
         ops, ex = self.ops, self.ex
         send_h, send_e, row_of, send_counts = ops.dispatch(idx, h, N, ex.world)
+        self._mark("dispatch")
         recv_counts = ex.counts(send_counts)
         rows_h = ex.rows(send_h, send_counts, recv_counts)
         rows_e = ex.rows(send_e, send_counts, recv_counts)
+        self._mark("exchange")
         M = sum(recv_counts)
         y = ops.experts(layer, rows_h, M, rows_e) if M else rows_h.new_empty((0, h.shape[1]), dtype=torch.float32)
+        self._mark("experts")
         y_back = ex.rows(y, recv_counts, send_counts)
-        ops.combine(N, w, y_back, row_of, ops.shared(layer, h, N), x)
+        self._mark("return")
+        y_shared = ops.shared(layer, h, N)
+        self._mark("shared")
+        ops.combine(N, w, y_back, row_of, y_shared, x)
+        self._mark("combine")
 
 
 def emulate(ops_by_rank, layer, xs, hs, Ns, routings):
