@@ -100,6 +100,14 @@ def kernel_traffic(kernel_bytes_per_launch):
     return None if rec is None else rec["traffic_over_algorithmic"] * kernel_bytes_per_launch
 
 
+def q2_traffic(bytes_per_call):
+    """DRAM bytes of the four expert launches of one Q2 call (GEMM and GEMV,
+    gate/up and down) from the committed ncu record, scaled to this run's
+    algorithmic expert bytes per call."""
+    rec = _traffic_record("q2_experts_traffic.json")
+    return None if rec is None else rec["traffic_over_algorithmic"] * bytes_per_call
+
+
 def prefill_traffic(flops_per_call):
     """DRAM bytes of the two grouped-GEMM launches of one 8192-token chunk,
     from the committed ncu record (scaled by FLOPs when this chunk's work
@@ -500,7 +508,8 @@ def measure(args, world, ctx, spec, n_rot, K, W):
             **({"launch_us_event_bracketed": bracketed_us,
                 "launch_timing": "timed region / launches (one decode_kernel per step)"}
                if single else {}),
-            "traffic": kernel_traffic(kern_bytes / K) if single else None,
+            "traffic": (kernel_traffic(kern_bytes / K) if single else
+                        q2_traffic(kern_bytes / K) if spec["kind"] == "q2" and spec["T"] == 256 else None),
             "peak_source": peak_source(peak_kind, "hbm"),
             "per_unit": per_unit,
         },
