@@ -291,3 +291,38 @@ def test_world_of_one_over_nccl(B):
         dist.destroy_process_group()
         B.moe_destroy(ref)
         B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("with_gamma", [False, True])
+def test_rmsnorm_call_against_the_oracle(B, with_gamma):
+    """moe_rmsnorm (the expert-parallel layer's router input) against the
+    oracle's RMSNorm: fp32 inside against fp64, one bf16 rounding each, so
+    equal or one bf16 ulp apart; and a copy of x on a layer without a norm."""
+    spec = LayerSpec(fmt=I.Q4, zipf=False, shared=False, **SMALL)
+    N = 300
+    ctx = make_ctx(B, spec, 64)
+    try:
+        gamma = I.router_np(9, 1, spec.d, 0)[0] * 50.0 + 1.0 if with_gamma else None
+        B.moe_set_norm(ctx, 0, gamma, 1e-5)
+        xb = I.hidden_np(8, N, spec.d, window=3)
+        h = torch.empty((N, spec.d), dtype=torch.int16, device="cuda")
+        B.moe_rmsnorm(ctx, 0, to_dev(xb), N, h)
+        torch.cuda.synchronize()
+        got = h.cpu().numpy().view(np.uint16).astype(np.int64)
+        want = O.rmsnorm(xb, gamma, 1e-5).astype(np.int64)
+        assert np.array_equal(got >> 15, want >> 15)
+        assert np.abs(got - want).max() <= 1
+        assert (got == want).mean() >= 0.999
+        B.moe_sync(ctx, 60000)
+    finally:
+        B.moe_destroy(ctx)
+    ctx = make_ctx(B, spec, 64)   # no norm configured: h is x
+    try:
+        B.moe_set_router(ctx, 0, spec.W, spec.bias)
+        x = to_dev(I.hidden_np(8, 40, spec.d))
+        h = torch.empty_like(x)
+        B.moe_rmsnorm(ctx, 0, x, 40, h)
+        torch.cuda.synchronize()
+        assert torch.equal(h, x)
+    finally:
+        B.moe_destroy(ctx)
