@@ -55,6 +55,8 @@ struct moe_ctx {
   uint8_t *h_arena = nullptr;            // host address of the arena (host tier)
   moe::TierCache tier;
   cudaStream_t tier_stream = nullptr;    // host -> HBM expert copies
+  cudaStream_t pf_side = nullptr;        // the chunk's GEMV experts, beside the GEMM
+  cudaEvent_t pf_fork = nullptr, pf_join = nullptr;
   cudaEvent_t tier_done = nullptr;       // the latest copies and slot-table update
   int32_t *tier_idx = nullptr;           // device [max_tokens * k] routing of the tiered forward
   float *tier_w = nullptr;
@@ -287,6 +289,9 @@ moe_status do_configure(moe_ctx *c) {
   c->abuf = (uint16_t *)(b + o_a);
   c->ybuf = (float *)(b + o_y);
   if (T > kDecMaxT) {  // prefill-capable: grouped-GEMM buffers
+    CUDA_TRY(c, cudaStreamCreateWithFlags(&c->pf_side, cudaStreamNonBlocking));
+    CUDA_TRY(c, cudaEventCreateWithFlags(&c->pf_fork, cudaEventDisableTiming));
+    CUDA_TRY(c, cudaEventCreateWithFlags(&c->pf_join, cudaEventDisableTiming));
     const long long rows = Ptot;
     const int blocks = (T + kPfTok - 1) / kPfTok;
     c->pf_rows = (int)rows;
@@ -982,13 +987,20 @@ moe_status pf_experts_impl(moe_ctx *c, const uint16_t *h, int N, int kk, cudaStr
   g2.region_off = c->lay.p1_bytes;
   g2.out_a = nullptr;
   g2.out_y = c->ybuf;
+  // the GEMV experts run on a second stream beside the grouped GEMM: their
+  // CTAs take the SMs that GEMM pairs leave idle in its last round of items
+  // (they read the same grouped inputs and write other buffers)
+  CUDA_TRY(c, cudaEventRecord(c->pf_fork, s));
+  CUDA_TRY(c, cudaStreamWaitEvent(c->pf_side, c->pf_fork, 0));
   if (c->fmt == MOE_Q4_SYM_G32_F16) {
     CUDA_TRY(c, launch_prefill_gemms<1>(c, s));
-    CUDA_TRY(c, launch_experts<1>(c, s, kColdChunk, g1, g2));
+    CUDA_TRY(c, launch_experts<1>(c, c->pf_side, kColdChunk, g1, g2));
   } else {
     CUDA_TRY(c, launch_prefill_gemms<2>(c, s));
-    CUDA_TRY(c, launch_experts<2>(c, s, kColdChunk, g1, g2));
+    CUDA_TRY(c, launch_experts<2>(c, c->pf_side, kColdChunk, g1, g2));
   }
+  CUDA_TRY(c, cudaEventRecord(c->pf_join, c->pf_side));
+  CUDA_TRY(c, cudaStreamWaitEvent(s, c->pf_join, 0));
   return MOE_OK;
 }
 
@@ -1362,6 +1374,9 @@ moe_status moe_destroy(moe_ctx *c) {
   if (c->h_tier_idx) cudaFreeHost(c->h_tier_idx);
   if (c->tier_done) cudaEventDestroy(c->tier_done);
   if (c->tier_stream) cudaStreamDestroy(c->tier_stream);
+  if (c->pf_side) cudaStreamDestroy(c->pf_side);
+  if (c->pf_fork) cudaEventDestroy(c->pf_fork);
+  if (c->pf_join) cudaEventDestroy(c->pf_join);
   dfree(c->shared);
   dfree(c->pool);
   dfree(c->d_slot_of);
