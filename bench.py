@@ -452,7 +452,7 @@ def measure(args, world, ctx, spec, n_rot, K, W):
         kern_ms = exp_ms
         kern_bytes = expert_bytes
         kern_name = ("the experts of one call: prefill_gemm_kernel (gate/up + down, experts with "
-                     ">= 16 tokens) + expert_gemv_kernel (gate/up + down, the other experts)")
+                     ">= 24 tokens) + expert_gemv_kernel (gate/up + down, the other experts, beside the GEMM)")
         per_unit = f"{Be} B per touched expert (codes+scales), shared expert included"
     kern_gbs = kern_bytes / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
     res = {
@@ -486,7 +486,7 @@ def measure(args, world, ctx, spec, n_rot, K, W):
         "roofline": {
             "bound": "tensor",
             "kernel": ("the experts of one call: prefill_gemm_kernel (gate/up + down grouped GEMMs, "
-                       "tcgen05 fp16, experts with >= 16 tokens) + expert_gemv_kernel (the other "
+                       "tcgen05 fp16, experts with >= 24 tokens) + expert_gemv_kernel (the other "
                        "experts)"),
             "achieved": gemm_tf,
             "peak": tflops,

@@ -254,7 +254,7 @@ MOE_API moe_status moe_rmsnorm(moe_ctx *ctx, int layer, const void *x_dev, int T
 
 /* moe_experts_given: the experts of `layer` on caller-given routing, with
  * the chunk path's kernels (bucketing by expert, grouped tcgen05 GEMM for
- * experts with at least 16 rows, GEMV for the others, combine): the
+ * experts with at least 24 rows, GEMV for the others, combine): the
  * "experts by residency, then combine" half of the engine article's
  * per-layer flow ("93 token/s on one 8 GB card", section "Architecture
  * overview") without its router.  It is what an expert-parallel owner runs
