@@ -326,3 +326,48 @@ def test_rmsnorm_call_against_the_oracle(B, with_gamma):
         assert torch.equal(h, x)
     finally:
         B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("fmt", [I.Q4, I.Q2])
+def test_one_rank_chain_into_delta(B, fmt):
+    """The expert-parallel steps by hand at one rank, ending in
+    moe_ep_combine's delta form: route, dispatch, the owner's experts (one
+    expert per row, weight 1), the shared expert, combine; equal to
+    moe_prefill_delta bit for bit."""
+    spec = LayerSpec(fmt=fmt, zipf=True, **SMALL)
+    N = 600
+    ref = make_ctx(B, spec, N)
+    ctx = make_ctx(B, spec, N * spec.k)
+    try:
+        load_layer(B, ref, spec)
+        load_owned(B, ctx, spec, 0, spec.E)
+        x = to_dev(I.hidden_np(3, N, spec.d, window=6))
+        want = torch.empty((N, spec.d), dtype=torch.float32, device="cuda")
+        B.moe_prefill_delta(ref, 0, x, N, want)
+        idx = torch.empty((N, spec.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((N, spec.k), dtype=torch.float32, device="cuda")
+        B.moe_prefill_route(ctx, 0, x, N, idx, w)
+        P = N * spec.k
+        send_h = torch.empty((P, spec.d), dtype=torch.int16, device="cuda")
+        send_e = torch.empty(P, dtype=torch.int32, device="cuda")
+        row_of = torch.empty(P, dtype=torch.int32, device="cuda")
+        counts = B.moe_ep_dispatch(ctx, idx, N, 1, x, send_h, send_e, row_of)
+        assert counts == [P]
+        y = torch.empty((P, spec.d), dtype=torch.float32, device="cuda")
+        ones = torch.ones(P, dtype=torch.float32, device="cuda")
+        B.moe_experts_given(ctx, 0, send_h, P, 1, send_e, ones, 0, y)
+        ysh = torch.empty((N, spec.d), dtype=torch.float32, device="cuda")
+        B.moe_experts_given(ctx, 0, x, N, 0, None, None, 1, ysh)
+        got = torch.empty_like(want)
+        B.moe_ep_combine(ctx, N, w, y, row_of, ysh, delta=got)
+        with pytest.raises(B.MoeError):
+            B.moe_ep_combine(ctx, N, w, y, row_of, ysh)            # neither x nor delta
+        with pytest.raises(B.MoeError):
+            B.moe_ep_combine(ctx, N, w, y, row_of, ysh, x=x, delta=got)   # both
+        torch.cuda.synchronize()
+        B.moe_sync(ref, 60000)
+        B.moe_sync(ctx, 60000)
+        assert torch.equal(got, want)
+    finally:
+        B.moe_destroy(ref)
+        B.moe_destroy(ctx)
