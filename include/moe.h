@@ -305,7 +305,9 @@ MOE_API moe_status moe_ep_dispatch(moe_ctx *ctx, const int32_t *idx_dev, int N, 
  * [N, d], updated in place: x <- bf16(x + acc)) and delta_dev (fp32 [N, d]
  * <- acc) is non-NULL; acc = sum_j w[t,j] y[row_of(t,j)] + y_shared[t],
  * j in order, the one-GPU combine's arithmetic, so an expert-parallel layer
- * matches moe_prefill bit for bit.  Errors: INVALID_ARG. */
+ * matches moe_prefill bit for bit.  row_of_dev must be the one
+ * moe_ep_dispatch wrote for the same routing (its entries are rows of y_dev
+ * or -1; they are not checked again).  Errors: INVALID_ARG. */
 MOE_API moe_status moe_ep_combine(moe_ctx *ctx, int N, const float *w_dev, const float *y_dev,
                                   const int32_t *row_of_dev, const float *y_shared_dev, void *x_dev,
                                   float *delta_dev, void *stream);
