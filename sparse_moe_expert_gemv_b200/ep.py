@@ -64,8 +64,8 @@ class DeviceOps:
         return send_h, send_e, row_of, counts
 
     def experts(self, layer, rows_h, M, rows_e):
-        """y [M, d] fp32: row i's output of expert rows_e[i].  More rows than
-        the context holds run in slices of max_tokens rows."""
+        """y [M, d] fp32: row i's output of expert rows_e[i] (M may be 0).
+        More rows than the context holds run in slices of max_tokens rows."""
         self.last_rows = M
         y = torch.empty((M, self.d), dtype=torch.float32, device=self.device)
         ones = torch.ones(min(M, self.max_tokens), dtype=torch.float32, device=self.device)
@@ -89,9 +89,14 @@ class DeviceOps:
 
 
 def _as_rows_of_bytes(t):
-    """A [n, ...] tensor as [n, row bytes] uint8 (the all-to-all splits count rows)."""
-    t = t.contiguous()
-    return t.reshape(t.shape[0], -1).view(torch.uint8)
+    """A [n, ...] tensor as [n, row bytes] uint8 (the all-to-all splits count
+    rows); n may be 0."""
+    row = 1
+    for s in t.shape[1:]:
+        row *= s
+    if t.shape[0] == 0:
+        return torch.empty((0, row * t.element_size()), dtype=torch.uint8, device=t.device)
+    return t.contiguous().reshape(t.shape[0], row).view(torch.uint8)
 
 
 class Exchange:
@@ -149,7 +154,7 @@ class ExpertParallelMoE:
         rows_e = ex.rows(send_e, send_counts, recv_counts)
         self._mark("exchange")
         M = sum(recv_counts)
-        y = ops.experts(layer, rows_h, M, rows_e) if M else rows_h.new_empty((0, h.shape[1]), dtype=torch.float32)
+        y = ops.experts(layer, rows_h, M, rows_e)   # M may be 0: an empty output of the ops' row type
         self._mark("experts")
         y_back = ex.rows(y, recv_counts, send_counts)
         self._mark("return")
@@ -184,8 +189,7 @@ def emulate(ops_by_rank, layer, xs, hs, Ns, routings):
     ys = []
     for r in range(R):
         M = sum(recv[r])
-        ys.append(ops_by_rank[r].experts(layer, rows_h[r], M, rows_e[r]) if M else
-                  torch.empty((0, hs[r].shape[1]), dtype=torch.float32, device=hs[r].device))
+        ys.append(ops_by_rank[r].experts(layer, rows_h[r], M, rows_e[r]))
     y_back = a2a(ys, recv)
     for r in range(R):
         ops = ops_by_rank[r]

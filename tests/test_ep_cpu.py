@@ -73,3 +73,64 @@ def test_expert_parallel_gloo_ranks_match_the_one_process_layer(tmp_path, world,
         assert np.array_equal(rec, np.sort(idx[(idx // per) == r]))
         rows += rec.size
     assert rows == sum(sizes) * 4
+
+
+EMPTY_PROG = r"""
+import json, os, sys
+sys.path.insert(0, sys.argv[1])
+import numpy as np, torch
+import torch.distributed as dist
+import oracle as O
+from sparse_moe_expert_gemv_b200 import inputs as I
+from sparse_moe_expert_gemv_b200.ep import Exchange, ExpertParallelMoE
+from tests._harness import LayerSpec
+from tests._ep_oracle_ops import OracleOps
+
+class FirstHalfRouting(OracleOps):
+    # every token picks experts from rank 0's half only: rank 1 receives no rows
+    def route(self, layer, h, N):
+        t = np.arange(N)[:, None]
+        j = np.arange(self.k)[None, :]
+        idx = ((3 * t + 5 * j) % (self.E // 2)).astype(np.int32)
+        w = np.full((N, self.k), 1.0 / self.k)
+        return torch.from_numpy(idx), torch.from_numpy(w)
+
+rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+dist.init_process_group("gloo", rank=rank, world_size=world)
+spec = LayerSpec(d=256, f=128, E=16, k=4, fmt=O.Q4, zipf=False, shared=True)
+N = 7
+x = torch.from_numpy(I.hidden_np(4, N, 256, window=rank).view(np.int16).copy())
+ops = FirstHalfRouting(spec, rank, world)
+ExpertParallelMoE(ops, Exchange()).forward(0, x, N)
+dist.barrier()
+dist.destroy_process_group()
+np.savez(os.path.join(sys.argv[2], f"rank{rank}.npz"), x=x.numpy().view(np.uint16), delta=ops.last_delta,
+         received=np.array(ops.received, np.int64))
+"""
+
+
+def test_a_rank_that_receives_no_rows(tmp_path):
+    """Rank 1 owns experts nobody selects: it sends its tokens' rows, receives
+    none, computes nothing, and still gets its outputs back."""
+    import oracle as O
+    from sparse_moe_expert_gemv_b200 import inputs as I
+    from tests._harness import LayerSpec
+
+    outs = launch(["-c", EMPTY_PROG, ROOT, str(tmp_path)], 2, free_port())
+    for rc, out, err in outs:
+        assert rc == 0, err[-3000:]
+    spec = LayerSpec(d=256, f=128, E=16, k=4, fmt=O.Q4, zipf=False, shared=True)
+    N, k = 7, 4
+    for r in range(2):
+        got = np.load(tmp_path / f"rank{r}.npz")
+        assert got["received"].size == (2 * N * k if r == 0 else 0)
+        xb = I.hidden_np(4, N, 256, window=r)
+        idx = (3 * np.arange(N)[:, None] + 5 * np.arange(k)[None, :]) % 8
+        acc = np.zeros((N, 256))
+        for j in range(k):
+            for t in range(N):
+                Wg, Wu, Wd = O.dequant_expert(spec.fmt, 256, 128, *spec.expert(int(idx[t, j])))
+                acc[t] += (1.0 / k) * O.expert(Wg, Wu, Wd, xb[t:t + 1])[0]
+        Wg, Wu, Wd = O.dequant_expert(spec.fmt, 256, 128, *spec.shared_expert())
+        acc += O.expert(Wg, Wu, Wd, xb)
+        assert np.array_equal(got["delta"], acc)
