@@ -139,11 +139,31 @@ class ExpertParallelMoE:
             self.on_phase(name)
 
     def forward(self, layer, x, N):
-        """x [N, d] bf16, in place: x <- x + MoE(norm(x)) for this rank's tokens."""
+        """x [N, d] bf16, in place: x <- x + MoE(norm(x)) for this rank's
+        tokens.  N may be 0: the rank still serves its experts to the others
+        and takes part in every collective."""
+        if N == 0:
+            self._serve_only(layer, x)
+            return
         h = self.ops.norm(layer, x, N)
         idx, w = self.ops.route(layer, h, N)
         self._mark("route")
         self.forward_routed(layer, x, h, N, idx, w)
+
+    def _serve_only(self, layer, x):
+        """A step with no tokens of this rank's own: empty send blocks, the
+        owner's work for the other ranks, nothing to combine."""
+        ops, ex = self.ops, self.ex
+        zero = [0] * ex.world
+        recv_counts = ex.counts(zero)
+        d = x.shape[1]
+        rows_h = ex.rows(x.new_empty((0, d)), zero, recv_counts)
+        rows_e = ex.rows(torch.empty(0, dtype=torch.int32, device=x.device), zero, recv_counts)
+        self._mark("exchange")
+        y = ops.experts(layer, rows_h, sum(recv_counts), rows_e)
+        self._mark("experts")
+        ex.rows(y, recv_counts, zero)
+        self._mark("return")
 
     def forward_routed(self, layer, x, h, N, idx, w):
         ops, ex = self.ops, self.ex
