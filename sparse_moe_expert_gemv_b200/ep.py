@@ -190,7 +190,15 @@ def emulate(ops_by_rank, layer, xs, hs, Ns, routings):
     ``ExpertParallelMoE.forward_routed``, rank by rank.  xs are updated in
     place.  Returns the rows each rank received (for inspection)."""
     R = len(ops_by_rank)
-    plans = [ops_by_rank[r].dispatch(routings[r][0], hs[r], Ns[r], R) for r in range(R)]
+
+    def plan(r):
+        if Ns[r] == 0:  # nothing to send: empty blocks of the same row types
+            h = hs[r]
+            return (h.new_empty((0, h.shape[1])), torch.empty(0, dtype=torch.int32, device=h.device),
+                    torch.empty(0, dtype=torch.int32, device=h.device), [0] * R)
+        return ops_by_rank[r].dispatch(routings[r][0], hs[r], Ns[r], R)
+
+    plans = [plan(r) for r in range(R)]
     splits = [p[3] for p in plans]
 
     def a2a(bufs, split):
@@ -212,6 +220,8 @@ def emulate(ops_by_rank, layer, xs, hs, Ns, routings):
         ys.append(ops_by_rank[r].experts(layer, rows_h[r], M, rows_e[r]))
     y_back = a2a(ys, recv)
     for r in range(R):
+        if Ns[r] == 0:
+            continue
         ops = ops_by_rank[r]
         ops.combine(Ns[r], routings[r][1], y_back[r], plans[r][2], ops.shared(layer, hs[r], Ns[r]), xs[r])
     return rows_e

@@ -248,6 +248,13 @@ def test_emulated_ranks_match_one_gpu_small(B, R, fmt):
     _emulated_vs_one_gpu(B, spec, [300, 77, 250, 173][:R] if R > 1 else [800], R, norm=True)
 
 
+def test_emulated_rank_without_tokens(B):
+    """Three ranks, the middle one with no tokens of its own: it still
+    computes its experts' rows for the others."""
+    spec = LayerSpec(fmt=I.Q4, zipf=True, d=512, f=256, E=60, k=4)
+    _emulated_vs_one_gpu(B, spec, [400, 0, 200], 3, norm=False)
+
+
 def test_emulated_ranks_match_one_gpu_full_shape(B):
     """d=2048 f=768 E=512 top-10 + shared, Zipf routing, four ranks of
     uneven size."""
