@@ -378,3 +378,37 @@ def test_one_rank_chain_into_delta(B, fmt):
     finally:
         B.moe_destroy(ref)
         B.moe_destroy(ctx)
+
+
+@pytest.mark.parametrize("fmt,N", [(I.Q2, 256), (I.Q4, 1500)])
+def test_chunk_path_under_graph_capture(B, fmt, N):
+    """The chunk path forks its GEMV experts to a second stream and joins
+    them before the combine; captured in a CUDA graph and replayed, it must
+    give the eager result bit for bit."""
+    spec = LayerSpec(fmt=fmt, zipf=True, **FULL)
+    ctx = make_ctx(B, spec, N)
+    try:
+        load_layer(B, ctx, spec)
+        x = to_dev(I.hidden_np(2, N, spec.d, window=8))
+        eager = torch.empty((N, spec.d), dtype=torch.float32, device="cuda")
+        B.moe_prefill_delta(ctx, 0, x, N, eager)
+        torch.cuda.synchronize()
+        out = torch.zeros_like(eager)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            B.moe_prefill_delta(ctx, 0, x, N, out, stream=s)   # warm-up on the capture stream
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        out.zero_()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            B.moe_prefill_delta(ctx, 0, x, N, out)
+        for _ in range(2):
+            out.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(out, eager)
+        B.moe_sync(ctx, 60000)
+    finally:
+        B.moe_destroy(ctx)
