@@ -928,7 +928,7 @@ def run_ep(args, world, rank, K, W):
     t_exp = (seg["experts"] + seg["shared"]) * 1e-3
     P = N * K_TOP
     gather_bytes = N * D * 2 + P * D * 2
-    combine_bytes = P * D * 4 + N * D * 4 + 2 * N * D * 2 + P * 8
+    combine_bytes = P * D * 2 + N * D * 4 + 2 * N * D * 2 + P * 8   # fp16 y rows, fp32 shared, x
     res = {
         "metric": "expert-parallel MoE tokens/s", "value": whole_job_rate(world, N * K, ms_max),
         "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_max / K,

@@ -277,6 +277,17 @@ MOE_API moe_status moe_experts_given(moe_ctx *ctx, int layer, const void *h_dev,
                                      const int32_t *idx_dev, const float *w_dev, int with_shared,
                                      float *delta_dev, void *stream);
 
+/* moe_experts_rows: the owner's step of an expert-parallel layer.  Row t
+ * of h_dev (bf16 [M, d], router input) goes through the one expert
+ * e_dev[t] (int32 [M], loaded, in [0, E)) with weight 1 and no shared
+ * expert, with the chunk path's kernels (as moe_experts_given with kk = 1);
+ * y_dev (fp16 [M, d], caller-owned, 16-byte aligned) receives each row's
+ * output y in row order, in the fp16 the chunk path keeps expert outputs in
+ * before its combine.  M <= max_tokens.  The ids are checked on the host
+ * first (one stream synchronisation).  Errors as moe_experts_given. */
+MOE_API moe_status moe_experts_rows(moe_ctx *ctx, int layer, const void *h_dev, int M,
+                                    const int32_t *e_dev, void *y_dev, void *stream);
+
 /* Expert parallelism over n_ranks ranks: expert e belongs to rank
  * e / (E / n_ranks) (E a multiple of n_ranks, n_ranks <= 64).
  *
@@ -297,8 +308,8 @@ MOE_API moe_status moe_ep_dispatch(moe_ctx *ctx, const int32_t *idx_dev, int N, 
                                    const void *h_dev, void *send_h_dev, int32_t *send_e_dev,
                                    int32_t *row_of_dev, int32_t *counts_host, void *stream);
 
-/* moe_ep_combine: the receive side.  y_dev fp32 [rows, d]: the expert
- * outputs returned by the owners, in send order (row_of_dev from
+/* moe_ep_combine: the receive side.  y_dev fp16 [rows, d]: the expert
+ * outputs returned by the owners (moe_experts_rows), in send order (row_of_dev from
  * moe_ep_dispatch maps pair q to its row); w_dev fp32 [N, k];
  * y_shared_dev fp32 [N, d] (the shared expert's output, e.g. from
  * moe_experts_given with kk = 0) or NULL.  Exactly one of x_dev (bf16
@@ -308,7 +319,7 @@ MOE_API moe_status moe_ep_dispatch(moe_ctx *ctx, const int32_t *idx_dev, int N, 
  * matches moe_prefill bit for bit.  row_of_dev must be the one
  * moe_ep_dispatch wrote for the same routing (its entries are rows of y_dev
  * or -1; they are not checked again).  Errors: INVALID_ARG. */
-MOE_API moe_status moe_ep_combine(moe_ctx *ctx, int N, const float *w_dev, const float *y_dev,
+MOE_API moe_status moe_ep_combine(moe_ctx *ctx, int N, const float *w_dev, const void *y_dev,
                                   const int32_t *row_of_dev, const float *y_shared_dev, void *x_dev,
                                   float *delta_dev, void *stream);
 

@@ -38,7 +38,7 @@ EXPORTS = ("moe_create", "moe_configure", "moe_destroy", "moe_load_experts",
            "moe_tier_prefetch", "moe_forward_tiered", "moe_tier_stats", "moe_tier_dump_trace",
            "moe_tier_sim_create", "moe_tier_sim_request", "moe_tier_sim_counts",
            "moe_tier_sim_destroy", "moe_rmsnorm", "moe_experts_given", "moe_ep_dispatch",
-           "moe_ep_combine")
+           "moe_ep_combine", "moe_experts_rows")
 
 
 class MoeError(RuntimeError):
@@ -100,6 +100,7 @@ def _load():
         "moe_experts_given": [P, I, P, I, I, P, P, I, P, P],
         "moe_ep_dispatch": [P, P, I, I, P, P, P, P, ctypes.POINTER(ctypes.c_int32), P],
         "moe_ep_combine": [P, I, P, P, P, P, P, P, P],
+        "moe_experts_rows": [P, I, P, I, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -246,6 +247,10 @@ def moe_rmsnorm(ctx, layer, x, T, h, stream=None):
 def moe_experts_given(ctx, layer, h, N, kk, idx, w, with_shared, delta, stream=None):
     _check(ctx, _lib.moe_experts_given(ctx, layer, _ptr(h), N, kk, _ptr(idx), _ptr(w),
                                        int(bool(with_shared)), _ptr(delta), _stream(stream)))
+
+
+def moe_experts_rows(ctx, layer, h, M, e, y16, stream=None):
+    _check(ctx, _lib.moe_experts_rows(ctx, layer, _ptr(h), M, _ptr(e), _ptr(y16), _stream(stream)))
 
 
 def moe_ep_dispatch(ctx, idx, N, n_ranks, h, send_h, send_e, row_of, stream=None):

@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kEpBlockPairs) ep_place_kernel(EpPlanParams p)
 }
 
 struct EpCombineParams {
-  const float *y;         // fp32 [rows][d] expert outputs, in send order
+  const __half *y;        // fp16 [rows][d] expert outputs, in send order
   const int *row_of;      // [N*k] row of pair q in y (negative: contributes nothing)
   const float *w;         // [N, k]
   const float *y_shared;  // fp32 [N, d] or null
@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(EpCombineParams p) {
       const int row = __ldg(p.row_of + (long long)t * p.k + j);
       if (row < 0) continue;
       const float wj = __ldg(p.w + (long long)t * p.k + j);
-      const float4 v = __ldcs(reinterpret_cast<const float4 *>(p.y + (long long)row * p.d + o));
+      const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p.y + (long long)row * p.d + o));
+      const float4 v = make_float4(half_lo(q.x), half_hi(q.x), half_lo(q.y), half_hi(q.y));
       a0 = fmaf(wj, v.x, a0);
       a1 = fmaf(wj, v.y, a1);
       a2 = fmaf(wj, v.z, a2);

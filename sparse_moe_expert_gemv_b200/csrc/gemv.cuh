@@ -48,6 +48,7 @@ struct GemvParams {
   long long region_off;
   uint16_t *out_a;     // gated: bf16 a [pairs][R]
   float *out_y;        // down: fp32 y [pairs][R]
+  __half *out_y16;     // down, instead of out_y when set: fp16 y [pairs][R]
   int *status;
 };
 
@@ -426,7 +427,7 @@ struct ItemRun {
 
   // Write the item's outputs: a = bf16(SiLU(g) * u) (gated) or y (down).
   static MOE_DEV void store(const float (&acc)[C::NM][NTA][4], const int (&epair)[2][2], int rb,
-                            int lane, int R, uint16_t *out_a, float *out_y) {
+                            int lane, int R, uint16_t *out_a, float *out_y, __half *out_y16 = nullptr) {
     const int g = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NTA; ++nt) {
@@ -440,7 +441,10 @@ struct ItemRun {
           const float av = gv / (1.0f + __expf(-gv)) * uv;
           out_a[(long long)pair * R + row] = __bfloat16_as_ushort(__float2bfloat16_rn(av));
         } else {
-          out_y[(long long)pair * R + row] = acc[0][nt][c];
+          if (out_y16)
+            out_y16[(long long)pair * R + row] = __float2half_rn(acc[0][nt][c]);
+          else
+            out_y[(long long)pair * R + row] = acc[0][nt][c];
         }
       }
     }
@@ -454,7 +458,7 @@ MOE_DEV bool whole_item(WarpRing &r, const Phase &ph, const GemvParams &p, int l
   using Run = ItemRun<FMT, GATED, NTA>;
   float acc[Run::C::NM][NTA][4];
   if (!Run::run(r, ph, lane, 0, ph.UPI, br, acc)) return false;
-  Run::store(acc, epair, rb, lane, p.R, p.out_a, p.out_y);
+  Run::store(acc, epair, rb, lane, p.R, p.out_a, p.out_y, p.out_y16);
   return true;
 }
 

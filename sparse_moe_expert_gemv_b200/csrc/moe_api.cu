@@ -990,7 +990,8 @@ moe_status pf_experts_impl(moe_ctx *c, const uint16_t *h, int N, int kk, cudaStr
   g2.R = c->d;
   g2.region_off = c->lay.p1_bytes;
   g2.out_a = nullptr;
-  g2.out_y = c->ybuf;
+  g2.out_y = nullptr;
+  g2.out_y16 = reinterpret_cast<__half *>(c->ybuf);  // fp16 y by pair id, as the GEMM's
   // the GEMV experts run on a second stream beside the grouped GEMM: their
   // CTAs take the SMs that GEMM pairs leave idle in its last round of items
   // (they read the same grouped inputs and write other buffers)
@@ -1013,7 +1014,8 @@ moe_status pf_experts_impl(moe_ctx *c, const uint16_t *h, int N, int kk, cudaStr
 moe_status pf_combine_impl(moe_ctx *c, int N, int kk, const float *w, bool with_shared, uint16_t *x,
                            float *delta, cudaStream_t s) {
   const int d = c->d;
-  PfCombineParams mp{c->pf_y16, c->ybuf, w, c->pf_row_of, N, kk, d, with_shared ? 1 : 0, x, delta};
+  PfCombineParams mp{c->pf_y16, reinterpret_cast<const __half *>(c->ybuf), w, c->pf_row_of, N, kk, d,
+                     with_shared ? 1 : 0, x, delta};
   const long long n4 = (long long)N * d / 4;
   const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
   CUDA_TRY(c, launch(prefill_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));
@@ -1049,7 +1051,7 @@ moe_status prefill_impl(moe_ctx *c, int layer, uint16_t *x, int N, float *delta,
 // from idx, then the chunk path's bucketing, experts and combine into
 // delta.  idx was checked on the host (ids in [0, E), distinct per token).
 moe_status given_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int kk, const int32_t *idx,
-                      const float *w, bool with_shared, float *delta, cudaStream_t s) {
+                      const float *w, bool with_shared, float *delta, cudaStream_t s, __half *rows16 = nullptr) {
   moe_status st = pf_maps(c);
   if (st) return st;
   const int blocks = (N + kPfTok - 1) / kPfTok;
@@ -1059,6 +1061,13 @@ moe_status given_impl(moe_ctx *c, int layer, const uint16_t *h, int N, int kk, c
   if (st) return st;
   st = pf_experts_impl(c, h, N, kk, s);
   if (st) return st;
+  if (rows16) {  // kk == 1, no weights, no shared expert: each row's y as it is
+    PfRowsParams rp{c->pf_y16, reinterpret_cast<const __half *>(c->ybuf), c->pf_row_of, N, c->d, rows16};
+    const long long n8 = (long long)N * c->d / 8;
+    const int blocks = (int)std::min<long long>((n8 + 255) / 256, 8LL * c->n_sm);
+    CUDA_TRY(c, launch(prefill_rows_kernel, dim3(blocks), dim3(256), 0, s, rp));
+    return MOE_OK;
+  }
   return pf_combine_impl(c, N, kk, w, with_shared, nullptr, delta, s);
 }
 
@@ -1793,24 +1802,21 @@ moe_status moe_rmsnorm(moe_ctx *c, int layer, const void *x, int T, void *h, voi
   return MOE_OK;
 }
 
-moe_status moe_experts_given(moe_ctx *c, int layer, const void *h, int N, int kk, const int32_t *idx,
-                             const float *w, int with_shared, float *delta, void *stream) {
-  if (!c) return MOE_ERR_INVALID_ARG;
+// Checks shared by the calls on given routing; the ids are copied to the
+// host and checked before any launch (one stream synchronisation).
+static moe_status given_check(moe_ctx *c, int layer, const void *h, int N, int kk, const int32_t *idx,
+                              int with_shared, const void *out, cudaStream_t s, const char *who) {
   if (!c->configured) return fail(c, MOE_ERR_STATE, "nothing loaded");
-  if (!valid_layer(c, layer) || !h || !delta || N < 1 || N > c->max_tokens || kk < 0 || kk > c->k ||
-      (kk > 0 && (!idx || !w)) || (kk == 0 && !with_shared) || !aligned16(h) || !aligned16(delta))
-    return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: bad arguments (N=%d max=%d kk=%d k=%d)", N,
-                c->max_tokens, kk, c->k);
-  if (with_shared && !c->n_shared)
-    return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: no shared expert configured");
+  if (!valid_layer(c, layer) || !h || !out || N < 1 || N > c->max_tokens || kk < 0 || kk > c->k ||
+      (kk > 0 && !idx) || (kk == 0 && !with_shared) || !aligned16(h) || !aligned16(out))
+    return fail(c, MOE_ERR_INVALID_ARG, "%s: bad arguments (N=%d max=%d kk=%d k=%d)", who, N, c->max_tokens,
+                kk, c->k);
+  if (with_shared && !c->n_shared) return fail(c, MOE_ERR_INVALID_ARG, "%s: no shared expert configured", who);
   if (!c->pf || c->pf_pairs <= 0 || c->d % (2 * kPfBN) != 0 || c->f % kPfBN != 0 || c->E > kPfMaxE)
     return fail(c, MOE_ERR_NOT_SUPPORTED,
-                "moe_experts_given: needs a chunk-configured context (max_tokens > 32) and the "
-                "grouped GEMM's shapes");
+                "%s: needs a chunk-configured context (max_tokens > 32) and the grouped GEMM's shapes", who);
   if (with_shared && !c->shared_loaded[layer])
     return fail(c, MOE_ERR_STATE, "shared expert of layer %d not loaded", layer);
-  cudaStream_t s = (cudaStream_t)stream;
-  c->last_stream = s;
   if (kk > 0) {
     // the ids index the kernels' tables: check them before any launch
     std::vector<int32_t> ids((size_t)N * kk);
@@ -1821,16 +1827,37 @@ moe_status moe_experts_given(moe_ctx *c, int layer, const void *h, int N, int kk
       for (int j = 0; j < kk; ++j) {
         const int e = ids[(size_t)t * kk + j];
         if (e < 0 || e >= c->E)
-          return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: id %d of token %d outside [0, %d)", e, t,
-                      c->E);
-        if (!loaded[e])
-          return fail(c, MOE_ERR_STATE, "moe_experts_given: expert %d of layer %d not loaded", e, layer);
+          return fail(c, MOE_ERR_INVALID_ARG, "%s: id %d of row %d outside [0, %d)", who, e, t, c->E);
+        if (!loaded[e]) return fail(c, MOE_ERR_STATE, "%s: expert %d of layer %d not loaded", who, e, layer);
         for (int i = 0; i < j; ++i)
           if (ids[(size_t)t * kk + i] == e)
-            return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: token %d selects expert %d twice", t, e);
+            return fail(c, MOE_ERR_INVALID_ARG, "%s: row %d selects expert %d twice", who, t, e);
       }
   }
+  return MOE_OK;
+}
+
+moe_status moe_experts_given(moe_ctx *c, int layer, const void *h, int N, int kk, const int32_t *idx,
+                             const float *w, int with_shared, float *delta, void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kk > 0 && !w) return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_given: weights missing");
+  moe_status st = given_check(c, layer, h, N, kk, idx, with_shared, delta, s, "moe_experts_given");
+  if (st) return st;
+  c->last_stream = s;
   return given_impl(c, layer, (const uint16_t *)h, N, kk, idx, w, with_shared != 0, delta, s);
+}
+
+moe_status moe_experts_rows(moe_ctx *c, int layer, const void *h, int M, const int32_t *e, void *y_dev,
+                            void *stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (!e) return fail(c, MOE_ERR_INVALID_ARG, "moe_experts_rows: expert ids missing");
+  moe_status st = given_check(c, layer, h, M, 1, e, 0, y_dev, s, "moe_experts_rows");
+  if (st) return st;
+  c->last_stream = s;
+  return given_impl(c, layer, (const uint16_t *)h, M, 1, e, nullptr, false, nullptr, s,
+                    reinterpret_cast<__half *>(y_dev));
 }
 
 moe_status moe_ep_dispatch(moe_ctx *c, const int32_t *idx, int N, int n_ranks, const void *h,
@@ -1865,7 +1892,7 @@ moe_status moe_ep_dispatch(moe_ctx *c, const int32_t *idx, int N, int n_ranks, c
   return MOE_OK;
 }
 
-moe_status moe_ep_combine(moe_ctx *c, int N, const float *w, const float *y, const int32_t *row_of,
+moe_status moe_ep_combine(moe_ctx *c, int N, const float *w, const void *y, const int32_t *row_of,
                           const float *y_shared, void *x, float *delta, void *stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (N < 1 || !w || !y || !row_of || (!x == !delta) || !aligned16(y) ||
@@ -1873,7 +1900,8 @@ moe_status moe_ep_combine(moe_ctx *c, int N, const float *w, const float *y, con
     return fail(c, MOE_ERR_INVALID_ARG, "moe_ep_combine: bad arguments");
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
-  EpCombineParams mp{y, row_of, w, y_shared, N, c->k, c->d, (uint16_t *)x, delta};
+  EpCombineParams mp{reinterpret_cast<const __half *>(y), row_of, w, y_shared, N, c->k, c->d, (uint16_t *)x,
+                     delta};
   const long long n4 = (long long)N * c->d / 4;
   const int cblocks = (int)std::min<long long>((n4 + 255) / 256, 8LL * c->n_sm);
   CUDA_TRY(c, launch(ep_combine_kernel, dim3(cblocks), dim3(256), 0, s, mp));

@@ -1440,7 +1440,7 @@ __global__ void __launch_bounds__(256, 1)
 
 struct PfCombineParams {
   const __half *y;    // fp16 [rows][d] grouped order (GEMM experts)
-  const float *y32;   // fp32 [T*k][d] by pair id (GEMV experts: row_of < 0)
+  const __half *yp;   // fp16 [T*k][d] by pair id (GEMV experts: row_of < 0)
   const float *w;     // [T][k]
   const int *row_of;  // [T*k + T]
   int T, k, d, has_shared;
@@ -1449,7 +1449,7 @@ struct PfCombineParams {
 };
 
 // x[t] <- bf16(x[t] + sum_j w[t,j] y[row(t,j)] + y[row(shared, t)]), j in order;
-// a pair of a GEMV expert reads its fp32 y by pair id instead.
+// a pair of a GEMV expert reads its y by pair id instead (fp16 as well).
 __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p) {
   pdl_wait();
   const int per_t = p.d / 4, P = p.T * p.k;
@@ -1459,21 +1459,21 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p)
     const int t = (int)(i / per_t), o = (int)(i - (long long)t * per_t) * 4;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     // four fp16 y values of a row: one 8-byte load
-    auto y4 = [&](long long row) {
-      const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(p.y + row * p.d + o));
+    auto y4 = [&](const __half *base, long long row) {
+      const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(base + row * p.d + o));
       return make_float4(half_lo(v.x), half_hi(v.x), half_lo(v.y), half_hi(v.y));
     };
     for (int j = 0; j < p.k; ++j) {
       const float wj = __ldg(p.w + (long long)t * p.k + j);
       const int row = __ldg(p.row_of + (long long)t * p.k + j);
-      const float4 v = row >= 0 ? y4(row) : __ldcg(reinterpret_cast<const float4 *>(p.y32 + (long long)~row * p.d + o));
+      const float4 v = row >= 0 ? y4(p.y, row) : y4(p.yp, ~row);
       a0 = fmaf(wj, v.x, a0);
       a1 = fmaf(wj, v.y, a1);
       a2 = fmaf(wj, v.z, a2);
       a3 = fmaf(wj, v.w, a3);
     }
     if (p.has_shared) {
-      const float4 sh = y4(P + t);
+      const float4 sh = y4(p.y, P + t);
       a0 += sh.x;
       a1 += sh.y;
       a2 += sh.z;
@@ -1492,6 +1492,31 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(PfCombineParams p)
       *reinterpret_cast<uint2 *>(xr) = o2;
     }
   }
+}
+
+// One expert per row (given routing with kk = 1, weight 1): row t's output
+// y in fp16, in row order, copied from the GEMM's grouped rows or the GEMV's
+// pair rows (an expert-parallel owner's result).
+struct PfRowsParams {
+  const __half *y;    // fp16 [rows][d] grouped order (GEMM experts)
+  const __half *yp;   // fp16 [T][d] by pair id (GEMV experts: row_of < 0)
+  const int *row_of;  // [T]
+  int T, d;
+  __half *out;        // fp16 [T][d]
+};
+
+__global__ void __launch_bounds__(256) prefill_rows_kernel(PfRowsParams p) {
+  pdl_wait();
+  const int per_t = p.d / 8;
+  const long long n = (long long)p.T * per_t;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / per_t), o = (int)(i - (long long)t * per_t) * 8;
+    const int row = __ldg(p.row_of + t);
+    const __half *src = row >= 0 ? p.y + (long long)row * p.d : p.yp + (long long)~row * p.d;
+    *reinterpret_cast<uint4 *>(p.out + (long long)t * p.d + o) = __ldcg(reinterpret_cast<const uint4 *>(src + o));
+  }
+  pdl_launch_dependents();
 }
 
 }  // namespace moe

@@ -12,10 +12,10 @@ route, run the selected experts, combine into the residual) becomes:
    by the expert's owner, and the rows' expert ids;
 3. an all-to-all of those rows and ids (the split sizes are exchanged first);
 4. each owner runs its experts on the rows it received
-   (``moe_experts_given``, one expert per row with weight 1, so a row's
-   output is that expert's y);
+   (``moe_experts_rows``: one expert per row, each row's output y in fp16);
 5. an all-to-all of the outputs back to their source ranks, and the shared
-   expert on the rank's own rows;
+   expert on the rank's own rows (``moe_experts_given`` with no routed
+   experts);
 6. ``moe_ep_combine``: ``x <- bf16(x + sum_j w_j y_j + y_shared)``, j in
    order, with the one-GPU combine's arithmetic.
 
@@ -64,15 +64,14 @@ class DeviceOps:
         return send_h, send_e, row_of, counts
 
     def experts(self, layer, rows_h, M, rows_e):
-        """y [M, d] fp32: row i's output of expert rows_e[i] (M may be 0).
-        More rows than the context holds run in slices of max_tokens rows."""
+        """y [M, d] fp16: row i's output of expert rows_e[i] (M may be 0), in
+        the fp16 the chunk path keeps expert outputs in.  More rows than the
+        context holds run in slices of max_tokens rows."""
         self.last_rows = M
-        y = torch.empty((M, self.d), dtype=torch.float32, device=self.device)
-        ones = torch.ones(min(M, self.max_tokens), dtype=torch.float32, device=self.device)
+        y = torch.empty((M, self.d), dtype=torch.float16, device=self.device)
         for a in range(0, M, self.max_tokens):
             n = min(self.max_tokens, M - a)
-            self.B.moe_experts_given(self.ctx, layer, rows_h[a:a + n], n, 1, rows_e[a:a + n],
-                                     ones[:n], 0, y[a:a + n])
+            self.B.moe_experts_rows(self.ctx, layer, rows_h[a:a + n], n, rows_e[a:a + n], y[a:a + n])
         return y
 
     def shared(self, layer, h, N):

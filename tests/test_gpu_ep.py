@@ -339,7 +339,7 @@ def test_rmsnorm_call_against_the_oracle(B, with_gamma):
 def test_one_rank_chain_into_delta(B, fmt):
     """The expert-parallel steps by hand at one rank, ending in
     moe_ep_combine's delta form: route, dispatch, the owner's experts (one
-    expert per row, weight 1), the shared expert, combine; equal to
+    expert per row, fp16 outputs), the shared expert, combine; equal to
     moe_prefill_delta bit for bit."""
     spec = LayerSpec(fmt=fmt, zipf=True, **SMALL)
     N = 600
@@ -360,9 +360,8 @@ def test_one_rank_chain_into_delta(B, fmt):
         row_of = torch.empty(P, dtype=torch.int32, device="cuda")
         counts = B.moe_ep_dispatch(ctx, idx, N, 1, x, send_h, send_e, row_of)
         assert counts == [P]
-        y = torch.empty((P, spec.d), dtype=torch.float32, device="cuda")
-        ones = torch.ones(P, dtype=torch.float32, device="cuda")
-        B.moe_experts_given(ctx, 0, send_h, P, 1, send_e, ones, 0, y)
+        y = torch.empty((P, spec.d), dtype=torch.float16, device="cuda")
+        B.moe_experts_rows(ctx, 0, send_h, P, send_e, y)
         ysh = torch.empty((N, spec.d), dtype=torch.float32, device="cuda")
         B.moe_experts_given(ctx, 0, x, N, 0, None, None, 1, ysh)
         got = torch.empty_like(want)
