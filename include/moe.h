@@ -30,7 +30,11 @@
  *  - Layouts are row-major and densely packed unless stated otherwise.
  *    Activations are bfloat16 bit patterns (uint16), router weights fp32.
  *  - A context is used from one host thread at a time and on the device that
- *    was current when it was created.
+ *    was current when it was created.  Its compute calls share the context's
+ *    scratch memory, so calls on different streams must not overlap: issue
+ *    them on one stream, or order the streams.  (Chunk calls fork internal
+ *    work to a stream of the context's own and join it before they return
+ *    to the caller's stream.)
  *
  * Packed expert format (input of moe_load_experts / moe_load_shared).  The
  * pages print no bit layout; these formats are this library's own:
