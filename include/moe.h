@@ -167,9 +167,10 @@ MOE_API moe_status moe_set_slots(moe_ctx *ctx, const int32_t *slot_of);
  * "Architecture overview": the router picks 10 of 512 experts per token;
  * the "Doorbell handshake" section ends the "pre" half of a block with the
  * router's ids and weights).  Windows of more than 32 tokens select the
- * top-k one warp per token; with E a multiple of 256 and a context
- * configured for chunks (max_tokens > 32), the logits come from the
- * tensor-core router (see moe_set_router).  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
+ * top-k one warp per token; in a context configured for chunks
+ * (max_tokens > 32) whose shapes the grouped GEMM takes, they route exactly
+ * as moe_prefill_route (logits on the tensor cores when E is a multiple of
+ * 256, see moe_set_router; the sort by expert over many CTAs).  h_dev: bf16 [T, d] router input.  idx_dev int32 [T, k] and
  * w_dev fp32 [T, k] receive each token's experts and renormalised weights,
  * ordered by descending logit (equal logits: lower expert id first).
  * bucket_off_dev int32 [E+1] (exclusive prefix of tokens per expert) and

@@ -1519,6 +1519,16 @@ moe_status moe_route(moe_ctx *c, int layer, const void *h, int T, int32_t *idx, 
   if (!c->has_router[layer]) return fail(c, MOE_ERR_STATE, "router of layer %d not set", layer);
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
+  if (use_prefill_gemm(c, T)) {
+    // a chunk in a chunk-configured context: the chunk path's routing, whose
+    // parallel sort by expert gives the same buckets as the one-CTA sort below
+    moe_status st = prefill_route_impl(c, layer, (const uint16_t *)h, T, idx, w, bperm, s, kHotMinTokens);
+    if (st) return st;
+    if (boff)
+      CUDA_TRY(c, cudaMemcpyAsync(boff, c->pf_eoff, (size_t)(c->E + 1) * sizeof(int32_t),
+                                  cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+  }
   FinishParams fp = finish_params(c, layer, T);
   fp.idx = idx;
   fp.w = w;
