@@ -515,8 +515,10 @@ def measure(args, world, ctx, spec, n_rot, K, W):
         },
         "e2e": {"value": whole_job_rate(world, tok, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * D * 2, "d2h_bytes_per_step": T * D * 2},
-        # chunks: router, top-k, column scan, scan, scatter, 2 GEMMs, 2 GEMVs, combine
-        "gpu_launches": K * (1 if single else 10),
+        # chunks: router, top-k, column scan, scan, scatter, 2 GEMMs, 2 GEMVs,
+        # combine, and one more: the split router's sum (the Q2 chunks of 64-320
+        # tokens) or the column scan's counting pass (8192 tokens)
+        "gpu_launches": K * (1 if single else 11),
         "clocks": clocks,
     }
     if single:
