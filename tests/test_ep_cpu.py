@@ -47,6 +47,7 @@ print(json.dumps({"rank": rank, "rows": len(ops.received)}))
     (2, 16, [37, 20], True, False),
     (3, 24, [9, 1, 30], False, True),
     (3, 24, [0, 25, 12], True, False),   # a rank with no tokens of its own still serves
+    (4, 32, [11, 0, 6, 19], True, True),
 ])
 def test_expert_parallel_gloo_ranks_match_the_one_process_layer(tmp_path, world, E, sizes, shared,
                                                                  norm):
